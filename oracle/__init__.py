@@ -1,0 +1,172 @@
+"""Float64 CPU oracle for the selective state-space scan (S6).
+
+TEST INFRASTRUCTURE ONLY.  The product path (the CUDA library and its Python
+binding) never imports this package.  Only ``tests/``, the package smoke check
+and the benchmark's CPU-baseline leg use it.
+
+The arithmetic lives in ``ssm_ref.c`` (plain C, double precision, sequential
+in time).  This module compiles it with gcc and marshals numpy arrays to it.
+Activations are passed as stored: ``float32`` arrays, or bfloat16 given as
+``uint16`` bit patterns; the C code widens each value exactly to double.
+
+Sources: the Mamba pages' description of the selection mechanism (input-
+dependent dt, B, C), the ZOH + Euler discretisation named in the "Mamba3"
+post, the recurrent one-step mode, and Gu & Dao Appendix D ("Speed": chunks
+continue from the carried state).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ssm_ref.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD, "libssm_ref.so")
+
+_lib = None
+
+
+def build(force: bool = False, src: str = _SRC, out: str = _LIB_PATH) -> str:
+    """Compile the C oracle into a shared library and return its path.
+
+    No fast-math and no FMA contraction: the double-precision arithmetic is
+    evaluated exactly as written.
+    """
+    os.makedirs(os.path.dirname(out), exist_ok=True)
+    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src):
+        cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+               "-shared", "-fPIC", "-o", out, src, "-lm"]
+        subprocess.check_call(cmd)
+    return out
+
+
+class Oracle:
+    """ctypes handle on one compiled copy of the oracle library."""
+
+    def __init__(self, path: str):
+        lib = ctypes.CDLL(path)
+        P, I, L = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+        lib.ssm_ref_fwd.argtypes = [P, P, P, I, P, P, P, P, P, P, I, L, L, L, L, P, P, I]
+        lib.ssm_ref_fwd.restype = I
+        lib.ssm_ref_fwd_channels.argtypes = [P, P, P, I, P, P, P, P, P, P, I, L, L, L, L,
+                                             P, L, P, P, I]
+        lib.ssm_ref_fwd_channels.restype = I
+        lib.ssm_ref_step.argtypes = [P, P, P, P, I, P, P, P, P, P, I, L, L, L, P, I]
+        lib.ssm_ref_step.restype = I
+        self._lib = lib
+
+    # -- marshalling helpers ---------------------------------------------
+    @staticmethod
+    def _act(a, dtype_code):
+        if a is None:
+            return None
+        a = np.ascontiguousarray(a)
+        want = np.uint16 if dtype_code == 1 else np.float32
+        if a.dtype != want:
+            raise TypeError(f"activation dtype {a.dtype}, expected {want}")
+        return a
+
+    @staticmethod
+    def _f32(a):
+        if a is None:
+            return None
+        return np.ascontiguousarray(a, dtype=np.float32)
+
+    @staticmethod
+    def _ptr(a):
+        return None if a is None else a.ctypes.data
+
+    @staticmethod
+    def _dtype_code(x):
+        if x.dtype == np.uint16:
+            return 1
+        if x.dtype == np.float32:
+            return 0
+        raise TypeError(f"activations must be float32 or bf16 bits (uint16), got {x.dtype}")
+
+    # -- entry points -----------------------------------------------------
+    def fwd(self, x, delta, delta_bias, softplus, A, B, C, D, z, h0, threads=0,
+            want_h_last=True):
+        """Full scan.  Returns (out [b,d,L] float64, h_last [b,d,N] float64 or None)."""
+        code = self._dtype_code(x)
+        x, delta, B, C, z = (self._act(t, code) for t in (x, delta, B, C, z))
+        A, D, delta_bias, h0 = (self._f32(t) for t in (A, D, delta_bias, h0))
+        batch, dim, L = x.shape
+        N = A.shape[1]
+        out = np.empty((batch, dim, L), np.float64)
+        hl = np.empty((batch, dim, N), np.float64) if want_h_last else None
+        rc = self._lib.ssm_ref_fwd(self._ptr(x), self._ptr(delta), self._ptr(delta_bias),
+                                   int(bool(softplus)), self._ptr(A), self._ptr(B), self._ptr(C),
+                                   self._ptr(D), self._ptr(z), self._ptr(h0), code,
+                                   batch, L, dim, N, self._ptr(out), self._ptr(hl), int(threads))
+        if rc != 0:
+            raise ValueError("oracle rejected the arguments")
+        return out, hl
+
+    def fwd_channels(self, x, delta, delta_bias, softplus, A, B, C, D, z, h0, channels,
+                     threads=0):
+        """Scan of selected channels (flat index b*dim + d).
+
+        Returns (out [nsel, L] float64, h_last [nsel, N] float64)."""
+        code = self._dtype_code(x)
+        x, delta, B, C, z = (self._act(t, code) for t in (x, delta, B, C, z))
+        A, D, delta_bias, h0 = (self._f32(t) for t in (A, D, delta_bias, h0))
+        batch, dim, L = x.shape
+        N = A.shape[1]
+        chan = np.ascontiguousarray(channels, dtype=np.int64)
+        out = np.empty((chan.size, L), np.float64)
+        hl = np.empty((chan.size, N), np.float64)
+        rc = self._lib.ssm_ref_fwd_channels(
+            self._ptr(x), self._ptr(delta), self._ptr(delta_bias), int(bool(softplus)),
+            self._ptr(A), self._ptr(B), self._ptr(C), self._ptr(D), self._ptr(z), self._ptr(h0),
+            code, batch, L, dim, N, self._ptr(chan), chan.size, self._ptr(out), self._ptr(hl),
+            int(threads))
+        if rc != 0:
+            raise ValueError("oracle rejected the arguments")
+        return out, hl
+
+    def step(self, state, x, delta, delta_bias, softplus, A, B, C, D, z, threads=0):
+        """One decode step.  `state` ([b,d,N] float64) is updated in place.
+
+        Token tensors: x, delta, z [b,d]; B, C [b,N].  Returns out [b,d] float64."""
+        if state.dtype != np.float64 or not state.flags.c_contiguous:
+            raise TypeError("state must be a contiguous float64 array")
+        code = self._dtype_code(x)
+        x, delta, B, C, z = (self._act(t, code) for t in (x, delta, B, C, z))
+        A, D, delta_bias = (self._f32(t) for t in (A, D, delta_bias))
+        batch, dim = x.shape
+        N = A.shape[1]
+        out = np.empty((batch, dim), np.float64)
+        rc = self._lib.ssm_ref_step(self._ptr(state), self._ptr(x), self._ptr(delta),
+                                    self._ptr(delta_bias), int(bool(softplus)), self._ptr(A),
+                                    self._ptr(B), self._ptr(C), self._ptr(D), self._ptr(z), code,
+                                    batch, dim, N, self._ptr(out), int(threads))
+        if rc != 0:
+            raise ValueError("oracle rejected the arguments")
+        return out
+
+
+def load(path: str | None = None) -> Oracle:
+    """Build (if needed) and load the oracle library; cached per process."""
+    global _lib
+    if path is not None:
+        return Oracle(path)
+    if _lib is None:
+        _lib = Oracle(build())
+    return _lib
+
+
+def fwd(*args, **kw):
+    return load().fwd(*args, **kw)
+
+
+def fwd_channels(*args, **kw):
+    return load().fwd_channels(*args, **kw)
+
+
+def step(*args, **kw):
+    return load().step(*args, **kw)

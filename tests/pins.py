@@ -1,0 +1,334 @@
+"""Checks that pin the float64 oracle to facts other than its own loop.
+
+Each pin takes an oracle handle (``oracle.Oracle``) and raises AssertionError
+when the oracle disagrees with what the mathematics fixes.  The expected values
+are computed here by independent routes: closed forms, numpy/scipy library
+routines, the convolutional mode of an LTI system, chunk-split invariance and
+brute-force evaluation of every bracketing of the associative combine.
+
+The mutation test runs every pin against deliberately broken copies of the
+oracle and requires each copy to fail at least one pin.
+"""
+from __future__ import annotations
+
+import itertools
+import math
+from functools import lru_cache
+
+import numpy as np
+from scipy.special import expit
+
+RTOL = 1e-11
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _f32(a):
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def _close(got, want, rtol=RTOL, atol=1e-13, what=""):
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    assert got.shape == want.shape, (what, got.shape, want.shape)
+    err = np.abs(got - want)
+    lim = atol + rtol * np.abs(want)
+    bad = err > lim
+    assert not bad.any(), f"{what}: max err {err.max():.3e} at {np.argwhere(bad)[0]}"
+
+
+def _rand_case(seed, b=2, d=3, n=4, L=5, h0=True, z=True, Dskip=True, bias=True):
+    r = _rng(seed)
+    return dict(
+        x=_f32(r.standard_normal((b, d, L))),
+        delta=_f32(r.standard_normal((b, d, L)) * 0.5),
+        z=_f32(r.standard_normal((b, d, L))) if z else None,
+        B=_f32(r.standard_normal((b, n, L))),
+        C=_f32(r.standard_normal((b, n, L))),
+        A=_f32(-r.uniform(0.2, 2.0, (d, n))),
+        D=_f32(r.standard_normal(d)) if Dskip else None,
+        delta_bias=_f32(r.standard_normal(d) * 0.3) if bias else None,
+        h0=_f32(r.standard_normal((b, d, n))) if h0 else None,
+        softplus=True,
+    )
+
+
+def _call(orc, c, **over):
+    a = dict(c)
+    a.update(over)
+    return orc.fwd(a["x"], a["delta"], a["delta_bias"], a["softplus"], a["A"], a["B"], a["C"],
+                   a["D"], a["z"], a["h0"])
+
+
+def _softplus_lib(v):
+    # numpy's log(exp(0) + exp(v)) is softplus without our formula
+    return np.logaddexp(0.0, v)
+
+
+# ---------------------------------------------------------------------------
+def pin_single_step_closed_form(orc):
+    """(a) L = 1: one ZOH/Euler step from h0, readout, D skip and silu gate,
+    written as one vectorised expression (no loop over t or n)."""
+    for seed, sp in ((1, True), (2, False)):
+        c = _rand_case(seed, L=1)
+        c["softplus"] = sp
+        x, v = c["x"].astype(np.float64), c["delta"].astype(np.float64)
+        v = v + c["delta_bias"].astype(np.float64)[None, :, None]
+        dt = _softplus_lib(v) if sp else v                       # [b,d,1]
+        A = c["A"].astype(np.float64)                              # [d,n]
+        Bm, Cm = c["B"].astype(np.float64), c["C"].astype(np.float64)  # [b,n,1]
+        h0 = c["h0"].astype(np.float64)                            # [b,d,n]
+        h1 = np.exp(dt * A[None]) * h0 + dt * x * np.transpose(Bm, (0, 2, 1))
+        y = np.einsum("bdn,bn->bd", h1, Cm[:, :, 0])[..., None] + c["D"][None, :, None] * x
+        zz = c["z"].astype(np.float64)
+        want = y * zz * expit(zz)
+        out, hl = _call(orc, c)
+        _close(out, want, what="L=1 out")
+        _close(hl, h1, what="L=1 h_last")
+
+
+def pin_hand_values(orc):
+    """(a') Exactly representable single step worked by hand: softplus off,
+    dt = ln 2 and A = -1 give Abar = 1/2; x = 2, B = 3, C = 5, D = 0.5,
+    h0 = 4, no gate.  h1 = 2 + 6 ln 2, y = 5 h1 + 1."""
+    ln2 = math.log(2.0)
+    one = lambda v: np.full((1, 1, 1), v, np.float32)
+    c = dict(x=one(2.0), delta=_f32(np.full((1, 1, 1), ln2)), z=None, B=one(3.0), C=one(5.0),
+             A=_f32([[-1.0]]), D=_f32([0.5]), delta_bias=None, h0=one(4.0), softplus=False)
+    dt = float(np.float32(ln2))
+    out, hl = _call(orc, c)
+    h1 = math.exp(-dt) * 4.0 + dt * 6.0
+    _close(hl[0, 0, 0], h1, rtol=1e-15, what="hand h1")
+    _close(out[0, 0, 0], 5.0 * h1 + 1.0, rtol=1e-15, what="hand y")
+    assert abs(hl[0, 0, 0] - (2.0 + 6.0 * ln2)) < 1e-6
+
+
+def pin_geometric_sum(orc):
+    """(b) dt, B, C, x (and z) constant over t: h_t = a^(t+1) h0 + u B (1 - a^(t+1)) / (1 - a),
+    a = exp(dt A), u = dt x; y_t = C.h_t + D x, gated."""
+    r = _rng(3)
+    b, d, n, L = 2, 3, 5, 40
+    xv = r.standard_normal((b, d, 1))
+    vv = r.standard_normal((b, d, 1)) * 0.5
+    zv = r.standard_normal((b, d, 1))
+    Bv = r.standard_normal((b, n, 1))
+    Cv = r.standard_normal((b, n, 1))
+    c = dict(x=_f32(np.repeat(xv, L, 2)), delta=_f32(np.repeat(vv, L, 2)),
+             z=_f32(np.repeat(zv, L, 2)), B=_f32(np.repeat(Bv, L, 2)), C=_f32(np.repeat(Cv, L, 2)),
+             A=_f32(-r.uniform(0.1, 1.5, (d, n))), D=_f32(r.standard_normal(d)),
+             delta_bias=_f32(r.standard_normal(d) * 0.2), h0=_f32(r.standard_normal((b, d, n))),
+             softplus=True)
+    dt = _softplus_lib(c["delta"][:, :, :1].astype(np.float64) + c["delta_bias"][None, :, None])
+    a = np.exp(dt * c["A"][None].astype(np.float64))                     # [b,d,n]
+    u = dt * c["x"][:, :, :1].astype(np.float64)                           # [b,d,1]
+    Bn = np.transpose(c["B"][:, :, :1].astype(np.float64), (0, 2, 1))      # [b,1,n]
+    Cn = np.transpose(c["C"][:, :, :1].astype(np.float64), (0, 2, 1))
+    t = np.arange(L)[None, None, None, :] + 1.0                            # [1,1,1,L]
+    ap = a[..., None] ** t                                                 # [b,d,n,L]
+    h = ap * c["h0"].astype(np.float64)[..., None] + (u * Bn)[..., None] * (1 - ap) / (1 - a)[..., None]
+    y = np.einsum("bdnl,bdn->bdl", h, np.broadcast_to(Cn, a.shape)) + \
+        c["D"][None, :, None] * c["x"].astype(np.float64)
+    zz = c["z"].astype(np.float64)
+    want = y * zz * expit(zz)
+    out, hl = _call(orc, c)
+    _close(out, want, rtol=1e-10, what="geometric out")
+    _close(hl, h[..., -1], rtol=1e-10, what="geometric h_last")
+
+
+def pin_convolution_mode(orc):
+    """(c) Input-independent dt, B, C with h0 = 0 make the system LTI, so the
+    scan equals the convolutional mode y = K * x + D x with kernel
+    K_k = sum_n C_n Abar_n^k dt B_n (computed with numpy.convolve)."""
+    r = _rng(4)
+    b, d, n, L = 2, 3, 6, 64
+    vv = r.standard_normal((1, d, 1)) * 0.5
+    Bv = r.standard_normal((b, n, 1))
+    Cv = r.standard_normal((b, n, 1))
+    x = _f32(r.standard_normal((b, d, L)))
+    c = dict(x=x, delta=_f32(np.repeat(np.repeat(vv, b, 0), L, 2)), z=None,
+             B=_f32(np.repeat(Bv, L, 2)), C=_f32(np.repeat(Cv, L, 2)),
+             A=_f32(-r.uniform(0.05, 1.0, (d, n))), D=_f32(r.standard_normal(d)),
+             delta_bias=_f32(r.standard_normal(d) * 0.2), h0=None, softplus=True)
+    out, _ = _call(orc, c)
+    dt = _softplus_lib(c["delta"][0, :, 0].astype(np.float64) + c["delta_bias"])   # [d]
+    k = np.arange(L)
+    for bi in range(b):
+        for di in range(d):
+            abar = np.exp(dt[di] * c["A"][di].astype(np.float64))                # [n]
+            K = ((c["C"][bi, :, 0].astype(np.float64) * dt[di] * c["B"][bi, :, 0])[:, None]
+                 * abar[:, None] ** k[None, :]).sum(0)
+            xs = x[bi, di].astype(np.float64)
+            want = np.convolve(xs, K)[:L] + c["D"][di] * xs
+            _close(out[bi, di], want, rtol=1e-10, atol=1e-12, what=f"conv b{bi} d{di}")
+
+
+def pin_chunk_split(orc):
+    """(d) Scanning [0, m) and then [m, L) from the carried state equals the
+    full scan, for several split points m."""
+    c = _rand_case(5, b=2, d=3, n=4, L=37)
+    out, hl = _call(orc, c)
+    seq_keys = ("x", "delta", "z", "B", "C")
+    for m in (1, 5, 16, 36):
+        first = {k: (np.ascontiguousarray(v[..., :m]) if k in seq_keys else v) for k, v in c.items()}
+        second = {k: (np.ascontiguousarray(v[..., m:]) if k in seq_keys else v) for k, v in c.items()}
+        o1, h1 = _call(orc, first)
+        second["h0"] = _f32(h1)
+        o2, h2 = _call(orc, second)
+        # the carried state is rounded to float32 between the two calls
+        _close(o1, out[..., :m], rtol=1e-12, what=f"split m={m} first")
+        _close(o2, out[..., m:], rtol=2e-5, atol=2e-5, what=f"split m={m} second")
+        _close(h2, hl, rtol=2e-5, atol=2e-5, what=f"split m={m} h_last")
+
+
+@lru_cache(maxsize=None)
+def _bracketings(lo, hi):
+    """All full bracketings of the elements lo..hi-1 as nested tuples."""
+    if hi - lo == 1:
+        return [lo]
+    res = []
+    for m in range(lo + 1, hi):
+        for left in _bracketings(lo, m):
+            for right in _bracketings(m, hi):
+                res.append((left, right))
+    return res
+
+
+def _eval_bracket(tree, pairs):
+    """Combine affine maps h -> a h + b, earlier map first:
+    (a1, b1) then (a2, b2) gives (a2 a1, a2 b1 + b2)."""
+    if isinstance(tree, int):
+        return pairs[tree]
+    a1, b1 = _eval_bracket(tree[0], pairs)
+    a2, b2 = _eval_bracket(tree[1], pairs)
+    return a2 * a1, a2 * b1 + b2
+
+
+def pin_associative_brute_force(orc):
+    """(e) On tiny L, every bracketing of the associative combine of the
+    per-step pairs (Abar_t, Bbar_t x_t) gives the state the oracle reaches; the
+    prefix of each t gives y_t.  This is the algebra a parallel scan relies on."""
+    for L in (1, 2, 3, 5, 6):
+        c = _rand_case(10 + L, b=1, d=2, n=3, L=L)
+        out, hl = _call(orc, c)
+        dt = _softplus_lib(c["delta"].astype(np.float64) + c["delta_bias"][None, :, None])  # [1,d,L]
+        for di in range(2):
+            for ni in range(3):
+                pairs = [(math.exp(dt[0, di, t] * float(c["A"][di, ni])),
+                          dt[0, di, t] * float(c["B"][0, ni, t]) * float(c["x"][0, di, t]))
+                         for t in range(L)]
+                h0 = float(c["h0"][0, di, ni])
+                for tree in _bracketings(0, L):
+                    a, bb = _eval_bracket(tree, pairs)
+                    assert abs(a * h0 + bb - hl[0, di, ni]) <= 1e-12 * (1 + abs(hl[0, di, ni])), \
+                        (L, di, ni, tree)
+        # outputs from prefixes, bracketed right-to-left
+        for di in range(2):
+            for t in range(L):
+                y = float(c["D"][di]) * float(c["x"][0, di, t])
+                for ni in range(3):
+                    pairs = [(math.exp(dt[0, di, s] * float(c["A"][di, ni])),
+                              dt[0, di, s] * float(c["B"][0, ni, s]) * float(c["x"][0, di, s]))
+                             for s in range(t + 1)]
+                    tree = _bracketings(0, t + 1)[-1]
+                    a, bb = _eval_bracket(tree, pairs)
+                    y += float(c["C"][0, ni, t]) * (a * float(c["h0"][0, di, ni]) + bb)
+                zz = float(c["z"][0, di, t])
+                y *= zz * expit(zz)
+                assert abs(y - out[0, di, t]) <= 1e-11 * (1 + abs(y)), (L, di, t)
+
+
+def pin_degenerate(orc):
+    """Special cases: dt = 0 keeps h = h0; A -> -inf makes the system
+    memoryless (h_t = dt B_t x_t); optional inputs absent mean zero / identity."""
+    c = _rand_case(20, L=7)
+    c0 = dict(c, delta=np.zeros_like(c["delta"]), delta_bias=None, softplus=False)
+    out, hl = _call(orc, c0)
+    _close(hl, c["h0"], rtol=0, atol=0, what="dt=0 state")
+    D64, x64 = c["D"].astype(np.float64), c["x"].astype(np.float64)
+    y = np.einsum("bdn,bnl->bdl", c["h0"].astype(np.float64), c["C"].astype(np.float64)) + \
+        D64[None, :, None] * x64
+    zz = c["z"].astype(np.float64)
+    _close(out, y * zz * expit(zz), rtol=1e-12, what="dt=0 out")
+
+    cinf = dict(c, A=np.full_like(c["A"], -1e30))
+    out, hl = _call(orc, cinf)
+    dt = _softplus_lib(c["delta"].astype(np.float64) + c["delta_bias"][None, :, None])
+    ht = dt[:, :, None, :] * c["B"].astype(np.float64)[:, None] * x64[:, :, None, :]
+    y = np.einsum("bdnl,bnl->bdl", ht, c["C"].astype(np.float64)) + D64[None, :, None] * x64
+    _close(out, y * zz * expit(zz), rtol=1e-12, what="memoryless out")
+    _close(hl, ht[..., -1], rtol=1e-12, what="memoryless h_last")
+
+    # no h0 / D / z / bias equals passing zeros / no gate
+    cn = dict(c, h0=None, D=None, z=None, delta_bias=None)
+    cz = dict(c, h0=np.zeros_like(c["h0"]), D=np.zeros_like(c["D"]), z=None,
+              delta_bias=np.zeros_like(c["delta_bias"]))
+    o1, h1 = _call(orc, cn)
+    o2, h2 = _call(orc, cz)
+    _close(o1, o2, rtol=0, atol=0, what="optional args")
+    _close(h1, h2, rtol=0, atol=0, what="optional args h")
+
+
+def pin_softplus_extremes(orc):
+    """dt = softplus(v) is read back through A = 0, h0 = 0, B = x = 1, L = 1
+    (then h1 = dt): compare with math.log1p(math.exp(v)) and its limits."""
+    vs = np.array([-80.0, -20.0, -3.0, 0.0, 0.5, 8.0, 30.0, 300.0], np.float32)
+    d = vs.size
+    c = dict(x=np.ones((1, d, 1), np.float32), delta=vs.reshape(1, d, 1).copy(), z=None,
+             B=np.ones((1, 1, 1), np.float32), C=np.ones((1, 1, 1), np.float32),
+             A=np.zeros((d, 1), np.float32), D=None, delta_bias=None, h0=None, softplus=True)
+    _, hl = _call(orc, c)
+    for i, v in enumerate(vs.astype(np.float64)):
+        want = math.log1p(math.exp(v))  # the definition; no overflow for these v
+        assert abs(hl[0, i, 0] - want) <= 1e-14 * max(1.0, abs(want)) + 1e-300, (v, hl[0, i, 0])
+    assert hl[0, 0, 0] > 0.0  # softplus(-80) = 1.8e-35 is not flushed to zero
+
+
+def pin_bf16_widening(orc):
+    """bf16 inputs are widened exactly: the oracle on bf16 bit patterns equals
+    the oracle on the same values given as float32."""
+    c = _rand_case(30, L=9)
+    def bits(a):
+        u = np.ascontiguousarray(a, np.float32).view(np.uint32)
+        return (u >> 16).astype(np.uint16)  # truncation: any bf16 value will do
+    cb = {k: (bits(v) if k in ("x", "delta", "z", "B", "C") else v) for k, v in c.items()}
+    cf = {k: ((bits(v).astype(np.uint32) << 16).view(np.float32) if k in ("x", "delta", "z", "B", "C")
+              else v) for k, v in c.items()}
+    o1, h1 = _call(orc, cb)
+    o2, h2 = _call(orc, cf)
+    _close(o1, o2, rtol=0, atol=0, what="bf16 widening")
+    _close(h1, h2, rtol=0, atol=0, what="bf16 widening h")
+
+
+def pin_step_equals_scan(orc):
+    """The recurrent mode: T single steps from h0 equal one scan over T tokens;
+    channel-subset entry equals the full scan on those channels."""
+    c = _rand_case(40, b=2, d=3, n=4, L=6)
+    out, hl = _call(orc, c)
+    state = c["h0"].astype(np.float64).copy()
+    for t in range(6):
+        tok = {k: np.ascontiguousarray(c[k][..., t]) for k in ("x", "delta", "z", "B", "C")}
+        o = orc.step(state, tok["x"], tok["delta"], c["delta_bias"], True, c["A"], tok["B"], tok["C"],
+                     c["D"], tok["z"])
+        _close(o, out[..., t], rtol=1e-13, what=f"step t={t}")
+    _close(state, hl, rtol=1e-13, what="step state")
+    sel = np.array([5, 0, 3])
+    o, h = orc.fwd_channels(c["x"], c["delta"], c["delta_bias"], True, c["A"], c["B"], c["C"],
+                            c["D"], c["z"], c["h0"], sel)
+    _close(o, out.reshape(6, 6)[sel], rtol=0, atol=0, what="channel subset out")
+    _close(h, hl.reshape(6, 4)[sel], rtol=0, atol=0, what="channel subset h")
+
+
+ALL_PINS = [
+    pin_single_step_closed_form,
+    pin_hand_values,
+    pin_geometric_sum,
+    pin_convolution_mode,
+    pin_chunk_split,
+    pin_associative_brute_force,
+    pin_degenerate,
+    pin_softplus_extremes,
+    pin_bf16_widening,
+    pin_step_equals_scan,
+]

@@ -1,0 +1,64 @@
+"""Plant plausible mistakes in copies of the oracle and check that the pins
+catch every one of them.  Each mutant is the oracle's C source with one text
+substitution, compiled into a temporary library (the oracle itself is never
+modified)."""
+import os
+
+import pytest
+
+import oracle
+import pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "ssm_ref.c")
+
+# (name, original text, mutated text) -- each original must occur in the source
+MUTANTS = [
+    ("h0 ignored", "h[n] = a->h0 ? (double)a->h0[chan * N + n] : 0.0;", "h[n] = 0.0;"),
+    ("A sign flipped", "exp(dt * (double)a->A[d * N + n])", "exp(-dt * (double)a->A[d * N + n])"),
+    ("Euler term without dt", "h[n] = abar * h[n] + dt * bt * xt;", "h[n] = abar * h[n] + bt * xt;"),
+    ("ZOH uses exp(A) not exp(dt A)", "exp(dt * (double)a->A[d * N + n])", "exp((double)a->A[d * N + n])"),
+    ("D skip dropped", "y += (double)a->D[d] * xt;", "y += 0.0;"),
+    ("gate is sigmoid not silu", "return z / (1.0 + exp(-z));", "return 1.0 / (1.0 + exp(-z));"),
+    ("softplus dropped", "const double dt = a->softplus ? softplus_ref(v) : v;", "const double dt = v;"),
+    ("bias ignored", "v += (double)a->delta_bias[d];", "v += 0.0;"),
+    ("softplus sign", "return (v > 0.0 ? v : 0.0) + log1p(exp(-fabs(v)));",
+     "return (v > 0.0 ? v : 0.0) + log1p(exp(fabs(v)));"),
+    ("B and C swapped", "y += load_act(a->C, (b * N + n) * L + t, a->dtype) * h[n];",
+     "y += load_act(a->B, (b * N + n) * L + t, a->dtype) * h[n];"),
+    ("B read transposed [b][t][n]", "load_act(a->B, (b * N + n) * L + t, a->dtype);",
+     "load_act(a->B, (b * L + t) * N + n, a->dtype);"),
+    ("x read one step late", "const double xt = load_act(a->x, chan * L + t, a->dtype);",
+     "const double xt = load_act(a->x, chan * L + (t + 1 < L ? t + 1 : t), a->dtype);"),
+    ("C readout dropped", "        double y = 0.0;\n        for (int64_t n = 0; n < N; n++)\n            y += load_act(a->C",
+     "        double y = 0.0;\n        for (int64_t n = 0; n < N; n++)\n            y += 0.0 * load_act(a->C"),
+    ("state decays twice", "h[n] = abar * h[n] + dt * bt * xt;", "h[n] = abar * abar * h[n] + dt * bt * xt;"),
+    ("A indexed [n][d]", "exp(dt * (double)a->A[d * N + n])", "exp(dt * (double)a->A[(n * a->dim + d) % (a->dim * N)])"),
+    ("h_last returns the initial state", "            hl[n] = h[n];",
+     "            hl[n] = a->h0 ? (double)a->h0[chan * N + n] : 0.0;"),
+    ("step ignores gate", "            y *= silu_ref(load_act(z, c, dtype));", "            y *= 1.0;"),
+    ("channel index b/d swapped", "scan_channel(&a, c / dim, c % dim,", "scan_channel(&a, c % batch, c / batch,"),
+]
+
+
+def _mutant(tmp_path, i, old, new):
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutant {i}: text not found"
+    msrc = src.replace(old, new)
+    c_path = tmp_path / f"mut{i}.c"
+    c_path.write_text(msrc)
+    so = str(tmp_path / f"libmut{i}.so")
+    oracle.build(force=True, src=str(c_path), out=so)
+    return oracle.load(so)
+
+
+@pytest.mark.parametrize("i", range(len(MUTANTS)), ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(tmp_path, i):
+    name, old, new = MUTANTS[i]
+    orc = _mutant(tmp_path, i, old, new)
+    caught = []
+    for pin in pins.ALL_PINS:
+        try:
+            pin(orc)
+        except (AssertionError, ValueError, FloatingPointError):
+            caught.append(pin.__name__)
+    assert caught, f"mutant '{name}' passed every pin"

@@ -1,0 +1,478 @@
+"""Benchmark of the selective-scan hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+One step = one forward scan of the Mamba-2.8B mixer-layer shape (batch 4,
+L 4096, D 5120, N 16, bf16 activations, fp32 state; also returns h_last) over
+inputs already resident in HBM.  The reported metric is achieved HBM
+bandwidth over the compulsory bytes (read x, delta, z, B, C, A, D, bias; write
+out and h_last), with Gtoken-channel/s and the fraction of the measured HBM
+peak alongside.  The recurrent decode step (256 x 5120 x 16 fp32 state,
+one bf16 token per sequence) is measured in the same run under "decode".
+
+Multi-GPU (torchrun): every rank scans its own independent copy of the
+workload (weak scaling, no data-path collective); the time is the maximum over
+ranks and the value the bytes of all ranks over that time.
+
+`--impl reference` times the float64 CPU oracle instead (the reference arm of
+this project), on bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import platform
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+FWD_CFG = 2
+DECODE_CFG = 4
+METRIC = "selective-scan fwd: achieved HBM GB/s (% of peak), Gtoken·ch/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def _cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor()
+
+
+def fwd_bytes(cfg):
+    c = workloads.CONFIGS[cfg]
+    return workloads.compulsory_bytes_fwd(c.batch, c.seqlen, c.dim, c.dstate,
+                                          2 if c.dtype == "bf16" else 4, c.has_h0, True)
+
+
+def step_bytes(cfg):
+    c = workloads.CONFIGS[cfg]
+    return workloads.compulsory_bytes_step(c.batch, c.dim, c.dstate, 2 if c.dtype == "bf16" else 4)
+
+
+def _source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "selective_state_space_38_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _profiled_traffic(kernel_key):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel
+    sources have not changed since it was taken (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)[kernel_key]
+    except (OSError, KeyError, ValueError):
+        return None
+    if rec.get("source_hash") != _source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index, period_s=0.005):
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # NVML unavailable: report no clocks
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def _max_over_ranks(value, world, device):
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def cpu_oracle_rate(cfg, target_s=10.0, threads=None):
+    """Time the float64 oracle (as it stands) on a bounded channel sample of
+    `cfg`; returns (GB/s-equivalent, seconds, channels, threads)."""
+    import oracle
+    orc = oracle.load()
+    c = workloads.CONFIGS[cfg]
+    threads = threads or _cores()
+    inp = workloads.make_inputs(cfg)
+    rng = np.random.default_rng(123)
+    nsel = 64
+    spent = 0.0
+    done = 0
+    while True:
+        chan = rng.choice(c.channels, nsel, replace=False)
+        t0 = time.perf_counter()
+        orc.fwd_channels(inp["x"], inp["delta"], inp["delta_bias"], True, inp["A"], inp["B"],
+                         inp["C"], inp["D"], inp["z"], inp["h0"], chan, threads=threads)
+        dt = time.perf_counter() - t0
+        spent += dt
+        done += nsel
+        if spent >= target_s or done >= c.channels:
+            break
+        # grow the sample towards the time budget
+        nsel = int(min(c.channels - done, max(nsel, nsel * max(1.0, (target_s - spent) / max(dt, 1e-3)))))
+        nsel = max(nsel, 1)
+    bytes_per_chan = fwd_bytes(cfg) / c.channels
+    return bytes_per_chan * done / spent / 1e9, spent, done, threads
+
+
+def run_reference(args):
+    world, rank, _ = _dist()
+    if rank != 0:
+        return 0
+    import oracle
+    orc = oracle.load()
+    c = workloads.CONFIGS[FWD_CFG]
+    inp = workloads.make_inputs(FWD_CFG)
+    threads = _cores()
+    rng = np.random.default_rng(7)
+    nsel = max(1, min(c.channels, int(os.environ.get("SSM_REF_CHANNELS", "256"))))
+    bytes_per_chan = fwd_bytes(FWD_CFG) / c.channels
+
+    def one():
+        chan = rng.choice(c.channels, nsel, replace=False)
+        t0 = time.perf_counter()
+        orc.fwd_channels(inp["x"], inp["delta"], inp["delta_bias"], True, inp["A"], inp["B"],
+                         inp["C"], inp["D"], inp["z"], inp["h0"], chan, threads=threads)
+        return time.perf_counter() - t0
+
+    for _ in range(args.warmup):
+        one()
+    times = [one() for _ in range(args.steps)]
+    total = sum(times)
+    value = bytes_per_chan * nsel * args.steps / total / 1e9
+    sample = (f"{nsel} random channels (full L={c.seqlen}) of the {c.name} forward scan per step; "
+              f"GB/s counts the compulsory bytes of those channels")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{c.name} forward scan (float64 CPU oracle, channel sample)",
+                   "batch": c.batch, "seqlen": c.seqlen, "dim": c.dim, "dstate": c.dstate},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": sample, "cpu": _cpu_model()},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+def _to_dev(a, device):
+    import torch
+    if a is None:
+        return None
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+    return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+
+def _to_pinned(a):
+    import torch
+    if a is None:
+        return None
+    if a.dtype == np.uint16:
+        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+    else:
+        t = torch.from_numpy(np.ascontiguousarray(a))
+    return t.pin_memory()
+
+
+def bench_fwd(args, device, world):
+    import torch
+    import selective_state_space_38_b200 as ssm
+    c = workloads.CONFIGS[FWD_CFG]
+    inp = workloads.make_inputs(FWD_CFG)
+    t = {k: _to_dev(v, device) for k, v in inp.items() if isinstance(v, np.ndarray)}
+    out = torch.empty_like(t["x"])
+    hl = torch.empty((c.batch, c.dim, c.dstate), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def launch():
+        ssm.ssm_scan_fwd(t["x"], t["delta"], t["delta_bias"], True, t["A"], t["B"], t["C"], t["D"],
+                         t["z"], None, out=out, h_last=hl)
+
+    for _ in range(args.warmup):
+        launch()
+    torch.cuda.synchronize(device)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    _barrier(world)
+    torch.cuda.synchronize(device)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device.index) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            launch()
+            ev[i][1].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize(device)
+    _barrier(world)
+    total_ms = start.elapsed_time(end)
+    per_launch = [a.elapsed_time(b) for a, b in ev]
+    total_ms = _max_over_ranks(total_ms, world, device)
+    return dict(total_ms=total_ms, launch_ms=statistics.mean(per_launch),
+                launch_ms_median=statistics.median(per_launch), clocks=clk.summary(), inputs=inp)
+
+
+def bench_e2e(args, device, world, inp):
+    """Same metric through the public API from pinned host buffers: H2D copy of
+    the step's inputs, the scan, D2H copy of out and h_last, every step."""
+    import torch
+    import selective_state_space_38_b200 as ssm
+    c = workloads.CONFIGS[FWD_CFG]
+    host = {k: _to_pinned(v) for k, v in inp.items() if isinstance(v, np.ndarray)}
+    dev = {k: torch.empty(v.shape, dtype=v.dtype, device=device) for k, v in host.items()}
+    out_h = torch.empty((c.batch, c.dim, c.seqlen), dtype=torch.bfloat16).pin_memory()
+    hl_h = torch.empty((c.batch, c.dim, c.dstate), dtype=torch.float32).pin_memory()
+    out_d = torch.empty(out_h.shape, dtype=out_h.dtype, device=device)
+    hl_d = torch.empty(hl_h.shape, dtype=hl_h.dtype, device=device)
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_h.numel() * out_h.element_size() + hl_h.numel() * hl_h.element_size()
+    stream = torch.cuda.current_stream(device)
+
+    def one():
+        for k, v in host.items():
+            dev[k].copy_(v, non_blocking=True)
+        ssm.ssm_scan_fwd(dev["x"], dev["delta"], dev["delta_bias"], True, dev["A"], dev["B"],
+                         dev["C"], dev["D"], dev["z"], None, out=out_d, h_last=hl_d)
+        out_h.copy_(out_d, non_blocking=True)
+        hl_h.copy_(hl_d, non_blocking=True)
+
+    steps = max(1, min(args.steps, 20))
+    for _ in range(max(1, min(args.warmup, 3))):
+        one()
+    torch.cuda.synchronize(device)
+    _barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    _barrier(world)
+    ms = _max_over_ranks(a.elapsed_time(b), world, device) / steps
+    return dict(ms=ms, h2d=h2d, d2h=d2h, steps=steps)
+
+
+def bench_decode(args, device):
+    """The recurrent step on the decode config: per-step kernel time with the
+    L2 flushed between steps (so the 84 MB state comes from HBM)."""
+    import torch
+    import selective_state_space_38_b200 as ssm
+    c = workloads.CONFIGS[DECODE_CFG]
+    prm = workloads.decode_params(DECODE_CFG)
+    p = {k: _to_dev(prm[k], device) for k in ("A", "D", "delta_bias")}
+    g = torch.Generator(device="cpu").manual_seed(4)
+    state = (torch.randn((c.batch, c.dim, c.dstate), generator=g) * 0.5).to(device)
+    pool = [{k: _to_dev(v, device) for k, v in workloads.decode_tokens(DECODE_CFG, s).items()}
+            for s in range(4)]
+    outb = torch.empty((c.batch, c.dim), dtype=torch.bfloat16, device=device)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+    steps = 64
+    times = []
+    for s in range(steps + 4):
+        tok = pool[s % len(pool)]
+        flush.fill_(float(s))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        ssm.ssm_scan_step(state, tok["x"], tok["delta"], p["delta_bias"], True, p["A"], tok["B"],
+                          tok["C"], p["D"], tok["z"], out=outb)
+        b.record(stream)
+        times.append((a, b))
+    torch.cuda.synchronize(device)
+    ms = statistics.median([a.elapsed_time(b) for a, b in times[4:]])
+    nb = step_bytes(DECODE_CFG)
+    return dict(ms=ms, gbs=nb / (ms * 1e-3) / 1e9, bytes=nb, steps=steps,
+                gtok_ch=c.batch * c.dim / (ms * 1e-3) / 1e9)
+
+
+def run_gpu(args):
+    import torch
+    world, rank, local = _dist()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    if not torch.cuda.is_available():
+        print(json.dumps({"metric": METRIC, "error": "no CUDA device"}))
+        return 1
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    hbm_peak, peak_kind = _peaks()
+    c = workloads.CONFIGS[FWD_CFG]
+
+    f = bench_fwd(args, device, world)
+    nb = fwd_bytes(FWD_CFG)
+    ms_step = f["total_ms"] / args.steps
+    value = world * nb / (ms_step * 1e-3) / 1e9
+    achieved = nb / (f["launch_ms"] * 1e-3) / 1e9
+    e = bench_e2e(args, device, world, f["inputs"])
+    e2e_gbs = world * nb / (e["ms"] * 1e-3) / 1e9
+    dec = bench_decode(args, device) if rank == 0 else None
+
+    if rank == 0:
+        cpu_val, cpu_s, cpu_ch, cores = cpu_oracle_rate(FWD_CFG, target_s=float(
+            os.environ.get("SSM_CPU_BASELINE_S", "10")))
+        tok_ch = c.batch * c.seqlen * c.dim
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": f"{c.name} forward scan (Mamba-2.8B mixer layer shape)",
+                       "batch": c.batch, "seqlen": c.seqlen, "dim": c.dim, "dstate": c.dstate,
+                       "state_dtype": "f32", "returns_h_last": True,
+                       "l2": f"inputs {nb / 1e6:.0f} MB > L2 126 MB; no flush needed",
+                       "parallelism": f"{world} independent replica(s)"},
+            "pct_of_hbm_peak": round(100.0 * value / world / hbm_peak, 2),
+            "gtok_ch_per_s": round(world * tok_ch / (ms_step * 1e-3) / 1e9, 2),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": hbm_peak,
+                         "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
+                         "peak_kind": peak_kind,
+                         "traffic": _profiled_traffic("scan_fwd_cfg2"),
+                         "algorithmic_bytes_per_launch": nb,
+                         "launch_ms_mean": round(f["launch_ms"], 5),
+                         "launch_ms_median": round(f["launch_ms_median"], 5)},
+            "e2e": {"value": round(e2e_gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": e["h2d"],
+                    "d2h_bytes_per_step": e["d2h"], "ms_per_step": round(e["ms"], 3),
+                    "steps": e["steps"]},
+            "cpu_baseline": {"value": round(cpu_val, 4), "unit": "GB/s", "cores": cores,
+                             "kind": "oracle", "cpu": _cpu_model(),
+                             "sample": f"{cpu_ch} channels (full L) of the same workload, "
+                                       f"{cpu_s:.1f} s of float64 oracle time"},
+            "decode": {"workload": workloads.CONFIGS[DECODE_CFG].name,
+                       "ms_per_step": round(dec["ms"], 5), "value": round(dec["gbs"], 2),
+                       "unit": "GB/s", "pct_of_hbm_peak": round(100 * dec["gbs"] / hbm_peak, 2),
+                       "gtok_ch_per_s": round(dec["gtok_ch"], 3),
+                       "bytes_per_step": dec["bytes"], "l2": "flushed between steps"},
+            "gpu_launches": args.steps,
+            "clocks": f["clocks"],
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

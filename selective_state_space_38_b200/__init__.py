@@ -1,0 +1,187 @@
+"""B200 (sm_100a) selective state-space scan (S6): Python binding.
+
+A thin ctypes layer over ``libssm_scan_b200.so`` (declared in
+``include/ssm_scan.h``).  It checks tensor dtypes, devices and contiguity and
+passes raw device pointers and the current CUDA stream; every step of the
+scan runs in the library's CUDA kernels.  PyTorch is used only to hold device
+memory and to name the stream.
+
+The library must have been built (``python -m selective_state_space_38_b200.build``);
+the first call without it raises ImportError -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "lib", "libssm_scan_b200.so")
+
+SSM_F32, SSM_BF16 = 0, 1
+DSTATE = 16
+
+
+class SSMError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"ssm_scan error {code}: {msg}")
+        self.code = code
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("dim", ctypes.c_int64),
+                ("dstate", ctypes.c_int64), ("act_dtype", ctypes.c_int32)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m selective_state_space_38_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I = ctypes.c_void_p, ctypes.c_int
+    DP = ctypes.POINTER(Dims)
+    lib.ssm_scan_fwd.argtypes = [P, P, P, I, P, P, P, P, P, P, P, P, DP, P]
+    lib.ssm_scan_fwd.restype = I
+    lib.ssm_scan_step.argtypes = [P, P, P, P, I, P, P, P, P, P, P, DP, P]
+    lib.ssm_scan_step.restype = I
+    lib.ssm_strerror.argtypes = [I]
+    lib.ssm_strerror.restype = ctypes.c_char_p
+    lib.ssm_version.argtypes = []
+    lib.ssm_version.restype = I
+    return lib
+
+
+_lib = None
+
+
+def get_lib():
+    """The loaded CUDA library (loaded on first use; ImportError if not built)."""
+    global _lib
+    if _lib is None:
+        _lib = _load()
+    return _lib
+
+
+EXPORTS = ("ssm_scan_fwd", "ssm_scan_step", "ssm_strerror", "ssm_version")
+
+
+def ssm_strerror(code: int) -> str:
+    return get_lib().ssm_strerror(int(code)).decode()
+
+
+def ssm_version() -> int:
+    return int(get_lib().ssm_version())
+
+
+def _act_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return SSM_BF16
+    if t.dtype == torch.float32:
+        return SSM_F32
+    raise TypeError(f"activations must be bfloat16 or float32, got {t.dtype}")
+
+
+def _ptr(t, *, dtype=None, device=None, shape=None, name=""):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _stream_ptr(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return stream.cuda_stream
+
+
+def _check(rc):
+    if rc != 0:
+        raise SSMError(rc, ssm_strerror(rc))
+
+
+def ssm_scan_fwd(x, delta, delta_bias, softplus, A, B, C, D=None, z=None, h0=None,
+                 out=None, h_last=None, return_last_state=True, stream=None):
+    """Forward selective scan.
+
+    x, delta, z: [batch, dim, L]; B, C: [batch, 16, L] (all bfloat16 or all
+    float32, on one CUDA device); A: [dim, 16], D, delta_bias: [dim], h0:
+    [batch, dim, 16] float32.  Returns (out, h_last); h_last is None when
+    ``return_last_state`` is False and no buffer is given.
+    """
+    if x.device.type != "cuda":
+        raise ValueError("ssm_scan_fwd needs CUDA tensors")
+    dev = x.device
+    batch, dim, L = x.shape
+    code = _act_code(x)
+    act = x.dtype
+    f32 = torch.float32
+    ptrs = dict(
+        x=_ptr(x, dtype=act, device=dev, name="x"),
+        delta=_ptr(delta, dtype=act, device=dev, shape=x.shape, name="delta"),
+        z=_ptr(z, dtype=act, device=dev, shape=x.shape, name="z"),
+        B=_ptr(B, dtype=act, device=dev, shape=(batch, DSTATE, L), name="B"),
+        C=_ptr(C, dtype=act, device=dev, shape=(batch, DSTATE, L), name="C"),
+        A=_ptr(A, dtype=f32, device=dev, shape=(dim, DSTATE), name="A"),
+        D=_ptr(D, dtype=f32, device=dev, shape=(dim,), name="D"),
+        delta_bias=_ptr(delta_bias, dtype=f32, device=dev, shape=(dim,), name="delta_bias"),
+        h0=_ptr(h0, dtype=f32, device=dev, shape=(batch, dim, DSTATE), name="h0"),
+    )
+    if out is None:
+        out = torch.empty_like(x)
+    if h_last is None and return_last_state:
+        h_last = torch.empty((batch, dim, DSTATE), dtype=f32, device=dev)
+    po = _ptr(out, dtype=act, device=dev, shape=x.shape, name="out")
+    ph = _ptr(h_last, dtype=f32, device=dev, shape=(batch, dim, DSTATE), name="h_last")
+    dims = Dims(batch, L, dim, DSTATE, code)
+    with torch.cuda.device(dev):
+        rc = get_lib().ssm_scan_fwd(ptrs["x"], ptrs["delta"], ptrs["delta_bias"], int(bool(softplus)),
+                              ptrs["A"], ptrs["B"], ptrs["C"], ptrs["D"], ptrs["z"], ptrs["h0"],
+                              po, ph, ctypes.byref(dims), _stream_ptr(stream, dev))
+    _check(rc)
+    return out, h_last
+
+
+def ssm_scan_step(state, x, delta, delta_bias, softplus, A, B, C, D=None, z=None, out=None,
+                  stream=None):
+    """One recurrent decode step; ``state`` ([batch, dim, 16] float32) is
+    updated in place.  x, delta, z: [batch, dim]; B, C: [batch, 16].
+    Returns out [batch, dim]."""
+    if x.device.type != "cuda":
+        raise ValueError("ssm_scan_step needs CUDA tensors")
+    dev = x.device
+    batch, dim = x.shape
+    code = _act_code(x)
+    act = x.dtype
+    f32 = torch.float32
+    ps = _ptr(state, dtype=f32, device=dev, shape=(batch, dim, DSTATE), name="state")
+    px = _ptr(x, dtype=act, device=dev, name="x")
+    pd = _ptr(delta, dtype=act, device=dev, shape=x.shape, name="delta")
+    pz = _ptr(z, dtype=act, device=dev, shape=x.shape, name="z")
+    pB = _ptr(B, dtype=act, device=dev, shape=(batch, DSTATE), name="B")
+    pC = _ptr(C, dtype=act, device=dev, shape=(batch, DSTATE), name="C")
+    pA = _ptr(A, dtype=f32, device=dev, shape=(dim, DSTATE), name="A")
+    pD = _ptr(D, dtype=f32, device=dev, shape=(dim,), name="D")
+    pb = _ptr(delta_bias, dtype=f32, device=dev, shape=(dim,), name="delta_bias")
+    if out is None:
+        out = torch.empty_like(x)
+    po = _ptr(out, dtype=act, device=dev, shape=x.shape, name="out")
+    dims = Dims(batch, 1, dim, DSTATE, code)
+    with torch.cuda.device(dev):
+        rc = get_lib().ssm_scan_step(ps, px, pd, pb, int(bool(softplus)), pA, pB, pC, pD, pz, po,
+                               ctypes.byref(dims), _stream_ptr(stream, dev))
+    _check(rc)
+    return out
+
+
+__all__ = ["ssm_scan_fwd", "ssm_scan_step", "ssm_strerror", "ssm_version", "SSMError", "Dims",
+           "LIB_PATH", "get_lib"]

@@ -1,0 +1,115 @@
+// common.cuh -- device helpers shared by the selective-scan kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace ssm {
+
+constexpr int kNState = 16;            // states per channel (N)
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// ---- MUFU (special-function unit) wrappers: PTX instructions, called as-is ----
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float lg2_approx(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// ---- activation element types ----------------------------------------------
+// bfloat16 values travel as raw 16-bit patterns; widening is a shift.
+struct bf16raw {
+    uint16_t bits;
+};
+
+template <typename T>
+struct Act;
+
+template <>
+struct Act<float> {
+    static constexpr int kBytes = 4;
+    static constexpr int kPerPiece = 4;  // elements per 16-byte piece
+    __device__ static float widen(float v) { return v; }
+    // element i (0..3) of a 16-byte piece
+    __device__ static float piece(const uint4 &v, int i) {
+        const uint32_t w = i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+        return __uint_as_float(w);
+    }
+    __device__ static float load(const void *p, int64_t i) { return static_cast<const float *>(p)[i]; }
+    __device__ static void store(void *p, int64_t i, float v) { static_cast<float *>(p)[i] = v; }
+};
+
+template <>
+struct Act<bf16raw> {
+    static constexpr int kBytes = 2;
+    static constexpr int kPerPiece = 8;
+    __device__ static float widen(uint16_t v) { return __uint_as_float(static_cast<uint32_t>(v) << 16); }
+    __device__ static float piece(const uint4 &v, int i) {
+        const uint32_t w = (i >> 1) == 0 ? v.x : (i >> 1) == 1 ? v.y : (i >> 1) == 2 ? v.z : v.w;
+        return (i & 1) ? __uint_as_float(w & 0xffff0000u) : __uint_as_float(w << 16);
+    }
+    __device__ static float load(const void *p, int64_t i) {
+        return widen(static_cast<const uint16_t *>(p)[i]);
+    }
+    __device__ static void store(void *p, int64_t i, float v) {
+        uint32_t r;
+        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(0.0f), "f"(v));
+        static_cast<uint16_t *>(p)[i] = static_cast<uint16_t>(r & 0xffffu);
+    }
+};
+
+// two floats -> packed bf16x2 (lo in the low half), round to nearest even
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// ---- step size, gate ----------------------------------------------------------
+// softplus(v) = ln(1 + e^v).  Fast form for bf16 activations: two MUFU ops,
+// identity above 15 (the remainder e^-v < 3.1e-7 is below float resolution of v).
+__device__ __forceinline__ float softplus_fast(float v) {
+    const float e = ex2_approx(v * kLog2e);
+    const float s = lg2_approx(1.0f + e) * kLn2;
+    return v > 15.0f ? v : s;
+}
+// Accurate form for float32 activations.
+__device__ __forceinline__ float softplus_accurate(float v) {
+    return v > 20.0f ? v : log1pf(expf(v));
+}
+// silu(z) = z / (1 + e^-z); e^-z may overflow to +inf, giving -0 for z << 0.
+__device__ __forceinline__ float silu_fast(float z) {
+    return z * rcp_approx(1.0f + ex2_approx(-z * kLog2e));
+}
+__device__ __forceinline__ float silu_accurate(float z) {
+    return z / (1.0f + expf(-z));
+}
+
+// ---- cp.async (16-byte, L1 bypass, zero-fill beyond src_bytes) ----------------
+__device__ __forceinline__ void cp_async16(uint32_t dst_smem, const void *src, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst_smem), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+}  // namespace ssm

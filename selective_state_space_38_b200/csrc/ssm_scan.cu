@@ -1,0 +1,167 @@
+// ssm_scan.cu -- C ABI entry points: host-side validation and kernel launch.
+//
+// Every argument check happens here, before anything is enqueued; a call that
+// fails a check launches nothing.  Kernels run asynchronously on the caller's
+// stream.
+
+#include <climits>
+#include <cstddef>
+#include <cstdint>
+#include <type_traits>
+
+#include <cuda_runtime.h>
+
+#include "ssm_scan.h"
+#include "common.cuh"
+#include "scan_fwd.cuh"
+#include "scan_step.cuh"
+
+namespace {
+
+using namespace ssm;
+
+constexpr int kVersion = 10000;  // 1.0.0
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+struct Span {
+    const void *p;
+    size_t bytes;
+};
+
+bool overlap(const Span &a, const Span &b) {
+    if (!a.p || !b.p || a.bytes == 0 || b.bytes == 0) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a.p), b0 = reinterpret_cast<uintptr_t>(b.p);
+    return a0 < b0 + b.bytes && b0 < a0 + a.bytes;
+}
+
+// sizes must be positive and every buffer must stay well inside int64 byte offsets
+bool dims_ok(int64_t batch, int64_t seqlen, int64_t dim) {
+    if (batch < 1 || seqlen < 1 || dim < 1) return false;
+    const double elems = static_cast<double>(batch) * static_cast<double>(seqlen) * static_cast<double>(dim);
+    return elems < 4.0e18 / 16.0;
+}
+
+template <typename T, bool VEC>
+int launch_fwd(const FwdParams &p, cudaStream_t stream) {
+    const int64_t tiles = (p.dim + kFwdThreads - 1) / kFwdThreads;
+    const int64_t ctas = tiles * p.batch;
+    if (ctas > INT_MAX) return SSM_ERR_UNSUPPORTED;
+    const int smem = FwdSmem<T>::kTotal;
+    auto kern = scan_fwd_kernel<T, VEC>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    kern<<<static_cast<unsigned>(ctas), kFwdThreads, smem, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+template <typename T>
+int launch_step(const StepParams &p, cudaStream_t stream) {
+    const int64_t threads = p.batch * p.dim * 4;
+    const int64_t blocks = (threads + kStepThreads - 1) / kStepThreads;
+    if (blocks > INT_MAX) return SSM_ERR_UNSUPPORTED;
+    scan_step_kernel<T><<<static_cast<unsigned>(blocks), kStepThreads, 0, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ssm_version(void) { return kVersion; }
+
+const char *ssm_strerror(int code) {
+    switch (code) {
+        case SSM_OK: return "ok";
+        case SSM_ERR_INVALID_ARG: return "invalid argument (NULL required pointer, size < 1, or out overlapping an input)";
+        case SSM_ERR_UNSUPPORTED: return "unsupported (dstate must be 16, dtype f32 or bf16, sizes within limits)";
+        case SSM_ERR_MISALIGNED: return "misaligned pointer (16-byte alignment required)";
+        case SSM_ERR_CUDA: return "CUDA launch error";
+        case SSM_ERR_TIMEOUT: return "bounded device wait timed out";
+        default: return "unknown error code";
+    }
+}
+
+int ssm_scan_fwd(const void *x, const void *delta, const float *delta_bias, int softplus,
+                 const float *A, const void *B, const void *C, const float *D, const void *z,
+                 const float *h0, void *out, float *h_last, const ssm_dims_t *dims,
+                 ssm_stream_t stream) {
+    if (!dims) return SSM_ERR_INVALID_ARG;
+    const int64_t batch = dims->batch, L = dims->seqlen, dim = dims->dim, N = dims->dstate;
+    if (!x || !delta || !A || !B || !C || !out) return SSM_ERR_INVALID_ARG;
+    if (!dims_ok(batch, L, dim) || N < 1) return SSM_ERR_INVALID_ARG;
+    if (N != kNState) return SSM_ERR_UNSUPPORTED;
+    if (dims->act_dtype != SSM_F32 && dims->act_dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
+    const size_t es = dims->act_dtype == SSM_F32 ? 4 : 2;
+    for (const void *ptr : {x, delta, (const void *)A, B, C, z, (const void *)h0, (const void *)out,
+                            (const void *)h_last})
+        if (ptr && !aligned16(ptr)) return SSM_ERR_MISALIGNED;
+    for (const void *ptr : {(const void *)delta_bias, (const void *)D})
+        if (ptr && !aligned4(ptr)) return SSM_ERR_MISALIGNED;
+
+    const size_t tok = static_cast<size_t>(batch) * dim * L;
+    const Span o{out, tok * es};
+    const Span ins[] = {{x, tok * es}, {delta, tok * es}, {z, z ? tok * es : 0},
+                        {B, static_cast<size_t>(batch) * N * L * es}, {C, static_cast<size_t>(batch) * N * L * es},
+                        {A, static_cast<size_t>(dim) * N * 4}, {D, D ? static_cast<size_t>(dim) * 4 : 0},
+                        {delta_bias, delta_bias ? static_cast<size_t>(dim) * 4 : 0},
+                        {h0, h0 ? static_cast<size_t>(batch) * dim * N * 4 : 0},
+                        {h_last, h_last ? static_cast<size_t>(batch) * dim * N * 4 : 0}};
+    for (const Span &s : ins)
+        if (overlap(o, s)) return SSM_ERR_INVALID_ARG;
+    if (h_last) {  // h_last may be h0 itself, but must not partially overlap any input
+        const Span hl{h_last, static_cast<size_t>(batch) * dim * N * 4};
+        for (int i = 0; i < 8; ++i)
+            if (overlap(hl, ins[i])) return SSM_ERR_INVALID_ARG;
+        if (h0 && h0 != h_last && overlap(hl, ins[8])) return SSM_ERR_INVALID_ARG;
+    }
+
+    FwdParams p;
+    p.x = x; p.delta = delta; p.z = z; p.B = B; p.C = C;
+    p.delta_bias = delta_bias; p.A = A; p.D = D; p.h0 = h0;
+    p.out = out; p.h_last = h_last;
+    p.batch = batch; p.seqlen = L; p.dim = dim;
+    p.softplus = softplus ? 1 : 0;
+    const bool vec = (static_cast<size_t>(L) * es) % 16 == 0;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (dims->act_dtype == SSM_BF16)
+        return vec ? launch_fwd<bf16raw, true>(p, s) : launch_fwd<bf16raw, false>(p, s);
+    return vec ? launch_fwd<float, true>(p, s) : launch_fwd<float, false>(p, s);
+}
+
+int ssm_scan_step(float *state, const void *x, const void *delta, const float *delta_bias,
+                  int softplus, const float *A, const void *B, const void *C, const float *D,
+                  const void *z, void *out, const ssm_dims_t *dims, ssm_stream_t stream) {
+    if (!dims) return SSM_ERR_INVALID_ARG;
+    const int64_t batch = dims->batch, dim = dims->dim, N = dims->dstate;
+    if (!state || !x || !delta || !A || !B || !C || !out) return SSM_ERR_INVALID_ARG;
+    if (!dims_ok(batch, 1, dim) || N < 1) return SSM_ERR_INVALID_ARG;
+    if (N != kNState) return SSM_ERR_UNSUPPORTED;
+    if (dims->act_dtype != SSM_F32 && dims->act_dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
+    const size_t es = dims->act_dtype == SSM_F32 ? 4 : 2;
+    if (!aligned16(state) || !aligned16(A)) return SSM_ERR_MISALIGNED;
+    for (const void *ptr : {x, delta, B, C, z, (const void *)out, (const void *)delta_bias, (const void *)D})
+        if (ptr && (reinterpret_cast<uintptr_t>(ptr) % (ptr == delta_bias || ptr == D ? 4 : es)) != 0)
+            return SSM_ERR_MISALIGNED;
+
+    const size_t nch = static_cast<size_t>(batch) * dim;
+    const Span o{out, nch * es};
+    const Span st{state, nch * N * 4};
+    const Span ins[] = {{x, nch * es}, {delta, nch * es}, {z, z ? nch * es : 0},
+                        {B, static_cast<size_t>(batch) * N * es}, {C, static_cast<size_t>(batch) * N * es},
+                        {A, static_cast<size_t>(dim) * N * 4}, {D, D ? static_cast<size_t>(dim) * 4 : 0},
+                        {delta_bias, delta_bias ? static_cast<size_t>(dim) * 4 : 0}};
+    if (overlap(o, st)) return SSM_ERR_INVALID_ARG;
+    for (const Span &s : ins)
+        if (overlap(o, s) || overlap(st, s)) return SSM_ERR_INVALID_ARG;
+
+    StepParams p;
+    p.state = state; p.x = x; p.delta = delta; p.z = z; p.B = B; p.C = C;
+    p.delta_bias = delta_bias; p.A = A; p.D = D; p.out = out;
+    p.batch = batch; p.dim = dim; p.softplus = softplus ? 1 : 0;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return dims->act_dtype == SSM_BF16 ? launch_step<bf16raw>(p, s) : launch_step<float>(p, s);
+}
+
+}  // extern "C"

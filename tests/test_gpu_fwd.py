@@ -1,0 +1,213 @@
+"""GPU parity of ssm_scan_fwd against the float64 oracle (element by element,
+same stored inputs).  Small and ragged shapes are compared in full; the large
+configs in full where the oracle is fast enough, otherwise on sampled channels
+over the whole sequence."""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from helpers import check, to_dev, to_np64
+
+pytestmark = pytest.mark.gpu
+
+
+def _gpu_fwd(inp, want_state=True, h0=None):
+    import selective_state_space_38_b200 as ssm
+    t = {k: to_dev(v) for k, v in inp.items() if isinstance(v, np.ndarray)}
+    out, hl = ssm.ssm_scan_fwd(t["x"], t["delta"], t.get("delta_bias"), inp["softplus"], t["A"],
+                               t["B"], t["C"], t.get("D"), t.get("z"),
+                               to_dev(h0) if h0 is not None else t.get("h0"),
+                               return_last_state=want_state)
+    torch.cuda.synchronize()
+    return out, hl
+
+
+def _oracle(orc, inp, channels=None):
+    args = (inp["x"], inp["delta"], inp.get("delta_bias"), inp["softplus"], inp["A"], inp["B"],
+            inp["C"], inp.get("D"), inp.get("z"), inp.get("h0"))
+    if channels is None:
+        return orc.fwd(*args)
+    return orc.fwd_channels(*args, channels)
+
+
+def _dt(inp):
+    return "f32" if inp["x"].dtype == np.float32 else "bf16"
+
+
+SMALL_L = [1, 7, 31, 33, 64, 255, 257, 1000]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("L", SMALL_L)
+def test_small_shapes(orc, dtype, L):
+    inp = workloads.custom_inputs(2, L, 130, 16, dtype=dtype, seed=L, has_h0=(L % 2 == 1))
+    out, hl = _gpu_fwd(inp)
+    ref_out, ref_hl = _oracle(orc, inp)
+    check(to_np64(out), ref_out, dtype, f"out L={L}")
+    check(to_np64(hl), ref_hl, dtype, f"h_last L={L}")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_optional_inputs_absent(orc, dtype):
+    inp = workloads.custom_inputs(1, 300, 200, 16, dtype=dtype, seed=5)
+    inp.update(z=None, D=None, delta_bias=None, h0=None)
+    inp["delta"] = inp["delta"]  # raw delta without bias; softplus keeps dt > 0
+    out, hl = _gpu_fwd(inp)
+    ref_out, ref_hl = _oracle(orc, inp)
+    check(to_np64(out), ref_out, dtype, "out (no z/D/bias/h0)")
+    check(to_np64(hl), ref_hl, dtype, "h_last (no z/D/bias/h0)")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_softplus_off(orc, dtype):
+    inp = workloads.custom_inputs(2, 129, 64, 16, dtype=dtype, seed=6)
+    inp["softplus"] = False
+    # dt = delta + bias must stay positive and small: use |delta| as stored values
+    if dtype == "f32":
+        inp["delta"] = np.abs(inp["delta"]) * np.float32(0.1)
+    else:
+        inp["delta"] = inp["delta"] & np.uint16(0x7FFF)  # clear the sign bit
+    inp["delta_bias"] = np.full_like(inp["delta_bias"], 0.01)
+    out, hl = _gpu_fwd(inp)
+    ref_out, ref_hl = _oracle(orc, inp)
+    check(to_np64(out), ref_out, dtype, "out softplus=0")
+    check(to_np64(hl), ref_hl, dtype, "h_last softplus=0")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_general_A(orc, dtype):
+    """A without the S4D-real structure takes the per-state exp path."""
+    inp = workloads.custom_inputs(2, 200, 96, 16, dtype=dtype, seed=7, has_h0=True)
+    rng = np.random.default_rng(70)
+    inp["A"] = -rng.uniform(0.05, 3.0, size=inp["A"].shape).astype(np.float32)
+    out, hl = _gpu_fwd(inp)
+    ref_out, ref_hl = _oracle(orc, inp)
+    check(to_np64(out), ref_out, dtype, "out general A")
+    check(to_np64(hl), ref_hl, dtype, "h_last general A")
+
+
+def test_mixed_A_rows(orc):
+    """Some channels S4D-structured, some not, within one warp."""
+    inp = workloads.custom_inputs(1, 100, 64, 16, dtype="bf16", seed=8)
+    inp["A"][5] = -np.linspace(0.3, 4.0, 16, dtype=np.float32)
+    out, hl = _gpu_fwd(inp)
+    ref_out, ref_hl = _oracle(orc, inp)
+    check(to_np64(out), ref_out, "bf16", "out mixed A")
+    check(to_np64(hl), ref_hl, "bf16", "h_last mixed A")
+
+
+def test_extreme_dt(orc):
+    """dt spanning 1e-6..50: state decay from ~1 (memory) to exactly 0 (reset)."""
+    inp = workloads.custom_inputs(1, 257, 64, 16, dtype="bf16", seed=9, has_h0=True)
+    bias = np.linspace(-14.0, 50.0, 64).astype(np.float32)
+    inp["delta_bias"] = bias
+    out, hl = _gpu_fwd(inp)
+    ref_out, ref_hl = _oracle(orc, inp)
+    check(to_np64(out), ref_out, "bf16", "out extreme dt")
+    check(to_np64(hl), ref_hl, "bf16", "h_last extreme dt")
+
+
+def test_h_last_in_place_over_h0(orc):
+    import selective_state_space_38_b200 as ssm
+    inp = workloads.custom_inputs(2, 96, 130, 16, dtype="bf16", seed=10, has_h0=True)
+    t = {k: to_dev(v) for k, v in inp.items() if isinstance(v, np.ndarray)}
+    h = t["h0"].clone()
+    out, hl = ssm.ssm_scan_fwd(t["x"], t["delta"], t["delta_bias"], True, t["A"], t["B"], t["C"],
+                               t["D"], t["z"], h, h_last=h)
+    torch.cuda.synchronize()
+    assert hl.data_ptr() == h.data_ptr()
+    ref_out, ref_hl = _oracle(orc, inp)
+    check(to_np64(out), ref_out, "bf16", "out in-place")
+    check(to_np64(h), ref_hl, "bf16", "h_last in-place")
+
+
+def test_chunk_split_matches_full_gpu_scan():
+    """Scanning [0, m) then [m, L) from the carried state equals one call."""
+    inp = workloads.custom_inputs(2, 1000, 200, 16, dtype="bf16", seed=11, has_h0=True)
+    out, hl = _gpu_fwd(inp)
+    for m in (1, 333, 512, 999):
+        a = {k: (np.ascontiguousarray(v[..., :m]) if k in ("x", "delta", "z", "B", "C") else v)
+             for k, v in inp.items()}
+        b = {k: (np.ascontiguousarray(v[..., m:]) if k in ("x", "delta", "z", "B", "C") else v)
+             for k, v in inp.items()}
+        o1, h1 = _gpu_fwd(a)
+        b["h0"] = None
+        o2, h2 = _gpu_fwd(b, h0=h1.cpu().numpy())
+        got = torch.cat([o1, o2], dim=-1)
+        check(to_np64(got), to_np64(out), "bf16", f"split m={m} out")
+        check(to_np64(h2), to_np64(hl), "bf16", f"split m={m} h_last")
+
+
+def test_output_guard_bands():
+    """The kernel writes exactly [batch][dim][L] and h_last: the bytes
+    around both stay untouched (NaN canary)."""
+    import selective_state_space_38_b200 as ssm
+    inp = workloads.custom_inputs(1, 77, 130, 16, dtype="bf16", seed=12)
+    t = {k: to_dev(v) for k, v in inp.items() if isinstance(v, np.ndarray)}
+    n_out = 130 * 77
+    guard = 64
+    big = torch.full((n_out + 2 * guard,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    out = big[guard:guard + n_out].view(1, 130, 77)
+    hbig = torch.full((130 * 16 + 2 * guard,), float("nan"), dtype=torch.float32, device="cuda")
+    hl = hbig[guard:guard + 130 * 16].view(1, 130, 16)
+    ssm.ssm_scan_fwd(t["x"], t["delta"], t["delta_bias"], True, t["A"], t["B"], t["C"], t["D"],
+                     t["z"], None, out=out, h_last=hl)
+    torch.cuda.synchronize()
+    assert torch.isnan(big[:guard].float()).all() and torch.isnan(big[-guard:].float()).all()
+    assert torch.isnan(hbig[:guard]).all() and torch.isnan(hbig[-guard:]).all()
+    assert torch.isfinite(out.float()).all() and torch.isfinite(hl).all()
+
+
+# ---- the configs ---------------------------------------------------------------
+def test_config0_full(orc):
+    inp = workloads.make_inputs(0)
+    out, hl = _gpu_fwd(inp)
+    ref_out, ref_hl = _oracle(orc, inp)
+    check(to_np64(out), ref_out, "f32", "config0 out")
+    check(to_np64(hl), ref_hl, "f32", "config0 h_last")
+
+
+def test_config1_full(orc):
+    inp = workloads.make_inputs(1)
+    out, hl = _gpu_fwd(inp)
+    ref_out, ref_hl = _oracle(orc, inp)
+    check(to_np64(out), ref_out, "bf16", "config1 out")
+    check(to_np64(hl), ref_hl, "bf16", "config1 h_last")
+
+
+def _sampled(orc, cfg, nsel, seed):
+    inp = workloads.make_inputs(cfg)
+    out, hl = _gpu_fwd(inp)
+    c = workloads.CONFIGS[cfg]
+    rng = np.random.default_rng(seed)
+    chan = np.unique(np.concatenate([
+        rng.choice(c.channels, nsel, replace=False),
+        [0, c.dim - 1, c.channels - 1, c.dim, 127, 128]]))
+    ref_out, ref_hl = _oracle(orc, inp, chan)
+    got = to_np64(out).reshape(c.channels, -1)[chan]
+    gothl = to_np64(hl).reshape(c.channels, -1)[chan]
+    check(got, ref_out, "bf16", f"config{cfg} out (sampled)")
+    check(gothl, ref_hl, "bf16", f"config{cfg} h_last (sampled)")
+    return inp, out, hl
+
+
+def test_config2_sampled(orc):
+    _sampled(orc, 2, 192, 2)
+
+
+def test_config3_sampled_and_split(orc):
+    inp, out, hl = _sampled(orc, 3, 48, 3)
+    # state carry across two calls at a non-aligned split point
+    m = 65536 + 777
+    a = {k: (np.ascontiguousarray(v[..., :m]) if k in ("x", "delta", "z", "B", "C") else v)
+         for k, v in inp.items()}
+    o1, h1 = _gpu_fwd(a)
+    del a
+    b = {k: (np.ascontiguousarray(v[..., m:]) if k in ("x", "delta", "z", "B", "C") else v)
+         for k, v in inp.items()}
+    b["h0"] = None
+    o2, h2 = _gpu_fwd(b, h0=h1.cpu().numpy())
+    check(to_np64(o1), to_np64(out[..., :m]), "bf16", "config3 split first")
+    check(to_np64(o2), to_np64(out[..., m:]), "bf16", "config3 split second")
+    check(to_np64(h2), to_np64(hl), "bf16", "config3 split h_last")

@@ -181,9 +181,9 @@ def _sampled(orc, cfg, nsel, seed):
     out, hl = _gpu_fwd(inp)
     c = workloads.CONFIGS[cfg]
     rng = np.random.default_rng(seed)
-    chan = np.unique(np.concatenate([
-        rng.choice(c.channels, nsel, replace=False),
-        [0, c.dim - 1, c.channels - 1, c.dim, 127, 128]]))
+    edge = np.array([0, 127, 128, c.dim - 1, c.dim, c.channels - 1])
+    chan = np.unique(np.concatenate([rng.choice(c.channels, nsel, replace=False),
+                                     edge[edge < c.channels]]))
     ref_out, ref_hl = _oracle(orc, inp, chan)
     got = to_np64(out).reshape(c.channels, -1)[chan]
     gothl = to_np64(hl).reshape(c.channels, -1)[chan]

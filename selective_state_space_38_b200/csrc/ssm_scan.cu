@@ -7,6 +7,7 @@
 #include <climits>
 #include <cstddef>
 #include <cstdint>
+#include <mutex>
 #include <type_traits>
 
 #include <cuda_runtime.h>
@@ -43,17 +44,64 @@ bool dims_ok(int64_t batch, int64_t seqlen, int64_t dim) {
     return elems < 4.0e18 / 16.0;
 }
 
+// Scratch memory comes from a library-owned stream-ordered pool per device that
+// keeps freed memory (release threshold = max), so after the first call an
+// allocation is a cheap pool hit and never waits on the operating system.
+cudaMemPool_t scratch_pool(int dev) {
+    static std::mutex mu;
+    static cudaMemPool_t pools[64] = {};
+    if (dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!pools[dev]) {
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t pool = nullptr;
+        if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return nullptr;
+        uint64_t keep = UINT64_MAX;
+        cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+        pools[dev] = pool;
+    }
+    return pools[dev];
+}
+
+// Persistent launch: one single-warp CTA per SM sub-partition (4 per SM), or
+// fewer when there are fewer items.  The work queue, segment flags and
+// carried states live in a stream-ordered scratch allocation of
+// fwd_scratch_bytes(groups) bytes, whose counter and flags are zeroed first.
 template <typename T, bool VEC>
 int launch_fwd(const FwdParams &p, cudaStream_t stream) {
-    const int64_t tiles = (p.dim + kFwdThreads - 1) / kFwdThreads;
-    const int64_t ctas = tiles * p.batch;
-    if (ctas > INT_MAX) return SSM_ERR_UNSUPPORTED;
-    const int smem = FwdSmem<T>::kTotal;
-    auto kern = scan_fwd_kernel<T, VEC>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    const int64_t groups = ((p.dim + 31) / 32) * p.batch;
+    const int64_t items = groups * ((p.seqlen + kSegSteps - 1) / kSegSteps);
+    if (items > static_cast<int64_t>(UINT32_MAX) / 2) return SSM_ERR_UNSUPPORTED;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return SSM_ERR_CUDA;
-    kern<<<static_cast<unsigned>(ctas), kFwdThreads, smem, stream>>>(p);
-    return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+    const int64_t workers = items < 4 * static_cast<int64_t>(sms) ? items : 4 * static_cast<int64_t>(sms);
+    const int smem = FwdSmem<T>::kWarpBytes;
+    auto k_s4d = scan_fwd_kernel<T, VEC, true>;
+    auto k_gen = scan_fwd_kernel<T, VEC, false>;
+    if (cudaFuncSetAttribute(k_s4d, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+        cudaFuncSetAttribute(k_gen, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    cudaMemPool_t pool = scratch_pool(dev);
+    if (!pool) return SSM_ERR_CUDA;
+    void *scratch = nullptr;
+    if (cudaMallocFromPoolAsync(&scratch, fwd_scratch_bytes(groups), pool, stream) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    int rc = SSM_OK;
+    if (cudaMemsetAsync(scratch, 0, fwd_scratch_flag_bytes(groups), stream) != cudaSuccess) {
+        rc = SSM_ERR_CUDA;
+    } else {
+        const FwdScratch sc = fwd_scratch_view(scratch, groups);
+        k_s4d<<<static_cast<unsigned>(workers), kFwdThreads, smem, stream>>>(p, sc);
+        k_gen<<<static_cast<unsigned>(workers), kFwdThreads, smem, stream>>>(p, sc);
+        if (cudaGetLastError() != cudaSuccess) rc = SSM_ERR_CUDA;
+    }
+    if (cudaFreeAsync(scratch, stream) != cudaSuccess) rc = SSM_ERR_CUDA;
+    return rc;
 }
 
 template <typename T>

@@ -450,7 +450,8 @@ def run_gpu(args):
                        "unit": "GB/s", "pct_of_hbm_peak": round(100 * dec["gbs"] / hbm_peak, 2),
                        "gtok_ch_per_s": round(dec["gtok_ch"], 3),
                        "bytes_per_step": dec["bytes"], "l2": "flushed between steps"},
-            "gpu_launches": args.steps,
+            # per forward call: the S4D-structured and the general kernel instance
+            "gpu_launches": 2 * args.steps,
             "clocks": f["clocks"],
         }
         print(json.dumps(line), flush=True)

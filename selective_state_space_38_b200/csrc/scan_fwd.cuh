@@ -33,6 +33,8 @@
 
 #include <type_traits>
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace ssm {
@@ -46,25 +48,37 @@ struct FwdParams {
     int softplus;
 };
 
-constexpr int kWarpsPerCTA = 1;
-constexpr int kFwdThreads = 32 * kWarpsPerCTA;
+// TMA descriptors of the aligned path: activations as 3-D [batch][dim][L]
+// tensors with [1][32][TC] boxes and the 64-byte swizzle (the same XOR layout
+// as swz()), B and C as [batch][16][L] with [1][16][TC] boxes.
+struct TmaMaps {
+    CUtensorMap x, delta, z, B, C, out;
+};
+
+constexpr int kPairs = 4;                    // warp triples per CTA (one per SM sub-partition)
+constexpr int kFwdThreads = 96 * kPairs;     // warps 0..3 scan, 4..7 stage + prepare, 8..11 finish
 constexpr int kRowBytes = 64;  // bytes of one channel row of a chunk
 constexpr int kPieces = kRowBytes / 16;
-constexpr int kStages = 2;     // chunks in flight per warp
+constexpr int kStages = 3;     // staged chunks per pair (post-processing, next, loading)
 constexpr int kBCPitch = 36;   // floats per time row of widened B|C (32 used)
 
+// Shared memory of one warp triple.  Stages hold raw chunks (x, delta, z
+// tiles and the B, C rows); bcf and ur are double-buffered per chunk parity.
+// bcf and ur carry one spare step row so that the scan warp's step-ahead
+// preparation can run unconditionally on a chunk's last step.
 template <typename T>
 struct FwdSmem {
-    static constexpr int kTC = kRowBytes / Act<T>::kBytes;         // timesteps per chunk
-    static constexpr int kTileBytes = 32 * kRowBytes;              // one [32 ch][TC] tile
-    static constexpr int kBCRowBytes = kRowBytes;                  // one [TC] row of B or C
-    static constexpr int kStageBytes = 3 * kTileBytes + 2 * kNState * kBCRowBytes;
+    static constexpr int kTC = kRowBytes / Act<T>::kBytes;          // timesteps per chunk
+    static constexpr int kTileBytes = 32 * kRowBytes;               // one [32 ch][TC] tile
+    static constexpr int kStageBytes = 3 * kTileBytes + 2 * kNState * kRowBytes;
+    static constexpr int kBCFBytes = (kTC + 1) * kBCPitch * 4;      // widened B|C, time-major
+    static constexpr int kURBytes = (kTC + 1) * 32 * 8;             // float2 (u, r) per [t][lane]
     static constexpr int kBCFOff = kStages * kStageBytes;
-    // one spare row at the end of bcf and ur lets the step-ahead preparation run
-    // unconditionally on the chunk's last step (its result is never used)
-    static constexpr int kUROff = kBCFOff + (kTC + 1) * kBCPitch * 4;  // float2 (u, r) per [t][lane]
-    static constexpr int kWarpBytes = kUROff + (kTC + 1) * 32 * 8;
-    static constexpr int kTotal = kWarpsPerCTA * kWarpBytes;
+    static constexpr int kUROff = kBCFOff + 2 * kBCFBytes;
+    static constexpr int kDescOff = kUROff + 2 * kURBytes;          // ring of 4 chunk descriptors
+    static constexpr int kBarOff = kDescOff + 4 * 64;               // mbarriers ready[2], done[2], posted[2], full[3]
+    static constexpr int kPairBytes = (kBarOff + 9 * 8 + 1023) / 1024 * 1024;
+    static constexpr int kTotal = kPairs * kPairBytes + 1024;       // + slack to align the base to 1 KB
 };
 
 __device__ __forceinline__ int swz(int row, int pc) { return pc ^ ((row >> 1) & 3); }
@@ -429,14 +443,14 @@ __device__ __forceinline__ void store_chunk(const FwdParams &p, const uint8_t *t
 // The sequence of each 32-channel group is cut into segments of kSegSteps
 // steps.  An item is one (group, segment) pair; items are handed out in
 // segment-major order through an atomic counter, so the work spreads evenly
-// over the persistent warps whatever the number of groups.  A segment other
+// over the persistent workers whatever the number of groups.  A segment other
 // than the first starts from the state its predecessor left in `carry` and
 // published by setting flag[group] = segment index; the predecessor was taken
-// from the queue earlier by a running warp, so the wait always ends.  Each
-// wait is still bounded: past kSpinLimit polls the warp records an error and
-// carries on.
+// from the queue earlier by a running worker, so the wait always ends.  Every
+// wait is still bounded: past its limit the warp records an error and goes on.
 constexpr int kSegSteps = 512;
-constexpr uint32_t kSpinLimit = 1u << 26;
+constexpr uint32_t kSpinLimit = 1u << 24;   // flag polls (64 ns apart)
+constexpr uint32_t kBarLimit = 1u << 20;    // mbarrier try_wait rounds
 
 struct FwdScratch {
     uint32_t *counter;  // [2] next item, one queue per kernel instance (S4D, general)
@@ -473,168 +487,316 @@ __device__ __forceinline__ void st_release(uint32_t *p, uint32_t v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// One segment [t_begin, t_end) of the warp's 32 channels, from state h.
-template <typename T, bool VEC, bool S4D>
-__device__ __forceinline__ void scan_segment(const FwdParams &p, uint8_t *ws, int64_t b, int64_t d0,
-                                             int64_t t_begin, int64_t t_end, int lane,
-                                             const ChanConst &cc, const float (&a2)[kNState],
-                                             float2 (&h)[8]) {
-    using SM = FwdSmem<T>;
-    constexpr int TC = SM::kTC;
-    const bool has_z = p.z != nullptr;
-    const bool softplus = p.softplus != 0;
-    float *bcf = reinterpret_cast<float *>(ws + SM::kBCFOff);
-    float2 *ur = reinterpret_cast<float2 *>(ws + SM::kUROff);
-    const int64_t nchunks = (t_end - t_begin + TC - 1) / TC;
-
-    if constexpr (VEC) load_chunk_async<T>(p, ws, b, d0, t_begin, lane);
-    else load_chunk_sync<T>(p, ws, b, d0, t_begin, lane);
-    cp_async_commit();
-    for (int64_t k = 0; k < nchunks; ++k) {
-        const int64_t t0 = t_begin + k * TC;
-        if (k + 1 < nchunks) {
-            uint8_t *st = ws + ((k + 1) % kStages) * SM::kStageBytes;
-            if constexpr (VEC) load_chunk_async<T>(p, st, b, d0, t0 + TC, lane);
-            else load_chunk_sync<T>(p, st, b, d0, t0 + TC, lane);
-        }
-        cp_async_commit();
-        cp_async_wait<1>();
-        __syncwarp();
-        uint8_t *stage = ws + (k % kStages) * SM::kStageBytes;
-        widen_bc<T>(stage + 3 * SM::kTileBytes, bcf, lane);
-        __syncwarp();
-        const int nvalid = static_cast<int>(t_end - t0 < TC ? t_end - t0 : TC);
-        chunk_prepass<T, S4D>(stage, ur, lane, cc, softplus);
-        __syncwarp();
-        if (nvalid == TC)
-            chunk_core<S4D, true>(bcf, ur, lane, TC, a2, h);
-        else
-            chunk_core<S4D, false>(bcf, ur, lane, nvalid, a2, h);
-        __syncwarp();
-        chunk_postpass<T>(stage, ur, lane, cc, has_z);
-        __syncwarp();
-        store_chunk<T, VEC>(p, stage, b, d0, t0, lane);
-        __syncwarp();
+// ---- mbarriers (shared memory), with bounded waits -------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+// wait for the completion of the phase with the given parity; false on timeout
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t *error) {
+    const uint32_t addr = smem_u32(bar);
+    for (uint32_t n = 0; n < kBarLimit; ++n) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(addr), "r"(parity)
+            : "memory");
+        if (done) return true;
     }
-    cp_async_wait<0>();
-    __syncwarp();
+    atomicOr(error, 2u);
+    return false;
 }
 
-// ---- the kernel -----------------------------------------------------------------
-// Persistent: every warp is a worker that takes (group, segment) items from the
-// queue until none are left.  grid: any number of one-warp CTAs (one per SM
-// sub-partition is the intent); dynamic smem FwdSmem<T>::kWarpBytes.
-// Two instances run back to back on the stream.  The S4D instance takes the
-// groups whose channels all have S4D-structured A rows and marks the scratch
-// when it meets any other group; the general instance then takes exactly
-// those (and returns at once when none was marked).
-template <typename T, bool VEC, bool S4D>
-__global__ void __launch_bounds__(kFwdThreads) scan_fwd_kernel(const FwdParams p, const FwdScratch sc) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    const int lane = threadIdx.x & 31;
-    if (!S4D && *reinterpret_cast<volatile uint32_t *>(sc.general) == 0) return;
-    uint32_t *counter = sc.counter + (S4D ? 0 : 1);
-    uint8_t *ws = smem;
-    const int64_t tiles = (p.dim + 31) / 32;
-    const int64_t groups = tiles * p.batch;
-    const int64_t nseg = (p.seqlen + kSegSteps - 1) / kSegSteps;
-    const int64_t items = groups * nseg;
+// One chunk of a worker's stream, as the helper hands it to the scan warp.
+struct ChunkDesc {
+    int64_t b, d0, t0, g, seg;
+    int32_t nvalid;
+    int32_t flags;  // kFirst: first chunk of its segment; kLast: last; kSeqEnd: segment ends the sequence; kStop
+};
+constexpr int32_t kFirst = 1, kLast = 2, kSeqEnd = 4, kStop = 8;
 
-    uint32_t item = 0;
-    if (lane == 0) item = atomicAdd(counter, 1u);
-    item = __shfl_sync(0xffffffffu, item, 0);
-    while (static_cast<int64_t>(item) < items) {
-        const int64_t seg = item / groups, g = item % groups;
-        const int64_t b = g / tiles, d0 = (g % tiles) * 32, d = d0 + lane;
-        const bool active = d < p.dim;
-        const int64_t dc = active ? d : p.dim - 1;
+// Per-lane constants of a channel for the helper's passes.
+__device__ __forceinline__ ChanConst chan_const(const FwdParams &p, int64_t dc) {
+    ChanConst cc;
+    const float a2 = p.A[dc * kNState] * kLog2e;
+    const float Dd = p.D ? p.D[dc] : 0.0f;
+    const float bias = p.delta_bias ? p.delta_bias[dc] : 0.0f;
+    cc.a2_0 = a2;
+    cc.a2_0x2 = make_float2(a2, a2);
+    cc.Dx2 = make_float2(Dd, Dd);
+    cc.biasx2 = make_float2(bias, bias);
+    return cc;
+}
 
-        ChanConst cc;
-        float a2[kNState];
-        bool s4d = true;
-        {
-            const float4 *ar = reinterpret_cast<const float4 *>(p.A + dc * kNState);
-            float a[kNState];
+// Whether all channels of the warp's group have S4D-structured A rows
+// (A[d, n] == (n + 1) A[d, 0] exactly); lanes past the last channel agree.
+__device__ __forceinline__ bool group_is_s4d(const FwdParams &p, int64_t d0, int lane) {
+    const int64_t d = d0 + lane;
+    bool ok = true;
+    if (d < p.dim) {
+        const float4 *ar = reinterpret_cast<const float4 *>(p.A + d * kNState);
+        float a[kNState];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float4 v = ar[q];
-                a[4 * q] = v.x; a[4 * q + 1] = v.y; a[4 * q + 2] = v.z; a[4 * q + 3] = v.w;
-            }
-#pragma unroll
-            for (int n = 0; n < kNState; ++n) {
-                a2[n] = a[n] * kLog2e;
-                s4d = s4d && (a[n] == __fmul_rn(static_cast<float>(n + 1), a[0]));
-            }
-            cc.a2_0 = a2[0];
-            cc.a2_0x2 = make_float2(a2[0], a2[0]);
-            const float Dd = p.D ? p.D[dc] : 0.0f;
-            const float bias = p.delta_bias ? p.delta_bias[dc] : 0.0f;
-            cc.Dx2 = make_float2(Dd, Dd);
-            cc.biasx2 = make_float2(bias, bias);
+        for (int q = 0; q < 4; ++q) {
+            const float4 v = ar[q];
+            a[4 * q] = v.x; a[4 * q + 1] = v.y; a[4 * q + 2] = v.z; a[4 * q + 3] = v.w;
         }
-        // inactive lanes (past the last channel) never disqualify a warp
-        const bool warp_s4d = __all_sync(0xffffffffu, s4d || !active);
-        if (warp_s4d != S4D) {
-            if (S4D && lane == 0) atomicOr(sc.general, 1u);
+#pragma unroll
+        for (int n = 0; n < kNState; ++n) ok = ok && (a[n] == __fmul_rn(static_cast<float>(n + 1), a[0]));
+    }
+    return __all_sync(0xffffffffu, ok);
+}
+
+// The helper's walk through the queue: the next chunk of its stream.
+template <typename T, bool S4D>
+struct ChunkCursor {
+    int64_t g = 0, seg = 0, b = 0, d0 = 0, t_begin = 0, t_next = 0, t_end = 0;
+    bool open = false;
+
+    __device__ __forceinline__ ChunkDesc next(const FwdParams &p, const FwdScratch &sc, uint32_t *counter,
+                                              int lane) {
+        constexpr int TC = FwdSmem<T>::kTC;
+        const int64_t tiles = (p.dim + 31) / 32;
+        const int64_t groups = tiles * p.batch;
+        const int64_t items = groups * ((p.seqlen + kSegSteps - 1) / kSegSteps);
+        ChunkDesc dsc;
+        while (!open || t_next >= t_end) {
+            uint32_t item = 0;
             if (lane == 0) item = atomicAdd(counter, 1u);
             item = __shfl_sync(0xffffffffu, item, 0);
-            continue;
+            if (static_cast<int64_t>(item) >= items) {
+                dsc.flags = kStop;
+                return dsc;
+            }
+            seg = item / groups;
+            g = item % groups;
+            b = g / tiles;
+            d0 = (g % tiles) * 32;
+            t_begin = seg * kSegSteps;
+            t_end = t_begin + kSegSteps < p.seqlen ? t_begin + kSegSteps : p.seqlen;
+            t_next = t_begin;
+            const bool s4d = group_is_s4d(p, d0, lane);
+            if (s4d != S4D) {
+                if (S4D && lane == 0) atomicOr(sc.general, 1u);
+                open = false;
+                continue;
+            }
+            open = true;
         }
+        dsc.b = b; dsc.d0 = d0; dsc.t0 = t_next; dsc.g = g; dsc.seg = seg;
+        dsc.nvalid = static_cast<int32_t>(t_end - t_next < TC ? t_end - t_next : TC);
+        dsc.flags = (t_next == t_begin ? kFirst : 0) | (t_next + TC >= t_end ? kLast : 0) |
+                    (t_end == p.seqlen ? kSeqEnd : 0);
+        t_next += TC;
+        return dsc;
+    }
+};
 
-        // the state entering this segment
-        float2 h[8];
-        if (seg == 0) {
-            if (active && p.h0) {
-                const float4 *hr = reinterpret_cast<const float4 *>(p.h0 + (b * p.dim + d) * kNState);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float4 v = hr[q];
-                    h[2 * q] = make_float2(v.x, v.y);
-                    h[2 * q + 1] = make_float2(v.z, v.w);
+// ---- the kernel -----------------------------------------------------------------
+// Persistent and warp-specialized.  grid: one CTA per SM; block: kPairs warp
+// triples; warps w, w + 4 and w + 8 share an SM sub-partition and their own
+// slice of shared memory.
+//   prep (w + 4): takes items from the queue, stages chunks with TMA (or
+//          element loads), widens B|C and computes the per-step scalars
+//          (u, r); hands the chunk over (mbarrier ready).
+//   scan (w):    the recurrence on (u, r) and B|C with the state in registers;
+//          at segment boundaries it takes the state from h0 or the
+//          predecessor's carry and leaves it in the carry or h_last (done).
+//   post (w + 8): D skip, silu gate, bf16 pack and the TMA store of the
+//          output tile (posted).
+// The three instruction streams (MUFU-heavy, FMA-heavy, store) overlap on the
+// sub-partition.  Two instances run back to back: the S4D one takes groups
+// whose A rows are all S4D-structured and marks the scratch when it meets
+// another group; the general one then takes those.
+template <typename T, bool VEC, bool S4D>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    scan_fwd_kernel(const FwdParams p, const FwdScratch sc, const __grid_constant__ TmaMaps tm) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    // 1 KB alignment keeps every tile on a whole period of the 64-byte swizzle
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    using SM = FwdSmem<T>;
+    constexpr int TC = SM::kTC;
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int pair = warp & (kPairs - 1);
+    const int role = warp / kPairs;  // 0 scan, 1 prep, 2 post
+    uint8_t *ps = smem + pair * SM::kPairBytes;
+    uint64_t *ready = reinterpret_cast<uint64_t *>(ps + SM::kBarOff);
+    uint64_t *done = ready + 2;
+    uint64_t *posted = ready + 4;
+    uint64_t *full = ready + 6;  // [kStages]: TMA bytes of a staged chunk have landed
+    ChunkDesc *ring = reinterpret_cast<ChunkDesc *>(ps + SM::kDescOff);
+    auto stage_of = [&](int64_t j) { return ps + (j % kStages) * SM::kStageBytes; };
+    auto bcf_of = [&](int64_t j) { return reinterpret_cast<float *>(ps + SM::kBCFOff + (j & 1) * SM::kBCFBytes); };
+    auto ur_of = [&](int64_t j) { return reinterpret_cast<float2 *>(ps + SM::kUROff + (j & 1) * SM::kURBytes); };
+    auto parity = [](int64_t j, int n) { return static_cast<uint32_t>((j / n) & 1); };
+
+    if (threadIdx.x < kPairs) {
+        uint64_t *r = reinterpret_cast<uint64_t *>(smem + threadIdx.x * SM::kPairBytes + SM::kBarOff);
+        for (int i = 0; i < 6; ++i) mbar_init(r + i, 32);
+        for (int i = 0; i < kStages; ++i) mbar_init(r + 6 + i, 1);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    __syncthreads();
+    if (!S4D && *reinterpret_cast<volatile uint32_t *>(sc.general) == 0) return;
+    uint32_t *counter = sc.counter + (S4D ? 0 : 1);
+
+    if (role == 1) {
+        // ------------------------------------------------------------------ prep
+        ChunkCursor<T, S4D> cur;
+        const uint32_t stage_tx = (p.z ? 3u : 2u) * SM::kTileBytes + 2u * kNState * kRowBytes;
+        // stage chunk j: TMA (one lane, completion on full[j % kStages]) or element loads
+        auto issue = [&](const ChunkDesc &dsc, int64_t j) {
+            if (dsc.flags & kStop) return;
+            uint8_t *st = stage_of(j);
+            if constexpr (VEC) {
+                if (lane == 0) {
+                    uint64_t *bar = full + (j % kStages);
+                    mbar_arrive_expect_tx(bar, stage_tx);
+                    const int t0 = static_cast<int>(dsc.t0), d0 = static_cast<int>(dsc.d0), b = static_cast<int>(dsc.b);
+                    tma_load_3d(st, &tm.x, t0, d0, b, bar);
+                    tma_load_3d(st + SM::kTileBytes, &tm.delta, t0, d0, b, bar);
+                    if (p.z) tma_load_3d(st + 2 * SM::kTileBytes, &tm.z, t0, d0, b, bar);
+                    tma_load_3d(st + 3 * SM::kTileBytes, &tm.B, t0, 0, b, bar);
+                    tma_load_3d(st + 3 * SM::kTileBytes + kNState * kRowBytes, &tm.C, t0, 0, b, bar);
                 }
             } else {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) h[j] = make_float2(0.0f, 0.0f);
+                load_chunk_sync<T>(p, st, dsc.b, dsc.d0, dsc.t0, lane);
             }
-        } else {
-            uint32_t spins = 0;
-            while (ld_acquire(sc.flags + g) < static_cast<uint32_t>(seg)) {
-                if (++spins > kSpinLimit) {
-                    atomicOr(sc.error, 1u);
-                    break;
+        };
+        const bool softplus = p.softplus != 0;
+        ChunkDesc dnext = cur.next(p, sc, counter, lane);
+        issue(dnext, 0);
+        for (int64_t j = 0;; ++j) {
+            const ChunkDesc dj = dnext;
+            // chunk j+1 goes to the stage that chunk j-2 used: wait until it is posted
+            if (j >= 2) mbar_wait(posted + (j & 1), parity(j - 2, 2), sc.error);
+            if (!(dj.flags & kStop)) {
+                dnext = cur.next(p, sc, counter, lane);
+                issue(dnext, j + 1);
+                if constexpr (VEC) mbar_wait(full + (j % kStages), parity(j, kStages), sc.error);
+                __syncwarp();
+                uint8_t *st = stage_of(j);
+                widen_bc<T>(st + 3 * SM::kTileBytes, bcf_of(j), lane);
+                const int64_t d = dj.d0 + lane;
+                const ChanConst cc = chan_const(p, d < p.dim ? d : p.dim - 1);
+                chunk_prepass<T, S4D>(st, ur_of(j), lane, cc, softplus);
+            }
+            if (lane == 0) ring[j & 3] = dj;
+            __syncwarp();
+            mbar_arrive(ready + (j & 1));
+            if (dj.flags & kStop) break;
+        }
+    } else if (role == 2) {
+        // ------------------------------------------------------------------ post
+        const bool has_z = p.z != nullptr;
+        for (int64_t j = 0;; ++j) {
+            mbar_wait(done + (j & 1), parity(j, 2), sc.error);
+            const ChunkDesc dj = ring[j & 3];
+            if (dj.flags & kStop) break;
+            uint8_t *st = stage_of(j);
+            const int64_t d = dj.d0 + lane;
+            const ChanConst cc = chan_const(p, d < p.dim ? d : p.dim - 1);
+            chunk_postpass<T>(st, ur_of(j), lane, cc, has_z);
+            if constexpr (VEC) {
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_3d(&tm.out, static_cast<int>(dj.t0), static_cast<int>(dj.d0), static_cast<int>(dj.b), st);
+                    tma_store_commit();
+                    tma_store_wait_read();  // the stage is handed back for loading right after
                 }
-                __nanosleep(128);
+            } else {
+                __syncwarp();
+                store_chunk<T, VEC>(p, st, dj.b, dj.d0, dj.t0, lane);
             }
             __syncwarp();
-            const float4 *cr = reinterpret_cast<const float4 *>(sc.carry + (g * 32 + lane) * kNState);
+            mbar_arrive(posted + (j & 1));
+        }
+        if (VEC && lane == 0) tma_store_wait_all();
+    } else {
+        // ------------------------------------------------------------------ scan
+        float2 h[8];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float4 v = __ldcg(cr + q);
-                h[2 * q] = make_float2(v.x, v.y);
-                h[2 * q + 1] = make_float2(v.z, v.w);
+        for (int j = 0; j < 8; ++j) h[j] = make_float2(0.0f, 0.0f);
+        float a2[kNState];
+#pragma unroll
+        for (int n = 0; n < kNState; ++n) a2[n] = 0.0f;
+        for (int64_t k = 0;; ++k) {
+            mbar_wait(ready + (k & 1), parity(k, 2), sc.error);
+            const ChunkDesc dk = ring[k & 3];
+            if (dk.flags & kStop) {
+                mbar_arrive(done + (k & 1));  // lets the post warp see the end
+                break;
             }
-        }
-
-        const int64_t t_begin = seg * kSegSteps;
-        const int64_t t_end = t_begin + kSegSteps < p.seqlen ? t_begin + kSegSteps : p.seqlen;
-        scan_segment<T, VEC, S4D>(p, ws, b, d0, t_begin, t_end, lane, cc, a2, h);
-
-        if (t_end < p.seqlen) {
-            // hand the state to the next segment of this group
-            float4 *cr = reinterpret_cast<float4 *>(sc.carry + (g * 32 + lane) * kNState);
+            const int64_t d = dk.d0 + lane;
+            const bool active = d < p.dim;
+            if (dk.flags & kFirst) {
+                if (!S4D) {
+                    const float *ar = p.A + (active ? d : p.dim - 1) * kNState;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) __stcg(cr + q, make_float4(h[2 * q].x, h[2 * q].y, h[2 * q + 1].x, h[2 * q + 1].y));
-            __threadfence();
+                    for (int n = 0; n < kNState; ++n) a2[n] = ar[n] * kLog2e;
+                }
+                if (dk.seg == 0) {
+                    if (active && p.h0) {
+                        const float4 *hr = reinterpret_cast<const float4 *>(p.h0 + (dk.b * p.dim + d) * kNState);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float4 v = hr[q];
+                            h[2 * q] = make_float2(v.x, v.y);
+                            h[2 * q + 1] = make_float2(v.z, v.w);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) h[j] = make_float2(0.0f, 0.0f);
+                    }
+                } else {
+                    uint32_t spins = 0;
+                    while (ld_acquire(sc.flags + dk.g) < static_cast<uint32_t>(dk.seg)) {
+                        if (++spins > kSpinLimit) {
+                            atomicOr(sc.error, 1u);
+                            break;
+                        }
+                        __nanosleep(64);
+                    }
+                    const float4 *cr = reinterpret_cast<const float4 *>(sc.carry + (dk.g * 32 + lane) * kNState);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float4 v = __ldcg(cr + q);
+                        h[2 * q] = make_float2(v.x, v.y);
+                        h[2 * q + 1] = make_float2(v.z, v.w);
+                    }
+                }
+            }
+            if (dk.nvalid == TC)
+                chunk_core<S4D, true>(bcf_of(k), ur_of(k), lane, TC, a2, h);
+            else
+                chunk_core<S4D, false>(bcf_of(k), ur_of(k), lane, dk.nvalid, a2, h);
+            if (dk.flags & kLast) {
+                if (!(dk.flags & kSeqEnd)) {
+                    // hand the state to the next segment of this group
+                    float4 *cr = reinterpret_cast<float4 *>(sc.carry + (dk.g * 32 + lane) * kNState);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        __stcg(cr + q, make_float4(h[2 * q].x, h[2 * q].y, h[2 * q + 1].x, h[2 * q + 1].y));
+                    __threadfence();
+                    __syncwarp();
+                    if (lane == 0) st_release(sc.flags + dk.g, static_cast<uint32_t>(dk.seg + 1));
+                } else if (active && p.h_last) {
+                    float4 *hr = reinterpret_cast<float4 *>(p.h_last + (dk.b * p.dim + d) * kNState);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        hr[q] = make_float4(h[2 * q].x, h[2 * q].y, h[2 * q + 1].x, h[2 * q + 1].y);
+                }
+            }
             __syncwarp();
-            if (lane == 0) st_release(sc.flags + g, static_cast<uint32_t>(seg + 1));
-        } else if (active && p.h_last) {
-            float4 *hr = reinterpret_cast<float4 *>(p.h_last + (b * p.dim + d) * kNState);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) hr[q] = make_float4(h[2 * q].x, h[2 * q].y, h[2 * q + 1].x, h[2 * q + 1].y);
+            mbar_arrive(done + (k & 1));
         }
-
-        if (lane == 0) item = atomicAdd(counter, 1u);
-        item = __shfl_sync(0xffffffffu, item, 0);
     }
 }
 

@@ -5,11 +5,14 @@
 // stream.
 
 #include <climits>
+#include <cstring>
 #include <cstddef>
 #include <cstdint>
 #include <mutex>
 #include <type_traits>
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include "ssm_scan.h"
@@ -66,10 +69,53 @@ cudaMemPool_t scratch_pool(int dev) {
     return pools[dev];
 }
 
-// Persistent launch: one single-warp CTA per SM sub-partition (4 per SM), or
-// fewer when there are fewer items.  The work queue, segment flags and
-// carried states live in a stream-ordered scratch allocation of
-// fwd_scratch_bytes(groups) bytes, whose counter and flags are zeroed first.
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime
+// (no link-time dependency on libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// A rank-3 [d2][d1][d0] tensor (d0 contiguous) with a [1][box1][box0] box.
+bool encode3d(CUtensorMap *m, CUtensorMapDataType dt, size_t es, const void *base, uint64_t d0, uint64_t d1,
+              uint64_t d2, uint32_t box0, uint32_t box1, CUtensorMapSwizzle sw) {
+    auto fn = tensor_map_encoder();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {d0, d1, d2};
+    const cuuint64_t strides[2] = {d0 * es, d0 * d1 * es};
+    const cuuint32_t box[3] = {box0, box1, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename T>
+bool make_maps(const FwdParams &p, TmaMaps *tm) {
+    const CUtensorMapDataType dt = Act<T>::kBytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const size_t es = Act<T>::kBytes;
+    const uint32_t tc = FwdSmem<T>::kTC;
+    const uint64_t L = p.seqlen, D = p.dim, Bt = p.batch;
+    bool ok = encode3d(&tm->x, dt, es, p.x, L, D, Bt, tc, 32, CU_TENSOR_MAP_SWIZZLE_64B) &&
+              encode3d(&tm->delta, dt, es, p.delta, L, D, Bt, tc, 32, CU_TENSOR_MAP_SWIZZLE_64B) &&
+              encode3d(&tm->out, dt, es, p.out, L, D, Bt, tc, 32, CU_TENSOR_MAP_SWIZZLE_64B) &&
+              encode3d(&tm->B, dt, es, p.B, L, kNState, Bt, tc, kNState, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+              encode3d(&tm->C, dt, es, p.C, L, kNState, Bt, tc, kNState, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (ok && p.z) ok = encode3d(&tm->z, dt, es, p.z, L, D, Bt, tc, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+    return ok;
+}
+
+// Persistent launch: one CTA of kPairs scan/helper warp pairs per SM (or fewer
+// when there are fewer items).  The work queue, segment flags and carried
+// states live in a scratch allocation of fwd_scratch_bytes(groups) bytes whose
+// counters and flags are zeroed first.
 template <typename T, bool VEC>
 int launch_fwd(const FwdParams &p, cudaStream_t stream) {
     const int64_t groups = ((p.dim + 31) / 32) * p.batch;
@@ -79,13 +125,17 @@ int launch_fwd(const FwdParams &p, cudaStream_t stream) {
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return SSM_ERR_CUDA;
-    const int64_t workers = items < 4 * static_cast<int64_t>(sms) ? items : 4 * static_cast<int64_t>(sms);
-    const int smem = FwdSmem<T>::kWarpBytes;
+    const int64_t want = (items + kPairs - 1) / kPairs;
+    const int64_t ctas = want < sms ? want : sms;
+    const int smem = FwdSmem<T>::kTotal;
     auto k_s4d = scan_fwd_kernel<T, VEC, true>;
     auto k_gen = scan_fwd_kernel<T, VEC, false>;
     if (cudaFuncSetAttribute(k_s4d, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
         cudaFuncSetAttribute(k_gen, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return SSM_ERR_CUDA;
+    TmaMaps tm;
+    memset(&tm, 0, sizeof tm);
+    if (VEC && !make_maps<T>(p, &tm)) return SSM_ERR_CUDA;
     cudaMemPool_t pool = scratch_pool(dev);
     if (!pool) return SSM_ERR_CUDA;
     void *scratch = nullptr;
@@ -96,8 +146,8 @@ int launch_fwd(const FwdParams &p, cudaStream_t stream) {
         rc = SSM_ERR_CUDA;
     } else {
         const FwdScratch sc = fwd_scratch_view(scratch, groups);
-        k_s4d<<<static_cast<unsigned>(workers), kFwdThreads, smem, stream>>>(p, sc);
-        k_gen<<<static_cast<unsigned>(workers), kFwdThreads, smem, stream>>>(p, sc);
+        k_s4d<<<static_cast<unsigned>(ctas), kFwdThreads, smem, stream>>>(p, sc, tm);
+        k_gen<<<static_cast<unsigned>(ctas), kFwdThreads, smem, stream>>>(p, sc, tm);
         if (cudaGetLastError() != cudaSuccess) rc = SSM_ERR_CUDA;
     }
     if (cudaFreeAsync(scratch, stream) != cudaSuccess) rc = SSM_ERR_CUDA;

@@ -115,6 +115,27 @@ int ssm_scan_step(float *state, const void *x, const void *delta, const float *d
                   const float *D, const void *z, void *out,
                   const ssm_dims_t *dims, ssm_stream_t stream);
 
+/*
+ * ssm_scan_fwd without any device allocation.  The pages have no counterpart:
+ * this entry point exists for callers that cannot allocate device memory
+ * while they run the scan (code running inside an allocator or memory-pool
+ * callback, runtimes that reserve all device memory up front and forbid
+ * later allocations).  Arguments, layout, results and error codes are those
+ * of ssm_scan_fwd.  Its work queue, segment flags and carried states use a
+ * fixed 2 MiB device array inside the library (held by every GPU that loads
+ * it), so shapes with batch * ceil(dim / 32) above about 1000 are rejected
+ * with SSM_ERR_UNSUPPORTED.  The first call on a device looks up that array's
+ * address; make that first call before any stream capture.  Every call
+ * shares the one array of its device: calls whose work overlaps on the GPU
+ * (for example calls on two streams of the same device) race on it and must be
+ * serialised by the caller.  It allocates nothing: no cudaMalloc/cudaFree and
+ * no memory-pool allocation.
+ */
+int ssm_scan_fwd_noalloc(const void *x, const void *delta, const float *delta_bias, int softplus,
+                         const float *A, const void *B, const void *C, const float *D,
+                         const void *z, const float *h0, void *out, float *h_last,
+                         const ssm_dims_t *dims, ssm_stream_t stream);
+
 /* Static, human-readable text for an SSM_* code (never NULL). */
 const char *ssm_strerror(int code);
 

@@ -263,3 +263,117 @@ int ssm_scan_step(float *state, const void *x, const void *delta, const float *d
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------
+// Allocation-free forward scan.
+//
+// Some callers cannot allocate device memory while they run the scan: code
+// inside a custom allocator or memory-pool callback, runtimes that reserve all
+// device memory up front and forbid later allocation, and processes that must
+// not touch the CUDA allocator at all.  ssm_scan_fwd_noalloc serves them: it
+// runs the same kernels as ssm_scan_fwd, but its work queue, segment flags and
+// carried states live in the fixed device array below instead of a pool
+// allocation.  The array is part of the library image, so every GPU that loads
+// the library holds kNoAllocScratchBytes for the life of the process.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(2) << 20;  // fits ~1000 groups of 32 channels
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of the array on device `dev` (taken once per device, with
+// that device current; the first call on a device does this look-up).
+void *noalloc_scratch(int dev) {
+    static std::mutex mu;
+    static void *addr[64] = {};
+    if (dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
+        addr[dev] = ptr;
+    }
+    return addr[dev];
+}
+
+template <typename T, bool VEC>
+int launch_fwd_noalloc(const FwdParams &p, cudaStream_t stream) {
+    const int64_t groups = ((p.dim + 31) / 32) * p.batch;
+    const int64_t items = groups * ((p.seqlen + kSegSteps - 1) / kSegSteps);
+    if (items > static_cast<int64_t>(UINT32_MAX) / 2 || fwd_scratch_bytes(groups) > kNoAllocScratchBytes)
+        return SSM_ERR_UNSUPPORTED;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    void *scratch = noalloc_scratch(dev);
+    if (!scratch) return SSM_ERR_CUDA;
+    const int64_t want = (items + kPairs - 1) / kPairs;
+    const int64_t ctas = want < sms ? want : sms;
+    const int smem = FwdSmem<T>::kTotal;
+    auto k_s4d = scan_fwd_kernel<T, VEC, true>;
+    auto k_gen = scan_fwd_kernel<T, VEC, false>;
+    if (cudaFuncSetAttribute(k_s4d, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+        cudaFuncSetAttribute(k_gen, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    TmaMaps tm;
+    memset(&tm, 0, sizeof tm);
+    if (VEC && !make_maps<T>(p, &tm)) return SSM_ERR_CUDA;
+    // the array keeps the previous call's contents: the queue counters, error
+    // word and segment flags must start at zero (the carries need not)
+    if (cudaMemsetAsync(scratch, 0, fwd_scratch_flag_bytes(groups), stream) != cudaSuccess) return SSM_ERR_CUDA;
+    const FwdScratch sc = fwd_scratch_view(scratch, groups);
+    k_s4d<<<static_cast<unsigned>(ctas), kFwdThreads, smem, stream>>>(p, sc, tm);
+    k_gen<<<static_cast<unsigned>(ctas), kFwdThreads, smem, stream>>>(p, sc, tm);
+    return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" int ssm_scan_fwd_noalloc(const void *x, const void *delta, const float *delta_bias, int softplus,
+                                    const float *A, const void *B, const void *C, const float *D,
+                                    const void *z, const float *h0, void *out, float *h_last,
+                                    const ssm_dims_t *dims, ssm_stream_t stream) {
+    if (!dims) return SSM_ERR_INVALID_ARG;
+    const int64_t batch = dims->batch, L = dims->seqlen, dim = dims->dim, N = dims->dstate;
+    if (!x || !delta || !A || !B || !C || !out) return SSM_ERR_INVALID_ARG;
+    if (!dims_ok(batch, L, dim) || N < 1) return SSM_ERR_INVALID_ARG;
+    if (N != kNState) return SSM_ERR_UNSUPPORTED;
+    if (dims->act_dtype != SSM_F32 && dims->act_dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
+    const size_t es = dims->act_dtype == SSM_F32 ? 4 : 2;
+    for (const void *ptr : {x, delta, (const void *)A, B, C, z, (const void *)h0, (const void *)out,
+                            (const void *)h_last})
+        if (ptr && !aligned16(ptr)) return SSM_ERR_MISALIGNED;
+    for (const void *ptr : {(const void *)delta_bias, (const void *)D})
+        if (ptr && !aligned4(ptr)) return SSM_ERR_MISALIGNED;
+    const size_t tok = static_cast<size_t>(batch) * dim * L;
+    const Span o{out, tok * es};
+    const Span ins[] = {{x, tok * es}, {delta, tok * es}, {z, z ? tok * es : 0},
+                        {B, static_cast<size_t>(batch) * N * L * es}, {C, static_cast<size_t>(batch) * N * L * es},
+                        {A, static_cast<size_t>(dim) * N * 4}, {D, D ? static_cast<size_t>(dim) * 4 : 0},
+                        {delta_bias, delta_bias ? static_cast<size_t>(dim) * 4 : 0},
+                        {h0, h0 ? static_cast<size_t>(batch) * dim * N * 4 : 0},
+                        {h_last, h_last ? static_cast<size_t>(batch) * dim * N * 4 : 0}};
+    for (const Span &s : ins)
+        if (overlap(o, s)) return SSM_ERR_INVALID_ARG;
+    if (h_last) {
+        const Span hl{h_last, static_cast<size_t>(batch) * dim * N * 4};
+        for (int i = 0; i < 8; ++i)
+            if (overlap(hl, ins[i])) return SSM_ERR_INVALID_ARG;
+        if (h0 && h0 != h_last && overlap(hl, ins[8])) return SSM_ERR_INVALID_ARG;
+    }
+    // the work queue of this shape must fit the fixed array
+    const int64_t groups = ((dim + 31) / 32) * batch;
+    if (fwd_scratch_bytes(groups) > kNoAllocScratchBytes) return SSM_ERR_UNSUPPORTED;
+
+    FwdParams p;
+    p.x = x; p.delta = delta; p.z = z; p.B = B; p.C = C;
+    p.delta_bias = delta_bias; p.A = A; p.D = D; p.h0 = h0;
+    p.out = out; p.h_last = h_last;
+    p.batch = batch; p.seqlen = L; p.dim = dim;
+    p.softplus = softplus ? 1 : 0;
+    const bool vec = (static_cast<size_t>(L) * es) % 16 == 0;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (dims->act_dtype == SSM_BF16)
+        return vec ? launch_fwd_noalloc<bf16raw, true>(p, s) : launch_fwd_noalloc<bf16raw, false>(p, s);
+    return vec ? launch_fwd_noalloc<float, true>(p, s) : launch_fwd_noalloc<float, false>(p, s);
+}

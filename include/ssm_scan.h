@@ -27,10 +27,13 @@
  * arithmetic is float32; the state is float32.
  *
  * Ownership and execution: every pointer is a device pointer owned by the
- * caller.  The library keeps no state between calls and allocates no memory.
- * Work is enqueued on `stream` and runs asynchronously; the call returns
- * after validating the arguments and launching.  Errors that the device meets
- * later surface through the CUDA stream.  Calls are thread-safe.
+ * caller.  ssm_scan_fwd takes a small scratch area for its work queue
+ * (16 KB + 2 KB per group of 32 channels) from a library-owned, stream-ordered
+ * memory pool per device and returns it on the same stream; the pool keeps the
+ * memory between calls.  ssm_scan_step allocates nothing.  Work is enqueued on
+ * `stream` and runs asynchronously; the call returns after validating the
+ * arguments and launching.  Errors that the device meets later surface
+ * through the CUDA stream.  Calls are thread-safe.
  *
  * Error behaviour: every check is made on the host before anything is
  * launched; a call that returns non-zero has launched nothing and touched no

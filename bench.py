@@ -406,8 +406,18 @@ def run_gpu(args):
     hbm_peak, peak_kind = _peaks()
     c = workloads.CONFIGS[FWD_CFG]
 
+    if args.only == "step":
+        dec = bench_decode(args, device)
+        print(json.dumps({"only": "step", "ms_per_step": round(dec["ms"], 5), "value": round(dec["gbs"], 2),
+                          "unit": "GB/s"}), flush=True)
+        return 0
     f = bench_fwd(args, device, world)
     nb = fwd_bytes(FWD_CFG)
+    if args.only == "fwd":
+        print(json.dumps({"only": "fwd", "launch_ms_mean": round(f["launch_ms"], 5),
+                          "value": round(nb / (f["launch_ms"] * 1e-3) / 1e9, 2), "unit": "GB/s"}),
+              flush=True)
+        return 0
     ms_step = f["total_ms"] / args.steps
     value = world * nb / (ms_step * 1e-3) / 1e9
     achieved = nb / (f["launch_ms"] * 1e-3) / 1e9
@@ -464,9 +474,11 @@ def run_gpu(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    # profiler runs: only the forward-scan or only the decode-step timing loop
+    ap.add_argument("--only", default=None, choices=["fwd", "step"])
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

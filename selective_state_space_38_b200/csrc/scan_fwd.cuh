@@ -617,8 +617,12 @@ template <typename T, bool VEC, bool S4D>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     scan_fwd_kernel(const FwdParams p, const FwdScratch sc, const __grid_constant__ TmaMaps tm) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    // 1 KB alignment keeps every tile on a whole period of the 64-byte swizzle
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1 KB alignment keeps every tile on a whole period of the 64-byte swizzle.  The
+    // offset is added to the shared-memory pointer itself (no round trip through an
+    // integer), so the compiler keeps the shared address space and emits ld/st.shared
+    // rather than generic accesses, which cost twice the data-pipe passes on a
+    // warp-uniform read.
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     using SM = FwdSmem<T>;
     constexpr int TC = SM::kTC;
     const int lane = threadIdx.x & 31;

@@ -27,10 +27,14 @@
  * arithmetic is float32; the state is float32.
  *
  * Ownership and execution: every pointer is a device pointer owned by the
- * caller.  ssm_scan_fwd takes a small scratch area for its work queue
- * (16 KB + 2 KB per group of 32 channels) from a library-owned, stream-ordered
- * memory pool per device and returns it on the same stream; the pool keeps the
- * memory between calls.  ssm_scan_step allocates nothing.  Work is enqueued on
+ * caller.  ssm_scan_fwd takes a scratch area for its work queue (16 KB + 2 KB
+ * per group of 32 channels) from a library-owned, stream-ordered memory pool per
+ * device and returns it on the same stream; the pool keeps the memory between
+ * calls.  When the channel groups (batch * ceil(dim / 32)) number fewer than
+ * half the GPU's SM sub-partitions, the call cuts each sequence into segments
+ * and scans them in parallel in two passes; the scratch then also holds 6 KB per
+ * (group, segment), with about 4 * (SM sub-partitions) segments in all (under
+ * 15 MB on a 148-SM GPU).  ssm_scan_step allocates nothing.  Work is enqueued on
  * `stream` and runs asynchronously; the call returns after validating the
  * arguments and launching.  Errors that the device meets later surface
  * through the CUDA stream.  Calls are thread-safe.
@@ -127,8 +131,11 @@ int ssm_scan_step(float *state, const void *x, const void *delta, const float *d
  * of ssm_scan_fwd.  Its work queue, segment flags and carried states use a
  * fixed 2 MiB device array inside the library (held by every GPU that loads
  * it), so shapes with batch * ceil(dim / 32) above about 1000 are rejected
- * with SSM_ERR_UNSUPPORTED.  The first call on a device looks up that array's
- * address; make that first call before any stream capture.  Every call
+ * with SSM_ERR_UNSUPPORTED.  It always scans the segments of a group in order
+ * (no two-pass parallel schedule), whatever the number of groups, so shapes
+ * with few channel groups run slower here than through ssm_scan_fwd.  The
+ * first call on a device looks up that array's address; make that first call
+ * before any stream capture.  Every call
  * shares the one array of its device: calls whose work overlaps on the GPU
  * (for example calls on two streams of the same device) race on it and must be
  * serialised by the caller.  It allocates nothing: no cudaMalloc/cudaFree and

@@ -46,7 +46,15 @@ struct FwdParams {
     float *h_last;
     int64_t batch, seqlen, dim;
     int softplus;
+    // kChained: segments of a group run in order, each starting from its
+    // predecessor's carried state.  kSummary and kFromStart are the two scan passes
+    // of the time-parallel schedule: every segment first runs from a zero state and
+    // records its end state and decay product; after segment_combine_kernel has
+    // turned those into start states, every segment runs again from its own.
+    int mode;
+    int64_t seg_steps;  // steps per segment, a multiple of 32
 };
+constexpr int kChained = 0, kSummary = 1, kFromStart = 2;
 
 // TMA descriptors of the aligned path: activations as 3-D [batch][dim][L]
 // tensors with [1][32][TC] boxes and the 64-byte swizzle (the same XOR layout
@@ -270,7 +278,7 @@ struct StepOps {
     float2 a[8], ub[8], c[8];
 };
 
-template <bool S4D>
+template <bool S4D, bool READOUT = true>
 __device__ __forceinline__ void prepare_step(const float *bcf, const float2 *ur, int t, int row,
                                              const float (&a2)[kNState], StepOps &s) {
     const float2 ut_rt = ur[t * 32 + row];
@@ -278,11 +286,14 @@ __device__ __forceinline__ void prepare_step(const float *bcf, const float2 *ur,
     const float2 U2 = make_float2(ut_rt.x, ut_rt.x);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-        const float4 b4 = p[q], c4 = p[4 + q];
+        const float4 b4 = p[q];
         s.ub[2 * q] = __fmul2_rn(U2, make_float2(b4.x, b4.y));
         s.ub[2 * q + 1] = __fmul2_rn(U2, make_float2(b4.z, b4.w));
-        s.c[2 * q] = make_float2(c4.x, c4.y);
-        s.c[2 * q + 1] = make_float2(c4.z, c4.w);
+        if (READOUT) {
+            const float4 c4 = p[4 + q];
+            s.c[2 * q] = make_float2(c4.x, c4.y);
+            s.c[2 * q + 1] = make_float2(c4.z, c4.w);
+        }
     }
     const float Rt = ut_rt.y;
     if constexpr (S4D) {
@@ -331,6 +342,32 @@ __device__ __forceinline__ void chunk_core(const float *bcf, float2 *ur, int row
             }
             const float2 ys = __fadd2_rn(ya, yb);
             ur[t * 32 + row].x = ys.x + ys.y;
+        }
+    }
+}
+
+// The summary pass of the time-parallel schedule: the same state update, with
+// the running product of the per-step decays P_n = prod_t Abar_{t,n} in place
+// of the readout (so P carries the rounding of the decays the sequential scan
+// applies).  No y is produced.
+template <bool S4D, bool FULL>
+__device__ __forceinline__ void chunk_summary(const float *bcf, const float2 *ur, int row, int nvalid,
+                                              const float (&a2)[kNState], float2 (&h)[8], float2 (&P)[8]) {
+    StepOps nxt;
+    prepare_step<S4D, false>(bcf, ur, 0, row, a2, nxt);
+#pragma unroll 1
+    for (int t0 = 0; t0 < nvalid; t0 += 8) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int t = t0 + i;
+            if (!FULL && t >= nvalid) break;
+            const StepOps cur = nxt;
+            if (FULL || t + 1 < nvalid) prepare_step<S4D, false>(bcf, ur, t + 1, row, a2, nxt);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                h[j] = __ffma2_rn(cur.a[j], h[j], cur.ub[j]);
+                P[j] = __fmul2_rn(cur.a[j], P[j]);
+            }
         }
     }
 }
@@ -440,8 +477,8 @@ __device__ __forceinline__ void store_chunk(const FwdParams &p, const uint8_t *t
 }
 
 // ---- work queue and carried state ----------------------------------------------
-// The sequence of each 32-channel group is cut into segments of kSegSteps
-// steps.  An item is one (group, segment) pair; items are handed out in
+// The sequence of each 32-channel group is cut into segments of p.seg_steps
+// steps (kSegSteps for the chained schedule).  An item is one (group, segment) pair; items are handed out in
 // segment-major order through an atomic counter, so the work spreads evenly
 // over the persistent workers whatever the number of groups.  A segment other
 // than the first starts from the state its predecessor left in `carry` and
@@ -458,16 +495,20 @@ struct FwdScratch {
     uint32_t *general;  // non-zero: some group has A rows without the S4D structure
     uint32_t *flags;    // [groups]: segments of the group finished
     float *carry;       // [groups][32 lanes][16 states]
+    float *summ;        // time-parallel schedule: [groups][segs][32 lanes][16 end states, 16 decay products]
+    float *start;       // time-parallel schedule: [groups][segs][32 lanes][16 start states]
 };
 
-// bytes of scratch for `groups` groups; the first flag_bytes(...) bytes must be zero at launch
+// bytes of scratch for `groups` groups (and, for the time-parallel schedule,
+// `segs` segments per group); the first flag_bytes(...) bytes must be zero at launch
 __host__ __device__ inline size_t fwd_scratch_flag_bytes(int64_t groups) {
     return (256 + 4 * static_cast<size_t>(groups) + 255) / 256 * 256;
 }
-__host__ __device__ inline size_t fwd_scratch_bytes(int64_t groups) {
-    return fwd_scratch_flag_bytes(groups) + static_cast<size_t>(groups) * 32 * kNState * 4;
+__host__ __device__ inline size_t fwd_scratch_bytes(int64_t groups, int64_t segs = 0) {
+    return fwd_scratch_flag_bytes(groups) + static_cast<size_t>(groups) * 32 * kNState * 4 +
+           static_cast<size_t>(groups) * segs * 32 * 3 * kNState * 4;
 }
-__host__ __device__ inline FwdScratch fwd_scratch_view(void *base, int64_t groups) {
+__host__ __device__ inline FwdScratch fwd_scratch_view(void *base, int64_t groups, int64_t segs = 0) {
     uint8_t *b = static_cast<uint8_t *>(base);
     FwdScratch s;
     s.counter = reinterpret_cast<uint32_t *>(b);
@@ -475,6 +516,8 @@ __host__ __device__ inline FwdScratch fwd_scratch_view(void *base, int64_t group
     s.general = reinterpret_cast<uint32_t *>(b + 12);
     s.flags = reinterpret_cast<uint32_t *>(b + 256);
     s.carry = reinterpret_cast<float *>(b + fwd_scratch_flag_bytes(groups));
+    s.summ = s.carry + static_cast<size_t>(groups) * 32 * kNState;
+    s.start = s.summ + static_cast<size_t>(groups) * segs * 32 * 2 * kNState;
     return s;
 }
 
@@ -507,6 +550,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32
             : "r"(addr), "r"(parity)
             : "memory");
         if (done) return true;
+        // once any wait of the launch has given up, stop waiting: the results are void
+        if ((n & 1023u) == 1023u && *reinterpret_cast<volatile uint32_t *>(error) != 0) return false;
     }
     atomicOr(error, 2u);
     return false;
@@ -563,7 +608,7 @@ struct ChunkCursor {
         constexpr int TC = FwdSmem<T>::kTC;
         const int64_t tiles = (p.dim + 31) / 32;
         const int64_t groups = tiles * p.batch;
-        const int64_t items = groups * ((p.seqlen + kSegSteps - 1) / kSegSteps);
+        const int64_t items = groups * ((p.seqlen + p.seg_steps - 1) / p.seg_steps);
         ChunkDesc dsc;
         while (!open || t_next >= t_end) {
             uint32_t item = 0;
@@ -577,8 +622,8 @@ struct ChunkCursor {
             g = item % groups;
             b = g / tiles;
             d0 = (g % tiles) * 32;
-            t_begin = seg * kSegSteps;
-            t_end = t_begin + kSegSteps < p.seqlen ? t_begin + kSegSteps : p.seqlen;
+            t_begin = seg * p.seg_steps;
+            t_end = t_begin + p.seg_steps < p.seqlen ? t_begin + p.seg_steps : p.seqlen;
             t_next = t_begin;
             const bool s4d = group_is_s4d(p, d0, lane);
             if (s4d != S4D) {
@@ -704,6 +749,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             const ChunkDesc dj = ring[j & 3];
             if (dj.flags & kStop) break;
             uint8_t *st = stage_of(j);
+            if (p.mode == kSummary) {  // the summary pass writes no output
+                __syncwarp();
+                mbar_arrive(posted + (j & 1));
+                continue;
+            }
             const int64_t d = dj.d0 + lane;
             const ChanConst cc = chan_const(p, d < p.dim ? d : p.dim - 1);
             chunk_postpass<T>(st, ur_of(j), lane, cc, has_z);
@@ -725,9 +775,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (VEC && lane == 0) tma_store_wait_all();
     } else {
         // ------------------------------------------------------------------ scan
-        float2 h[8];
+        const int64_t segs = (p.seqlen + p.seg_steps - 1) / p.seg_steps;
+        float2 h[8], P[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) h[j] = make_float2(0.0f, 0.0f);
+        for (int j = 0; j < 8; ++j) h[j] = P[j] = make_float2(0.0f, 0.0f);
         float a2[kNState];
 #pragma unroll
         for (int n = 0; n < kNState; ++n) a2[n] = 0.0f;
@@ -740,25 +791,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             }
             const int64_t d = dk.d0 + lane;
             const bool active = d < p.dim;
+            const int64_t gs = (dk.g * segs + dk.seg) * 32 + lane;  // (group, segment, lane) slot
             if (dk.flags & kFirst) {
                 if (!S4D) {
                     const float *ar = p.A + (active ? d : p.dim - 1) * kNState;
 #pragma unroll
                     for (int n = 0; n < kNState; ++n) a2[n] = ar[n] * kLog2e;
                 }
-                if (dk.seg == 0) {
-                    if (active && p.h0) {
-                        const float4 *hr = reinterpret_cast<const float4 *>(p.h0 + (dk.b * p.dim + d) * kNState);
+                const float4 *src = nullptr;
+                if (p.mode == kSummary) {
+                    // every segment starts from zero; P starts as the identity
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const float4 v = hr[q];
-                            h[2 * q] = make_float2(v.x, v.y);
-                            h[2 * q + 1] = make_float2(v.z, v.w);
-                        }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) h[j] = make_float2(0.0f, 0.0f);
-                    }
+                    for (int j = 0; j < 8; ++j) P[j] = make_float2(1.0f, 1.0f);
+                } else if (dk.seg == 0) {
+                    if (active && p.h0) src = reinterpret_cast<const float4 *>(p.h0 + (dk.b * p.dim + d) * kNState);
+                } else if (p.mode == kFromStart) {
+                    src = reinterpret_cast<const float4 *>(sc.start + gs * kNState);
                 } else {
                     uint32_t spins = 0;
                     while (ld_acquire(sc.flags + dk.g) < static_cast<uint32_t>(dk.seg)) {
@@ -768,29 +816,45 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                         }
                         __nanosleep(64);
                     }
-                    const float4 *cr = reinterpret_cast<const float4 *>(sc.carry + (dk.g * 32 + lane) * kNState);
+                    src = reinterpret_cast<const float4 *>(sc.carry + (dk.g * 32 + lane) * kNState);
+                }
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const float4 v = __ldcg(cr + q);
-                        h[2 * q] = make_float2(v.x, v.y);
-                        h[2 * q + 1] = make_float2(v.z, v.w);
-                    }
+                for (int q = 0; q < 4; ++q) {
+                    const float4 v = src ? __ldcg(src + q) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                    h[2 * q] = make_float2(v.x, v.y);
+                    h[2 * q + 1] = make_float2(v.z, v.w);
                 }
             }
-            if (dk.nvalid == TC)
+            if (p.mode == kSummary) {
+                if (dk.nvalid == TC)
+                    chunk_summary<S4D, true>(bcf_of(k), ur_of(k), lane, TC, a2, h, P);
+                else
+                    chunk_summary<S4D, false>(bcf_of(k), ur_of(k), lane, dk.nvalid, a2, h, P);
+            } else if (dk.nvalid == TC) {
                 chunk_core<S4D, true>(bcf_of(k), ur_of(k), lane, TC, a2, h);
-            else
+            } else {
                 chunk_core<S4D, false>(bcf_of(k), ur_of(k), lane, dk.nvalid, a2, h);
+            }
             if (dk.flags & kLast) {
-                if (!(dk.flags & kSeqEnd)) {
-                    // hand the state to the next segment of this group
-                    float4 *cr = reinterpret_cast<float4 *>(sc.carry + (dk.g * 32 + lane) * kNState);
+                if (p.mode == kSummary) {
+                    // the segment's end state from zero and its decay product
+                    float4 *sm = reinterpret_cast<float4 *>(sc.summ + gs * 2 * kNState);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        __stcg(cr + q, make_float4(h[2 * q].x, h[2 * q].y, h[2 * q + 1].x, h[2 * q + 1].y));
-                    __threadfence();
-                    __syncwarp();
-                    if (lane == 0) st_release(sc.flags + dk.g, static_cast<uint32_t>(dk.seg + 1));
+                    for (int q = 0; q < 4; ++q) {
+                        __stcg(sm + q, make_float4(h[2 * q].x, h[2 * q].y, h[2 * q + 1].x, h[2 * q + 1].y));
+                        __stcg(sm + 4 + q, make_float4(P[2 * q].x, P[2 * q].y, P[2 * q + 1].x, P[2 * q + 1].y));
+                    }
+                } else if (!(dk.flags & kSeqEnd)) {
+                    if (p.mode == kChained) {
+                        // hand the state to the next segment of this group
+                        float4 *cr = reinterpret_cast<float4 *>(sc.carry + (dk.g * 32 + lane) * kNState);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            __stcg(cr + q, make_float4(h[2 * q].x, h[2 * q].y, h[2 * q + 1].x, h[2 * q + 1].y));
+                        __threadfence();
+                        __syncwarp();
+                        if (lane == 0) st_release(sc.flags + dk.g, static_cast<uint32_t>(dk.seg + 1));
+                    }
                 } else if (active && p.h_last) {
                     float4 *hr = reinterpret_cast<float4 *>(p.h_last + (dk.b * p.dim + d) * kNState);
 #pragma unroll
@@ -800,6 +864,45 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             }
             __syncwarp();
             mbar_arrive(done + (k & 1));
+        }
+    }
+}
+
+// Start states of every segment for the time-parallel schedule, from the
+// summaries of the segments before it: h_0 = h0 (or 0), h_{s+1} = P_s h_s + e_s
+// with e_s the end state of segment s run from zero and P_s its decay product
+// (the splitting of the recurrence into chunks that continue from a carried
+// state, applied to the carries themselves).  One thread per (group, lane).
+__global__ void segment_combine_kernel(const FwdParams p, const FwdScratch sc) {
+    const int64_t tiles = (p.dim + 31) / 32;
+    const int64_t groups = tiles * p.batch;
+    const int64_t segs = (p.seqlen + p.seg_steps - 1) / p.seg_steps;
+    const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t g = tid / 32;
+    const int lane = static_cast<int>(tid % 32);
+    if (g >= groups) return;
+    const int64_t d = (g % tiles) * 32 + lane, b = g / tiles;
+    float h[kNState];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        if (p.h0 && d < p.dim) v = reinterpret_cast<const float4 *>(p.h0 + (b * p.dim + d) * kNState)[q];
+        h[4 * q] = v.x; h[4 * q + 1] = v.y; h[4 * q + 2] = v.z; h[4 * q + 3] = v.w;
+    }
+    for (int64_t s = 0; s < segs; ++s) {
+        const int64_t gs = (g * segs + s) * 32 + lane;
+        float4 *st = reinterpret_cast<float4 *>(sc.start + gs * kNState);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) st[q] = make_float4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
+        if (s + 1 == segs) break;
+        const float4 *sm = reinterpret_cast<const float4 *>(sc.summ + gs * 2 * kNState);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 e = sm[q], pr = sm[4 + q];
+            h[4 * q] = fmaf(pr.x, h[4 * q], e.x);
+            h[4 * q + 1] = fmaf(pr.y, h[4 * q + 1], e.y);
+            h[4 * q + 2] = fmaf(pr.z, h[4 * q + 2], e.z);
+            h[4 * q + 3] = fmaf(pr.w, h[4 * q + 3], e.w);
         }
     }
 }

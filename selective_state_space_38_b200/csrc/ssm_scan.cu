@@ -112,12 +112,73 @@ bool make_maps(const FwdParams &p, TmaMaps *tm) {
     return ok;
 }
 
-// Persistent launch: one CTA of kPairs scan/helper warp pairs per SM (or fewer
-// when there are fewer items).  The work queue, segment flags and carried
-// states live in a scratch allocation of fwd_scratch_bytes(groups) bytes whose
-// counters and flags are zeroed first.
+// The schedule for a shape.  Segments of a group form a chain; when the groups
+// alone cannot keep every SM sub-partition's scan warp busy (fewer than half as
+// many groups as sub-partitions), the time-parallel schedule cuts each sequence
+// into enough segments for about four items per warp and pays a summary pass
+// (about two thirds of a scan) to run them all at once.  Returns the segment
+// count of the time-parallel schedule, or 0 for the chained one.
+int64_t parallel_segments(const FwdParams &p, int sms, int64_t *seg_steps) {
+    const int64_t groups = ((p.dim + 31) / 32) * p.batch;
+    const int64_t workers = static_cast<int64_t>(kPairs) * sms;
+    if (2 * groups > workers) return 0;
+    const int64_t want = (4 * workers + groups - 1) / groups;
+    int64_t steps = (p.seqlen + want - 1) / want;
+    steps = (steps + 31) / 32 * 32;
+    if (steps < 256) steps = 256;
+    const int64_t segs = (p.seqlen + steps - 1) / steps;
+    if (segs < 2) return 0;
+    *seg_steps = steps;
+    return segs;
+}
+
+// Persistent launch: one CTA of kPairs warp triples per SM (or fewer when there
+// are fewer items); the S4D instance, then the general one.
 template <typename T, bool VEC>
-int launch_fwd(const FwdParams &p, cudaStream_t stream) {
+int launch_pass(const FwdParams &p, const FwdScratch &sc, const TmaMaps &tm, int sms, cudaStream_t stream) {
+    const int64_t groups = ((p.dim + 31) / 32) * p.batch;
+    const int64_t items = groups * ((p.seqlen + p.seg_steps - 1) / p.seg_steps);
+    const int64_t want = (items + kPairs - 1) / kPairs;
+    const int64_t ctas = want < sms ? want : sms;
+    const int smem = FwdSmem<T>::kTotal;
+    scan_fwd_kernel<T, VEC, true><<<static_cast<unsigned>(ctas), kFwdThreads, smem, stream>>>(p, sc, tm);
+    scan_fwd_kernel<T, VEC, false><<<static_cast<unsigned>(ctas), kFwdThreads, smem, stream>>>(p, sc, tm);
+    return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+// The kernels of one forward call on zeroed scratch: one chained pass, or the
+// summary pass, the segment combine and the second pass of the time-parallel
+// schedule (the queue is re-armed between the passes).
+template <typename T, bool VEC>
+int launch_fwd_kernels(FwdParams p, void *scratch, int64_t segs, int sms, cudaStream_t stream) {
+    const int64_t groups = ((p.dim + 31) / 32) * p.batch;
+    const int smem = FwdSmem<T>::kTotal;
+    if (cudaFuncSetAttribute(scan_fwd_kernel<T, VEC, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(scan_fwd_kernel<T, VEC, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess)
+        return SSM_ERR_CUDA;
+    TmaMaps tm;
+    memset(&tm, 0, sizeof tm);
+    if (VEC && !make_maps<T>(p, &tm)) return SSM_ERR_CUDA;
+    const FwdScratch sc = fwd_scratch_view(scratch, groups, segs);
+    if (segs == 0) {
+        p.mode = kChained;
+        p.seg_steps = kSegSteps;
+        return launch_pass<T, VEC>(p, sc, tm, sms, stream);
+    }
+    p.mode = kSummary;
+    int rc = launch_pass<T, VEC>(p, sc, tm, sms, stream);
+    if (rc != SSM_OK) return rc;
+    const int64_t threads = groups * 32;
+    segment_combine_kernel<<<static_cast<unsigned>((threads + 127) / 128), 128, 0, stream>>>(p, sc);
+    if (cudaMemsetAsync(scratch, 0, fwd_scratch_flag_bytes(groups), stream) != cudaSuccess) return SSM_ERR_CUDA;
+    p.mode = kFromStart;
+    return launch_pass<T, VEC>(p, sc, tm, sms, stream);
+}
+
+template <typename T, bool VEC>
+int launch_fwd(FwdParams p, cudaStream_t stream) {
     const int64_t groups = ((p.dim + 31) / 32) * p.batch;
     const int64_t items = groups * ((p.seqlen + kSegSteps - 1) / kSegSteps);
     if (items > static_cast<int64_t>(UINT32_MAX) / 2) return SSM_ERR_UNSUPPORTED;
@@ -125,31 +186,17 @@ int launch_fwd(const FwdParams &p, cudaStream_t stream) {
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return SSM_ERR_CUDA;
-    const int64_t want = (items + kPairs - 1) / kPairs;
-    const int64_t ctas = want < sms ? want : sms;
-    const int smem = FwdSmem<T>::kTotal;
-    auto k_s4d = scan_fwd_kernel<T, VEC, true>;
-    auto k_gen = scan_fwd_kernel<T, VEC, false>;
-    if (cudaFuncSetAttribute(k_s4d, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
-        cudaFuncSetAttribute(k_gen, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-        return SSM_ERR_CUDA;
-    TmaMaps tm;
-    memset(&tm, 0, sizeof tm);
-    if (VEC && !make_maps<T>(p, &tm)) return SSM_ERR_CUDA;
+    const int64_t segs = parallel_segments(p, sms, &p.seg_steps);
     cudaMemPool_t pool = scratch_pool(dev);
     if (!pool) return SSM_ERR_CUDA;
     void *scratch = nullptr;
-    if (cudaMallocFromPoolAsync(&scratch, fwd_scratch_bytes(groups), pool, stream) != cudaSuccess)
+    if (cudaMallocFromPoolAsync(&scratch, fwd_scratch_bytes(groups, segs), pool, stream) != cudaSuccess)
         return SSM_ERR_CUDA;
     int rc = SSM_OK;
-    if (cudaMemsetAsync(scratch, 0, fwd_scratch_flag_bytes(groups), stream) != cudaSuccess) {
+    if (cudaMemsetAsync(scratch, 0, fwd_scratch_flag_bytes(groups), stream) != cudaSuccess)
         rc = SSM_ERR_CUDA;
-    } else {
-        const FwdScratch sc = fwd_scratch_view(scratch, groups);
-        k_s4d<<<static_cast<unsigned>(ctas), kFwdThreads, smem, stream>>>(p, sc, tm);
-        k_gen<<<static_cast<unsigned>(ctas), kFwdThreads, smem, stream>>>(p, sc, tm);
-        if (cudaGetLastError() != cudaSuccess) rc = SSM_ERR_CUDA;
-    }
+    else
+        rc = launch_fwd_kernels<T, VEC>(p, scratch, segs, sms, stream);
     if (cudaFreeAsync(scratch, stream) != cudaSuccess) rc = SSM_ERR_CUDA;
     return rc;
 }
@@ -295,6 +342,7 @@ void *noalloc_scratch(int dev) {
     return addr[dev];
 }
 
+// Always the chained schedule: its scratch does not grow with the sequence.
 template <typename T, bool VEC>
 int launch_fwd_noalloc(const FwdParams &p, cudaStream_t stream) {
     const int64_t groups = ((p.dim + 31) / 32) * p.batch;
@@ -307,24 +355,10 @@ int launch_fwd_noalloc(const FwdParams &p, cudaStream_t stream) {
         return SSM_ERR_CUDA;
     void *scratch = noalloc_scratch(dev);
     if (!scratch) return SSM_ERR_CUDA;
-    const int64_t want = (items + kPairs - 1) / kPairs;
-    const int64_t ctas = want < sms ? want : sms;
-    const int smem = FwdSmem<T>::kTotal;
-    auto k_s4d = scan_fwd_kernel<T, VEC, true>;
-    auto k_gen = scan_fwd_kernel<T, VEC, false>;
-    if (cudaFuncSetAttribute(k_s4d, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
-        cudaFuncSetAttribute(k_gen, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-        return SSM_ERR_CUDA;
-    TmaMaps tm;
-    memset(&tm, 0, sizeof tm);
-    if (VEC && !make_maps<T>(p, &tm)) return SSM_ERR_CUDA;
     // the array keeps the previous call's contents: the queue counters, error
     // word and segment flags must start at zero (the carries need not)
     if (cudaMemsetAsync(scratch, 0, fwd_scratch_flag_bytes(groups), stream) != cudaSuccess) return SSM_ERR_CUDA;
-    const FwdScratch sc = fwd_scratch_view(scratch, groups);
-    k_s4d<<<static_cast<unsigned>(ctas), kFwdThreads, smem, stream>>>(p, sc, tm);
-    k_gen<<<static_cast<unsigned>(ctas), kFwdThreads, smem, stream>>>(p, sc, tm);
-    return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+    return launch_fwd_kernels<T, VEC>(p, scratch, 0, sms, stream);
 }
 
 }  // namespace

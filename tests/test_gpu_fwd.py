@@ -97,6 +97,28 @@ def test_mixed_A_rows(orc):
     check(to_np64(hl), ref_hl, "bf16", "h_last mixed A")
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("A_kind", ["s4d", "general", "mixed"])
+@pytest.mark.parametrize("L", [4000, 4001])
+def test_time_parallel_schedule(orc, dtype, A_kind, L):
+    """Few channel groups over a long sequence take the time-parallel schedule:
+    every segment is summarised from a zero state, the summaries are combined
+    into start states, and every segment runs again from its own.  Here 2 groups
+    (40 channels, the second ragged) over 4000 or 4001 steps, which the schedule
+    cuts into 16 segments of 256 with a ragged last one, from a random h0; 4001
+    also takes the element-wise (unaligned) loads."""
+    inp = workloads.custom_inputs(1, L, 40, 16, dtype=dtype, seed=L + len(A_kind), has_h0=True)
+    rng = np.random.default_rng(L)
+    if A_kind == "general":
+        inp["A"] = -rng.uniform(0.05, 3.0, size=inp["A"].shape).astype(np.float32)
+    elif A_kind == "mixed":
+        inp["A"][3] = -np.linspace(0.3, 4.0, 16, dtype=np.float32)
+    out, hl = _gpu_fwd(inp)
+    ref_out, ref_hl = _oracle(orc, inp)
+    check(to_np64(out), ref_out, dtype, f"out time-parallel {A_kind} L={L}")
+    check(to_np64(hl), ref_hl, dtype, f"h_last time-parallel {A_kind} L={L}")
+
+
 def test_extreme_dt(orc):
     """dt spanning 1e-6..50: state decay from ~1 (memory) to exactly 0 (reset)."""
     inp = workloads.custom_inputs(1, 257, 64, 16, dtype="bf16", seed=9, has_h0=True)

@@ -316,8 +316,8 @@ __device__ __forceinline__ void prepare_step(const float *bcf, const float2 *ur,
 
 // The state update over the chunk's first `nvalid` steps, software-pipelined
 // by hand: the operands of step t+1 are prepared while step t updates the
-// state.  y_t = C_t . h_t (without the D skip and the gate) replaces u in
-// ur[t][lane].x.  Full chunks run a branch-free body (the preparation of the
+// state.  y_t = C_t . h_t (without the D skip and the gate) is stored densely
+// as float `lane` of row t of ur, over (u, r) pairs the warp has already read.  Full chunks run a branch-free body (the preparation of the
 // step after the chunk reads the spare table row); only the last, partial
 // chunk of a sequence tests the step index.
 template <bool S4D, bool FULL>
@@ -341,7 +341,7 @@ __device__ __forceinline__ void chunk_core(const float *bcf, float2 *ur, int row
                 else ya = __ffma2_rn(cur.c[j], h[j], ya);
             }
             const float2 ys = __fadd2_rn(ya, yb);
-            ur[t * 32 + row].x = ys.x + ys.y;
+            reinterpret_cast<float *>(ur + t * 32)[row] = ys.x + ys.y;  // dense: one wavefront
         }
     }
 }
@@ -375,6 +375,7 @@ __device__ __forceinline__ void chunk_summary(const float *bcf, const float2 *ur
 // ---- phase 3: D skip, gate, output -----------------------------------------------
 // out_t = (y_t + D x_t) silu(z_t), written over the lane's own x row of the
 // stage (already consumed); stage by stage over step pairs as in phase 1.
+// y_t is float `lane` of row t of ur.
 template <typename T>
 __device__ __forceinline__ void chunk_postpass(uint8_t *stage, const float2 *ur, int row,
                                                const ChanConst &cc, bool has_z) {
@@ -395,7 +396,8 @@ __device__ __forceinline__ void chunk_postpass(uint8_t *stage, const float2 *ur,
     for (int k = 0; k < NP; ++k) {
         const int pc = (2 * k) / PP, i = (2 * k) % PP;
         const float2 X = make_float2(AT::piece(xv[pc], i), AT::piece(xv[pc], i + 1));
-        O[k] = __ffma2_rn(X, cc.Dx2, make_float2(ur[(2 * k) * 32 + row].x, ur[(2 * k + 1) * 32 + row].x));
+        O[k] = __ffma2_rn(X, cc.Dx2, make_float2(reinterpret_cast<const float *>(ur + (2 * k) * 32)[row],
+                                                 reinterpret_cast<const float *>(ur + (2 * k + 1) * 32)[row]));
     }
     if (has_z) {
         float2 Z[NP], E[NP];

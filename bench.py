@@ -82,6 +82,16 @@ def step_bytes(cfg):
     return workloads.compulsory_bytes_step(c.batch, c.dim, c.dstate, 2 if c.dtype == "bf16" else 4)
 
 
+def fwd_config(world):
+    """The workload both arms report: the forward scan of the Mamba-2.8B layer shape."""
+    c = workloads.CONFIGS[FWD_CFG]
+    return {"workload": f"{c.name} forward scan (Mamba-2.8B mixer layer shape)",
+            "batch": c.batch, "seqlen": c.seqlen, "dim": c.dim, "dstate": c.dstate,
+            "state_dtype": "f32", "returns_h_last": True,
+            "l2": f"inputs {fwd_bytes(FWD_CFG) / 1e6:.0f} MB > L2 126 MB; no flush needed",
+            "parallelism": f"{world} independent replica(s)"}
+
+
 def _source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "selective_state_space_38_b200", "csrc")
@@ -246,8 +256,7 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{c.name} forward scan (float64 CPU oracle, channel sample)",
-                   "batch": c.batch, "seqlen": c.seqlen, "dim": c.dim, "dstate": c.dstate},
+        "config": fwd_config(1),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
                          "sample": sample, "cpu": _cpu_model()},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -406,6 +415,8 @@ def run_gpu(args):
     hbm_peak, peak_kind = _peaks()
     c = workloads.CONFIGS[FWD_CFG]
 
+    if args.only and world > 1:
+        raise SystemExit("--only is a single-GPU profiling mode")
     if args.only == "step":
         dec = bench_decode(args, device)
         print(json.dumps({"only": "step", "ms_per_step": round(dec["ms"], 5), "value": round(dec["gbs"], 2),
@@ -434,11 +445,7 @@ def run_gpu(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": f"{c.name} forward scan (Mamba-2.8B mixer layer shape)",
-                       "batch": c.batch, "seqlen": c.seqlen, "dim": c.dim, "dstate": c.dstate,
-                       "state_dtype": "f32", "returns_h_last": True,
-                       "l2": f"inputs {nb / 1e6:.0f} MB > L2 126 MB; no flush needed",
-                       "parallelism": f"{world} independent replica(s)"},
+            "config": fwd_config(world),
             "pct_of_hbm_peak": round(100.0 * value / world / hbm_peak, 2),
             "gtok_ch_per_s": round(world * tok_ch / (ms_step * 1e-3) / 1e9, 2),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": hbm_peak,

@@ -599,31 +599,38 @@ __device__ __forceinline__ bool group_is_s4d(const FwdParams &p, int64_t d0, int
     return __all_sync(0xffffffffu, ok);
 }
 
-// The helper's walk through the queue: the next chunk of its stream.
+// The helper's walk through the queue: the next chunk of its stream.  The
+// shape's counts are fixed at construction; item indices are below 2^31 (the
+// host checks), so an item is split with 32-bit arithmetic.
 template <typename T, bool S4D>
 struct ChunkCursor {
+    uint32_t tiles, groups, items;
     int64_t g = 0, seg = 0, b = 0, d0 = 0, t_begin = 0, t_next = 0, t_end = 0;
     bool open = false;
+
+    __device__ __forceinline__ explicit ChunkCursor(const FwdParams &p) {
+        tiles = static_cast<uint32_t>((p.dim + 31) / 32);
+        groups = tiles * static_cast<uint32_t>(p.batch);
+        items = groups * static_cast<uint32_t>((p.seqlen + p.seg_steps - 1) / p.seg_steps);
+    }
 
     __device__ __forceinline__ ChunkDesc next(const FwdParams &p, const FwdScratch &sc, uint32_t *counter,
                                               int lane) {
         constexpr int TC = FwdSmem<T>::kTC;
-        const int64_t tiles = (p.dim + 31) / 32;
-        const int64_t groups = tiles * p.batch;
-        const int64_t items = groups * ((p.seqlen + p.seg_steps - 1) / p.seg_steps);
         ChunkDesc dsc;
         while (!open || t_next >= t_end) {
             uint32_t item = 0;
             if (lane == 0) item = atomicAdd(counter, 1u);
             item = __shfl_sync(0xffffffffu, item, 0);
-            if (static_cast<int64_t>(item) >= items) {
+            if (item >= items) {
                 dsc.flags = kStop;
                 return dsc;
             }
+            const uint32_t gi = item % groups;
             seg = item / groups;
-            g = item % groups;
-            b = g / tiles;
-            d0 = (g % tiles) * 32;
+            g = gi;
+            b = gi / tiles;
+            d0 = static_cast<int64_t>(gi % tiles) * 32;
             t_begin = seg * p.seg_steps;
             t_end = t_begin + p.seg_steps < p.seqlen ? t_begin + p.seg_steps : p.seqlen;
             t_next = t_begin;
@@ -699,7 +706,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
     if (role == 1) {
         // ------------------------------------------------------------------ prep
-        ChunkCursor<T, S4D> cur;
+        ChunkCursor<T, S4D> cur(p);
         const uint32_t stage_tx = (p.z ? 3u : 2u) * SM::kTileBytes + 2u * kNState * kRowBytes;
         // stage chunk j: TMA (one lane, completion on full[j % kStages]) or element loads
         auto issue = [&](const ChunkDesc &dsc, int64_t j) {

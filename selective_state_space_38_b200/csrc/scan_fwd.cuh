@@ -728,6 +728,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             }
         };
         const bool softplus = p.softplus != 0;
+        ChanConst cc;
+        int64_t cc_d0 = -1;
         ChunkDesc dnext = cur.next(p, sc, counter, lane);
         issue(dnext, 0);
         for (int64_t j = 0;; ++j) {
@@ -741,8 +743,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 __syncwarp();
                 uint8_t *st = stage_of(j);
                 widen_bc<T>(st + 3 * SM::kTileBytes, bcf_of(j), lane);
-                const int64_t d = dj.d0 + lane;
-                const ChanConst cc = chan_const(p, d < p.dim ? d : p.dim - 1);
+                if (dj.d0 != cc_d0) {  // the channel constants change only with the group
+                    const int64_t d = dj.d0 + lane;
+                    cc = chan_const(p, d < p.dim ? d : p.dim - 1);
+                    cc_d0 = dj.d0;
+                }
                 chunk_prepass<T, S4D>(st, ur_of(j), lane, cc, softplus);
             }
             if (lane == 0) ring[j & 3] = dj;
@@ -753,6 +758,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     } else if (role == 2) {
         // ------------------------------------------------------------------ post
         const bool has_z = p.z != nullptr;
+        ChanConst cc;
+        int64_t cc_d0 = -1;
         for (int64_t j = 0;; ++j) {
             mbar_wait(done + (j & 1), parity(j, 2), sc.error);
             const ChunkDesc dj = ring[j & 3];
@@ -763,8 +770,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 mbar_arrive(posted + (j & 1));
                 continue;
             }
-            const int64_t d = dj.d0 + lane;
-            const ChanConst cc = chan_const(p, d < p.dim ? d : p.dim - 1);
+            if (dj.d0 != cc_d0) {
+                const int64_t d = dj.d0 + lane;
+                cc = chan_const(p, d < p.dim ? d : p.dim - 1);
+                cc_d0 = dj.d0;
+            }
             chunk_postpass<T>(st, ur_of(j), lane, cc, has_z);
             if constexpr (VEC) {
                 fence_proxy_async_smem();

@@ -26,7 +26,21 @@ struct StepParams {
 
 constexpr int kStepThreads = 256;
 
+// four consecutive B or C values of one sequence (an 8- or 16-byte vector load;
+// the API requires 16-byte aligned B and C, and the offset is a multiple of 4)
 template <typename T>
+__device__ __forceinline__ float4 load4(const void *p, int64_t i) {
+    if constexpr (Act<T>::kBytes == 4) {
+        return *reinterpret_cast<const float4 *>(static_cast<const float *>(p) + i);
+    } else {
+        const uint2 w = *reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(p) + i);
+        return make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u), __uint_as_float(w.y << 16),
+                           __uint_as_float(w.y & 0xffff0000u));
+    }
+}
+
+// SMALL: every channel index fits in 32 bits, so (b, d) come from a 32-bit division.
+template <typename T, bool SMALL>
 __global__ void __launch_bounds__(kStepThreads) scan_step_kernel(const StepParams p) {
     using AT = Act<T>;
     constexpr bool kAccurate = AT::kBytes == 4;
@@ -36,26 +50,32 @@ __global__ void __launch_bounds__(kStepThreads) scan_step_kernel(const StepParam
     const int q = static_cast<int>(gid & 3);
     const bool active = chan < nchan;
     const int64_t c = active ? chan : nchan - 1;  // inactive lanes still join the shuffles
-    const int64_t b = c / p.dim, d = c % p.dim;
+    int64_t b, d;
+    if constexpr (SMALL) {
+        const uint32_t c32 = static_cast<uint32_t>(c), dim32 = static_cast<uint32_t>(p.dim);
+        b = c32 / dim32;
+        d = c32 - static_cast<uint32_t>(b) * dim32;
+    } else {
+        b = c / p.dim;
+        d = c % p.dim;
+    }
 
     float4 h = *reinterpret_cast<const float4 *>(p.state + c * kNState + q * 4);
     const float4 a = *reinterpret_cast<const float4 *>(p.A + d * kNState + q * 4);
     const float xf = AT::load(p.x, c);
     float v = AT::load(p.delta, c);
     if (p.delta_bias) v += p.delta_bias[d];
+    const int64_t bn = b * kNState + q * 4;
+    const float4 Bv = load4<T>(p.B, bn), Cv = load4<T>(p.C, bn);
     const float dt = p.softplus ? (kAccurate ? softplus_accurate(v) : softplus_fast(v)) : v;
     const float u = dt * xf;
-    const int64_t bn = b * kNState + q * 4;
-    const float B0 = AT::load(p.B, bn), B1 = AT::load(p.B, bn + 1), B2 = AT::load(p.B, bn + 2),
-                B3 = AT::load(p.B, bn + 3);
-    const float C0 = AT::load(p.C, bn), C1 = AT::load(p.C, bn + 1), C2 = AT::load(p.C, bn + 2),
-                C3 = AT::load(p.C, bn + 3);
+    const float e = kLog2e * dt;
 
-    h.x = ex2_approx(a.x * kLog2e * dt) * h.x + u * B0;
-    h.y = ex2_approx(a.y * kLog2e * dt) * h.y + u * B1;
-    h.z = ex2_approx(a.z * kLog2e * dt) * h.z + u * B2;
-    h.w = ex2_approx(a.w * kLog2e * dt) * h.w + u * B3;
-    float y = (C0 * h.x + C1 * h.y) + (C2 * h.z + C3 * h.w);
+    h.x = ex2_approx(a.x * e) * h.x + u * Bv.x;
+    h.y = ex2_approx(a.y * e) * h.y + u * Bv.y;
+    h.z = ex2_approx(a.z * e) * h.z + u * Bv.z;
+    h.w = ex2_approx(a.w * e) * h.w + u * Bv.w;
+    float y = (Cv.x * h.x + Cv.y * h.y) + (Cv.z * h.z + Cv.w * h.w);
     y += __shfl_xor_sync(0xffffffffu, y, 1);
     y += __shfl_xor_sync(0xffffffffu, y, 2);
 

@@ -206,7 +206,10 @@ int launch_step(const StepParams &p, cudaStream_t stream) {
     const int64_t threads = p.batch * p.dim * 4;
     const int64_t blocks = (threads + kStepThreads - 1) / kStepThreads;
     if (blocks > INT_MAX) return SSM_ERR_UNSUPPORTED;
-    scan_step_kernel<T><<<static_cast<unsigned>(blocks), kStepThreads, 0, stream>>>(p);
+    if (p.batch * p.dim < (int64_t(1) << 31))
+        scan_step_kernel<T, true><<<static_cast<unsigned>(blocks), kStepThreads, 0, stream>>>(p);
+    else
+        scan_step_kernel<T, false><<<static_cast<unsigned>(blocks), kStepThreads, 0, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 

@@ -96,18 +96,6 @@ __device__ __forceinline__ float silu_accurate(float z) {
     return z / (1.0f + expf(-z));
 }
 
-// ---- cp.async (16-byte, L1 bypass, zero-fill beyond src_bytes) ----------------
-__device__ __forceinline__ void cp_async16(uint32_t dst_smem, const void *src, int src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst_smem), "l"(src),
-                 "r"(src_bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -182,20 +182,20 @@ def test_output_guard_bands():
 
 
 # ---- the configs ---------------------------------------------------------------
-def test_config0_full(orc):
+def test_tiny_fp32_full(orc):
     inp = workloads.make_inputs(0)
     out, hl = _gpu_fwd(inp)
     ref_out, ref_hl = _oracle(orc, inp)
-    check(to_np64(out), ref_out, "f32", "config0 out")
-    check(to_np64(hl), ref_hl, "f32", "config0 h_last")
+    check(to_np64(out), ref_out, "f32", "tiny fp32 out")
+    check(to_np64(hl), ref_hl, "f32", "tiny fp32 h_last")
 
 
-def test_config1_full(orc):
+def test_mamba130m_layer_full(orc):
     inp = workloads.make_inputs(1)
     out, hl = _gpu_fwd(inp)
     ref_out, ref_hl = _oracle(orc, inp)
-    check(to_np64(out), ref_out, "bf16", "config1 out")
-    check(to_np64(hl), ref_hl, "bf16", "config1 h_last")
+    check(to_np64(out), ref_out, "bf16", "mamba-130m layer out")
+    check(to_np64(hl), ref_hl, "bf16", "mamba-130m layer h_last")
 
 
 def _sampled(orc, cfg, nsel, seed):
@@ -209,16 +209,16 @@ def _sampled(orc, cfg, nsel, seed):
     ref_out, ref_hl = _oracle(orc, inp, chan)
     got = to_np64(out).reshape(c.channels, -1)[chan]
     gothl = to_np64(hl).reshape(c.channels, -1)[chan]
-    check(got, ref_out, "bf16", f"config{cfg} out (sampled)")
-    check(gothl, ref_hl, "bf16", f"config{cfg} h_last (sampled)")
+    check(got, ref_out, "bf16", f"{c.name} out (sampled)")
+    check(gothl, ref_hl, "bf16", f"{c.name} h_last (sampled)")
     return inp, out, hl
 
 
-def test_config2_sampled(orc):
+def test_mamba2p8b_layer_sampled(orc):
     _sampled(orc, 2, 192, 2)
 
 
-def test_config3_sampled_and_split(orc):
+def test_long_sequence_sampled_and_split(orc):
     inp, out, hl = _sampled(orc, 3, 48, 3)
     # state carry across two calls at a non-aligned split point
     m = 65536 + 777
@@ -230,6 +230,6 @@ def test_config3_sampled_and_split(orc):
          for k, v in inp.items()}
     b["h0"] = None
     o2, h2 = _gpu_fwd(b, h0=h1.cpu().numpy())
-    check(to_np64(o1), to_np64(out[..., :m]), "bf16", "config3 split first")
-    check(to_np64(o2), to_np64(out[..., m:]), "bf16", "config3 split second")
-    check(to_np64(h2), to_np64(hl), "bf16", "config3 split h_last")
+    check(to_np64(o1), to_np64(out[..., :m]), "bf16", "long sequence split, first part")
+    check(to_np64(o2), to_np64(out[..., m:]), "bf16", "long sequence split, second part")
+    check(to_np64(h2), to_np64(hl), "bf16", "long sequence split h_last")

@@ -54,7 +54,7 @@ def test_steps_equal_fwd_scan():
 
 
 def decode_prefill_state(orc, cfg=4):
-    """The decode config's initial state: 64 oracle steps from zero on the
+    """The decode workload's initial state: 64 oracle steps from zero on the
     prefill tokens, rounded to float32."""
     c = workloads.CONFIGS[cfg]
     prm = workloads.decode_params(cfg)
@@ -66,7 +66,7 @@ def decode_prefill_state(orc, cfg=4):
     return state64.astype(np.float32)
 
 
-def test_config4_decode(orc):
+def test_decode_batch_256x5120(orc):
     """256 sequences x 5120 channels x 16 fp32 states, 1024 consecutive steps.
     Every step: out and state of a 16-sequence subset against the oracle.
     Steps 1 and 2: out of all 256 sequences.  After 1024 steps: the final

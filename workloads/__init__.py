@@ -18,7 +18,7 @@ default, draws in float32 in this order):
   h0 ~ N(0, 1) [batch][dim][dstate] when the config has an initial state.
   A[d, n] = -(n + 1) (S4D-real), D = 1, float32.
 Activations are rounded to bfloat16 (round to nearest even) from float32 for
-the bf16 configs and kept as float32 for config 0.  bfloat16 arrays are carried
+the bf16 workloads and kept as float32 for the tiny fp32 one.  bfloat16 arrays are carried
 as uint16 bit patterns.
 
 The decode config draws each step's tokens from its own stream

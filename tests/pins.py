@@ -182,6 +182,29 @@ def pin_chunk_split(orc):
         _close(h2, hl, rtol=2e-5, atol=2e-5, what=f"split m={m} h_last")
 
 
+def pin_segment_summaries(orc):
+    """(d') The identity behind the time-parallel schedule: scanning segment s
+    from a zero state gives e_s, the decays of the segment multiply to
+    P_s[n] = exp(A[d, n] sum_t dt_t), and the state at the end of segment s is
+    P_s h_s + e_s, where h_s is the state entering it (h_0 = h0).  P_s is
+    computed here from its closed form (softplus by numpy's logaddexp), not by
+    the oracle, so a wrong decay or a wrong state carry fails."""
+    c = _rand_case(13, b=2, d=3, n=4, L=40)
+    seq_keys = ("x", "delta", "z", "B", "C")
+    dt = np.logaddexp(0.0, c["delta"].astype(np.float64) + c["delta_bias"].astype(np.float64)[None, :, None])
+    A = c["A"].astype(np.float64)
+    h = c["h0"].astype(np.float64)
+    for lo in range(0, 40, 8):
+        hi = lo + 8
+        seg = {k: (np.ascontiguousarray(v[..., lo:hi]) if k in seq_keys else v) for k, v in c.items()}
+        _, e = _call(orc, seg, h0=None)
+        P = np.exp(A[None, :, :] * dt[..., lo:hi].sum(-1)[..., None])
+        h = P * h + e
+        prefix = {k: (np.ascontiguousarray(v[..., :hi]) if k in seq_keys else v) for k, v in c.items()}
+        _, want = _call(orc, prefix)
+        _close(h, want, rtol=1e-11, atol=1e-13, what=f"segment summaries up to t={hi}")
+
+
 @lru_cache(maxsize=None)
 def _bracketings(lo, hi):
     """All full bracketings of the elements lo..hi-1 as nested tuples."""
@@ -326,6 +349,7 @@ ALL_PINS = [
     pin_geometric_sum,
     pin_convolution_mode,
     pin_chunk_split,
+    pin_segment_summaries,
     pin_associative_brute_force,
     pin_degenerate,
     pin_softplus_extremes,

@@ -102,9 +102,10 @@ def _source_hash():
     return h.hexdigest()[:16]
 
 
-def _profiled_traffic(kernel_key):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel
-    sources have not changed since it was taken (else None)."""
+def _profiled(kernel_key):
+    """The committed ncu summary of a kernel (profiles/traffic.json): DRAM bytes
+    per launch and pipe utilisation, if the kernel sources have not changed
+    since it was taken (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -113,7 +114,18 @@ def _profiled_traffic(kernel_key):
         return None
     if rec.get("source_hash") != _source_hash():
         return None
-    return rec.get("dram_bytes_per_launch")
+    return rec
+
+
+def _pipes(kernel_key):
+    rec = _profiled(kernel_key)
+    if rec is None:
+        return None
+    keys = ("fma_pipe_pct", "xu_pipe_pct", "dram_throughput_pct", "issue_active_pct", "smem_pipe_pct",
+            "smem_bank_conflicts_ld", "smem_bank_conflicts_st")
+    out = {k: rec[k] for k in keys if k in rec}
+    out["source"] = "ncu, profiles/traffic.json"
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -287,32 +299,42 @@ def _to_pinned(a):
     return t.pin_memory()
 
 
-def bench_fwd(args, device, world):
+def bench_fwd(args, device, world, cfg=FWD_CFG, steps=None, warmup=None):
+    """Event-timed forward scans of `cfg` over inputs resident in HBM (all
+    configs' inputs exceed the 126 MB L2, so no flush is needed).  One launch =
+    the forward call (its S4D and general kernel instances, and for few-group
+    shapes the summary pass, the combine and the second pass)."""
     import torch
     import selective_state_space_38_b200 as ssm
-    c = workloads.CONFIGS[FWD_CFG]
-    inp = workloads.make_inputs(FWD_CFG)
+    steps = args.steps if steps is None else steps
+    warmup = args.warmup if warmup is None else warmup
+    c = workloads.CONFIGS[cfg]
+    inp = workloads.make_inputs(cfg)
     t = {k: _to_dev(v, device) for k, v in inp.items() if isinstance(v, np.ndarray)}
     out = torch.empty_like(t["x"])
     hl = torch.empty((c.batch, c.dim, c.dstate), dtype=torch.float32, device=device)
+    ws = torch.empty(ssm.ssm_scan_fwd_workspace_size(c.batch, c.seqlen, c.dim, device), dtype=torch.uint8,
+                     device=device)
     stream = torch.cuda.current_stream(device)
 
     def launch():
         ssm.ssm_scan_fwd(t["x"], t["delta"], t["delta_bias"], True, t["A"], t["B"], t["C"], t["D"],
-                         t["z"], None, out=out, h_last=hl)
+                         t["z"], t.get("h0"), out=out, h_last=hl, workspace=ws)
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         launch()
     torch.cuda.synchronize(device)
+    if ssm.ssm_scan_fwd_status(ws, stream) != 0:
+        raise RuntimeError("a bounded device wait gave up during the warm-up")
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
+          for _ in range(steps)]
     _barrier(world)
     torch.cuda.synchronize(device)
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     with ClockSampler(device.index) as clk:
         start.record(stream)
-        for i in range(args.steps):
+        for i in range(steps):
             ev[i][0].record(stream)
             launch()
             ev[i][1].record(stream)
@@ -322,8 +344,11 @@ def bench_fwd(args, device, world):
     total_ms = start.elapsed_time(end)
     per_launch = [a.elapsed_time(b) for a, b in ev]
     total_ms = _max_over_ranks(total_ms, world, device)
+    segs_schedule = ssm.ssm_scan_fwd_workspace_size(c.batch, c.seqlen, c.dim, device) > \
+        ssm.ssm_scan_fwd_workspace_size(c.batch, 1, c.dim, device)
     return dict(total_ms=total_ms, launch_ms=statistics.mean(per_launch),
-                launch_ms_median=statistics.median(per_launch), clocks=clk.summary(), inputs=inp)
+                launch_ms_median=statistics.median(per_launch), clocks=clk.summary(), inputs=inp,
+                kernels_per_call=5 if segs_schedule else 2)
 
 
 def bench_e2e(args, device, world, inp):
@@ -342,11 +367,14 @@ def bench_e2e(args, device, world, inp):
     d2h = out_h.numel() * out_h.element_size() + hl_h.numel() * hl_h.element_size()
     stream = torch.cuda.current_stream(device)
 
+    ws = torch.empty(ssm.ssm_scan_fwd_workspace_size(c.batch, c.seqlen, c.dim, device), dtype=torch.uint8,
+                     device=device)
+
     def one():
         for k, v in host.items():
             dev[k].copy_(v, non_blocking=True)
         ssm.ssm_scan_fwd(dev["x"], dev["delta"], dev["delta_bias"], True, dev["A"], dev["B"],
-                         dev["C"], dev["D"], dev["z"], None, out=out_d, h_last=hl_d)
+                         dev["C"], dev["D"], dev["z"], None, out=out_d, h_last=hl_d, workspace=ws)
         out_h.copy_(out_d, non_blocking=True)
         hl_h.copy_(hl_d, non_blocking=True)
 
@@ -366,37 +394,71 @@ def bench_e2e(args, device, world, inp):
     return dict(ms=ms, h2d=h2d, d2h=d2h, steps=steps)
 
 
-def bench_decode(args, device):
-    """The recurrent step on the decode config: per-step kernel time with the
-    L2 flushed between steps (so the 84 MB state comes from HBM)."""
+def _device_tokens(c, n, gen, device):
+    """n decode token sets drawn on the device with the decode config's
+    distributions (x, z, B, C ~ N(0,1), delta ~ N(0, 0.1^2)), rounded to bf16."""
+    import torch
+
+    def draw(shape, scale=1.0):
+        return (torch.randn(shape, generator=gen, device=device) * scale).to(torch.bfloat16)
+    return dict(x=draw((n, c.batch, c.dim)), delta=draw((n, c.batch, c.dim), 0.1),
+                z=draw((n, c.batch, c.dim)), B=draw((n, c.batch, c.dstate)), C=draw((n, c.batch, c.dstate)))
+
+
+def bench_decode(args, device, flushed_steps=64):
+    """The recurrent step on the decode config (256 sequences x 5120 channels x
+    16 fp32 states): 1024 consecutive steps, back to back, from the state a
+    64-step prefill leaves; the per-step mean is the headline.  Beside it, the
+    median of single steps with the L2 flushed before each one (so the 84 MB
+    state comes from HBM)."""
     import torch
     import selective_state_space_38_b200 as ssm
     c = workloads.CONFIGS[DECODE_CFG]
     prm = workloads.decode_params(DECODE_CFG)
     p = {k: _to_dev(prm[k], device) for k in ("A", "D", "delta_bias")}
-    g = torch.Generator(device="cpu").manual_seed(4)
-    state = (torch.randn((c.batch, c.dim, c.dstate), generator=g) * 0.5).to(device)
-    pool = [{k: _to_dev(v, device) for k, v in workloads.decode_tokens(DECODE_CFG, s).items()}
-            for s in range(4)]
+    gen = torch.Generator(device=device)
+    gen.manual_seed(4)
+    pre = _device_tokens(c, c.prefill_steps, gen, device)
+    tok = _device_tokens(c, c.decode_steps, gen, device)
+    state = torch.zeros((c.batch, c.dim, c.dstate), dtype=torch.float32, device=device)
     outb = torch.empty((c.batch, c.dim), dtype=torch.bfloat16, device=device)
-    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
-    steps = 64
-    times = []
-    for s in range(steps + 4):
-        tok = pool[s % len(pool)]
-        flush.fill_(float(s))
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        ssm.ssm_scan_step(state, tok["x"], tok["delta"], p["delta_bias"], True, p["A"], tok["B"],
-                          tok["C"], p["D"], tok["z"], out=outb)
-        b.record(stream)
-        times.append((a, b))
+
+    def step(src, i):
+        ssm.ssm_scan_step(state, src["x"][i], src["delta"][i], p["delta_bias"], True, p["A"], src["B"][i],
+                          src["C"][i], p["D"], src["z"][i], out=outb)
+
+    for i in range(c.prefill_steps):
+        step(pre, i)
+    prefill_state = state.clone()
+    for i in range(8):  # warm-up
+        step(tok, i)
+    state.copy_(prefill_state)
     torch.cuda.synchronize(device)
-    ms = statistics.median([a.elapsed_time(b) for a, b in times[4:]])
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(c.decode_steps):
+        step(tok, i)
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    ms_b2b = a.elapsed_time(b) / c.decode_steps
+
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+    times = []
+    for s in range(flushed_steps + 4):
+        flush.fill_(float(s))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step(tok, s)
+        e1.record(stream)
+        times.append((e0, e1))
+    torch.cuda.synchronize(device)
+    ms_flushed = statistics.median([x.elapsed_time(y) for x, y in times[4:]])
     nb = step_bytes(DECODE_CFG)
-    return dict(ms=ms, gbs=nb / (ms * 1e-3) / 1e9, bytes=nb, steps=steps,
-                gtok_ch=c.batch * c.dim / (ms * 1e-3) / 1e9)
+    return dict(ms=ms_b2b, gbs=nb / (ms_b2b * 1e-3) / 1e9, bytes=nb, steps=c.decode_steps,
+                gtok_ch=c.batch * c.dim / (ms_b2b * 1e-3) / 1e9,
+                ms_flushed=ms_flushed, gbs_flushed=nb / (ms_flushed * 1e-3) / 1e9,
+                launches=c.prefill_steps + 8 + c.decode_steps + flushed_steps + 4)
 
 
 def run_gpu(args):
@@ -420,21 +482,43 @@ def run_gpu(args):
     if args.only == "step":
         dec = bench_decode(args, device)
         print(json.dumps({"only": "step", "ms_per_step": round(dec["ms"], 5), "value": round(dec["gbs"], 2),
-                          "unit": "GB/s"}), flush=True)
+                          "unit": "GB/s", "ms_per_step_flushed": round(dec["ms_flushed"], 5)}), flush=True)
         return 0
-    f = bench_fwd(args, device, world)
-    nb = fwd_bytes(FWD_CFG)
     if args.only == "fwd":
-        print(json.dumps({"only": "fwd", "launch_ms_mean": round(f["launch_ms"], 5),
+        f = bench_fwd(args, device, world, cfg=args.config)
+        nb = fwd_bytes(args.config)
+        print(json.dumps({"only": "fwd", "config": args.config, "launch_ms_mean": round(f["launch_ms"], 5),
                           "value": round(nb / (f["launch_ms"] * 1e-3) / 1e9, 2), "unit": "GB/s"}),
               flush=True)
         return 0
+    f = bench_fwd(args, device, world)
+    nb = fwd_bytes(FWD_CFG)
     ms_step = f["total_ms"] / args.steps
     value = world * nb / (ms_step * 1e-3) / 1e9
     achieved = nb / (f["launch_ms"] * 1e-3) / 1e9
     e = bench_e2e(args, device, world, f["inputs"])
+    del f["inputs"]
     e2e_gbs = world * nb / (e["ms"] * 1e-3) / 1e9
     dec = bench_decode(args, device) if rank == 0 else None
+    launches = f["kernels_per_call"] * args.steps
+
+    subs = {}
+    if rank == 0:
+        # the other forward configs, one sub-line each (same timing, fewer steps)
+        for cfg, steps in ((1, 50), (3, 10)):
+            cs = workloads.CONFIGS[cfg]
+            g = bench_fwd(args, device, 1, cfg=cfg, steps=steps, warmup=3)
+            del g["inputs"]
+            nbs = fwd_bytes(cfg)
+            gbs = nbs / (g["launch_ms"] * 1e-3) / 1e9
+            subs[cs.name] = {"launch_ms_mean": round(g["launch_ms"], 5), "value": round(gbs, 2), "unit": "GB/s",
+                             "frac": round(gbs / hbm_peak, 4),
+                             "gtok_ch_per_s": round(cs.batch * cs.seqlen * cs.dim / (g["launch_ms"] * 1e-3) / 1e9, 2),
+                             "algorithmic_bytes_per_launch": nbs, "steps": steps,
+                             "kernels_per_call": g["kernels_per_call"], "clocks": g["clocks"],
+                             "pipes": _pipes(f"scan_fwd_cfg{cfg}")}
+            launches += g["kernels_per_call"] * (steps + 3)
+        launches += dec["launches"]
 
     if rank == 0:
         cpu_val, cpu_s, cpu_ch, cores = cpu_oracle_rate(FWD_CFG, target_s=float(
@@ -451,10 +535,11 @@ def run_gpu(args):
             "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": hbm_peak,
                          "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
                          "peak_kind": peak_kind,
-                         "traffic": _profiled_traffic("scan_fwd_cfg2"),
+                         "traffic": (_profiled("scan_fwd_cfg2") or {}).get("dram_bytes_per_launch"),
                          "algorithmic_bytes_per_launch": nb,
                          "launch_ms_mean": round(f["launch_ms"], 5),
                          "launch_ms_median": round(f["launch_ms_median"], 5)},
+            "pipes": _pipes("scan_fwd_cfg2"),
             "e2e": {"value": round(e2e_gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": e["h2d"],
                     "d2h_bytes_per_step": e["d2h"], "ms_per_step": round(e["ms"], 3),
                     "steps": e["steps"]},
@@ -462,13 +547,23 @@ def run_gpu(args):
                              "kind": "oracle", "cpu": _cpu_model(),
                              "sample": f"{cpu_ch} channels (full L) of the same workload, "
                                        f"{cpu_s:.1f} s of float64 oracle time"},
+            "other_configs": subs,
             "decode": {"workload": workloads.CONFIGS[DECODE_CFG].name,
                        "ms_per_step": round(dec["ms"], 5), "value": round(dec["gbs"], 2),
                        "unit": "GB/s", "pct_of_hbm_peak": round(100 * dec["gbs"] / hbm_peak, 2),
-                       "gtok_ch_per_s": round(dec["gtok_ch"], 3),
-                       "bytes_per_step": dec["bytes"], "l2": "flushed between steps"},
-            # per forward call: the S4D-structured and the general kernel instance
-            "gpu_launches": 2 * args.steps,
+                       "gtok_ch_per_s": round(dec["gtok_ch"], 3), "steps": dec["steps"],
+                       "bytes_per_step": dec["bytes"],
+                       "l2": "back to back from the 64-step prefill state (the 84 MB state partly stays in L2)",
+                       "flushed": {"ms_per_step": round(dec["ms_flushed"], 5),
+                                   "value": round(dec["gbs_flushed"], 2),
+                                   "pct_of_hbm_peak": round(100 * dec["gbs_flushed"] / hbm_peak, 2),
+                                   "l2": "flushed before each step"},
+                       "pipes": _pipes("scan_step_cfg4")},
+            # kernels of this library launched inside the timed region: per forward call its
+            # S4D and general instances (five kernels on the two-pass schedule)
+            "gpu_launches": f["kernels_per_call"] * args.steps,
+            # and over the whole run (warm-up, end-to-end leg, other configs, decode)
+            "gpu_launches_run": launches,
             "clocks": f["clocks"],
         }
         print(json.dumps(line), flush=True)
@@ -486,6 +581,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     # profiler runs: only the forward-scan or only the decode-step timing loop
     ap.add_argument("--only", default=None, choices=["fwd", "step"])
+    ap.add_argument("--config", type=int, default=FWD_CFG, choices=[0, 1, 2, 3],
+                    help="forward config of --only fwd")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

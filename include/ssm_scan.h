@@ -27,17 +27,20 @@
  * arithmetic is float32; the state is float32.
  *
  * Ownership and execution: every pointer is a device pointer owned by the
- * caller.  ssm_scan_fwd takes a scratch area for its work queue (16 KB + 2 KB
- * per group of 32 channels) from a library-owned, stream-ordered memory pool per
- * device and returns it on the same stream; the pool keeps the memory between
- * calls.  When the channel groups (batch * ceil(dim / 32)) number fewer than
- * half the GPU's SM sub-partitions, the call cuts each sequence into segments
- * and scans them in parallel in two passes; the scratch then also holds 6 KB per
- * (group, segment), with about 4 * (SM sub-partitions) segments in all (under
- * 15 MB on a 148-SM GPU).  ssm_scan_step allocates nothing.  Work is enqueued on
- * `stream` and runs asynchronously; the call returns after validating the
- * arguments and launching.  Errors that the device meets later surface
- * through the CUDA stream.  Calls are thread-safe.
+ * caller, and the library allocates no device memory.  ssm_scan_fwd needs a
+ * workspace for its work queue, segment flags and carried states; the caller
+ * sizes it with ssm_scan_fwd_workspace_size and passes it in.  Its size is
+ * 16 KB + 2 KB per group of 32 channels (groups = batch * ceil(dim / 32)); when
+ * the groups number fewer than half the GPU's SM sub-partitions (4 per SM),
+ * the call cuts each sequence into segments and scans them in parallel in two
+ * passes, and the workspace also holds 6 KB per (group, segment), with about
+ * 16 * SMs segments in all (under 15 MB on a 148-SM GPU).  Calls that share a
+ * workspace must not overlap on the GPU (the same stream serialises them).
+ * ssm_scan_step needs no workspace.  Work is enqueued on `stream` and runs
+ * asynchronously; the call returns after validating the arguments and
+ * launching.  Errors that the device meets later surface through the CUDA
+ * stream, and a bounded device wait that gave up is reported by
+ * ssm_scan_fwd_status.  Calls are thread-safe.
  *
  * Error behaviour: every check is made on the host before anything is
  * launched; a call that returns non-zero has launched nothing and touched no
@@ -46,6 +49,7 @@
 #ifndef SSM_SCAN_H
 #define SSM_SCAN_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -70,12 +74,20 @@ typedef struct {
 
 enum {
     SSM_OK = 0,
-    SSM_ERR_INVALID_ARG = 1, /* NULL required pointer, a dimension < 1, or aliasing out with an input */
-    SSM_ERR_UNSUPPORTED = 2, /* dstate or dtype not supported, or sizes beyond 32-bit indexing limits */
+    SSM_ERR_INVALID_ARG = 1, /* NULL required pointer, a dimension < 1, overlapping buffers, or a too small workspace */
+    SSM_ERR_UNSUPPORTED = 2, /* dstate or dtype not supported, or batch, seqlen or dim beyond 2^31 - 65 */
     SSM_ERR_MISALIGNED = 3,  /* a pointer is not 16-byte aligned */
     SSM_ERR_CUDA = 4,        /* a CUDA launch or query failed */
-    SSM_ERR_TIMEOUT = 5      /* reserved: a bounded device wait gave up */
+    SSM_ERR_TIMEOUT = 5      /* a bounded device wait gave up (from ssm_scan_fwd_status) */
 };
+
+/*
+ * Workspace bytes that ssm_scan_fwd needs for the shape `dims` on a GPU with
+ * `sm_count` SMs (sm_count <= 0: the current device, which needs a CUDA
+ * context).  The size depends only on batch, seqlen, dim and the SM count.
+ * Returns SSM_OK and writes *bytes, or an SSM_ERR_* code.
+ */
+int ssm_scan_fwd_workspace_size(const ssm_dims_t *dims, int sm_count, size_t *bytes);
 
 /*
  * Forward scan over the whole sequence (the fused, chunked scan of Appendix D
@@ -91,14 +103,31 @@ enum {
  *   h0             optional [batch][dim][dstate] (NULL = zero initial state)
  *   out            required [batch][dim][seqlen]; must not overlap any input
  *   h_last         optional [batch][dim][dstate] (NULL = not written); may be h0
+ *   workspace      required device buffer of workspace_bytes, at least
+ *                  ssm_scan_fwd_workspace_size for this shape and device; its
+ *                  contents on entry do not matter; it must not overlap any
+ *                  input or output
  *   dims           sizes and activation dtype
  *   stream         CUDA stream
+ * Alignment: every pointer 16-byte aligned, except delta_bias and D (4 bytes).
  * Returns SSM_OK or an SSM_ERR_* code.
  */
 int ssm_scan_fwd(const void *x, const void *delta, const float *delta_bias, int softplus,
                  const float *A, const void *B, const void *C, const float *D,
                  const void *z, const float *h0, void *out, float *h_last,
+                 void *workspace, size_t workspace_bytes,
                  const ssm_dims_t *dims, ssm_stream_t stream);
+
+/*
+ * Whether the last forward call on `workspace` ran to completion: waits for
+ * `stream` to finish, then reads the call's error word from the workspace.
+ * Returns SSM_OK, SSM_ERR_TIMEOUT when one of the call's bounded device waits
+ * gave up (its out and h_last are then void; every wait is bounded, so the
+ * kernels always end), or SSM_ERR_CUDA when the stream reports a CUDA error.
+ * workspace == NULL asks about the last ssm_scan_fwd_noalloc call on the
+ * current device.  This call blocks the host; the forward calls never do.
+ */
+int ssm_scan_fwd_status(const void *workspace, ssm_stream_t stream);
 
 /*
  * One recurrent (decode) step for every sequence: the pages' recurrent mode,
@@ -115,6 +144,8 @@ int ssm_scan_fwd(const void *x, const void *delta, const float *delta_bias, int 
  *   z              optional [batch][dim]
  *   out            required [batch][dim]; must not overlap any input or state
  *   dims           batch, dim, dstate, act_dtype (seqlen is ignored)
+ * Alignment: state, A, B and C 16-byte aligned (they are read as vectors);
+ * x, delta, z and out aligned to their element size; D and delta_bias 4 bytes.
  * Returns SSM_OK or an SSM_ERR_* code.
  */
 int ssm_scan_step(float *state, const void *x, const void *delta, const float *delta_bias,
@@ -123,28 +154,42 @@ int ssm_scan_step(float *state, const void *x, const void *delta, const float *d
                   const ssm_dims_t *dims, ssm_stream_t stream);
 
 /*
- * ssm_scan_fwd without any device allocation.  The pages have no counterpart:
- * this entry point exists for callers that cannot allocate device memory
- * while they run the scan (code running inside an allocator or memory-pool
- * callback, runtimes that reserve all device memory up front and forbid
- * later allocations).  Arguments, layout, results and error codes are those
- * of ssm_scan_fwd.  Its work queue, segment flags and carried states use a
- * fixed 2 MiB device array inside the library (held by every GPU that loads
- * it), so shapes with batch * ceil(dim / 32) above about 1000 are rejected
- * with SSM_ERR_UNSUPPORTED.  It always scans the segments of a group in order
- * (no two-pass parallel schedule), whatever the number of groups, so shapes
- * with few channel groups run slower here than through ssm_scan_fwd.  The
- * first call on a device looks up that array's address; make that first call
- * before any stream capture.  Every call
- * shares the one array of its device: calls whose work overlaps on the GPU
- * (for example calls on two streams of the same device) race on it and must be
- * serialised by the caller.  It allocates nothing: no cudaMalloc/cudaFree and
- * no memory-pool allocation.
+ * ssm_scan_fwd without a workspace.  The pages have no counterpart: this
+ * entry point exists for callers that cannot allocate any device memory while
+ * they run the scan, not even a workspace (code running inside an allocator or
+ * memory-pool callback, runtimes that reserve all device memory up front and
+ * forbid later allocations).  Arguments, layout, results and error codes are
+ * those of ssm_scan_fwd without the two workspace arguments.  Its work queue,
+ * segment flags and carried states use a fixed 2 MiB device array inside the
+ * library (held by every GPU that loads it), so shapes with
+ * batch * ceil(dim / 32) above about 1000 are rejected with
+ * SSM_ERR_UNSUPPORTED.  It always scans the segments of a group in order (no
+ * two-pass parallel schedule), whatever the number of groups, so shapes with
+ * few channel groups run slower here than through ssm_scan_fwd.  The first
+ * call on a device looks up that array's address; make that first call before
+ * any stream capture.  Every call shares the one array of its device: calls
+ * whose work overlaps on the GPU (for example calls on two streams of the same
+ * device) race on it and must be serialised by the caller.
+ * ssm_scan_fwd_status(NULL, stream) reports on the last call.  It allocates
+ * nothing: no cudaMalloc/cudaFree and no memory-pool allocation.
  */
 int ssm_scan_fwd_noalloc(const void *x, const void *delta, const float *delta_bias, int softplus,
                          const float *A, const void *B, const void *C, const float *D,
                          const void *z, const float *h0, void *out, float *h_last,
                          const ssm_dims_t *dims, ssm_stream_t stream);
+
+/*
+ * Test support, not part of the operation: ssm_scan_fwd with the chained
+ * schedule, where each segment's wait for its predecessor's flag awaits a
+ * count that no flag ever reaches and gives up after `spin_limit` polls (0:
+ * at once).  The kernels still end normally; ssm_scan_fwd_status then reports
+ * SSM_ERR_TIMEOUT.  Arguments as for ssm_scan_fwd.
+ */
+int ssm_debug_fwd_flag_timeout(const void *x, const void *delta, const float *delta_bias, int softplus,
+                               const float *A, const void *B, const void *C, const float *D,
+                               const void *z, const float *h0, void *out, float *h_last,
+                               void *workspace, size_t workspace_bytes, uint32_t spin_limit,
+                               const ssm_dims_t *dims, ssm_stream_t stream);
 
 /* Static, human-readable text for an SSM_* code (never NULL). */
 const char *ssm_strerror(int code);

@@ -41,8 +41,17 @@ def _load():
     lib = ctypes.CDLL(LIB_PATH)
     P, I = ctypes.c_void_p, ctypes.c_int
     DP = ctypes.POINTER(Dims)
-    lib.ssm_scan_fwd.argtypes = [P, P, P, I, P, P, P, P, P, P, P, P, DP, P]
+    S = ctypes.c_size_t
+    lib.ssm_scan_fwd_workspace_size.argtypes = [DP, I, ctypes.POINTER(S)]
+    lib.ssm_scan_fwd_workspace_size.restype = I
+    lib.ssm_scan_fwd.argtypes = [P, P, P, I, P, P, P, P, P, P, P, P, P, S, DP, P]
     lib.ssm_scan_fwd.restype = I
+    lib.ssm_scan_fwd_status.argtypes = [P, P]
+    lib.ssm_scan_fwd_status.restype = I
+    lib.ssm_scan_fwd_noalloc.argtypes = [P, P, P, I, P, P, P, P, P, P, P, P, DP, P]
+    lib.ssm_scan_fwd_noalloc.restype = I
+    lib.ssm_debug_fwd_flag_timeout.argtypes = [P, P, P, I, P, P, P, P, P, P, P, P, P, S, ctypes.c_uint32, DP, P]
+    lib.ssm_debug_fwd_flag_timeout.restype = I
     lib.ssm_scan_step.argtypes = [P, P, P, P, I, P, P, P, P, P, P, DP, P]
     lib.ssm_scan_step.restype = I
     lib.ssm_strerror.argtypes = [I]
@@ -63,7 +72,8 @@ def get_lib():
     return _lib
 
 
-EXPORTS = ("ssm_scan_fwd", "ssm_scan_step", "ssm_strerror", "ssm_version")
+EXPORTS = ("ssm_scan_fwd_workspace_size", "ssm_scan_fwd", "ssm_scan_fwd_status", "ssm_scan_step",
+           "ssm_scan_fwd_noalloc", "ssm_debug_fwd_flag_timeout", "ssm_strerror", "ssm_version")
 
 
 def ssm_strerror(code: int) -> str:
@@ -72,6 +82,37 @@ def ssm_strerror(code: int) -> str:
 
 def ssm_version() -> int:
     return int(get_lib().ssm_version())
+
+
+_ws_sizes = {}
+
+
+def ssm_scan_fwd_workspace_size(batch: int, seqlen: int, dim: int, device=None, sm_count: int = 0) -> int:
+    """Workspace bytes ssm_scan_fwd needs for this shape (on `device`, or on a
+    GPU with `sm_count` SMs when that is given)."""
+    key = (batch, seqlen, dim, sm_count, None if sm_count > 0 else torch.device(device or "cuda").index)
+    n = _ws_sizes.get(key)
+    if n is None:
+        out = ctypes.c_size_t(0)
+        dims = Dims(batch, seqlen, dim, DSTATE, SSM_BF16)
+        if sm_count > 0:
+            rc = get_lib().ssm_scan_fwd_workspace_size(ctypes.byref(dims), int(sm_count), ctypes.byref(out))
+        else:
+            with torch.cuda.device(device):
+                rc = get_lib().ssm_scan_fwd_workspace_size(ctypes.byref(dims), 0, ctypes.byref(out))
+        _check(rc)
+        n = _ws_sizes[key] = int(out.value)
+    return n
+
+
+def ssm_scan_fwd_status(workspace=None, stream=None, device=None) -> int:
+    """Block until `stream` is done and return the status code of the last
+    forward call on `workspace` (a uint8 CUDA tensor; None: the last
+    ssm_scan_fwd_noalloc call): 0, or 5 when a bounded device wait gave up."""
+    dev = workspace.device if workspace is not None else torch.device(device or "cuda")
+    with torch.cuda.device(dev):
+        return int(get_lib().ssm_scan_fwd_status(
+            None if workspace is None else workspace.data_ptr(), _stream_ptr(stream, dev)))
 
 
 def _act_code(t: torch.Tensor) -> int:
@@ -110,13 +151,17 @@ def _check(rc):
 
 
 def ssm_scan_fwd(x, delta, delta_bias, softplus, A, B, C, D=None, z=None, h0=None,
-                 out=None, h_last=None, return_last_state=True, stream=None):
+                 out=None, h_last=None, return_last_state=True, stream=None, workspace=None,
+                 check=False):
     """Forward selective scan.
 
     x, delta, z: [batch, dim, L]; B, C: [batch, 16, L] (all bfloat16 or all
     float32, on one CUDA device); A: [dim, 16], D, delta_bias: [dim], h0:
     [batch, dim, 16] float32.  Returns (out, h_last); h_last is None when
-    ``return_last_state`` is False and no buffer is given.
+    ``return_last_state`` is False and no buffer is given.  ``workspace`` is
+    a uint8 CUDA tensor of at least ssm_scan_fwd_workspace_size bytes (taken
+    from torch's caching allocator when None).  ``check=True`` waits for the
+    call and raises SSMError when a bounded device wait gave up.
     """
     if x.device.type != "cuda":
         raise ValueError("ssm_scan_fwd needs CUDA tensors")
@@ -143,11 +188,18 @@ def ssm_scan_fwd(x, delta, delta_bias, softplus, A, B, C, D=None, z=None, h0=Non
     po = _ptr(out, dtype=act, device=dev, shape=x.shape, name="out")
     ph = _ptr(h_last, dtype=f32, device=dev, shape=(batch, dim, DSTATE), name="h_last")
     dims = Dims(batch, L, dim, DSTATE, code)
+    if workspace is None:
+        workspace = torch.empty(ssm_scan_fwd_workspace_size(batch, L, dim, dev), dtype=torch.uint8,
+                                device=dev)
+    pw = _ptr(workspace, dtype=torch.uint8, device=dev, name="workspace")
+    sp = _stream_ptr(stream, dev)
     with torch.cuda.device(dev):
         rc = get_lib().ssm_scan_fwd(ptrs["x"], ptrs["delta"], ptrs["delta_bias"], int(bool(softplus)),
-                              ptrs["A"], ptrs["B"], ptrs["C"], ptrs["D"], ptrs["z"], ptrs["h0"],
-                              po, ph, ctypes.byref(dims), _stream_ptr(stream, dev))
-    _check(rc)
+                                    ptrs["A"], ptrs["B"], ptrs["C"], ptrs["D"], ptrs["z"], ptrs["h0"],
+                                    po, ph, pw, workspace.numel(), ctypes.byref(dims), sp)
+        _check(rc)
+        if check:
+            _check(get_lib().ssm_scan_fwd_status(pw, sp))
     return out, h_last
 
 
@@ -183,5 +235,5 @@ def ssm_scan_step(state, x, delta, delta_bias, softplus, A, B, C, D=None, z=None
     return out
 
 
-__all__ = ["ssm_scan_fwd", "ssm_scan_step", "ssm_strerror", "ssm_version", "SSMError", "Dims",
-           "LIB_PATH", "get_lib"]
+__all__ = ["ssm_scan_fwd", "ssm_scan_fwd_workspace_size", "ssm_scan_fwd_status", "ssm_scan_step",
+           "ssm_strerror", "ssm_version", "SSMError", "Dims", "LIB_PATH", "get_lib"]

@@ -52,7 +52,14 @@ struct FwdParams {
     // records its end state and decay product; after segment_combine_kernel has
     // turned those into start states, every segment runs again from its own.
     int mode;
+    int pass;           // 0: the only or the summary pass; 1: the second pass (its own queues)
     int64_t seg_steps;  // steps per segment, a multiple of 32
+    // Bound of the inter-segment flag wait (polls 64 ns apart), and an offset
+    // added to the awaited segment count.  The library passes kSpinLimit and 0;
+    // the wait-timeout test entry point passes a small bound and an offset no
+    // flag ever reaches, so the wait gives up deterministically.
+    uint32_t spin_limit;
+    uint32_t flag_bias;
 };
 constexpr int kChained = 0, kSummary = 1, kFromStart = 2;
 
@@ -430,8 +437,8 @@ constexpr uint32_t kSpinLimit = 1u << 24;   // flag polls (64 ns apart)
 constexpr uint32_t kBarLimit = 1u << 20;    // mbarrier try_wait rounds
 
 struct FwdScratch {
-    uint32_t *counter;  // [2] next item, one queue per kernel instance (S4D, general)
-    uint32_t *error;    // non-zero: a bounded wait gave up
+    uint32_t *counter;  // [4] next item: one queue per (pass, kernel instance S4D / general)
+    uint32_t *error;    // non-zero: a bounded wait gave up (bit 0: segment flag, bit 1: mbarrier)
     uint32_t *general;  // non-zero: some group has A rows without the S4D structure
     uint32_t *flags;    // [groups]: segments of the group finished
     float *carry;       // [groups][32 lanes][16 states]
@@ -452,8 +459,8 @@ __host__ __device__ inline FwdScratch fwd_scratch_view(void *base, int64_t group
     uint8_t *b = static_cast<uint8_t *>(base);
     FwdScratch s;
     s.counter = reinterpret_cast<uint32_t *>(b);
-    s.error = reinterpret_cast<uint32_t *>(b + 8);
-    s.general = reinterpret_cast<uint32_t *>(b + 12);
+    s.error = reinterpret_cast<uint32_t *>(b + 16);
+    s.general = reinterpret_cast<uint32_t *>(b + 20);
     s.flags = reinterpret_cast<uint32_t *>(b + 256);
     s.carry = reinterpret_cast<float *>(b + fwd_scratch_flag_bytes(groups));
     s.summ = s.carry + static_cast<size_t>(groups) * 32 * kNState;
@@ -478,23 +485,37 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar))
                  : "memory");
 }
-// wait for the completion of the phase with the given parity; false on timeout
+// Wait for the completion of the phase with the given parity.  Returns false
+// when the wait gives up: after kBarLimit polls (the error word gets bit 1), or
+// early, once another wait of the launch has given up (the error word is
+// non-zero) -- its results are void, so the caller leaves its loop.  A caller
+// that gives up never touches the chunk it waited for.
+__device__ __forceinline__ bool mbar_try_parity(uint32_t addr, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    return done != 0;
+}
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t *error) {
     const uint32_t addr = smem_u32(bar);
     for (uint32_t n = 0; n < kBarLimit; ++n) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(done)
-            : "r"(addr), "r"(parity)
-            : "memory");
-        if (done) return true;
-        // once any wait of the launch has given up, stop waiting: the results are void
+        if (mbar_try_parity(addr, parity)) return true;
         if ((n & 1023u) == 1023u && *reinterpret_cast<volatile uint32_t *>(error) != 0) return false;
     }
     atomicOr(error, 2u);
     return false;
+}
+// The same wait for a TMA load's completion before the CTA may exit: it does not
+// stop early on the error word (a load must never be in flight when the CTA ends).
+__device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity, uint32_t *error) {
+    const uint32_t addr = smem_u32(bar);
+    for (uint32_t n = 0; n < kBarLimit; ++n)
+        if (mbar_try_parity(addr, parity)) return;
+    atomicOr(error, 2u);
 }
 
 // One chunk of a worker's stream, as the helper hands it to the scan warp.
@@ -640,12 +661,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     __syncthreads();
     if (!S4D && *reinterpret_cast<volatile uint32_t *>(sc.general) == 0) return;
-    uint32_t *counter = sc.counter + (S4D ? 0 : 1);
+    uint32_t *counter = sc.counter + 2 * p.pass + (S4D ? 0 : 1);
 
     if (role == 1) {
         // ------------------------------------------------------------------ prep
         ChunkCursor<T, S4D> cur(p);
         const uint32_t stage_tx = (p.z ? 3u : 2u) * SM::kTileBytes + 2u * kNState * kRowBytes;
+        // TMA loads issued and waited for, in chunk order: every issued load is
+        // waited for before the warp leaves, also when it gives up early
+        int64_t n_issued = 0, n_waited = 0;
         // stage chunk j: TMA (one lane, completion on full[j % kStages]) or element loads
         auto issue = [&](const ChunkDesc &dsc, int64_t j) {
             if (dsc.flags & kStop) return;
@@ -661,6 +685,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     tma_load_3d(st + 3 * SM::kTileBytes, &tm.B, t0, 0, b, bar);
                     tma_load_3d(st + 3 * SM::kTileBytes + kNState * kRowBytes, &tm.C, t0, 0, b, bar);
                 }
+                n_issued = j + 1;
             } else {
                 load_chunk_sync<T>(p, st, dsc.b, dsc.d0, dsc.t0, lane);
             }
@@ -673,11 +698,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int64_t j = 0;; ++j) {
             const ChunkDesc dj = dnext;
             // chunk j+1 goes to the stage that chunk j-2 used: wait until it is posted
-            if (j >= 2) mbar_wait(posted + (j & 1), parity(j - 2, 2), sc.error);
+            if (j >= 2 && !mbar_wait(posted + (j & 1), parity(j - 2, 2), sc.error)) break;
             if (!(dj.flags & kStop)) {
                 dnext = cur.next(p, sc, counter, lane);
                 issue(dnext, j + 1);
-                if constexpr (VEC) mbar_wait(full + (j % kStages), parity(j, kStages), sc.error);
+                if constexpr (VEC) {
+                    if (!mbar_wait(full + (j % kStages), parity(j, kStages), sc.error)) break;
+                    n_waited = j + 1;
+                }
                 __syncwarp();
                 uint8_t *st = stage_of(j);
                 widen_bc<T>(st + 3 * SM::kTileBytes, bcf_of(j), lane);
@@ -693,13 +721,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             mbar_arrive(ready + (j & 1));
             if (dj.flags & kStop) break;
         }
+        // loads still in flight after a wait gave up (none on the normal path)
+        for (int64_t j = n_waited; j < n_issued; ++j) mbar_drain(full + (j % kStages), parity(j, kStages), sc.error);
     } else if (role == 2) {
         // ------------------------------------------------------------------ post
         const bool has_z = p.z != nullptr;
         ChanConst cc;
         int64_t cc_d0 = -1;
         for (int64_t j = 0;; ++j) {
-            mbar_wait(done + (j & 1), parity(j, 2), sc.error);
+            if (!mbar_wait(done + (j & 1), parity(j, 2), sc.error)) break;
             const ChunkDesc dj = ring[j & 3];
             if (dj.flags & kStop) break;
             uint8_t *st = stage_of(j);
@@ -740,7 +770,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
         for (int n = 0; n < kNState; ++n) a2[n] = 0.0f;
         for (int64_t k = 0;; ++k) {
-            mbar_wait(ready + (k & 1), parity(k, 2), sc.error);
+            if (!mbar_wait(ready + (k & 1), parity(k, 2), sc.error)) break;
             const ChunkDesc dk = ring[k & 3];
             if (dk.flags & kStop) {
                 mbar_arrive(done + (k & 1));  // lets the post warp see the end
@@ -760,14 +790,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     // every segment starts from zero; P starts as the identity
 #pragma unroll
                     for (int j = 0; j < 8; ++j) P[j] = make_float2(1.0f, 1.0f);
+                } else if (p.mode == kFromStart) {
+                    // every segment, the first one included, starts from the state the
+                    // combine kernel left; h0 is not read here, so h_last may alias it
+                    src = reinterpret_cast<const float4 *>(sc.start + gs * kNState);
                 } else if (dk.seg == 0) {
                     if (active && p.h0) src = reinterpret_cast<const float4 *>(p.h0 + (dk.b * p.dim + d) * kNState);
-                } else if (p.mode == kFromStart) {
-                    src = reinterpret_cast<const float4 *>(sc.start + gs * kNState);
                 } else {
+                    const uint32_t want = static_cast<uint32_t>(dk.seg) + p.flag_bias;
                     uint32_t spins = 0;
-                    while (ld_acquire(sc.flags + dk.g) < static_cast<uint32_t>(dk.seg)) {
-                        if (++spins > kSpinLimit) {
+                    while (ld_acquire(sc.flags + dk.g) < want) {
+                        if (++spins > p.spin_limit) {
                             atomicOr(sc.error, 1u);
                             break;
                         }

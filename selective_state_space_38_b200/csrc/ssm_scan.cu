@@ -47,28 +47,6 @@ bool dims_ok(int64_t batch, int64_t seqlen, int64_t dim) {
     return elems < 4.0e18 / 16.0;
 }
 
-// Scratch memory comes from a library-owned stream-ordered pool per device that
-// keeps freed memory (release threshold = max), so after the first call an
-// allocation is a cheap pool hit and never waits on the operating system.
-cudaMemPool_t scratch_pool(int dev) {
-    static std::mutex mu;
-    static cudaMemPool_t pools[64] = {};
-    if (dev < 0 || dev >= 64) return nullptr;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!pools[dev]) {
-        cudaMemPoolProps props = {};
-        props.allocType = cudaMemAllocationTypePinned;
-        props.location.type = cudaMemLocationTypeDevice;
-        props.location.id = dev;
-        cudaMemPool_t pool = nullptr;
-        if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return nullptr;
-        uint64_t keep = UINT64_MAX;
-        cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
-        pools[dev] = pool;
-    }
-    return pools[dev];
-}
-
 // cuTensorMapEncodeTiled from the driver, looked up once through the runtime
 // (no link-time dependency on libcuda).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -164,41 +142,48 @@ int launch_fwd_kernels(FwdParams p, void *scratch, int64_t segs, int sms, cudaSt
     const FwdScratch sc = fwd_scratch_view(scratch, groups, segs);
     if (segs == 0) {
         p.mode = kChained;
+        p.pass = 0;
         p.seg_steps = kSegSteps;
         return launch_pass<T, VEC>(p, sc, tm, sms, stream);
     }
     p.mode = kSummary;
+    p.pass = 0;
     int rc = launch_pass<T, VEC>(p, sc, tm, sms, stream);
     if (rc != SSM_OK) return rc;
     const int64_t threads = groups * 32;
     segment_combine_kernel<<<static_cast<unsigned>((threads + 127) / 128), 128, 0, stream>>>(p, sc);
-    if (cudaMemsetAsync(scratch, 0, fwd_scratch_flag_bytes(groups), stream) != cudaSuccess) return SSM_ERR_CUDA;
+    // the second pass takes items from its own queues; the error word of the
+    // first pass stays set for the status query
     p.mode = kFromStart;
+    p.pass = 1;
     return launch_pass<T, VEC>(p, sc, tm, sms, stream);
 }
 
-template <typename T, bool VEC>
-int launch_fwd(FwdParams p, cudaStream_t stream) {
-    const int64_t groups = ((p.dim + 31) / 32) * p.batch;
-    const int64_t items = groups * ((p.seqlen + kSegSteps - 1) / kSegSteps);
-    if (items > static_cast<int64_t>(UINT32_MAX) / 2) return SSM_ERR_UNSUPPORTED;
-    int dev = 0, sms = 0;
+// SMs of the current device (the schedule, and so the workspace size, depend on it)
+int current_sms(int *sms) {
+    int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || *sms < 1)
         return SSM_ERR_CUDA;
-    const int64_t segs = parallel_segments(p, sms, &p.seg_steps);
-    cudaMemPool_t pool = scratch_pool(dev);
-    if (!pool) return SSM_ERR_CUDA;
-    void *scratch = nullptr;
-    if (cudaMallocFromPoolAsync(&scratch, fwd_scratch_bytes(groups, segs), pool, stream) != cudaSuccess)
-        return SSM_ERR_CUDA;
-    int rc = SSM_OK;
-    if (cudaMemsetAsync(scratch, 0, fwd_scratch_flag_bytes(groups), stream) != cudaSuccess)
-        rc = SSM_ERR_CUDA;
-    else
-        rc = launch_fwd_kernels<T, VEC>(p, scratch, segs, sms, stream);
-    if (cudaFreeAsync(scratch, stream) != cudaSuccess) rc = SSM_ERR_CUDA;
-    return rc;
+    return SSM_OK;
+}
+
+// Workspace bytes of a validated shape on a GPU with `sms` SMs.
+size_t fwd_workspace_bytes(const FwdParams &p, int sms) {
+    FwdParams q = p;
+    const int64_t groups = ((p.dim + 31) / 32) * p.batch;
+    const int64_t segs = parallel_segments(q, sms, &q.seg_steps);
+    return fwd_scratch_bytes(groups, segs);
+}
+
+// One forward call on the caller's workspace: zero its flag words, then the kernels.
+template <typename T, bool VEC>
+int launch_fwd(FwdParams p, void *ws, size_t ws_bytes, int sms, bool force_chained, cudaStream_t stream) {
+    const int64_t groups = ((p.dim + 31) / 32) * p.batch;
+    const int64_t segs = force_chained ? 0 : parallel_segments(p, sms, &p.seg_steps);
+    if (ws_bytes < fwd_scratch_bytes(groups, segs)) return SSM_ERR_INVALID_ARG;
+    if (cudaMemsetAsync(ws, 0, fwd_scratch_flag_bytes(groups), stream) != cudaSuccess) return SSM_ERR_CUDA;
+    return launch_fwd_kernels<T, VEC>(p, ws, segs, sms, stream);
 }
 
 template <typename T>
@@ -213,6 +198,82 @@ int launch_step(const StepParams &p, cudaStream_t stream) {
     return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
+// Every check of a forward call's arguments (all three forward entry points
+// share it); on success fills `p` and the activation element size.  The
+// workspace, when given, must not overlap any input or output.
+int validate_fwd(const void *x, const void *delta, const float *delta_bias, int softplus, const float *A,
+                 const void *B, const void *C, const float *D, const void *z, const float *h0, void *out,
+                 float *h_last, const void *ws, size_t ws_bytes, const ssm_dims_t *dims, FwdParams *p,
+                 size_t *es_out) {
+    if (!dims) return SSM_ERR_INVALID_ARG;
+    const int64_t batch = dims->batch, L = dims->seqlen, dim = dims->dim, N = dims->dstate;
+    if (!x || !delta || !A || !B || !C || !out) return SSM_ERR_INVALID_ARG;
+    if (!dims_ok(batch, L, dim) || N < 1) return SSM_ERR_INVALID_ARG;
+    if (N != kNState) return SSM_ERR_UNSUPPORTED;
+    if (dims->act_dtype != SSM_F32 && dims->act_dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
+    // TMA coordinates and the work queue's item split are 32-bit
+    if (batch > INT32_MAX || L > INT32_MAX - 64 || dim > INT32_MAX - 64) return SSM_ERR_UNSUPPORTED;
+    const int64_t groups = ((dim + 31) / 32) * batch;
+    if (groups * ((L + 255) / 256) > static_cast<int64_t>(UINT32_MAX) / 2) return SSM_ERR_UNSUPPORTED;
+    const size_t es = dims->act_dtype == SSM_F32 ? 4 : 2;
+    for (const void *ptr : {x, delta, (const void *)A, B, C, z, (const void *)h0, (const void *)out,
+                            (const void *)h_last, ws})
+        if (ptr && !aligned16(ptr)) return SSM_ERR_MISALIGNED;
+    for (const void *ptr : {(const void *)delta_bias, (const void *)D})
+        if (ptr && !aligned4(ptr)) return SSM_ERR_MISALIGNED;
+
+    const size_t tok = static_cast<size_t>(batch) * dim * L;
+    const size_t st = static_cast<size_t>(batch) * dim * N * 4;
+    const Span o{out, tok * es};
+    const Span ins[] = {{x, tok * es}, {delta, tok * es}, {z, z ? tok * es : 0},
+                        {B, static_cast<size_t>(batch) * N * L * es}, {C, static_cast<size_t>(batch) * N * L * es},
+                        {A, static_cast<size_t>(dim) * N * 4}, {D, D ? static_cast<size_t>(dim) * 4 : 0},
+                        {delta_bias, delta_bias ? static_cast<size_t>(dim) * 4 : 0},
+                        {h0, h0 ? st : 0}, {h_last, h_last ? st : 0}};
+    for (const Span &s : ins)
+        if (overlap(o, s)) return SSM_ERR_INVALID_ARG;
+    if (h_last) {  // h_last may be h0 itself, but must not partially overlap any input
+        const Span hl{h_last, st};
+        for (int i = 0; i < 8; ++i)
+            if (overlap(hl, ins[i])) return SSM_ERR_INVALID_ARG;
+        if (h0 && h0 != h_last && overlap(hl, ins[8])) return SSM_ERR_INVALID_ARG;
+    }
+    if (ws) {
+        // the chained schedule's workspace is the least any device needs (the
+        // exact size, which depends on the SM count, is checked at launch)
+        if (ws_bytes < fwd_scratch_bytes(((dim + 31) / 32) * batch)) return SSM_ERR_INVALID_ARG;
+        const Span w{ws, ws_bytes};
+        if (overlap(w, o)) return SSM_ERR_INVALID_ARG;
+        for (const Span &s : ins)
+            if (overlap(w, s)) return SSM_ERR_INVALID_ARG;
+    }
+
+    memset(p, 0, sizeof *p);
+    p->x = x; p->delta = delta; p->z = z; p->B = B; p->C = C;
+    p->delta_bias = delta_bias; p->A = A; p->D = D; p->h0 = h0;
+    p->out = out; p->h_last = h_last;
+    p->batch = batch; p->seqlen = L; p->dim = dim;
+    p->softplus = softplus ? 1 : 0;
+    p->seg_steps = kSegSteps;
+    p->spin_limit = kSpinLimit;
+    p->flag_bias = 0;
+    *es_out = es;
+    return SSM_OK;
+}
+
+// The forward call on a validated shape and a workspace of ws_bytes.
+int dispatch_fwd(const FwdParams &p, size_t es, int act_dtype, void *ws, size_t ws_bytes, bool force_chained,
+                 cudaStream_t s) {
+    int sms = 0;
+    if (current_sms(&sms) != SSM_OK) return SSM_ERR_CUDA;
+    const bool vec = (static_cast<size_t>(p.seqlen) * es) % 16 == 0;
+    if (act_dtype == SSM_BF16)
+        return vec ? launch_fwd<bf16raw, true>(p, ws, ws_bytes, sms, force_chained, s)
+                   : launch_fwd<bf16raw, false>(p, ws, ws_bytes, sms, force_chained, s);
+    return vec ? launch_fwd<float, true>(p, ws, ws_bytes, sms, force_chained, s)
+               : launch_fwd<float, false>(p, ws, ws_bytes, sms, force_chained, s);
+}
+
 }  // namespace
 
 extern "C" {
@@ -222,60 +283,57 @@ int ssm_version(void) { return kVersion; }
 const char *ssm_strerror(int code) {
     switch (code) {
         case SSM_OK: return "ok";
-        case SSM_ERR_INVALID_ARG: return "invalid argument (NULL required pointer, size < 1, or out overlapping an input)";
+        case SSM_ERR_INVALID_ARG: return "invalid argument (NULL required pointer, size < 1, overlapping buffers, or a workspace that is too small)";
         case SSM_ERR_UNSUPPORTED: return "unsupported (dstate must be 16, dtype f32 or bf16, sizes within limits)";
         case SSM_ERR_MISALIGNED: return "misaligned pointer (16-byte alignment required)";
-        case SSM_ERR_CUDA: return "CUDA launch error";
-        case SSM_ERR_TIMEOUT: return "bounded device wait timed out";
+        case SSM_ERR_CUDA: return "CUDA launch or query error";
+        case SSM_ERR_TIMEOUT: return "bounded device wait timed out; the call's results are void";
         default: return "unknown error code";
     }
 }
 
+int ssm_scan_fwd_workspace_size(const ssm_dims_t *dims, int sm_count, size_t *bytes) {
+    if (!dims || !bytes) return SSM_ERR_INVALID_ARG;
+    if (!dims_ok(dims->batch, dims->seqlen, dims->dim) || dims->dstate < 1) return SSM_ERR_INVALID_ARG;
+    if (dims->dstate != kNState) return SSM_ERR_UNSUPPORTED;
+    if (sm_count <= 0 && current_sms(&sm_count) != SSM_OK) return SSM_ERR_CUDA;
+    FwdParams p;
+    memset(&p, 0, sizeof p);
+    p.batch = dims->batch; p.seqlen = dims->seqlen; p.dim = dims->dim;
+    p.seg_steps = kSegSteps;
+    *bytes = fwd_workspace_bytes(p, sm_count);
+    return SSM_OK;
+}
+
 int ssm_scan_fwd(const void *x, const void *delta, const float *delta_bias, int softplus,
                  const float *A, const void *B, const void *C, const float *D, const void *z,
-                 const float *h0, void *out, float *h_last, const ssm_dims_t *dims,
-                 ssm_stream_t stream) {
-    if (!dims) return SSM_ERR_INVALID_ARG;
-    const int64_t batch = dims->batch, L = dims->seqlen, dim = dims->dim, N = dims->dstate;
-    if (!x || !delta || !A || !B || !C || !out) return SSM_ERR_INVALID_ARG;
-    if (!dims_ok(batch, L, dim) || N < 1) return SSM_ERR_INVALID_ARG;
-    if (N != kNState) return SSM_ERR_UNSUPPORTED;
-    if (dims->act_dtype != SSM_F32 && dims->act_dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
-    const size_t es = dims->act_dtype == SSM_F32 ? 4 : 2;
-    for (const void *ptr : {x, delta, (const void *)A, B, C, z, (const void *)h0, (const void *)out,
-                            (const void *)h_last})
-        if (ptr && !aligned16(ptr)) return SSM_ERR_MISALIGNED;
-    for (const void *ptr : {(const void *)delta_bias, (const void *)D})
-        if (ptr && !aligned4(ptr)) return SSM_ERR_MISALIGNED;
-
-    const size_t tok = static_cast<size_t>(batch) * dim * L;
-    const Span o{out, tok * es};
-    const Span ins[] = {{x, tok * es}, {delta, tok * es}, {z, z ? tok * es : 0},
-                        {B, static_cast<size_t>(batch) * N * L * es}, {C, static_cast<size_t>(batch) * N * L * es},
-                        {A, static_cast<size_t>(dim) * N * 4}, {D, D ? static_cast<size_t>(dim) * 4 : 0},
-                        {delta_bias, delta_bias ? static_cast<size_t>(dim) * 4 : 0},
-                        {h0, h0 ? static_cast<size_t>(batch) * dim * N * 4 : 0},
-                        {h_last, h_last ? static_cast<size_t>(batch) * dim * N * 4 : 0}};
-    for (const Span &s : ins)
-        if (overlap(o, s)) return SSM_ERR_INVALID_ARG;
-    if (h_last) {  // h_last may be h0 itself, but must not partially overlap any input
-        const Span hl{h_last, static_cast<size_t>(batch) * dim * N * 4};
-        for (int i = 0; i < 8; ++i)
-            if (overlap(hl, ins[i])) return SSM_ERR_INVALID_ARG;
-        if (h0 && h0 != h_last && overlap(hl, ins[8])) return SSM_ERR_INVALID_ARG;
-    }
-
+                 const float *h0, void *out, float *h_last, void *workspace, size_t workspace_bytes,
+                 const ssm_dims_t *dims, ssm_stream_t stream) {
+    if (!workspace) return SSM_ERR_INVALID_ARG;
     FwdParams p;
-    p.x = x; p.delta = delta; p.z = z; p.B = B; p.C = C;
-    p.delta_bias = delta_bias; p.A = A; p.D = D; p.h0 = h0;
-    p.out = out; p.h_last = h_last;
-    p.batch = batch; p.seqlen = L; p.dim = dim;
-    p.softplus = softplus ? 1 : 0;
-    const bool vec = (static_cast<size_t>(L) * es) % 16 == 0;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (dims->act_dtype == SSM_BF16)
-        return vec ? launch_fwd<bf16raw, true>(p, s) : launch_fwd<bf16raw, false>(p, s);
-    return vec ? launch_fwd<float, true>(p, s) : launch_fwd<float, false>(p, s);
+    size_t es = 0;
+    const int rc = validate_fwd(x, delta, delta_bias, softplus, A, B, C, D, z, h0, out, h_last, workspace,
+                                workspace_bytes, dims, &p, &es);
+    if (rc != SSM_OK) return rc;
+    return dispatch_fwd(p, es, dims->act_dtype, workspace, workspace_bytes, false,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+int ssm_debug_fwd_flag_timeout(const void *x, const void *delta, const float *delta_bias, int softplus,
+                               const float *A, const void *B, const void *C, const float *D, const void *z,
+                               const float *h0, void *out, float *h_last, void *workspace,
+                               size_t workspace_bytes, uint32_t spin_limit, const ssm_dims_t *dims,
+                               ssm_stream_t stream) {
+    if (!workspace) return SSM_ERR_INVALID_ARG;
+    FwdParams p;
+    size_t es = 0;
+    const int rc = validate_fwd(x, delta, delta_bias, softplus, A, B, C, D, z, h0, out, h_last, workspace,
+                                workspace_bytes, dims, &p, &es);
+    if (rc != SSM_OK) return rc;
+    p.spin_limit = spin_limit;
+    p.flag_bias = 1u << 30;  // no segment flag ever reaches this
+    return dispatch_fwd(p, es, dims->act_dtype, workspace, workspace_bytes, true,
+                        reinterpret_cast<cudaStream_t>(stream));
 }
 
 int ssm_scan_step(float *state, const void *x, const void *delta, const float *delta_bias,
@@ -288,8 +346,10 @@ int ssm_scan_step(float *state, const void *x, const void *delta, const float *d
     if (N != kNState) return SSM_ERR_UNSUPPORTED;
     if (dims->act_dtype != SSM_F32 && dims->act_dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
     const size_t es = dims->act_dtype == SSM_F32 ? 4 : 2;
-    if (!aligned16(state) || !aligned16(A)) return SSM_ERR_MISALIGNED;
-    for (const void *ptr : {x, delta, B, C, z, (const void *)out, (const void *)delta_bias, (const void *)D})
+    // state, A, B and C are read (and the state written) as 16-byte vectors per lane
+    for (const void *ptr : {(const void *)state, (const void *)A, B, C})
+        if (!aligned16(ptr)) return SSM_ERR_MISALIGNED;
+    for (const void *ptr : {x, delta, z, (const void *)out, (const void *)delta_bias, (const void *)D})
         if (ptr && (reinterpret_cast<uintptr_t>(ptr) % (ptr == delta_bias || ptr == D ? 4 : es)) != 0)
             return SSM_ERR_MISALIGNED;
 
@@ -322,8 +382,8 @@ int ssm_scan_step(float *state, const void *x, const void *delta, const float *d
 // device memory up front and forbid later allocation, and processes that must
 // not touch the CUDA allocator at all.  ssm_scan_fwd_noalloc serves them: it
 // runs the same kernels as ssm_scan_fwd, but its work queue, segment flags and
-// carried states live in the fixed device array below instead of a pool
-// allocation.  The array is part of the library image, so every GPU that loads
+// carried states live in the fixed device array below instead of a caller
+// workspace.  The array is part of the library image, so every GPU that loads
 // the library holds kNoAllocScratchBytes for the life of the process.
 namespace {
 
@@ -345,72 +405,45 @@ void *noalloc_scratch(int dev) {
     return addr[dev];
 }
 
-// Always the chained schedule: its scratch does not grow with the sequence.
-template <typename T, bool VEC>
-int launch_fwd_noalloc(const FwdParams &p, cudaStream_t stream) {
-    const int64_t groups = ((p.dim + 31) / 32) * p.batch;
-    const int64_t items = groups * ((p.seqlen + kSegSteps - 1) / kSegSteps);
-    if (items > static_cast<int64_t>(UINT32_MAX) / 2 || fwd_scratch_bytes(groups) > kNoAllocScratchBytes)
-        return SSM_ERR_UNSUPPORTED;
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return SSM_ERR_CUDA;
-    void *scratch = noalloc_scratch(dev);
-    if (!scratch) return SSM_ERR_CUDA;
-    // the array keeps the previous call's contents: the queue counters, error
-    // word and segment flags must start at zero (the carries need not)
-    if (cudaMemsetAsync(scratch, 0, fwd_scratch_flag_bytes(groups), stream) != cudaSuccess) return SSM_ERR_CUDA;
-    return launch_fwd_kernels<T, VEC>(p, scratch, 0, sms, stream);
-}
-
 }  // namespace
 
 extern "C" int ssm_scan_fwd_noalloc(const void *x, const void *delta, const float *delta_bias, int softplus,
                                     const float *A, const void *B, const void *C, const float *D,
                                     const void *z, const float *h0, void *out, float *h_last,
                                     const ssm_dims_t *dims, ssm_stream_t stream) {
-    if (!dims) return SSM_ERR_INVALID_ARG;
-    const int64_t batch = dims->batch, L = dims->seqlen, dim = dims->dim, N = dims->dstate;
-    if (!x || !delta || !A || !B || !C || !out) return SSM_ERR_INVALID_ARG;
-    if (!dims_ok(batch, L, dim) || N < 1) return SSM_ERR_INVALID_ARG;
-    if (N != kNState) return SSM_ERR_UNSUPPORTED;
-    if (dims->act_dtype != SSM_F32 && dims->act_dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
-    const size_t es = dims->act_dtype == SSM_F32 ? 4 : 2;
-    for (const void *ptr : {x, delta, (const void *)A, B, C, z, (const void *)h0, (const void *)out,
-                            (const void *)h_last})
-        if (ptr && !aligned16(ptr)) return SSM_ERR_MISALIGNED;
-    for (const void *ptr : {(const void *)delta_bias, (const void *)D})
-        if (ptr && !aligned4(ptr)) return SSM_ERR_MISALIGNED;
-    const size_t tok = static_cast<size_t>(batch) * dim * L;
-    const Span o{out, tok * es};
-    const Span ins[] = {{x, tok * es}, {delta, tok * es}, {z, z ? tok * es : 0},
-                        {B, static_cast<size_t>(batch) * N * L * es}, {C, static_cast<size_t>(batch) * N * L * es},
-                        {A, static_cast<size_t>(dim) * N * 4}, {D, D ? static_cast<size_t>(dim) * 4 : 0},
-                        {delta_bias, delta_bias ? static_cast<size_t>(dim) * 4 : 0},
-                        {h0, h0 ? static_cast<size_t>(batch) * dim * N * 4 : 0},
-                        {h_last, h_last ? static_cast<size_t>(batch) * dim * N * 4 : 0}};
-    for (const Span &s : ins)
-        if (overlap(o, s)) return SSM_ERR_INVALID_ARG;
-    if (h_last) {
-        const Span hl{h_last, static_cast<size_t>(batch) * dim * N * 4};
-        for (int i = 0; i < 8; ++i)
-            if (overlap(hl, ins[i])) return SSM_ERR_INVALID_ARG;
-        if (h0 && h0 != h_last && overlap(hl, ins[8])) return SSM_ERR_INVALID_ARG;
-    }
-    // the work queue of this shape must fit the fixed array
-    const int64_t groups = ((dim + 31) / 32) * batch;
-    if (fwd_scratch_bytes(groups) > kNoAllocScratchBytes) return SSM_ERR_UNSUPPORTED;
-
     FwdParams p;
-    p.x = x; p.delta = delta; p.z = z; p.B = B; p.C = C;
-    p.delta_bias = delta_bias; p.A = A; p.D = D; p.h0 = h0;
-    p.out = out; p.h_last = h_last;
-    p.batch = batch; p.seqlen = L; p.dim = dim;
-    p.softplus = softplus ? 1 : 0;
-    const bool vec = (static_cast<size_t>(L) * es) % 16 == 0;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (dims->act_dtype == SSM_BF16)
-        return vec ? launch_fwd_noalloc<bf16raw, true>(p, s) : launch_fwd_noalloc<bf16raw, false>(p, s);
-    return vec ? launch_fwd_noalloc<float, true>(p, s) : launch_fwd_noalloc<float, false>(p, s);
+    size_t es = 0;
+    const int rc = validate_fwd(x, delta, delta_bias, softplus, A, B, C, D, z, h0, out, h_last, nullptr, 0, dims,
+                                &p, &es);
+    if (rc != SSM_OK) return rc;
+    // the work queue of this shape (chained schedule: its scratch does not grow
+    // with the sequence) must fit the fixed array
+    const int64_t groups = ((p.dim + 31) / 32) * p.batch;
+    if (fwd_scratch_bytes(groups) > kNoAllocScratchBytes) return SSM_ERR_UNSUPPORTED;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SSM_ERR_CUDA;
+    void *scratch = noalloc_scratch(dev);
+    if (!scratch) return SSM_ERR_CUDA;
+    // the array keeps the previous call's contents: launch_fwd zeroes the queue
+    // counters, error word and segment flags (the carries need not start at zero)
+    return dispatch_fwd(p, es, dims->act_dtype, scratch, kNoAllocScratchBytes, true,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int ssm_scan_fwd_status(const void *workspace, ssm_stream_t stream) {
+    const uint8_t *ws = static_cast<const uint8_t *>(workspace);
+    if (!ws) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return SSM_ERR_CUDA;
+        ws = static_cast<const uint8_t *>(noalloc_scratch(dev));
+        if (!ws) return SSM_ERR_CUDA;
+    }
+    if (!aligned16(ws)) return SSM_ERR_MISALIGNED;
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return SSM_ERR_CUDA;
+    // the error word sits in the fixed header of every workspace layout
+    const FwdScratch view = fwd_scratch_view(const_cast<uint8_t *>(ws), 0);
+    uint32_t err = 0;
+    if (cudaMemcpy(&err, view.error, sizeof err, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    return err ? SSM_ERR_TIMEOUT : SSM_OK;
 }

@@ -25,8 +25,11 @@ def lib():
 
 def test_header_declares_entry_points():
     names = _declared()
-    for n in ("ssm_scan_fwd", "ssm_scan_step", "ssm_strerror", "ssm_version"):
+    for n in ("ssm_scan_fwd_workspace_size", "ssm_scan_fwd", "ssm_scan_fwd_status", "ssm_scan_step",
+              "ssm_scan_fwd_noalloc", "ssm_debug_fwd_flag_timeout", "ssm_strerror", "ssm_version"):
         assert n in names
+    import selective_state_space_38_b200 as m
+    assert sorted(m.EXPORTS) == names
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -51,12 +54,20 @@ def _dims(m, batch=2, L=64, dim=128, N=16, dt=1):
     return ctypes.byref(m.Dims(batch, L, dim, N, dt))
 
 
-def _fwd(lib, m, **over):
+WS = 1 << 20  # bytes of the fake workspace (enough for the default shape)
+
+
+def _fwd(lib, m, fn="ssm_scan_fwd", **over):
     a = dict(x=_p(1), delta=_p(2), bias=None, sp=1, A=_p(3), B=_p(4), C=_p(5), D=None, z=_p(6),
-             h0=None, out=_p(7), hl=None, dims=_dims(m))
+             h0=None, out=_p(7), hl=None, ws=_p(9), wsb=WS, dims=_dims(m))
     a.update(over)
-    return lib.ssm_scan_fwd(a["x"], a["delta"], a["bias"], a["sp"], a["A"], a["B"], a["C"], a["D"],
-                            a["z"], a["h0"], a["out"], a["hl"], a["dims"], None)
+    args = [a["x"], a["delta"], a["bias"], a["sp"], a["A"], a["B"], a["C"], a["D"], a["z"], a["h0"],
+            a["out"], a["hl"]]
+    if fn == "ssm_scan_fwd_noalloc":
+        return lib.ssm_scan_fwd_noalloc(*args, a["dims"], None)
+    if fn == "ssm_debug_fwd_flag_timeout":
+        return lib.ssm_debug_fwd_flag_timeout(*args, a["ws"], a["wsb"], 0, a["dims"], None)
+    return lib.ssm_scan_fwd(*args, a["ws"], a["wsb"], a["dims"], None)
 
 
 def test_fwd_rejects_bad_arguments(lib):
@@ -77,6 +88,54 @@ def test_fwd_rejects_bad_arguments(lib):
     assert _fwd(lib, m, out=ctypes.c_void_p(0x11000000 + 0x100)) == 1
     # h_last overlapping an activation input
     assert _fwd(lib, m, hl=_p(2)) == 1
+    # the workspace: required, 16-byte aligned, large enough, disjoint from every buffer
+    assert _fwd(lib, m, ws=None) == 1
+    assert _fwd(lib, m, ws=ctypes.c_void_p(0x19000008)) == 3
+    assert _fwd(lib, m, wsb=100) == 1
+    assert _fwd(lib, m, ws=_p(3)) == 1
+    assert _fwd(lib, m, ws=ctypes.c_void_p(0x17000000 - 0x100)) == 1  # runs into out
+    # sizes beyond the kernels' 32-bit coordinates
+    assert _fwd(lib, m, dims=_dims(m, batch=1, L=1 << 31, dim=1)) == 2
+    assert _fwd(lib, m, dims=_dims(m, batch=1, L=8, dim=1 << 31)) == 2
+
+
+@pytest.mark.parametrize("fn", ["ssm_scan_fwd_noalloc", "ssm_debug_fwd_flag_timeout"])
+def test_other_fwd_entries_share_the_checks(lib, fn):
+    import selective_state_space_38_b200 as m
+    assert _fwd(lib, m, fn, x=None) == 1
+    assert _fwd(lib, m, fn, dims=_dims(m, N=8)) == 2
+    assert _fwd(lib, m, fn, x=ctypes.c_void_p(0x10000002)) == 3
+    assert _fwd(lib, m, fn, out=_p(1)) == 1
+    assert _fwd(lib, m, fn, dims=_dims(m, batch=1, L=1 << 31, dim=1)) == 2
+    if fn == "ssm_debug_fwd_flag_timeout":
+        assert _fwd(lib, m, fn, ws=None) == 1
+
+
+def test_workspace_size_query(lib):
+    """Sizes for a given SM count, computed on the host: 16 KB of header and
+    flags plus a 2 KB carry per 32-channel group; the two-pass schedule adds
+    6 KB per (group, segment) when groups are fewer than half of 4 x SMs."""
+    import selective_state_space_38_b200 as m
+
+    def size(batch, L, dim, sms=148):
+        out = ctypes.c_size_t(0)
+        rc = lib.ssm_scan_fwd_workspace_size(ctypes.byref(m.Dims(batch, L, dim, 16, 1)), sms,
+                                             ctypes.byref(out))
+        assert rc == 0, m.ssm_strerror(rc)
+        return out.value
+
+    def flag_bytes(groups):
+        return (256 + 4 * groups + 255) // 256 * 256
+
+    groups = 4 * 160  # the Mamba-2.8B layer: 640 groups >= 592 / 2: chained
+    assert size(4, 4096, 5120) == flag_bytes(groups) + groups * 2048
+    groups = 64       # the long sequence: 64 groups, 4 x 592 / 64 = 37 segments of 3552 steps
+    segs = -(-131072 // 3552)
+    assert size(1, 131072, 2048) == flag_bytes(groups) + groups * 2048 + groups * segs * 6144
+    assert size(1, 64, 2048) == flag_bytes(groups) + groups * 2048  # too short to split
+    bad = ctypes.c_size_t(0)
+    assert lib.ssm_scan_fwd_workspace_size(None, 148, ctypes.byref(bad)) == 1
+    assert lib.ssm_scan_fwd_workspace_size(ctypes.byref(m.Dims(1, 8, 8, 8, 1)), 148, ctypes.byref(bad)) == 2
 
 
 def test_step_rejects_bad_arguments(lib):
@@ -94,6 +153,12 @@ def test_step_rejects_bad_arguments(lib):
     assert step(dims=_dims(m, N=32)) == 2
     assert step(st=ctypes.c_void_p(0x10000004)) == 3
     assert step(out=_p(0)) == 1  # out overlapping the state
+    # B and C are read as 16-byte vectors: an element-aligned but not 16-byte
+    # aligned B or C is refused (it would be a misaligned vector load)
+    assert step(B=ctypes.c_void_p(0x14000004)) == 3
+    assert step(C=ctypes.c_void_p(0x15000008)) == 3
+    assert step(B=ctypes.c_void_p(0x14000002), dims=_dims(m, dt=1)) == 3
+    assert step(A=ctypes.c_void_p(0x13000004)) == 3
 
 
 def test_python_binding_refuses_cpu_tensors():

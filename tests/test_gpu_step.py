@@ -67,29 +67,21 @@ def decode_prefill_state(orc, cfg=4):
 
 
 def test_decode_batch_256x5120(orc):
-    """256 sequences x 5120 channels x 16 fp32 states, 1024 consecutive steps.
-    Every step: out and state of a 16-sequence subset against the oracle.
-    Steps 1 and 2: out of all 256 sequences.  After 1024 steps: the final
-    state of the subset."""
+    """256 sequences x 5120 channels x 16 fp32 states, 1024 consecutive steps
+    from the 64-step prefill state.  Every step: out of all 256 sequences
+    against the oracle.  After steps 1, 2, 64 and 1024: the whole state."""
     c = workloads.CONFIGS[4]
     prm_np = workloads.decode_params(4)
     state0 = decode_prefill_state(orc)
     state = to_dev(state0)
     prm = {k: to_dev(prm_np[k]) for k in ("A", "D", "delta_bias")}
     prm["softplus"] = True
-    sub = np.arange(0, c.batch, c.batch // 16)  # 16 sequences
-    sub_state = state0[sub].astype(np.float64)
-    full_state = state0.astype(np.float64)
+    ref_state = state0.astype(np.float64)
     for s in range(c.decode_steps):
         tok_np = workloads.decode_tokens(4, s)
         out = _step(state, {k: to_dev(v) for k, v in tok_np.items()}, prm)
-        if s < 2:
-            ref = orc.step(full_state, tok_np["x"], tok_np["delta"], prm_np["delta_bias"], True,
-                           prm_np["A"], tok_np["B"], tok_np["C"], prm_np["D"], tok_np["z"])
-            check(to_np64(out), ref, "bf16", f"decode step {s} out (all sequences)")
-        tsub = {k: np.ascontiguousarray(v[sub]) for k, v in tok_np.items()}
-        ref_sub = orc.step(sub_state, tsub["x"], tsub["delta"], prm_np["delta_bias"], True,
-                           prm_np["A"], tsub["B"], tsub["C"], prm_np["D"], tsub["z"])
-        check(to_np64(out)[sub], ref_sub, "bf16", f"decode step {s} out (subset)")
-        if s in (0, 63, c.decode_steps - 1):
-            check(to_np64(state)[sub], sub_state, "bf16", f"decode step {s} state (subset)")
+        ref = orc.step(ref_state, tok_np["x"], tok_np["delta"], prm_np["delta_bias"], True,
+                       prm_np["A"], tok_np["B"], tok_np["C"], prm_np["D"], tok_np["z"])
+        check(to_np64(out), ref, "bf16", f"decode step {s + 1} out (all sequences)")
+        if s + 1 in (1, 2, 64, c.decode_steps):
+            check(to_np64(state), ref_state, "bf16", f"decode step {s + 1} state (all sequences)")

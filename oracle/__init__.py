@@ -57,6 +57,13 @@ class Oracle:
         lib.ssm_ref_fwd_channels.restype = I
         lib.ssm_ref_step.argtypes = [P, P, P, P, I, P, P, P, P, P, I, L, L, L, P, I]
         lib.ssm_ref_step.restype = I
+        lib.ssm_ref_conv1d.argtypes = [P, P, P, L, P, I, I, L, L, L, P, P, I]
+        lib.ssm_ref_conv1d.restype = I
+        lib.ssm_ref_conv_fwd.argtypes = [P, P, P, L, P, P, P, I, P, P, P, P, P, P, I, L, L, L, L,
+                                         P, P, P, I]
+        lib.ssm_ref_conv_fwd.restype = I
+        lib.ssm_ref_conv_step.argtypes = [P, P, P, P, P, L, P, P, I, P, P, P, P, P, I, L, L, L, P, I]
+        lib.ssm_ref_conv_step.restype = I
         self._lib = lib
 
     # -- marshalling helpers ---------------------------------------------
@@ -150,6 +157,72 @@ class Oracle:
         return out
 
 
+    # -- the short causal convolution in front of the scan -----------------
+    def conv1d(self, x, w, bias, conv_state=None, silu=True, threads=0):
+        """Causal depthwise convolution of width K = w.shape[1] (then silu).
+
+        x: [b,d,L] stored activations; w: [d,K]; bias: [d] or None;
+        conv_state: [b,d,K-1] stored activations or None (zeros).
+        Returns (xc [b,d,L] float64, new state [b,d,K-1] float64)."""
+        code = self._dtype_code(x)
+        x, conv_state = (self._act(t, code) for t in (x, conv_state))
+        w, bias = self._f32(w), self._f32(bias)
+        batch, dim, L = x.shape
+        K = w.shape[1]
+        xc = np.empty((batch, dim, L), np.float64)
+        st = np.empty((batch, dim, K - 1), np.float64)
+        rc = self._lib.ssm_ref_conv1d(self._ptr(x), self._ptr(w), self._ptr(bias), K,
+                                      self._ptr(conv_state), int(bool(silu)), code, batch, L, dim,
+                                      self._ptr(xc), self._ptr(st), int(threads))
+        if rc != 0:
+            raise ValueError("oracle rejected the arguments")
+        return xc, st
+
+    def conv_fwd(self, x, w, cbias, conv_state, delta, delta_bias, softplus, A, B, C, D, z, h0,
+                 threads=0):
+        """Convolution + silu, then the scan on its output.
+
+        Returns (out [b,d,L], h_last [b,d,N], new conv state [b,d,K-1]), float64."""
+        code = self._dtype_code(x)
+        x, conv_state, delta, B, C, z = (self._act(t, code) for t in (x, conv_state, delta, B, C, z))
+        w, cbias, A, D, delta_bias, h0 = (self._f32(t) for t in (w, cbias, A, D, delta_bias, h0))
+        batch, dim, L = x.shape
+        N, K = A.shape[1], w.shape[1]
+        out = np.empty((batch, dim, L), np.float64)
+        hl = np.empty((batch, dim, N), np.float64)
+        st = np.empty((batch, dim, K - 1), np.float64)
+        rc = self._lib.ssm_ref_conv_fwd(
+            self._ptr(x), self._ptr(w), self._ptr(cbias), K, self._ptr(conv_state), self._ptr(delta),
+            self._ptr(delta_bias), int(bool(softplus)), self._ptr(A), self._ptr(B), self._ptr(C),
+            self._ptr(D), self._ptr(z), self._ptr(h0), code, batch, L, dim, N, self._ptr(out),
+            self._ptr(hl), self._ptr(st), int(threads))
+        if rc != 0:
+            raise ValueError("oracle rejected the arguments")
+        return out, hl, st
+
+    def conv_step(self, conv_state, state, x, w, cbias, delta, delta_bias, softplus, A, B, C, D, z,
+                  threads=0):
+        """One decode step of convolution + scan.  conv_state ([b,d,K-1]) and
+        state ([b,d,N]), both contiguous float64, are updated in place.
+        Returns out [b,d] float64."""
+        for name, a in (("conv_state", conv_state), ("state", state)):
+            if a.dtype != np.float64 or not a.flags.c_contiguous:
+                raise TypeError(f"{name} must be a contiguous float64 array")
+        code = self._dtype_code(x)
+        x, delta, B, C, z = (self._act(t, code) for t in (x, delta, B, C, z))
+        w, cbias, A, D, delta_bias = (self._f32(t) for t in (w, cbias, A, D, delta_bias))
+        batch, dim = x.shape
+        N, K = A.shape[1], w.shape[1]
+        out = np.empty((batch, dim), np.float64)
+        rc = self._lib.ssm_ref_conv_step(
+            self._ptr(conv_state), self._ptr(state), self._ptr(x), self._ptr(w), self._ptr(cbias), K,
+            self._ptr(delta), self._ptr(delta_bias), int(bool(softplus)), self._ptr(A), self._ptr(B),
+            self._ptr(C), self._ptr(D), self._ptr(z), code, batch, dim, N, self._ptr(out), int(threads))
+        if rc != 0:
+            raise ValueError("oracle rejected the arguments")
+        return out
+
+
 def load(path: str | None = None) -> Oracle:
     """Build (if needed) and load the oracle library; cached per process."""
     global _lib
@@ -170,3 +243,15 @@ def fwd_channels(*args, **kw):
 
 def step(*args, **kw):
     return load().step(*args, **kw)
+
+
+def conv1d(*args, **kw):
+    return load().conv1d(*args, **kw)
+
+
+def conv_fwd(*args, **kw):
+    return load().conv_fwd(*args, **kw)
+
+
+def conv_step(*args, **kw):
+    return load().conv_step(*args, **kw)

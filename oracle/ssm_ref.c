@@ -92,8 +92,11 @@ typedef struct {
 } ref_args;
 
 /* The recurrence for one channel (b, d) over all t.  out_row gets seqlen
- * values (stride 1); hl gets dstate values (may be NULL). */
-static void scan_channel(const ref_args *a, int64_t b, int64_t d, double *out_row, double *hl)
+ * values (stride 1); hl gets dstate values (may be NULL).  xrow, when not
+ * NULL, holds the channel's x values in double precision (the output of the
+ * causal convolution in front of the scan) and replaces the stored x. */
+static void scan_channel_x(const ref_args *a, int64_t b, int64_t d, const double *xrow, double *out_row,
+                           double *hl)
 {
     const int64_t L = a->seqlen, N = a->dstate, Dm = a->dim;
     double h[REF_MAX_DSTATE];
@@ -106,7 +109,7 @@ static void scan_channel(const ref_args *a, int64_t b, int64_t d, double *out_ro
         if (a->delta_bias)
             v += (double)a->delta_bias[d];
         const double dt = a->softplus ? softplus_ref(v) : v;
-        const double xt = load_act(a->x, chan * L + t, a->dtype);
+        const double xt = xrow ? xrow[t] : load_act(a->x, chan * L + t, a->dtype);
 
         for (int64_t n = 0; n < N; n++) {
             const double abar = exp(dt * (double)a->A[d * N + n]);
@@ -125,6 +128,11 @@ static void scan_channel(const ref_args *a, int64_t b, int64_t d, double *out_ro
     if (hl)
         for (int64_t n = 0; n < N; n++)
             hl[n] = h[n];
+}
+
+static void scan_channel(const ref_args *a, int64_t b, int64_t d, double *out_row, double *hl)
+{
+    scan_channel_x(a, b, d, NULL, out_row, hl);
 }
 
 static int check_dims(int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate)
@@ -211,6 +219,161 @@ int ssm_ref_step(double *state, const void *x, const void *delta, const float *d
             v += (double)delta_bias[d];
         const double dt = softplus ? softplus_ref(v) : v;
         const double xt = load_act(x, c, dtype);
+        double y = 0.0;
+        for (int64_t n = 0; n < dstate; n++) {
+            const double abar = exp(dt * (double)A[d * dstate + n]);
+            h[n] = abar * h[n] + dt * load_act(B, b * dstate + n, dtype) * xt;
+        }
+        for (int64_t n = 0; n < dstate; n++)
+            y += load_act(C, b * dstate + n, dtype) * h[n];
+        if (D)
+            y += (double)D[d] * xt;
+        if (z)
+            y *= silu_ref(load_act(z, c, dtype));
+        out[c] = y;
+    }
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * Short causal convolution in front of the scan.
+ *
+ * Gu & Dao, "Mamba", Appendix D "Hardware-aware Algorithm For Selective
+ * SSMs", paragraph "Memory": the block runs input projection, convolution,
+ * activation, scan, output projection; "A Secret Weapon For mamba paper"
+ * names the causal_conv1d kernels; "Rumored Buzz on mamba paper": the
+ * inference cache holds the convolution state beside the SSM state.  The
+ * pages print no formula; the plain reading is a depthwise causal convolution
+ * of width K over each channel's sequence followed by silu:
+ *
+ *   xc[b,d,t] = silu( sum_{k=0}^{K-1} w[d,k] * xin(b,d,t-K+1+k) + bias[d] )
+ *
+ * (w[d,K-1] multiplies the current input), where xin(b,d,s) = x[b,d,s] for
+ * s >= 0 and conv_state[b,d,K-1+s] for -(K-1) <= s < 0: the K-1 inputs that
+ * came before this call (zero when conv_state is NULL).  After the call the
+ * state holds xin(b,d,L-K+1 .. L-1), the last K-1 inputs.
+ *
+ * Storage: w [dim][K] float32, bias [dim] float32 (NULL = 0), conv_state
+ * [batch][dim][K-1] in the activation dtype for the input (its values are
+ * raw inputs), double for the output.
+ */
+#define REF_MAX_CONV 64
+
+/* xin(b,d,s) of one channel, for -(K-1) <= s < L */
+static double conv_input(const void *x, const void *conv_state, int dtype, int64_t chan, int64_t L,
+                         int64_t K, int64_t s)
+{
+    if (s >= 0)
+        return load_act(x, chan * L + s, dtype);
+    if (!conv_state)
+        return 0.0;
+    return load_act(conv_state, chan * (K - 1) + (K - 1 + s), dtype);
+}
+
+/* The convolution of one channel: xc[0..L) (with silu when `silu`), and the
+ * channel's new state (K-1 values) into state_out when not NULL. */
+static void conv_channel(const void *x, const float *w, const float *bias, int64_t K,
+                         const void *conv_state, int silu, int dtype, int64_t chan, int64_t d,
+                         int64_t L, double *xc, double *state_out)
+{
+    for (int64_t t = 0; t < L; t++) {
+        double acc = bias ? (double)bias[d] : 0.0;
+        for (int64_t k = 0; k < K; k++)
+            acc += (double)w[d * K + k] * conv_input(x, conv_state, dtype, chan, L, K, t - K + 1 + k);
+        xc[t] = silu ? silu_ref(acc) : acc;
+    }
+    if (state_out)
+        for (int64_t j = 0; j < K - 1; j++)
+            state_out[j] = conv_input(x, conv_state, dtype, chan, L, K, L - (K - 1) + j);
+}
+
+/* The convolution alone.  xc: [batch][dim][seqlen] double; state_out:
+ * [batch][dim][K-1] double or NULL.  Returns 0, or 1 on bad sizes. */
+int ssm_ref_conv1d(const void *x, const float *w, const float *bias, int64_t K, const void *conv_state,
+                   int silu, int dtype, int64_t batch, int64_t seqlen, int64_t dim, double *xc,
+                   double *state_out, int nthreads)
+{
+    if (check_dims(batch, seqlen, dim, 1) || K < 1 || K > REF_MAX_CONV || !x || !w || !xc)
+        return 1;
+    set_threads(nthreads);
+    const int64_t nchan = batch * dim;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t c = 0; c < nchan; c++)
+        conv_channel(x, w, bias, K, conv_state, silu, dtype, c, c % dim, seqlen, xc + c * seqlen,
+                     state_out ? state_out + c * (K - 1) : NULL);
+    return 0;
+}
+
+/* Convolution + silu, then the scan on its output (the fused block path):
+ * the same outputs as ssm_ref_fwd with x replaced by xc, plus the new
+ * convolution state.  out: [batch][dim][seqlen]; h_last: [batch][dim][dstate]
+ * or NULL; state_out: [batch][dim][K-1] or NULL (all double). */
+int ssm_ref_conv_fwd(const void *x, const float *w, const float *cbias, int64_t K, const void *conv_state,
+                     const void *delta, const float *delta_bias, int softplus, const float *A,
+                     const void *B, const void *C, const float *D, const void *z, const float *h0,
+                     int dtype, int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
+                     double *out, double *h_last, double *state_out, int nthreads)
+{
+    if (check_dims(batch, seqlen, dim, dstate) || K < 1 || K > REF_MAX_CONV || !x || !w || !delta ||
+        !A || !B || !C || !out)
+        return 1;
+    const ref_args a = {x, delta, delta_bias, softplus, A, B, C, D, z, h0, dtype,
+                        batch, seqlen, dim, dstate};
+    set_threads(nthreads);
+    const int64_t nchan = batch * dim;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t c = 0; c < nchan; c++) {
+        double *xc = (double *)malloc((size_t)seqlen * sizeof(double));
+        if (!xc) {
+#pragma omp atomic write
+            bad = 1;
+            continue;
+        }
+        conv_channel(x, w, cbias, K, conv_state, 1, dtype, c, c % dim, seqlen, xc,
+                     state_out ? state_out + c * (K - 1) : NULL);
+        scan_channel_x(&a, c / dim, c % dim, xc, out + c * seqlen, h_last ? h_last + c * dstate : NULL);
+        free(xc);
+    }
+    return bad ? 2 : 0;
+}
+
+/* One decode step of the fused block: the convolution window is the channel's
+ * K-1 stored inputs followed by this token's x; xc = silu(window . w + bias);
+ * the state shifts by one input; then the SSM step of ssm_ref_step with x = xc.
+ * conv_state: [batch][dim][K-1] double, read and written; state:
+ * [batch][dim][dstate] double, read and written; out: [batch][dim] double. */
+int ssm_ref_conv_step(double *conv_state, double *state, const void *x, const float *w,
+                      const float *cbias, int64_t K, const void *delta, const float *delta_bias,
+                      int softplus, const float *A, const void *B, const void *C, const float *D,
+                      const void *z, int dtype, int64_t batch, int64_t dim, int64_t dstate,
+                      double *out, int nthreads)
+{
+    if (check_dims(batch, 1, dim, dstate) || K < 1 || K > REF_MAX_CONV || !conv_state || !state ||
+        !x || !w || !delta || !A || !B || !C || !out)
+        return 1;
+    set_threads(nthreads);
+    const int64_t nchan = batch * dim;
+#pragma omp parallel for schedule(static)
+    for (int64_t c = 0; c < nchan; c++) {
+        const int64_t b = c / dim, d = c % dim;
+        double *cs = conv_state + c * (K - 1);
+        const double xt_raw = load_act(x, c, dtype);
+        double acc = cbias ? (double)cbias[d] : 0.0;
+        for (int64_t k = 0; k < K - 1; k++)
+            acc += (double)w[d * K + k] * cs[k];
+        acc += (double)w[d * K + K - 1] * xt_raw;
+        for (int64_t k = 0; k + 1 < K - 1; k++)
+            cs[k] = cs[k + 1];
+        if (K > 1)
+            cs[K - 2] = xt_raw;
+        const double xt = silu_ref(acc);
+
+        double *h = state + c * dstate;
+        double v = load_act(delta, c, dtype);
+        if (delta_bias)
+            v += (double)delta_bias[d];
+        const double dt = softplus ? softplus_ref(v) : v;
         double y = 0.0;
         for (int64_t n = 0; n < dstate; n++) {
             const double abar = exp(dt * (double)A[d * dstate + n]);

@@ -343,6 +343,125 @@ def pin_step_equals_scan(orc):
     _close(h, hl.reshape(6, 4)[sel], rtol=0, atol=0, what="channel subset h")
 
 
+# ---------------------------------------------------------------------------
+# The short causal convolution in front of the scan (convolution, activation,
+# then the scan: Mamba, Appendix D "Memory").
+
+def _conv_case(seed, b=2, d=3, n=4, L=11, K=4, state=True):
+    r = _rng(seed)
+    c = _rand_case(seed, b=b, d=d, n=n, L=L)
+    c["w"] = _f32(r.standard_normal((d, K)) * 0.7)
+    c["cbias"] = _f32(r.standard_normal(d) * 0.3)
+    c["conv_state"] = _f32(r.standard_normal((b, d, K - 1))) if (state and K > 1) else None
+    return c
+
+
+def _conv_fwd(orc, c, **over):
+    a = dict(c)
+    a.update(over)
+    return orc.conv_fwd(a["x"], a["w"], a["cbias"], a["conv_state"], a["delta"], a["delta_bias"],
+                        a["softplus"], a["A"], a["B"], a["C"], a["D"], a["z"], a["h0"])
+
+
+def pin_conv_numpy_convolve(orc):
+    """The convolution is numpy.convolve of the state-padded row with the
+    reversed taps (the last tap multiplies the current input), plus the bias,
+    then silu (scipy's expit); the new state is the last K-1 inputs."""
+    for K, L, state in ((4, 11, True), (4, 2, True), (3, 9, False), (1, 5, False), (2, 1, True)):
+        c = _conv_case(50 + K + L, K=K, L=L, state=state)
+        xc, st = orc.conv1d(c["x"], c["w"], c["cbias"], c["conv_state"], silu=True)
+        pre, _ = orc.conv1d(c["x"], c["w"], c["cbias"], c["conv_state"], silu=False)
+        b, d, _ = c["x"].shape
+        for bi in range(b):
+            for di in range(d):
+                hist = (c["conv_state"][bi, di].astype(np.float64) if c["conv_state"] is not None
+                        else np.zeros(K - 1))
+                row = np.concatenate([hist, c["x"][bi, di].astype(np.float64)])
+                want = np.convolve(row, c["w"][di, ::-1].astype(np.float64), mode="valid") + c["cbias"][di]
+                _close(pre[bi, di], want, rtol=1e-13, atol=1e-14, what=f"conv K={K} L={L}")
+                _close(xc[bi, di], want * expit(want), rtol=1e-13, atol=1e-14, what=f"conv silu K={K}")
+                _close(st[bi, di], row[len(row) - (K - 1):], rtol=0, atol=0, what=f"conv state K={K} L={L}")
+
+
+def pin_conv_impulse(orc):
+    """Brute force on the tap order: a unit impulse at step s, zero bias and
+    no silu, gives w[d, K-1-j] at step s+j for j < K and zero elsewhere; an
+    impulse held in the state (j steps before the call) appears at t = K-2-j."""
+    K, L = 4, 9
+    w = _f32(np.arange(1, 2 * K + 1, dtype=np.float32).reshape(2, K))
+    for s in range(L):
+        x = np.zeros((1, 2, L), np.float32)
+        x[0, :, s] = 1.0
+        pre, _ = orc.conv1d(x, w, None, None, silu=False)
+        for di in range(2):
+            want = np.zeros(L)
+            for j in range(K):
+                if s + j < L:
+                    want[s + j] = w[di, K - 1 - j]
+            _close(pre[0, di], want, rtol=0, atol=0, what=f"impulse at {s}")
+    for j in range(K - 1):
+        st = np.zeros((1, 2, K - 1), np.float32)
+        st[0, :, K - 2 - j] = 1.0  # the input j steps before t = 0
+        pre, _ = orc.conv1d(np.zeros((1, 2, L), np.float32), w, None, st, silu=False)
+        for di in range(2):
+            want = np.zeros(L)
+            for t in range(L):
+                k = K - 1 - (t + 1 + j)  # the impulse sits at s = -1 - j
+                if 0 <= k < K:
+                    want[t] = w[di, k]
+            _close(pre[0, di], want, rtol=0, atol=0, what=f"state impulse {j}")
+
+
+def pin_conv_feeds_scan(orc):
+    """The fused path is the composition of the convolution (pinned above) and
+    the scan (pinned by the pins before): conv_fwd equals fwd run on the
+    convolution's output, up to the float32 rounding of that output."""
+    for K in (4, 1):
+        c = _conv_case(60 + K, K=K, L=13)
+        out, hl, st = _conv_fwd(orc, c)
+        xc, st2 = orc.conv1d(c["x"], c["w"], c["cbias"], c["conv_state"], silu=True)
+        o2, h2 = _call(orc, c, x=_f32(xc))
+        _close(out, o2, rtol=1e-6, atol=1e-6, what=f"conv then scan K={K}")
+        _close(hl, h2, rtol=1e-6, atol=1e-6, what=f"conv then scan h K={K}")
+        _close(st, st2, rtol=0, atol=0, what=f"conv then scan state K={K}")
+
+
+def pin_conv_split(orc):
+    """Two calls continue one: [0, m) and then [m, L) with the new convolution
+    state and h_last carried over equal one call over [0, L), including splits
+    shorter than the convolution window."""
+    c = _conv_case(70, L=17, K=4)
+    out, hl, st = _conv_fwd(orc, c)
+    seq_keys = ("x", "delta", "z", "B", "C")
+    for m in (1, 2, 3, 8, 16):
+        first = {k: (np.ascontiguousarray(v[..., :m]) if k in seq_keys else v) for k, v in c.items()}
+        second = {k: (np.ascontiguousarray(v[..., m:]) if k in seq_keys else v) for k, v in c.items()}
+        o1, h1, s1 = _conv_fwd(orc, first)
+        second["h0"] = _f32(h1)
+        second["conv_state"] = _f32(s1)  # raw float32 inputs: exact
+        o2, h2, s2 = _conv_fwd(orc, second)
+        _close(o1, out[..., :m], rtol=1e-12, what=f"conv split m={m} first")
+        _close(o2, out[..., m:], rtol=2e-5, atol=2e-5, what=f"conv split m={m} second")
+        _close(h2, hl, rtol=2e-5, atol=2e-5, what=f"conv split m={m} h_last")
+        _close(s2, st, rtol=0, atol=0, what=f"conv split m={m} state")
+
+
+def pin_conv_step_equals_fwd(orc):
+    """The recurrent mode of the block: T single steps (convolution window from
+    the carried inputs, then the SSM step) equal one call over T tokens."""
+    c = _conv_case(80, L=7, K=4)
+    out, hl, st = _conv_fwd(orc, c)
+    cs = c["conv_state"].astype(np.float64).copy()
+    state = c["h0"].astype(np.float64).copy()
+    for t in range(7):
+        tok = {k: np.ascontiguousarray(c[k][..., t]) for k in ("x", "delta", "z", "B", "C")}
+        o = orc.conv_step(cs, state, tok["x"], c["w"], c["cbias"], tok["delta"], c["delta_bias"], True,
+                          c["A"], tok["B"], tok["C"], c["D"], tok["z"])
+        _close(o, out[..., t], rtol=1e-13, atol=1e-15, what=f"conv step t={t}")
+    _close(state, hl, rtol=1e-13, what="conv step state")
+    _close(cs, st, rtol=0, atol=0, what="conv step window")
+
+
 ALL_PINS = [
     pin_single_step_closed_form,
     pin_hand_values,
@@ -355,4 +474,9 @@ ALL_PINS = [
     pin_softplus_extremes,
     pin_bf16_widening,
     pin_step_equals_scan,
+    pin_conv_numpy_convolve,
+    pin_conv_impulse,
+    pin_conv_feeds_scan,
+    pin_conv_split,
+    pin_conv_step_equals_fwd,
 ]

@@ -27,8 +27,8 @@ MUTANTS = [
      "y += load_act(a->B, (b * N + n) * L + t, a->dtype) * h[n];"),
     ("B read transposed [b][t][n]", "load_act(a->B, (b * N + n) * L + t, a->dtype);",
      "load_act(a->B, (b * L + t) * N + n, a->dtype);"),
-    ("x read one step late", "const double xt = load_act(a->x, chan * L + t, a->dtype);",
-     "const double xt = load_act(a->x, chan * L + (t + 1 < L ? t + 1 : t), a->dtype);"),
+    ("x read one step late", "const double xt = xrow ? xrow[t] : load_act(a->x, chan * L + t, a->dtype);",
+     "const double xt = xrow ? xrow[t] : load_act(a->x, chan * L + (t + 1 < L ? t + 1 : t), a->dtype);"),
     ("C readout dropped", "        double y = 0.0;\n        for (int64_t n = 0; n < N; n++)\n            y += load_act(a->C",
      "        double y = 0.0;\n        for (int64_t n = 0; n < N; n++)\n            y += 0.0 * load_act(a->C"),
     ("state decays twice", "h[n] = abar * h[n] + dt * bt * xt;", "h[n] = abar * abar * h[n] + dt * bt * xt;"),
@@ -37,6 +37,21 @@ MUTANTS = [
      "            hl[n] = a->h0 ? (double)a->h0[chan * N + n] : 0.0;"),
     ("step ignores gate", "            y *= silu_ref(load_act(z, c, dtype));", "            y *= 1.0;"),
     ("channel index b/d swapped", "scan_channel(&a, c / dim, c % dim,", "scan_channel(&a, c % batch, c / batch,"),
+    # the causal convolution in front of the scan
+    ("conv taps reversed", "acc += (double)w[d * K + k] * conv_input(",
+     "acc += (double)w[d * K + (K - 1 - k)] * conv_input("),
+    ("conv state ignored", "    if (!conv_state)\n        return 0.0;", "    if (1)\n        return 0.0;"),
+    ("conv window one step late", "conv_input(x, conv_state, dtype, chan, L, K, t - K + 1 + k);",
+     "conv_input(x, conv_state, dtype, chan, L, K, t - K + k);"),
+    ("conv bias dropped", "        double acc = bias ? (double)bias[d] : 0.0;\n        for (int64_t k = 0; k < K; k++)",
+     "        double acc = 0.0;\n        for (int64_t k = 0; k < K; k++)"),
+    ("conv output not activated", "conv_channel(x, w, cbias, K, conv_state, 1, dtype,",
+     "conv_channel(x, w, cbias, K, conv_state, 0, dtype,"),
+    ("conv scan reads raw x", "scan_channel_x(&a, c / dim, c % dim, xc,", "scan_channel_x(&a, c / dim, c % dim, NULL,"),
+    ("new conv state one input early", "conv_input(x, conv_state, dtype, chan, L, K, L - (K - 1) + j);",
+     "conv_input(x, conv_state, dtype, chan, L, K, L - K + j);"),
+    ("conv step does not shift", "            cs[k] = cs[k + 1];", "            cs[k] = cs[k];"),
+    ("conv step window reversed", "acc += (double)w[d * K + k] * cs[k];", "acc += (double)w[d * K + k] * cs[K - 2 - k];"),
 ]
 
 

@@ -154,6 +154,53 @@ int ssm_scan_step(float *state, const void *x, const void *delta, const float *d
                   const ssm_dims_t *dims, ssm_stream_t stream);
 
 /*
+ * The block's short causal convolution and activation fused in front of the
+ * forward scan (Appendix D "Memory": input projection, convolution,
+ * activation, scan, output projection; the convolution's output never goes
+ * to device memory).  The scan runs on
+ *
+ *   xc[b,d,t] = silu( sum_{k<K} conv_w[d,k] * xin(b,d,t-K+1+k) + conv_bias[d] )
+ *
+ * in place of x, where xin(b,d,s) = x[b,d,s] for s >= 0 and the stored input
+ * conv_state[b,d,K-1+s] for -(K-1) <= s < 0 (zero when conv_state is NULL).
+ * The D skip uses xc, rounded to the activation dtype.
+ *
+ *   x              required [batch][dim][seqlen], the raw input
+ *   conv_w         required [dim][conv_width] float32 (conv_w[d][conv_width-1]
+ *                  multiplies the current input), 4-byte aligned
+ *   conv_bias      optional [dim] float32 (NULL = 0), 4-byte aligned
+ *   conv_width     K, 1..4
+ *   conv_state     optional [batch][dim][K-1] activation dtype: the K-1 raw
+ *                  inputs before t = 0, oldest first (NULL = zeros)
+ *   conv_state_out optional [batch][dim][K-1] activation dtype: receives the
+ *                  last K-1 raw inputs (the window for the next call or for
+ *                  ssm_conv_scan_step); may be conv_state itself
+ * The remaining arguments, the workspace, errors and ssm_scan_fwd_status are
+ * those of ssm_scan_fwd.
+ */
+int ssm_conv_scan_fwd(const void *x, const float *conv_w, const float *conv_bias, int conv_width,
+                      const void *conv_state, void *conv_state_out,
+                      const void *delta, const float *delta_bias, int softplus,
+                      const float *A, const void *B, const void *C, const float *D,
+                      const void *z, const float *h0, void *out, float *h_last,
+                      void *workspace, size_t workspace_bytes,
+                      const ssm_dims_t *dims, ssm_stream_t stream);
+
+/*
+ * One decode step of the same block: the token x passes the convolution
+ * window (the K-1 stored raw inputs followed by x), silu, then the recurrent
+ * step of ssm_scan_step.  conv_state ([batch][dim][K-1], activation dtype,
+ * element aligned; required when K > 1) is read and shifted in place: its
+ * oldest input is dropped and x appended.  Other arguments as for
+ * ssm_scan_step and ssm_conv_scan_fwd.
+ */
+int ssm_conv_scan_step(void *conv_state, float *state, const void *x, const float *conv_w,
+                       const float *conv_bias, int conv_width, const void *delta,
+                       const float *delta_bias, int softplus, const float *A, const void *B,
+                       const void *C, const float *D, const void *z, void *out,
+                       const ssm_dims_t *dims, ssm_stream_t stream);
+
+/*
  * ssm_scan_fwd without a workspace.  The pages have no counterpart: this
  * entry point exists for callers that cannot allocate any device memory while
  * they run the scan, not even a workspace (code running inside an allocator or

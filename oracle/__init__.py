@@ -64,6 +64,10 @@ class Oracle:
         lib.ssm_ref_conv_fwd.restype = I
         lib.ssm_ref_conv_step.argtypes = [P, P, P, P, P, L, P, P, I, P, P, P, P, P, I, L, L, L, P, I]
         lib.ssm_ref_conv_step.restype = I
+        lib.ssm_ref_trap_fwd.argtypes = [P, P, P, I, P, P, P, P, P, P, P, P, P, I, L, L, L, L, P, P, I]
+        lib.ssm_ref_trap_fwd.restype = I
+        lib.ssm_ref_trap_step.argtypes = [P, P, P, P, I, P, P, P, P, P, P, P, P, I, L, L, L, P, I]
+        lib.ssm_ref_trap_step.restype = I
         self._lib = lib
 
     # -- marshalling helpers ---------------------------------------------
@@ -223,6 +227,51 @@ class Oracle:
         return out
 
 
+    # -- the exponential-trapezoidal rule (Mamba-3) -------------------------
+    def trap_fwd(self, x, delta, delta_bias, softplus, lam, A, B, C, D, z, h0, x_prev=None, B_prev=None,
+                 threads=0):
+        """Scan with the exponential-trapezoidal discretisation.  lam: [b,d,L]
+        stored activations; x_prev [b,d] and B_prev [b,N]: the input before
+        t = 0 (None: zero).  Returns (out [b,d,L], h_last [b,d,N]), float64."""
+        code = self._dtype_code(x)
+        x, delta, lam, B, C, z, x_prev, B_prev = (self._act(t, code) for t in
+                                                  (x, delta, lam, B, C, z, x_prev, B_prev))
+        A, D, delta_bias, h0 = (self._f32(t) for t in (A, D, delta_bias, h0))
+        batch, dim, L = x.shape
+        N = A.shape[1]
+        out = np.empty((batch, dim, L), np.float64)
+        hl = np.empty((batch, dim, N), np.float64)
+        rc = self._lib.ssm_ref_trap_fwd(
+            self._ptr(x), self._ptr(delta), self._ptr(delta_bias), int(bool(softplus)), self._ptr(lam),
+            self._ptr(A), self._ptr(B), self._ptr(C), self._ptr(D), self._ptr(z), self._ptr(h0),
+            self._ptr(x_prev), self._ptr(B_prev), code, batch, L, dim, N, self._ptr(out), self._ptr(hl),
+            int(threads))
+        if rc != 0:
+            raise ValueError("oracle rejected the arguments")
+        return out, hl
+
+    def trap_step(self, state, x, delta, delta_bias, softplus, lam, A, B, C, D, z, x_prev=None,
+                  B_prev=None, threads=0):
+        """One trapezoidal decode step; `state` ([b,d,N] float64) is updated in
+        place.  x_prev [b,d], B_prev [b,N]: the previous token's.  Returns out."""
+        if state.dtype != np.float64 or not state.flags.c_contiguous:
+            raise TypeError("state must be a contiguous float64 array")
+        code = self._dtype_code(x)
+        x, delta, lam, B, C, z, x_prev, B_prev = (self._act(t, code) for t in
+                                                  (x, delta, lam, B, C, z, x_prev, B_prev))
+        A, D, delta_bias = (self._f32(t) for t in (A, D, delta_bias))
+        batch, dim = x.shape
+        N = A.shape[1]
+        out = np.empty((batch, dim), np.float64)
+        rc = self._lib.ssm_ref_trap_step(
+            self._ptr(state), self._ptr(x), self._ptr(delta), self._ptr(delta_bias), int(bool(softplus)),
+            self._ptr(lam), self._ptr(A), self._ptr(B), self._ptr(C), self._ptr(D), self._ptr(z),
+            self._ptr(x_prev), self._ptr(B_prev), code, batch, dim, N, self._ptr(out), int(threads))
+        if rc != 0:
+            raise ValueError("oracle rejected the arguments")
+        return out
+
+
 def load(path: str | None = None) -> Oracle:
     """Build (if needed) and load the oracle library; cached per process."""
     global _lib
@@ -255,3 +304,11 @@ def conv_fwd(*args, **kw):
 
 def conv_step(*args, **kw):
     return load().conv_step(*args, **kw)
+
+
+def trap_fwd(*args, **kw):
+    return load().trap_fwd(*args, **kw)
+
+
+def trap_step(*args, **kw):
+    return load().trap_step(*args, **kw)

@@ -389,3 +389,130 @@ int ssm_ref_conv_step(double *conv_state, double *state, const void *x, const fl
     }
     return 0;
 }
+
+/* ---------------------------------------------------------------------------
+ * Exponential-trapezoidal discretisation (Mamba-3).
+ *
+ * The "Mamba3" posts (tginsight), section on the new discretisation scheme:
+ * Mamba-1/2 combine zero-order hold and Euler; Mamba-3 approximates the
+ * integral of the state update with both ends of the interval, mixed by a
+ * data-dependent coefficient lambda, which is a second-order rule.  The pages
+ * print no formula; the plain reading of that description, for
+ * h'(s) = A h(s) + B(s) x(s) over a step of length dt, is
+ *
+ *   h_t = alpha_t h_{t-1} + beta_t B_{t-1} x_{t-1} + gamma_t B_t x_t
+ *   alpha_t = exp(dt_t A),  beta_t = (1 - lambda_t) dt_t alpha_t,  gamma_t = lambda_t dt_t
+ *
+ * (the integrand exp((t - s) A) B(s) x(s) taken at the interval's start,
+ * weight 1 - lambda, and at its end, weight lambda).  lambda = 1 is the
+ * Euler input step of Mamba-1; lambda = 1/2 is the trapezoidal rule.  The
+ * input before t = 0 is x_prev[b,d] B_prev[b,:] (zero when either is NULL),
+ * which lets a sequence be split into calls.
+ *
+ * Storage: lam [batch][dim][seqlen] activation dtype; x_prev [batch][dim] and
+ * B_prev [batch][dstate] activation dtype; everything else as ssm_ref_fwd.
+ */
+static void trap_channel(const ref_args *a, const void *lam, const void *x_prev, const void *B_prev,
+                         int64_t b, int64_t d, double *out_row, double *hl)
+{
+    const int64_t L = a->seqlen, N = a->dstate, Dm = a->dim;
+    double h[REF_MAX_DSTATE], vprev[REF_MAX_DSTATE];
+    const int64_t chan = b * Dm + d;
+    const double xp = (x_prev && B_prev) ? load_act(x_prev, chan, a->dtype) : 0.0;
+    for (int64_t n = 0; n < N; n++) {
+        h[n] = a->h0 ? (double)a->h0[chan * N + n] : 0.0;
+        vprev[n] = (x_prev && B_prev) ? load_act(B_prev, b * N + n, a->dtype) * xp : 0.0;
+    }
+    for (int64_t t = 0; t < L; t++) {
+        double v = load_act(a->delta, chan * L + t, a->dtype);
+        if (a->delta_bias)
+            v += (double)a->delta_bias[d];
+        const double dt = a->softplus ? softplus_ref(v) : v;
+        const double lt = load_act(lam, chan * L + t, a->dtype);
+        const double xt = load_act(a->x, chan * L + t, a->dtype);
+        for (int64_t n = 0; n < N; n++) {
+            const double alpha = exp(dt * (double)a->A[d * N + n]);
+            const double beta = (1.0 - lt) * dt * alpha;
+            const double gamma = lt * dt;
+            const double vt = load_act(a->B, (b * N + n) * L + t, a->dtype) * xt;
+            h[n] = alpha * h[n] + beta * vprev[n] + gamma * vt;
+            vprev[n] = vt;
+        }
+        double y = 0.0;
+        for (int64_t n = 0; n < N; n++)
+            y += load_act(a->C, (b * N + n) * L + t, a->dtype) * h[n];
+        if (a->D)
+            y += (double)a->D[d] * xt;
+        if (a->z)
+            y *= silu_ref(load_act(a->z, chan * L + t, a->dtype));
+        out_row[t] = y;
+    }
+    if (hl)
+        for (int64_t n = 0; n < N; n++)
+            hl[n] = h[n];
+}
+
+int ssm_ref_trap_fwd(const void *x, const void *delta, const float *delta_bias, int softplus,
+                     const void *lam, const float *A, const void *B, const void *C, const float *D,
+                     const void *z, const float *h0, const void *x_prev, const void *B_prev, int dtype,
+                     int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
+                     double *out, double *h_last, int nthreads)
+{
+    if (check_dims(batch, seqlen, dim, dstate) || !x || !delta || !lam || !A || !B || !C || !out)
+        return 1;
+    const ref_args a = {x, delta, delta_bias, softplus, A, B, C, D, z, h0, dtype,
+                        batch, seqlen, dim, dstate};
+    set_threads(nthreads);
+    const int64_t nchan = batch * dim;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t c = 0; c < nchan; c++)
+        trap_channel(&a, lam, x_prev, B_prev, c / dim, c % dim, out + c * seqlen,
+                     h_last ? h_last + c * dstate : NULL);
+    return 0;
+}
+
+/* One recurrent step of the trapezoidal rule: the token's x, B, lambda and
+ * the previous token's x_prev [batch][dim] and B_prev [batch][dstate] (NULL:
+ * no previous input).  state: [batch][dim][dstate] double, read and written. */
+int ssm_ref_trap_step(double *state, const void *x, const void *delta, const float *delta_bias,
+                      int softplus, const void *lam, const float *A, const void *B, const void *C,
+                      const float *D, const void *z, const void *x_prev, const void *B_prev, int dtype,
+                      int64_t batch, int64_t dim, int64_t dstate, double *out, int nthreads)
+{
+    if (check_dims(batch, 1, dim, dstate) || !state || !x || !delta || !lam || !A || !B || !C || !out)
+        return 1;
+    set_threads(nthreads);
+    const int64_t nchan = batch * dim;
+#pragma omp parallel for schedule(static)
+    for (int64_t c = 0; c < nchan; c++) {
+        double hl[REF_MAX_DSTATE];
+        const int64_t b = c / dim, d = c % dim;
+        double *h = state + c * dstate;
+        double vprev[REF_MAX_DSTATE];
+        const double xp = (x_prev && B_prev) ? load_act(x_prev, c, dtype) : 0.0;
+        for (int64_t n = 0; n < dstate; n++)
+            vprev[n] = (x_prev && B_prev) ? load_act(B_prev, b * dstate + n, dtype) * xp : 0.0;
+        double v = load_act(delta, c, dtype);
+        if (delta_bias)
+            v += (double)delta_bias[d];
+        const double dt = softplus ? softplus_ref(v) : v;
+        const double lt = load_act(lam, c, dtype);
+        const double xt = load_act(x, c, dtype);
+        for (int64_t n = 0; n < dstate; n++) {
+            const double alpha = exp(dt * (double)A[d * dstate + n]);
+            const double vt = load_act(B, b * dstate + n, dtype) * xt;
+            hl[n] = alpha * h[n] + (1.0 - lt) * dt * alpha * vprev[n] + lt * dt * vt;
+        }
+        double y = 0.0;
+        for (int64_t n = 0; n < dstate; n++) {
+            h[n] = hl[n];
+            y += load_act(C, b * dstate + n, dtype) * h[n];
+        }
+        if (D)
+            y += (double)D[d] * xt;
+        if (z)
+            y *= silu_ref(load_act(z, c, dtype));
+        out[c] = y;
+    }
+    return 0;
+}

@@ -52,6 +52,10 @@ def _load():
     lib.ssm_scan_fwd_noalloc.restype = I
     lib.ssm_debug_fwd_flag_timeout.argtypes = [P, P, P, I, P, P, P, P, P, P, P, P, P, S, ctypes.c_uint32, DP, P]
     lib.ssm_debug_fwd_flag_timeout.restype = I
+    lib.ssm_conv_scan_fwd.argtypes = [P, P, P, I, P, P, P, P, I, P, P, P, P, P, P, P, P, P, S, DP, P]
+    lib.ssm_conv_scan_fwd.restype = I
+    lib.ssm_conv_scan_step.argtypes = [P, P, P, P, P, I, P, P, I, P, P, P, P, P, P, DP, P]
+    lib.ssm_conv_scan_step.restype = I
     lib.ssm_scan_step.argtypes = [P, P, P, P, I, P, P, P, P, P, P, DP, P]
     lib.ssm_scan_step.restype = I
     lib.ssm_strerror.argtypes = [I]
@@ -73,7 +77,8 @@ def get_lib():
 
 
 EXPORTS = ("ssm_scan_fwd_workspace_size", "ssm_scan_fwd", "ssm_scan_fwd_status", "ssm_scan_step",
-           "ssm_scan_fwd_noalloc", "ssm_debug_fwd_flag_timeout", "ssm_strerror", "ssm_version")
+           "ssm_conv_scan_fwd", "ssm_conv_scan_step", "ssm_scan_fwd_noalloc", "ssm_debug_fwd_flag_timeout",
+           "ssm_strerror", "ssm_version")
 
 
 def ssm_strerror(code: int) -> str:
@@ -203,6 +208,98 @@ def ssm_scan_fwd(x, delta, delta_bias, softplus, A, B, C, D=None, z=None, h0=Non
     return out, h_last
 
 
+def ssm_conv_scan_fwd(x, conv_w, conv_bias, conv_state, delta, delta_bias, softplus, A, B, C, D=None,
+                      z=None, h0=None, out=None, h_last=None, conv_state_out=None, return_conv_state=True,
+                      stream=None, workspace=None, check=False):
+    """Causal convolution (width conv_w.shape[1] <= 4) + silu fused in front of
+    the forward scan.  x is the raw input [batch, dim, L]; conv_w [dim, K] and
+    conv_bias [dim] float32; conv_state [batch, dim, K-1] in x's dtype (None:
+    zeros).  Returns (out, h_last, conv_state_out); the new convolution state
+    is written into ``conv_state_out`` (may be ``conv_state``) or a new tensor."""
+    if x.device.type != "cuda":
+        raise ValueError("ssm_conv_scan_fwd needs CUDA tensors")
+    dev = x.device
+    batch, dim, L = x.shape
+    code = _act_code(x)
+    act = x.dtype
+    f32 = torch.float32
+    K = int(conv_w.shape[1])
+    ptrs = dict(
+        x=_ptr(x, dtype=act, device=dev, name="x"),
+        w=_ptr(conv_w, dtype=f32, device=dev, shape=(dim, K), name="conv_w"),
+        cb=_ptr(conv_bias, dtype=f32, device=dev, shape=(dim,), name="conv_bias"),
+        cs=_ptr(conv_state, dtype=act, device=dev, shape=(batch, dim, K - 1), name="conv_state"),
+        delta=_ptr(delta, dtype=act, device=dev, shape=x.shape, name="delta"),
+        z=_ptr(z, dtype=act, device=dev, shape=x.shape, name="z"),
+        B=_ptr(B, dtype=act, device=dev, shape=(batch, DSTATE, L), name="B"),
+        C=_ptr(C, dtype=act, device=dev, shape=(batch, DSTATE, L), name="C"),
+        A=_ptr(A, dtype=f32, device=dev, shape=(dim, DSTATE), name="A"),
+        D=_ptr(D, dtype=f32, device=dev, shape=(dim,), name="D"),
+        delta_bias=_ptr(delta_bias, dtype=f32, device=dev, shape=(dim,), name="delta_bias"),
+        h0=_ptr(h0, dtype=f32, device=dev, shape=(batch, dim, DSTATE), name="h0"),
+    )
+    if out is None:
+        out = torch.empty_like(x)
+    if h_last is None:
+        h_last = torch.empty((batch, dim, DSTATE), dtype=f32, device=dev)
+    if conv_state_out is None and return_conv_state and K > 1:
+        conv_state_out = torch.empty((batch, dim, K - 1), dtype=act, device=dev)
+    po = _ptr(out, dtype=act, device=dev, shape=x.shape, name="out")
+    ph = _ptr(h_last, dtype=f32, device=dev, shape=(batch, dim, DSTATE), name="h_last")
+    pcs = _ptr(conv_state_out, dtype=act, device=dev, shape=(batch, dim, K - 1), name="conv_state_out")
+    dims = Dims(batch, L, dim, DSTATE, code)
+    if workspace is None:
+        workspace = torch.empty(ssm_scan_fwd_workspace_size(batch, L, dim, dev), dtype=torch.uint8,
+                                device=dev)
+    pw = _ptr(workspace, dtype=torch.uint8, device=dev, name="workspace")
+    sp = _stream_ptr(stream, dev)
+    with torch.cuda.device(dev):
+        rc = get_lib().ssm_conv_scan_fwd(ptrs["x"], ptrs["w"], ptrs["cb"], K, ptrs["cs"], pcs, ptrs["delta"],
+                                         ptrs["delta_bias"], int(bool(softplus)), ptrs["A"], ptrs["B"], ptrs["C"],
+                                         ptrs["D"], ptrs["z"], ptrs["h0"], po, ph, pw, workspace.numel(),
+                                         ctypes.byref(dims), sp)
+        _check(rc)
+        if check:
+            _check(get_lib().ssm_scan_fwd_status(pw, sp))
+    return out, h_last, conv_state_out
+
+
+def ssm_conv_scan_step(conv_state, state, x, conv_w, conv_bias, delta, delta_bias, softplus, A, B, C,
+                       D=None, z=None, out=None, stream=None):
+    """One decode step of convolution + scan; ``conv_state`` ([batch, dim,
+    K-1], x's dtype) and ``state`` ([batch, dim, 16] float32) are updated in
+    place.  Returns out [batch, dim]."""
+    if x.device.type != "cuda":
+        raise ValueError("ssm_conv_scan_step needs CUDA tensors")
+    dev = x.device
+    batch, dim = x.shape
+    code = _act_code(x)
+    act = x.dtype
+    f32 = torch.float32
+    K = int(conv_w.shape[1])
+    pcs = _ptr(conv_state, dtype=act, device=dev, shape=(batch, dim, K - 1), name="conv_state")
+    ps = _ptr(state, dtype=f32, device=dev, shape=(batch, dim, DSTATE), name="state")
+    px = _ptr(x, dtype=act, device=dev, name="x")
+    pw = _ptr(conv_w, dtype=f32, device=dev, shape=(dim, K), name="conv_w")
+    pcb = _ptr(conv_bias, dtype=f32, device=dev, shape=(dim,), name="conv_bias")
+    pd = _ptr(delta, dtype=act, device=dev, shape=x.shape, name="delta")
+    pz = _ptr(z, dtype=act, device=dev, shape=x.shape, name="z")
+    pB = _ptr(B, dtype=act, device=dev, shape=(batch, DSTATE), name="B")
+    pC = _ptr(C, dtype=act, device=dev, shape=(batch, DSTATE), name="C")
+    pA = _ptr(A, dtype=f32, device=dev, shape=(dim, DSTATE), name="A")
+    pD = _ptr(D, dtype=f32, device=dev, shape=(dim,), name="D")
+    pb = _ptr(delta_bias, dtype=f32, device=dev, shape=(dim,), name="delta_bias")
+    if out is None:
+        out = torch.empty_like(x)
+    po = _ptr(out, dtype=act, device=dev, shape=x.shape, name="out")
+    dims = Dims(batch, 1, dim, DSTATE, code)
+    with torch.cuda.device(dev):
+        rc = get_lib().ssm_conv_scan_step(pcs, ps, px, pw, pcb, K, pd, pb, int(bool(softplus)), pA, pB, pC,
+                                          pD, pz, po, ctypes.byref(dims), _stream_ptr(stream, dev))
+    _check(rc)
+    return out
+
+
 def ssm_scan_step(state, x, delta, delta_bias, softplus, A, B, C, D=None, z=None, out=None,
                   stream=None):
     """One recurrent decode step; ``state`` ([batch, dim, 16] float32) is
@@ -236,4 +333,5 @@ def ssm_scan_step(state, x, delta, delta_bias, softplus, A, B, C, D=None, z=None
 
 
 __all__ = ["ssm_scan_fwd", "ssm_scan_fwd_workspace_size", "ssm_scan_fwd_status", "ssm_scan_step",
+           "ssm_conv_scan_fwd", "ssm_conv_scan_step",
            "ssm_strerror", "ssm_version", "SSMError", "Dims", "LIB_PATH", "get_lib"]

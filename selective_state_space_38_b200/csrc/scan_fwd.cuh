@@ -60,6 +60,13 @@ struct FwdParams {
     // flag ever reaches, so the wait gives up deterministically.
     uint32_t spin_limit;
     uint32_t flag_bias;
+    // The short causal convolution in front of the scan (conv_k = 0: none).
+    // x is then the raw input, and the scan's x is silu(conv(x)), with
+    // conv_w[d][k] multiplying x[t - conv_k + 1 + k] (1 <= conv_k <= 4).
+    int conv_k;
+    const float *conv_w;        // [dim][conv_k]
+    const float *conv_bias;     // [dim] or NULL
+    const void *conv_state;     // [batch][dim][conv_k - 1] raw inputs before t = 0, or NULL
 };
 constexpr int kChained = 0, kSummary = 1, kFromStart = 2;
 
@@ -163,7 +170,28 @@ struct ChanConst {
     float2 a2_0x2;   // (a2_0, a2_0)
     float2 Dx2;      // (D[d], D[d])
     float2 biasx2;   // (bias[d], bias[d])
+    float cw[4];     // convolution taps (old to new), when the scan has a convolution in front
+    float cb;        // convolution bias
 };
+
+// The convolution's input history of a lane at a segment start t0: the three
+// raw inputs x[t0-3 .. t0-1], taken from x itself, from the stored state of
+// the K-1 inputs before t = 0, or zero.
+template <typename T>
+__device__ __forceinline__ void conv_halo(const FwdParams &p, int64_t b, int64_t d, int64_t t0, float (&halo)[3]) {
+    using AT = Act<T>;
+    const int64_t chan = b * p.dim + d;
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+        const int64_t s = t0 - 3 + i;
+        float v = 0.0f;
+        if (s >= 0)
+            v = AT::load(p.x, chan * p.seqlen + s);
+        else if (p.conv_state && s >= -(p.conv_k - 1))
+            v = AT::load(p.conv_state, chan * (p.conv_k - 1) + (p.conv_k - 1 + s));
+        halo[i] = v;
+    }
+}
 
 // ---- phase 1: per-step scalars of the chunk -----------------------------------
 // For every step t of the chunk: dt = softplus(delta + bias) (or delta + bias),
@@ -171,20 +199,57 @@ struct ChanConst {
 // (u, r) in ur[t][lane].  The work is laid out stage by stage over all step
 // pairs, so consecutive instructions are independent and the latency of each
 // special-function op is covered by the other pairs' work.
-template <typename T, bool S4D>
-__device__ __forceinline__ void chunk_prepass(const uint8_t *stage, float2 *ur, int row,
-                                              const ChanConst &cc, bool softplus) {
+// With CONV, x first becomes silu(conv(x)): the lane's raw row and the three
+// inputs before it (halo, updated to this chunk's last three) give the
+// convolution, whose output replaces the raw row in the stage (in the
+// activation dtype, for the post warp's D skip) and feeds u = dt x in float32.
+template <typename T, bool S4D, bool CONV>
+__device__ __forceinline__ void chunk_prepass(uint8_t *stage, float2 *ur, int row,
+                                              const ChanConst &cc, bool softplus, float (&halo)[3]) {
     using AT = Act<T>;
     constexpr bool kAccurate = AT::kBytes == 4;
     constexpr int PP = AT::kPerPiece, TC = FwdSmem<T>::kTC, NP = TC / 2;
     constexpr int TB = FwdSmem<T>::kTileBytes;
-    const uint8_t *xr = stage + row * kRowBytes;
+    uint8_t *xr = stage + row * kRowBytes;
     uint4 xv[kPieces], dv[kPieces];
 #pragma unroll
     for (int pc = 0; pc < kPieces; ++pc) {
         const int off = swz(row, pc) << 4;
         xv[pc] = *reinterpret_cast<const uint4 *>(xr + off);
         dv[pc] = *reinterpret_cast<const uint4 *>(xr + TB + off);
+    }
+    float XC[TC];  // the scan's x: the raw input, or the convolution's output
+#pragma unroll
+    for (int t = 0; t < TC; ++t) XC[t] = AT::piece(xv[t / PP], t % PP);
+    if constexpr (CONV) {
+        float raw[TC + 3];
+#pragma unroll
+        for (int i = 0; i < 3; ++i) raw[i] = halo[i];
+#pragma unroll
+        for (int t = 0; t < TC; ++t) raw[t + 3] = XC[t];
+#pragma unroll
+        for (int i = 0; i < 3; ++i) halo[i] = raw[TC + i];
+#pragma unroll
+        for (int t = 0; t < TC; ++t) {
+            float acc = cc.cb;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) acc = fmaf(cc.cw[k], raw[t + k], acc);
+            XC[t] = kAccurate ? acc * (1.0f / (1.0f + expf(-acc))) : silu_fast(acc);
+        }
+#pragma unroll
+        for (int pc = 0; pc < kPieces; ++pc) {
+            uint4 pk;
+            if constexpr (AT::kBytes == 2) {
+                const int t = pc * PP;
+                pk = make_uint4(pack_bf16x2(XC[t], XC[t + 1]), pack_bf16x2(XC[t + 2], XC[t + 3]),
+                                pack_bf16x2(XC[t + 4], XC[t + 5]), pack_bf16x2(XC[t + 6], XC[t + 7]));
+            } else {
+                const int t = pc * PP;
+                pk = make_uint4(__float_as_uint(XC[t]), __float_as_uint(XC[t + 1]), __float_as_uint(XC[t + 2]),
+                                __float_as_uint(XC[t + 3]));
+            }
+            *reinterpret_cast<uint4 *>(xr + (swz(row, pc) << 4)) = pk;
+        }
     }
     float2 V[NP], E[NP];
 #pragma unroll
@@ -226,8 +291,7 @@ __device__ __forceinline__ void chunk_prepass(const uint8_t *stage, float2 *ur, 
     }
 #pragma unroll
     for (int k = 0; k < NP; ++k) {
-        const int pc = (2 * k) / PP, i = (2 * k) % PP;
-        const float2 U = __fmul2_rn(V[k], make_float2(AT::piece(xv[pc], i), AT::piece(xv[pc], i + 1)));
+        const float2 U = __fmul2_rn(V[k], make_float2(XC[2 * k], XC[2 * k + 1]));
         ur[(2 * k) * 32 + row] = make_float2(U.x, E[k].x);
         ur[(2 * k + 1) * 32 + row] = make_float2(U.y, E[k].y);
     }
@@ -536,6 +600,13 @@ __device__ __forceinline__ ChanConst chan_const(const FwdParams &p, int64_t dc) 
     cc.a2_0x2 = make_float2(a2, a2);
     cc.Dx2 = make_float2(Dd, Dd);
     cc.biasx2 = make_float2(bias, bias);
+    // taps padded to four at the old end: cw[k] multiplies x[t - 3 + k]
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int kk = k - (4 - p.conv_k);
+        cc.cw[k] = (p.conv_k && kk >= 0) ? p.conv_w[dc * p.conv_k + kk] : 0.0f;
+    }
+    cc.cb = (p.conv_k && p.conv_bias) ? p.conv_bias[dc] : 0.0f;
     return cc;
 }
 
@@ -626,7 +697,7 @@ struct ChunkCursor {
 // sub-partition.  Two instances run back to back: the S4D one takes groups
 // whose A rows are all S4D-structured and marks the scratch when it meets
 // another group; the general one then takes those.
-template <typename T, bool VEC, bool S4D>
+template <typename T, bool VEC, bool S4D, bool CONV>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     scan_fwd_kernel(const FwdParams p, const FwdScratch sc, const __grid_constant__ TmaMaps tm) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -693,6 +764,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const bool softplus = p.softplus != 0;
         ChanConst cc;
         int64_t cc_d0 = -1;
+        float halo[3] = {0.0f, 0.0f, 0.0f};  // convolution inputs before the chunk (CONV)
         ChunkDesc dnext = cur.next(p, sc, counter, lane);
         issue(dnext, 0);
         for (int64_t j = 0;; ++j) {
@@ -714,7 +786,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     cc = chan_const(p, d < p.dim ? d : p.dim - 1);
                     cc_d0 = dj.d0;
                 }
-                chunk_prepass<T, S4D>(st, ur_of(j), lane, cc, softplus);
+                if (CONV && (dj.flags & kFirst)) {
+                    const int64_t d = dj.d0 + lane;
+                    conv_halo<T>(p, dj.b, d < p.dim ? d : p.dim - 1, dj.t0, halo);
+                }
+                chunk_prepass<T, S4D, CONV>(st, ur_of(j), lane, cc, softplus, halo);
             }
             if (lane == 0) ring[j & 3] = dj;
             __syncwarp();
@@ -895,6 +971,32 @@ __global__ void segment_combine_kernel(const FwdParams p, const FwdScratch sc) {
             h[4 * q + 3] = fmaf(pr.w, h[4 * q + 3], e.w);
         }
     }
+}
+
+// The convolution state after a forward call: the last K-1 raw inputs of
+// every channel, from x or (for sequences shorter than K-1) from the state
+// before the call.  One thread per channel reads all its values before it
+// writes, so the new state may overwrite the old one in place.
+template <typename T>
+__global__ void conv_state_kernel(const FwdParams p, void *state_out) {
+    using AT = Act<T>;
+    const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (c >= p.batch * p.dim) return;
+    const int K1 = p.conv_k - 1;
+    float v[3];
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+        v[j] = 0.0f;
+        if (j >= K1) continue;
+        const int64_t s = p.seqlen - K1 + j;
+        if (s >= 0)
+            v[j] = AT::load(p.x, c * p.seqlen + s);
+        else if (p.conv_state)
+            v[j] = AT::load(p.conv_state, c * K1 + (K1 + s));
+    }
+#pragma unroll
+    for (int j = 0; j < 3; ++j)
+        if (j < K1) AT::store(state_out, c * K1 + j, v[j]);
 }
 
 }  // namespace ssm

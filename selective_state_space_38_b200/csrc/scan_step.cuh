@@ -22,6 +22,12 @@ struct StepParams {
     void *out;
     int64_t batch, dim;
     int softplus;
+    // the short causal convolution in front of the scan (conv_k = 0: none):
+    // x is the raw token, the scan's x is silu(conv_w . [window, x] + conv_bias)
+    int conv_k;                 // width, 1..4
+    const float *conv_w;        // [dim][conv_k]
+    const float *conv_bias;     // [dim] or NULL
+    void *conv_state;           // [batch][dim][conv_k - 1] raw inputs, oldest first; read and shifted
 };
 
 constexpr int kStepThreads = 256;
@@ -40,7 +46,9 @@ __device__ __forceinline__ float4 load4(const void *p, int64_t i) {
 }
 
 // SMALL: every channel index fits in 32 bits, so (b, d) come from a 32-bit division.
-template <typename T, bool SMALL>
+// CONV: the token first passes the convolution window (every lane of a
+// channel computes it; the first lane shifts the stored window).
+template <typename T, bool SMALL, bool CONV>
 __global__ void __launch_bounds__(kStepThreads) scan_step_kernel(const StepParams p) {
     using AT = Act<T>;
     constexpr bool kAccurate = AT::kBytes == 4;
@@ -62,7 +70,27 @@ __global__ void __launch_bounds__(kStepThreads) scan_step_kernel(const StepParam
 
     float4 h = *reinterpret_cast<const float4 *>(p.state + c * kNState + q * 4);
     const float4 a = *reinterpret_cast<const float4 *>(p.A + d * kNState + q * 4);
-    const float xf = AT::load(p.x, c);
+    float xf = AT::load(p.x, c);
+    float window[3] = {0.0f, 0.0f, 0.0f};
+    if constexpr (CONV) {
+        const int K1 = p.conv_k - 1;
+        float acc = p.conv_bias ? p.conv_bias[d] : 0.0f;
+#pragma unroll
+        for (int k = 0; k < 3; ++k)
+            if (k < K1) {
+                window[k] = AT::load(p.conv_state, c * K1 + k);
+                acc = fmaf(p.conv_w[d * p.conv_k + k], window[k], acc);
+            }
+        acc = fmaf(p.conv_w[d * p.conv_k + K1], xf, acc);
+        // the window moves on by one input: oldest dropped, this token last
+        __syncwarp();  // every lane of the channel has read the window
+        if (active && q == 0) {
+#pragma unroll
+            for (int k = 0; k < 3; ++k)
+                if (k < K1) AT::store(p.conv_state, c * K1 + k, k + 1 < K1 ? window[k + 1] : xf);
+        }
+        xf = kAccurate ? silu_accurate(acc) : silu_fast(acc);
+    }
     float v = AT::load(p.delta, c);
     if (p.delta_bias) v += p.delta_bias[d];
     const int64_t bn = b * kNState + q * 4;

@@ -112,29 +112,29 @@ int64_t parallel_segments(const FwdParams &p, int sms, int64_t *seg_steps) {
 
 // Persistent launch: one CTA of kPairs warp triples per SM (or fewer when there
 // are fewer items); the S4D instance, then the general one.
-template <typename T, bool VEC>
+template <typename T, bool VEC, bool CONV>
 int launch_pass(const FwdParams &p, const FwdScratch &sc, const TmaMaps &tm, int sms, cudaStream_t stream) {
     const int64_t groups = ((p.dim + 31) / 32) * p.batch;
     const int64_t items = groups * ((p.seqlen + p.seg_steps - 1) / p.seg_steps);
     const int64_t want = (items + kPairs - 1) / kPairs;
     const int64_t ctas = want < sms ? want : sms;
     const int smem = FwdSmem<T>::kTotal;
-    scan_fwd_kernel<T, VEC, true><<<static_cast<unsigned>(ctas), kFwdThreads, smem, stream>>>(p, sc, tm);
-    scan_fwd_kernel<T, VEC, false><<<static_cast<unsigned>(ctas), kFwdThreads, smem, stream>>>(p, sc, tm);
+    scan_fwd_kernel<T, VEC, true, CONV><<<static_cast<unsigned>(ctas), kFwdThreads, smem, stream>>>(p, sc, tm);
+    scan_fwd_kernel<T, VEC, false, CONV><<<static_cast<unsigned>(ctas), kFwdThreads, smem, stream>>>(p, sc, tm);
     return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
 // The kernels of one forward call on zeroed scratch: one chained pass, or the
 // summary pass, the segment combine and the second pass of the time-parallel
 // schedule (the queue is re-armed between the passes).
-template <typename T, bool VEC>
+template <typename T, bool VEC, bool CONV>
 int launch_fwd_kernels(FwdParams p, void *scratch, int64_t segs, int sms, cudaStream_t stream) {
     const int64_t groups = ((p.dim + 31) / 32) * p.batch;
     const int smem = FwdSmem<T>::kTotal;
-    if (cudaFuncSetAttribute(scan_fwd_kernel<T, VEC, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-            cudaSuccess ||
-        cudaFuncSetAttribute(scan_fwd_kernel<T, VEC, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-            cudaSuccess)
+    if (cudaFuncSetAttribute(scan_fwd_kernel<T, VEC, true, CONV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess ||
+        cudaFuncSetAttribute(scan_fwd_kernel<T, VEC, false, CONV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
         return SSM_ERR_CUDA;
     TmaMaps tm;
     memset(&tm, 0, sizeof tm);
@@ -144,11 +144,11 @@ int launch_fwd_kernels(FwdParams p, void *scratch, int64_t segs, int sms, cudaSt
         p.mode = kChained;
         p.pass = 0;
         p.seg_steps = kSegSteps;
-        return launch_pass<T, VEC>(p, sc, tm, sms, stream);
+        return launch_pass<T, VEC, CONV>(p, sc, tm, sms, stream);
     }
     p.mode = kSummary;
     p.pass = 0;
-    int rc = launch_pass<T, VEC>(p, sc, tm, sms, stream);
+    int rc = launch_pass<T, VEC, CONV>(p, sc, tm, sms, stream);
     if (rc != SSM_OK) return rc;
     const int64_t threads = groups * 32;
     segment_combine_kernel<<<static_cast<unsigned>((threads + 127) / 128), 128, 0, stream>>>(p, sc);
@@ -156,7 +156,7 @@ int launch_fwd_kernels(FwdParams p, void *scratch, int64_t segs, int sms, cudaSt
     // first pass stays set for the status query
     p.mode = kFromStart;
     p.pass = 1;
-    return launch_pass<T, VEC>(p, sc, tm, sms, stream);
+    return launch_pass<T, VEC, CONV>(p, sc, tm, sms, stream);
 }
 
 // SMs of the current device (the schedule, and so the workspace size, depend on it)
@@ -177,40 +177,110 @@ size_t fwd_workspace_bytes(const FwdParams &p, int sms) {
 }
 
 // One forward call on the caller's workspace: zero its flag words, then the kernels.
-template <typename T, bool VEC>
+template <typename T, bool VEC, bool CONV>
 int launch_fwd(FwdParams p, void *ws, size_t ws_bytes, int sms, bool force_chained, cudaStream_t stream) {
     const int64_t groups = ((p.dim + 31) / 32) * p.batch;
     const int64_t segs = force_chained ? 0 : parallel_segments(p, sms, &p.seg_steps);
     if (ws_bytes < fwd_scratch_bytes(groups, segs)) return SSM_ERR_INVALID_ARG;
     if (cudaMemsetAsync(ws, 0, fwd_scratch_flag_bytes(groups), stream) != cudaSuccess) return SSM_ERR_CUDA;
-    return launch_fwd_kernels<T, VEC>(p, ws, segs, sms, stream);
+    return launch_fwd_kernels<T, VEC, CONV>(p, ws, segs, sms, stream);
 }
 
-template <typename T>
+// The convolution in front of the scan, when a forward call has one.
+struct ConvArgs {
+    const float *w;      // [dim][k]
+    const float *bias;   // [dim] or NULL
+    int k;               // width, 1..4
+    const void *state;   // [batch][dim][k-1] activation dtype, or NULL
+    void *state_out;     // [batch][dim][k-1] activation dtype, or NULL; may be `state`
+};
+
+template <typename T, bool CONV>
 int launch_step(const StepParams &p, cudaStream_t stream) {
     const int64_t threads = p.batch * p.dim * 4;
     const int64_t blocks = (threads + kStepThreads - 1) / kStepThreads;
     if (blocks > INT_MAX) return SSM_ERR_UNSUPPORTED;
     if (p.batch * p.dim < (int64_t(1) << 31))
-        scan_step_kernel<T, true><<<static_cast<unsigned>(blocks), kStepThreads, 0, stream>>>(p);
+        scan_step_kernel<T, true, CONV><<<static_cast<unsigned>(blocks), kStepThreads, 0, stream>>>(p);
     else
-        scan_step_kernel<T, false><<<static_cast<unsigned>(blocks), kStepThreads, 0, stream>>>(p);
+        scan_step_kernel<T, false, CONV><<<static_cast<unsigned>(blocks), kStepThreads, 0, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
-// Every check of a forward call's arguments (all three forward entry points
-// share it); on success fills `p` and the activation element size.  The
-// workspace, when given, must not overlap any input or output.
+// Every check of a decode step's arguments; on success fills `p`.  The state
+// and the convolution window are read and written in place; out must not
+// overlap anything.
+int validate_step(float *state, const void *x, const void *delta, const float *delta_bias, int softplus,
+                  const float *A, const void *B, const void *C, const float *D, const void *z, void *out,
+                  const ConvArgs *conv, const ssm_dims_t *dims, StepParams *p) {
+    if (!dims) return SSM_ERR_INVALID_ARG;
+    const int64_t batch = dims->batch, dim = dims->dim, N = dims->dstate;
+    if (!state || !x || !delta || !A || !B || !C || !out) return SSM_ERR_INVALID_ARG;
+    if (conv && (!conv->w || (conv->k > 1 && !conv->state_out))) return SSM_ERR_INVALID_ARG;
+    if (!dims_ok(batch, 1, dim) || N < 1) return SSM_ERR_INVALID_ARG;
+    if (N != kNState) return SSM_ERR_UNSUPPORTED;
+    if (dims->act_dtype != SSM_F32 && dims->act_dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
+    if (conv && (conv->k < 1 || conv->k > 4)) return SSM_ERR_UNSUPPORTED;
+    const size_t es = dims->act_dtype == SSM_F32 ? 4 : 2;
+    // state, A, B and C are read (and the state written) as 16-byte vectors per lane
+    for (const void *ptr : {(const void *)state, (const void *)A, B, C})
+        if (!aligned16(ptr)) return SSM_ERR_MISALIGNED;
+    for (const void *ptr : {x, delta, z, (const void *)out})
+        if (ptr && reinterpret_cast<uintptr_t>(ptr) % es != 0) return SSM_ERR_MISALIGNED;
+    for (const void *ptr : {(const void *)delta_bias, (const void *)D})
+        if (ptr && !aligned4(ptr)) return SSM_ERR_MISALIGNED;
+    if (conv) {
+        for (const void *ptr : {(const void *)conv->w, (const void *)conv->bias})
+            if (ptr && !aligned4(ptr)) return SSM_ERR_MISALIGNED;
+        if (conv->state_out && reinterpret_cast<uintptr_t>(conv->state_out) % es != 0) return SSM_ERR_MISALIGNED;
+    }
+
+    const size_t nch = static_cast<size_t>(batch) * dim;
+    const Span ins[] = {{x, nch * es}, {delta, nch * es}, {z, z ? nch * es : 0},
+                        {B, static_cast<size_t>(batch) * N * es}, {C, static_cast<size_t>(batch) * N * es},
+                        {A, static_cast<size_t>(dim) * N * 4}, {D, D ? static_cast<size_t>(dim) * 4 : 0},
+                        {delta_bias, delta_bias ? static_cast<size_t>(dim) * 4 : 0},
+                        {conv ? conv->w : nullptr, conv ? static_cast<size_t>(dim) * conv->k * 4 : 0},
+                        {conv && conv->bias ? conv->bias : nullptr, static_cast<size_t>(dim) * 4}};
+    const Span outs[] = {{out, nch * es}, {state, nch * N * 4},
+                         {conv && conv->k > 1 ? conv->state_out : nullptr, conv ? nch * (conv->k - 1) * es : 0}};
+    for (int o = 0; o < 3; ++o) {
+        for (const Span &in : ins)
+            if (overlap(outs[o], in)) return SSM_ERR_INVALID_ARG;
+        for (int q = o + 1; q < 3; ++q)
+            if (overlap(outs[o], outs[q])) return SSM_ERR_INVALID_ARG;
+    }
+
+    memset(p, 0, sizeof *p);
+    p->state = state; p->x = x; p->delta = delta; p->z = z; p->B = B; p->C = C;
+    p->delta_bias = delta_bias; p->A = A; p->D = D; p->out = out;
+    p->batch = batch; p->dim = dim; p->softplus = softplus ? 1 : 0;
+    if (conv) {
+        p->conv_k = conv->k;
+        p->conv_w = conv->w;
+        p->conv_bias = conv->bias;
+        p->conv_state = conv->state_out;
+    }
+    return SSM_OK;
+}
+
+// Every check of a forward call's arguments (all forward entry points share
+// it); on success fills `p` and the activation element size.  Outputs (out,
+// h_last, the workspace, the new convolution state) must not overlap any
+// input or each other, except that h_last may be h0 itself and the new
+// convolution state may be the old one itself.
 int validate_fwd(const void *x, const void *delta, const float *delta_bias, int softplus, const float *A,
                  const void *B, const void *C, const float *D, const void *z, const float *h0, void *out,
-                 float *h_last, const void *ws, size_t ws_bytes, const ssm_dims_t *dims, FwdParams *p,
-                 size_t *es_out) {
+                 float *h_last, const void *ws, size_t ws_bytes, const ConvArgs *conv, const ssm_dims_t *dims,
+                 FwdParams *p, size_t *es_out) {
     if (!dims) return SSM_ERR_INVALID_ARG;
     const int64_t batch = dims->batch, L = dims->seqlen, dim = dims->dim, N = dims->dstate;
     if (!x || !delta || !A || !B || !C || !out) return SSM_ERR_INVALID_ARG;
+    if (conv && !conv->w) return SSM_ERR_INVALID_ARG;
     if (!dims_ok(batch, L, dim) || N < 1) return SSM_ERR_INVALID_ARG;
     if (N != kNState) return SSM_ERR_UNSUPPORTED;
     if (dims->act_dtype != SSM_F32 && dims->act_dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
+    if (conv && (conv->k < 1 || conv->k > 4)) return SSM_ERR_UNSUPPORTED;
     // TMA coordinates and the work queue's item split are 32-bit
     if (batch > INT32_MAX || L > INT32_MAX - 64 || dim > INT32_MAX - 64) return SSM_ERR_UNSUPPORTED;
     const int64_t groups = ((dim + 31) / 32) * batch;
@@ -221,32 +291,35 @@ int validate_fwd(const void *x, const void *delta, const float *delta_bias, int 
         if (ptr && !aligned16(ptr)) return SSM_ERR_MISALIGNED;
     for (const void *ptr : {(const void *)delta_bias, (const void *)D})
         if (ptr && !aligned4(ptr)) return SSM_ERR_MISALIGNED;
+    if (conv) {
+        for (const void *ptr : {(const void *)conv->w, (const void *)conv->bias})
+            if (ptr && !aligned4(ptr)) return SSM_ERR_MISALIGNED;
+        for (const void *ptr : {conv->state, (const void *)conv->state_out})
+            if (ptr && reinterpret_cast<uintptr_t>(ptr) % es != 0) return SSM_ERR_MISALIGNED;
+    }
 
     const size_t tok = static_cast<size_t>(batch) * dim * L;
     const size_t st = static_cast<size_t>(batch) * dim * N * 4;
-    const Span o{out, tok * es};
+    const size_t cst = conv ? static_cast<size_t>(batch) * dim * (conv->k - 1) * es : 0;
     const Span ins[] = {{x, tok * es}, {delta, tok * es}, {z, z ? tok * es : 0},
                         {B, static_cast<size_t>(batch) * N * L * es}, {C, static_cast<size_t>(batch) * N * L * es},
                         {A, static_cast<size_t>(dim) * N * 4}, {D, D ? static_cast<size_t>(dim) * 4 : 0},
-                        {delta_bias, delta_bias ? static_cast<size_t>(dim) * 4 : 0},
-                        {h0, h0 ? st : 0}, {h_last, h_last ? st : 0}};
-    for (const Span &s : ins)
-        if (overlap(o, s)) return SSM_ERR_INVALID_ARG;
-    if (h_last) {  // h_last may be h0 itself, but must not partially overlap any input
-        const Span hl{h_last, st};
-        for (int i = 0; i < 8; ++i)
-            if (overlap(hl, ins[i])) return SSM_ERR_INVALID_ARG;
-        if (h0 && h0 != h_last && overlap(hl, ins[8])) return SSM_ERR_INVALID_ARG;
+                        {delta_bias, delta_bias ? static_cast<size_t>(dim) * 4 : 0}, {h0, h0 ? st : 0},
+                        {conv ? conv->w : nullptr, conv ? static_cast<size_t>(dim) * conv->k * 4 : 0},
+                        {conv && conv->bias ? conv->bias : nullptr, static_cast<size_t>(dim) * 4},
+                        {conv ? conv->state : nullptr, cst}};
+    const Span outs[] = {{out, tok * es}, {h_last, h_last ? st : 0}, {ws, ws ? ws_bytes : 0},
+                         {conv ? conv->state_out : nullptr, cst}};
+    const void *alias_of[] = {nullptr, h0, nullptr, conv ? conv->state : nullptr};  // allowed exact alias
+    for (int o = 0; o < 4; ++o) {
+        for (const Span &in : ins)
+            if (overlap(outs[o], in) && !(in.p == alias_of[o] && in.p == outs[o].p)) return SSM_ERR_INVALID_ARG;
+        for (int q = o + 1; q < 4; ++q)
+            if (overlap(outs[o], outs[q])) return SSM_ERR_INVALID_ARG;
     }
-    if (ws) {
-        // the chained schedule's workspace is the least any device needs (the
-        // exact size, which depends on the SM count, is checked at launch)
-        if (ws_bytes < fwd_scratch_bytes(((dim + 31) / 32) * batch)) return SSM_ERR_INVALID_ARG;
-        const Span w{ws, ws_bytes};
-        if (overlap(w, o)) return SSM_ERR_INVALID_ARG;
-        for (const Span &s : ins)
-            if (overlap(w, s)) return SSM_ERR_INVALID_ARG;
-    }
+    // the chained schedule's workspace is the least any device needs (the exact
+    // size, which depends on the SM count, is checked at launch)
+    if (ws && ws_bytes < fwd_scratch_bytes(groups)) return SSM_ERR_INVALID_ARG;
 
     memset(p, 0, sizeof *p);
     p->x = x; p->delta = delta; p->z = z; p->B = B; p->C = C;
@@ -257,21 +330,45 @@ int validate_fwd(const void *x, const void *delta, const float *delta_bias, int 
     p->seg_steps = kSegSteps;
     p->spin_limit = kSpinLimit;
     p->flag_bias = 0;
+    if (conv) {
+        p->conv_k = conv->k;
+        p->conv_w = conv->w;
+        p->conv_bias = conv->bias;
+        p->conv_state = conv->state;
+    }
     *es_out = es;
     return SSM_OK;
 }
 
-// The forward call on a validated shape and a workspace of ws_bytes.
+// The forward call on a validated shape and a workspace of ws_bytes; then,
+// for a call with a convolution, the new convolution state.
 int dispatch_fwd(const FwdParams &p, size_t es, int act_dtype, void *ws, size_t ws_bytes, bool force_chained,
-                 cudaStream_t s) {
+                 void *conv_state_out, cudaStream_t s) {
     int sms = 0;
     if (current_sms(&sms) != SSM_OK) return SSM_ERR_CUDA;
     const bool vec = (static_cast<size_t>(p.seqlen) * es) % 16 == 0;
-    if (act_dtype == SSM_BF16)
-        return vec ? launch_fwd<bf16raw, true>(p, ws, ws_bytes, sms, force_chained, s)
-                   : launch_fwd<bf16raw, false>(p, ws, ws_bytes, sms, force_chained, s);
-    return vec ? launch_fwd<float, true>(p, ws, ws_bytes, sms, force_chained, s)
-               : launch_fwd<float, false>(p, ws, ws_bytes, sms, force_chained, s);
+    const bool bf = act_dtype == SSM_BF16;
+    int rc;
+    if (p.conv_k) {
+        rc = bf ? (vec ? launch_fwd<bf16raw, true, true>(p, ws, ws_bytes, sms, force_chained, s)
+                       : launch_fwd<bf16raw, false, true>(p, ws, ws_bytes, sms, force_chained, s))
+                : (vec ? launch_fwd<float, true, true>(p, ws, ws_bytes, sms, force_chained, s)
+                       : launch_fwd<float, false, true>(p, ws, ws_bytes, sms, force_chained, s));
+        if (rc == SSM_OK && conv_state_out && p.conv_k > 1) {
+            const int64_t nch = p.batch * p.dim;
+            const unsigned blocks = static_cast<unsigned>((nch + 255) / 256);
+            if (bf)
+                conv_state_kernel<bf16raw><<<blocks, 256, 0, s>>>(p, conv_state_out);
+            else
+                conv_state_kernel<float><<<blocks, 256, 0, s>>>(p, conv_state_out);
+            rc = cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+        }
+        return rc;
+    }
+    return bf ? (vec ? launch_fwd<bf16raw, true, false>(p, ws, ws_bytes, sms, force_chained, s)
+                     : launch_fwd<bf16raw, false, false>(p, ws, ws_bytes, sms, force_chained, s))
+              : (vec ? launch_fwd<float, true, false>(p, ws, ws_bytes, sms, force_chained, s)
+                     : launch_fwd<float, false, false>(p, ws, ws_bytes, sms, force_chained, s));
 }
 
 }  // namespace
@@ -313,9 +410,9 @@ int ssm_scan_fwd(const void *x, const void *delta, const float *delta_bias, int 
     FwdParams p;
     size_t es = 0;
     const int rc = validate_fwd(x, delta, delta_bias, softplus, A, B, C, D, z, h0, out, h_last, workspace,
-                                workspace_bytes, dims, &p, &es);
+                                workspace_bytes, nullptr, dims, &p, &es);
     if (rc != SSM_OK) return rc;
-    return dispatch_fwd(p, es, dims->act_dtype, workspace, workspace_bytes, false,
+    return dispatch_fwd(p, es, dims->act_dtype, workspace, workspace_bytes, false, nullptr,
                         reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -328,48 +425,50 @@ int ssm_debug_fwd_flag_timeout(const void *x, const void *delta, const float *de
     FwdParams p;
     size_t es = 0;
     const int rc = validate_fwd(x, delta, delta_bias, softplus, A, B, C, D, z, h0, out, h_last, workspace,
-                                workspace_bytes, dims, &p, &es);
+                                workspace_bytes, nullptr, dims, &p, &es);
     if (rc != SSM_OK) return rc;
     p.spin_limit = spin_limit;
     p.flag_bias = 1u << 30;  // no segment flag ever reaches this
-    return dispatch_fwd(p, es, dims->act_dtype, workspace, workspace_bytes, true,
+    return dispatch_fwd(p, es, dims->act_dtype, workspace, workspace_bytes, true, nullptr,
                         reinterpret_cast<cudaStream_t>(stream));
 }
 
 int ssm_scan_step(float *state, const void *x, const void *delta, const float *delta_bias,
                   int softplus, const float *A, const void *B, const void *C, const float *D,
                   const void *z, void *out, const ssm_dims_t *dims, ssm_stream_t stream) {
-    if (!dims) return SSM_ERR_INVALID_ARG;
-    const int64_t batch = dims->batch, dim = dims->dim, N = dims->dstate;
-    if (!state || !x || !delta || !A || !B || !C || !out) return SSM_ERR_INVALID_ARG;
-    if (!dims_ok(batch, 1, dim) || N < 1) return SSM_ERR_INVALID_ARG;
-    if (N != kNState) return SSM_ERR_UNSUPPORTED;
-    if (dims->act_dtype != SSM_F32 && dims->act_dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
-    const size_t es = dims->act_dtype == SSM_F32 ? 4 : 2;
-    // state, A, B and C are read (and the state written) as 16-byte vectors per lane
-    for (const void *ptr : {(const void *)state, (const void *)A, B, C})
-        if (!aligned16(ptr)) return SSM_ERR_MISALIGNED;
-    for (const void *ptr : {x, delta, z, (const void *)out, (const void *)delta_bias, (const void *)D})
-        if (ptr && (reinterpret_cast<uintptr_t>(ptr) % (ptr == delta_bias || ptr == D ? 4 : es)) != 0)
-            return SSM_ERR_MISALIGNED;
-
-    const size_t nch = static_cast<size_t>(batch) * dim;
-    const Span o{out, nch * es};
-    const Span st{state, nch * N * 4};
-    const Span ins[] = {{x, nch * es}, {delta, nch * es}, {z, z ? nch * es : 0},
-                        {B, static_cast<size_t>(batch) * N * es}, {C, static_cast<size_t>(batch) * N * es},
-                        {A, static_cast<size_t>(dim) * N * 4}, {D, D ? static_cast<size_t>(dim) * 4 : 0},
-                        {delta_bias, delta_bias ? static_cast<size_t>(dim) * 4 : 0}};
-    if (overlap(o, st)) return SSM_ERR_INVALID_ARG;
-    for (const Span &s : ins)
-        if (overlap(o, s) || overlap(st, s)) return SSM_ERR_INVALID_ARG;
-
     StepParams p;
-    p.state = state; p.x = x; p.delta = delta; p.z = z; p.B = B; p.C = C;
-    p.delta_bias = delta_bias; p.A = A; p.D = D; p.out = out;
-    p.batch = batch; p.dim = dim; p.softplus = softplus ? 1 : 0;
+    const int rc = validate_step(state, x, delta, delta_bias, softplus, A, B, C, D, z, out, nullptr, dims, &p);
+    if (rc != SSM_OK) return rc;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    return dims->act_dtype == SSM_BF16 ? launch_step<bf16raw>(p, s) : launch_step<float>(p, s);
+    return dims->act_dtype == SSM_BF16 ? launch_step<bf16raw, false>(p, s) : launch_step<float, false>(p, s);
+}
+
+int ssm_conv_scan_fwd(const void *x, const float *conv_w, const float *conv_bias, int conv_width,
+                      const void *conv_state, void *conv_state_out, const void *delta, const float *delta_bias,
+                      int softplus, const float *A, const void *B, const void *C, const float *D, const void *z,
+                      const float *h0, void *out, float *h_last, void *workspace, size_t workspace_bytes,
+                      const ssm_dims_t *dims, ssm_stream_t stream) {
+    if (!workspace) return SSM_ERR_INVALID_ARG;
+    const ConvArgs conv{conv_w, conv_bias, conv_width, conv_state, conv_state_out};
+    FwdParams p;
+    size_t es = 0;
+    const int rc = validate_fwd(x, delta, delta_bias, softplus, A, B, C, D, z, h0, out, h_last, workspace,
+                                workspace_bytes, &conv, dims, &p, &es);
+    if (rc != SSM_OK) return rc;
+    return dispatch_fwd(p, es, dims->act_dtype, workspace, workspace_bytes, false, conv_state_out,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+int ssm_conv_scan_step(void *conv_state, float *state, const void *x, const float *conv_w,
+                       const float *conv_bias, int conv_width, const void *delta, const float *delta_bias,
+                       int softplus, const float *A, const void *B, const void *C, const float *D,
+                       const void *z, void *out, const ssm_dims_t *dims, ssm_stream_t stream) {
+    const ConvArgs conv{conv_w, conv_bias, conv_width, nullptr, conv_state};
+    StepParams p;
+    const int rc = validate_step(state, x, delta, delta_bias, softplus, A, B, C, D, z, out, &conv, dims, &p);
+    if (rc != SSM_OK) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return dims->act_dtype == SSM_BF16 ? launch_step<bf16raw, true>(p, s) : launch_step<float, true>(p, s);
 }
 
 }  // extern "C"
@@ -413,8 +512,8 @@ extern "C" int ssm_scan_fwd_noalloc(const void *x, const void *delta, const floa
                                     const ssm_dims_t *dims, ssm_stream_t stream) {
     FwdParams p;
     size_t es = 0;
-    const int rc = validate_fwd(x, delta, delta_bias, softplus, A, B, C, D, z, h0, out, h_last, nullptr, 0, dims,
-                                &p, &es);
+    const int rc = validate_fwd(x, delta, delta_bias, softplus, A, B, C, D, z, h0, out, h_last, nullptr, 0, nullptr,
+                                dims, &p, &es);
     if (rc != SSM_OK) return rc;
     // the work queue of this shape (chained schedule: its scratch does not grow
     // with the sequence) must fit the fixed array
@@ -426,7 +525,7 @@ extern "C" int ssm_scan_fwd_noalloc(const void *x, const void *delta, const floa
     if (!scratch) return SSM_ERR_CUDA;
     // the array keeps the previous call's contents: launch_fwd zeroes the queue
     // counters, error word and segment flags (the carries need not start at zero)
-    return dispatch_fwd(p, es, dims->act_dtype, scratch, kNoAllocScratchBytes, true,
+    return dispatch_fwd(p, es, dims->act_dtype, scratch, kNoAllocScratchBytes, true, nullptr,
                         reinterpret_cast<cudaStream_t>(stream));
 }
 

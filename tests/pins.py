@@ -462,6 +462,145 @@ def pin_conv_step_equals_fwd(orc):
     _close(cs, st, rtol=0, atol=0, what="conv step window")
 
 
+# ---------------------------------------------------------------------------
+# The exponential-trapezoidal discretisation ("Mamba3" posts: both ends of the
+# interval, mixed by a data-dependent lambda; second order).
+
+def _trap_case(seed, b=2, d=3, n=4, L=9, prev=True):
+    r = _rng(seed)
+    c = _rand_case(seed, b=b, d=d, n=n, L=L)
+    c["lam"] = _f32(r.uniform(0.0, 1.0, (b, d, L)))
+    c["x_prev"] = _f32(r.standard_normal((b, d))) if prev else None
+    c["B_prev"] = _f32(r.standard_normal((b, n))) if prev else None
+    return c
+
+
+def _trap(orc, c, **over):
+    a = dict(c)
+    a.update(over)
+    return orc.trap_fwd(a["x"], a["delta"], a["delta_bias"], a["softplus"], a["lam"], a["A"], a["B"],
+                        a["C"], a["D"], a["z"], a["h0"], a["x_prev"], a["B_prev"])
+
+
+def pin_trap_lambda_one_is_euler(orc):
+    """lambda = 1 drops the interval's start: the rule is Mamba-1's Euler
+    input step, whatever the previous input."""
+    c = _trap_case(90, L=12)
+    out, hl = _trap(orc, c, lam=np.ones_like(c["lam"]))
+    o2, h2 = _call(orc, c)
+    _close(out, o2, rtol=1e-13, atol=1e-14, what="trap lambda=1 out")
+    _close(hl, h2, rtol=1e-13, atol=1e-14, what="trap lambda=1 h_last")
+
+
+def pin_trap_constant_inputs(orc):
+    """Constant dt, lambda, B, x: h_0 = alpha h0 + beta v_prev + gamma v and
+    h_t = alpha h_{t-1} + (beta + gamma) v after it, a geometric sum; v = B x,
+    alpha = exp(dt A), beta = (1 - lambda) dt alpha, gamma = lambda dt."""
+    r = _rng(91)
+    b, d, n, L = 2, 3, 4, 30
+    rep = lambda a: _f32(np.repeat(a, L, -1))
+    c = dict(x=rep(r.standard_normal((b, d, 1))), delta=rep(r.standard_normal((b, d, 1)) * 0.4),
+             z=None, B=rep(r.standard_normal((b, n, 1))), C=rep(r.standard_normal((b, n, 1))),
+             A=_f32(-r.uniform(0.1, 1.5, (d, n))), D=None, delta_bias=_f32(r.standard_normal(d) * 0.2),
+             h0=_f32(r.standard_normal((b, d, n))), softplus=True,
+             lam=rep(r.uniform(0, 1, (b, d, 1))), x_prev=_f32(r.standard_normal((b, d))),
+             B_prev=_f32(r.standard_normal((b, n))))
+    dt = np.logaddexp(0.0, c["delta"][..., :1].astype(np.float64) + c["delta_bias"][None, :, None])  # [b,d,1]
+    lam = c["lam"][..., :1].astype(np.float64)
+    al = np.exp(dt * c["A"][None].astype(np.float64))                                             # [b,d,n]
+    be, ga = (1 - lam) * dt * al, lam * dt
+    v = c["x"][..., :1].astype(np.float64) * np.transpose(c["B"][..., :1], (0, 2, 1)).astype(np.float64)
+    vp = c["x_prev"][..., None].astype(np.float64) * c["B_prev"][:, None, :].astype(np.float64)
+    h_first = al * c["h0"] + be * vp + ga * v
+    t = np.arange(L)[None, None, None, :]
+    ap = al[..., None] ** t
+    h = ap * h_first[..., None] + ((be + ga) * v)[..., None] * (1 - ap) / (1 - al)[..., None]
+    y = np.einsum("bdnl,bn->bdl", h, c["C"][..., 0].astype(np.float64))
+    out, hl = _trap(orc, c)
+    _close(out, y, rtol=1e-10, atol=1e-12, what="trap constant out")
+    _close(hl, h[..., -1], rtol=1e-10, atol=1e-12, what="trap constant h_last")
+
+
+def pin_trap_second_order(orc):
+    """The rule is second order for lambda = 1/2 and first order for lambda = 1.
+    The scalar system h' = a h + b cos(w s), h(0) = 0, has the exact solution
+    h(T) = b (a e^{aT} - a cos wT + w sin wT) / (a^2 + w^2); n steps of
+    dt = T / n with x_t = cos(w (t+1) dt) and x_prev = cos(0) approximate it,
+    and halving dt divides the error by about 4 (lambda = 1/2) or 2 (lambda = 1)."""
+    a, bb, w, T = -0.7, 1.3, 2.0, 3.0
+    exact = bb * (a * math.exp(a * T) - a * math.cos(w * T) + w * math.sin(w * T)) / (a * a + w * w)
+
+    def err(n, lam):
+        dtv = T / n
+        s = (np.arange(n) + 1) * dtv
+        c = dict(x=_f32(np.cos(w * s)).reshape(1, 1, n), delta=_f32(np.full((1, 1, n), dtv)), z=None,
+                 B=_f32(np.full((1, 1, n), bb)), C=np.zeros((1, 1, n), np.float32), A=_f32([[a]]), D=None,
+                 delta_bias=None, h0=None, softplus=False, lam=_f32(np.full((1, 1, n), lam)),
+                 x_prev=_f32([[1.0]]), B_prev=_f32([[bb]]))
+        _, hl = _trap(orc, c)
+        return abs(hl[0, 0, 0] - exact)
+
+    for lam, lo, hi in ((0.5, 3.6, 4.4), (1.0, 1.8, 2.2)):
+        errs = [err(n, lam) for n in (32, 64, 128)]
+        for e1, e2 in zip(errs, errs[1:]):
+            assert lo < e1 / e2 < hi, (lam, errs)
+    assert err(128, 0.5) < 1e-3 * err(128, 1.0) ** 0.5
+
+
+def pin_trap_convolution_mode(orc):
+    """LTI case (constant dt, lambda, B, C; h0 = 0; nothing before t = 0):
+    y = K * x + D x with K_0 = sum_n C_n gamma B_n and
+    K_k = sum_n C_n alpha_n^(k-1) (alpha_n gamma + beta_n) B_n for k >= 1."""
+    r = _rng(92)
+    b, d, n, L = 1, 2, 5, 40
+    c = _trap_case(92, b=b, d=d, n=n, L=L, prev=False)
+    vv = r.standard_normal((1, d, 1)) * 0.4
+    c.update(delta=_f32(np.repeat(vv, L, 2)), B=_f32(np.repeat(r.standard_normal((b, n, 1)), L, 2)),
+             C=_f32(np.repeat(r.standard_normal((b, n, 1)), L, 2)), h0=None, z=None,
+             lam=_f32(np.repeat(r.uniform(0, 1, (1, d, 1)), L, 2)))
+    out, _ = _trap(orc, c)
+    dt = np.logaddexp(0.0, c["delta"][0, :, 0].astype(np.float64) + c["delta_bias"].astype(np.float64))
+    for di in range(d):
+        lam = float(c["lam"][0, di, 0])
+        al = np.exp(dt[di] * c["A"][di].astype(np.float64))
+        be, ga = (1 - lam) * dt[di] * al, lam * dt[di]
+        Bn, Cn = c["B"][0, :, 0].astype(np.float64), c["C"][0, :, 0].astype(np.float64)
+        K = np.empty(L)
+        K[0] = (Cn * ga * Bn).sum()
+        for k in range(1, L):
+            K[k] = (Cn * al ** (k - 1) * (al * ga + be) * Bn).sum()
+        xs = c["x"][0, di].astype(np.float64)
+        want = np.convolve(xs, K)[:L] + c["D"][di] * xs
+        _close(out[0, di], want, rtol=1e-10, atol=1e-12, what=f"trap conv mode d{di}")
+
+
+def pin_trap_split_and_step(orc):
+    """Two calls continue one when h_last and the last token's x and B are
+    carried over; T decode steps (each given the previous token) equal one call."""
+    c = _trap_case(93, L=15)
+    out, hl = _trap(orc, c)
+    seq = ("x", "delta", "z", "B", "C", "lam")
+    for m in (1, 6, 14):
+        first = {k: (np.ascontiguousarray(v[..., :m]) if k in seq else v) for k, v in c.items()}
+        second = {k: (np.ascontiguousarray(v[..., m:]) if k in seq else v) for k, v in c.items()}
+        o1, h1 = _trap(orc, first)
+        second.update(h0=_f32(h1), x_prev=np.ascontiguousarray(c["x"][..., m - 1]),
+                      B_prev=np.ascontiguousarray(c["B"][..., m - 1]))
+        o2, h2 = _trap(orc, second)
+        _close(o1, out[..., :m], rtol=1e-12, what=f"trap split m={m} first")
+        _close(o2, out[..., m:], rtol=2e-5, atol=2e-5, what=f"trap split m={m} second")
+        _close(h2, hl, rtol=2e-5, atol=2e-5, what=f"trap split m={m} h_last")
+    state = c["h0"].astype(np.float64).copy()
+    xp, bp = c["x_prev"], c["B_prev"]
+    for t in range(15):
+        tok = {k: np.ascontiguousarray(c[k][..., t]) for k in seq}
+        o = orc.trap_step(state, tok["x"], tok["delta"], c["delta_bias"], True, tok["lam"], c["A"], tok["B"],
+                          tok["C"], c["D"], tok["z"], xp, bp)
+        _close(o, out[..., t], rtol=1e-13, atol=1e-15, what=f"trap step t={t}")
+        xp, bp = tok["x"], tok["B"]
+    _close(state, hl, rtol=1e-13, what="trap step state")
+
+
 ALL_PINS = [
     pin_single_step_closed_form,
     pin_hand_values,
@@ -479,4 +618,9 @@ ALL_PINS = [
     pin_conv_feeds_scan,
     pin_conv_split,
     pin_conv_step_equals_fwd,
+    pin_trap_lambda_one_is_euler,
+    pin_trap_constant_inputs,
+    pin_trap_second_order,
+    pin_trap_convolution_mode,
+    pin_trap_split_and_step,
 ]

@@ -167,3 +167,43 @@ def test_python_binding_refuses_cpu_tensors():
     x = torch.zeros(1, 4, 8, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         m.ssm_scan_fwd(x, x, None, True, torch.zeros(4, 16), x, x)
+
+
+def test_conv_entries_reject_bad_arguments(lib):
+    """The fused convolution entries share the forward and step checks and add
+    their own: taps required, width 1..4, the new window disjoint from every
+    other buffer (it may only be the old window itself)."""
+    import selective_state_space_38_b200 as m
+
+    def fwd(**over):
+        a = dict(x=_p(1), w=_p(10), cb=None, k=4, cs=None, cso=_p(11), delta=_p(2), bias=None, sp=1, A=_p(3),
+                 B=_p(4), C=_p(5), D=None, z=_p(6), h0=None, out=_p(7), hl=None, ws=_p(9), wsb=WS,
+                 dims=_dims(m))
+        a.update(over)
+        return lib.ssm_conv_scan_fwd(a["x"], a["w"], a["cb"], a["k"], a["cs"], a["cso"], a["delta"], a["bias"],
+                                     a["sp"], a["A"], a["B"], a["C"], a["D"], a["z"], a["h0"], a["out"], a["hl"],
+                                     a["ws"], a["wsb"], a["dims"], None)
+    assert fwd(w=None) == 1
+    assert fwd(k=5) == 2
+    assert fwd(k=0) == 2
+    assert fwd(w=ctypes.c_void_p(0x1A000002)) == 3
+    assert fwd(cso=ctypes.c_void_p(0x1B000001)) == 3      # bf16 window at an odd byte
+    assert fwd(cso=_p(1)) == 1                            # new window over x
+    assert fwd(cso=_p(7)) == 1                            # ... over out
+    assert fwd(cso=_p(10)) == 1                           # ... over the taps
+    assert fwd(cs=_p(12), cso=ctypes.c_void_p(0x1C000002)) == 1  # partly over the old window
+    assert fwd(out=_p(10)) == 1                           # out over the taps
+    assert fwd(ws=None) == 1
+
+    def step(**over):
+        a = dict(cs=_p(12), st=_p(0), x=_p(1), w=_p(10), cb=None, k=4, delta=_p(2), bias=None, sp=1, A=_p(3),
+                 B=_p(4), C=_p(5), D=None, z=None, out=_p(7), dims=_dims(m))
+        a.update(over)
+        return lib.ssm_conv_scan_step(a["cs"], a["st"], a["x"], a["w"], a["cb"], a["k"], a["delta"], a["bias"],
+                                      a["sp"], a["A"], a["B"], a["C"], a["D"], a["z"], a["out"], a["dims"], None)
+    assert step(cs=None) == 1                             # the window is required for K > 1
+    assert step(w=None) == 1
+    assert step(k=7) == 2
+    assert step(cs=_p(0)) == 1                            # window over the state
+    assert step(cs=_p(1)) == 1                            # window over x
+    assert step(B=ctypes.c_void_p(0x14000004)) == 3

@@ -52,6 +52,18 @@ MUTANTS = [
      "conv_input(x, conv_state, dtype, chan, L, K, L - K + j);"),
     ("conv step does not shift", "            cs[k] = cs[k + 1];", "            cs[k] = cs[k];"),
     ("conv step window reversed", "acc += (double)w[d * K + k] * cs[k];", "acc += (double)w[d * K + k] * cs[K - 2 - k];"),
+    # the exponential-trapezoidal rule
+    ("trap weights swapped", "const double beta = (1.0 - lt) * dt * alpha;", "const double beta = lt * dt * alpha;"),
+    ("trap start term not decayed", "const double beta = (1.0 - lt) * dt * alpha;",
+     "const double beta = (1.0 - lt) * dt;"),
+    ("trap end weight without dt", "const double gamma = lt * dt;", "const double gamma = lt;"),
+    ("trap previous input never moves on", "            vprev[n] = vt;", "            vprev[n] = vprev[n];"),
+    ("trap input before t = 0 ignored", "const double xp = (x_prev && B_prev) ? load_act(x_prev, chan, a->dtype) : 0.0;",
+     "const double xp = 0.0;"),
+    ("trap step mixes by 1 - lambda twice", "hl[n] = alpha * h[n] + (1.0 - lt) * dt * alpha * vprev[n] + lt * dt * vt;",
+     "hl[n] = alpha * h[n] + (1.0 - lt) * dt * alpha * vprev[n] + (1.0 - lt) * dt * vt;"),
+    ("trap step drops the previous token", "hl[n] = alpha * h[n] + (1.0 - lt) * dt * alpha * vprev[n] + lt * dt * vt;",
+     "hl[n] = alpha * h[n] + lt * dt * vt;"),
 ]
 
 

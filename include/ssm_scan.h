@@ -201,6 +201,42 @@ int ssm_conv_scan_step(void *conv_state, float *state, const void *x, const floa
                        const ssm_dims_t *dims, ssm_stream_t stream);
 
 /*
+ * Forward scan with the exponential-trapezoidal discretisation ("Mamba3"
+ * posts, section on the new discretisation scheme: the integral over each
+ * step is approximated with both ends of the interval, mixed by a
+ * data-dependent lambda, a second-order rule):
+ *
+ *   h_t = alpha_t h_{t-1} + (1 - lam_t) dt_t alpha_t B_{t-1} x_{t-1} + lam_t dt_t B_t x_t
+ *   alpha_t = exp(dt_t A),  y_t and out as for ssm_scan_fwd
+ *
+ * lam = 1 gives ssm_scan_fwd's Euler input step; lam = 1/2 the trapezoidal rule.
+ *
+ *   lam            required [batch][dim][seqlen], activation dtype, 16-byte aligned
+ *   x_prev, B_prev optional [batch][dim] and [batch][dstate], activation dtype:
+ *                  the input before t = 0 (the previous call's last x and B);
+ *                  no previous input unless both are given
+ * The remaining arguments, the workspace, errors and ssm_scan_fwd_status are
+ * those of ssm_scan_fwd.  A sequence split into calls continues exactly when
+ * each call gets the previous call's h_last and its last x and B.
+ */
+int ssm_trap_scan_fwd(const void *x, const void *delta, const float *delta_bias, int softplus,
+                      const void *lam, const float *A, const void *B, const void *C, const float *D,
+                      const void *z, const float *h0, const void *x_prev, const void *B_prev,
+                      void *out, float *h_last, void *workspace, size_t workspace_bytes,
+                      const ssm_dims_t *dims, ssm_stream_t stream);
+
+/*
+ * One recurrent step with the exponential-trapezoidal rule: ssm_scan_step's
+ * arguments plus lam [batch][dim] (element aligned) and the previous token's
+ * x_prev [batch][dim] (element aligned) and B_prev [batch][dstate] (16-byte
+ * aligned); no previous input unless both are given.
+ */
+int ssm_trap_scan_step(float *state, const void *x, const void *delta, const float *delta_bias,
+                       int softplus, const void *lam, const float *A, const void *B, const void *C,
+                       const float *D, const void *z, const void *x_prev, const void *B_prev,
+                       void *out, const ssm_dims_t *dims, ssm_stream_t stream);
+
+/*
  * ssm_scan_fwd without a workspace.  The pages have no counterpart: this
  * entry point exists for callers that cannot allocate any device memory while
  * they run the scan, not even a workspace (code running inside an allocator or

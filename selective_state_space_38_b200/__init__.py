@@ -56,6 +56,10 @@ def _load():
     lib.ssm_conv_scan_fwd.restype = I
     lib.ssm_conv_scan_step.argtypes = [P, P, P, P, P, I, P, P, I, P, P, P, P, P, P, DP, P]
     lib.ssm_conv_scan_step.restype = I
+    lib.ssm_trap_scan_fwd.argtypes = [P, P, P, I, P, P, P, P, P, P, P, P, P, P, P, P, S, DP, P]
+    lib.ssm_trap_scan_fwd.restype = I
+    lib.ssm_trap_scan_step.argtypes = [P, P, P, P, I, P, P, P, P, P, P, P, P, P, DP, P]
+    lib.ssm_trap_scan_step.restype = I
     lib.ssm_scan_step.argtypes = [P, P, P, P, I, P, P, P, P, P, P, DP, P]
     lib.ssm_scan_step.restype = I
     lib.ssm_strerror.argtypes = [I]
@@ -77,7 +81,8 @@ def get_lib():
 
 
 EXPORTS = ("ssm_scan_fwd_workspace_size", "ssm_scan_fwd", "ssm_scan_fwd_status", "ssm_scan_step",
-           "ssm_conv_scan_fwd", "ssm_conv_scan_step", "ssm_scan_fwd_noalloc", "ssm_debug_fwd_flag_timeout",
+           "ssm_conv_scan_fwd", "ssm_conv_scan_step", "ssm_trap_scan_fwd", "ssm_trap_scan_step",
+           "ssm_scan_fwd_noalloc", "ssm_debug_fwd_flag_timeout",
            "ssm_strerror", "ssm_version")
 
 
@@ -300,6 +305,88 @@ def ssm_conv_scan_step(conv_state, state, x, conv_w, conv_bias, delta, delta_bia
     return out
 
 
+def ssm_trap_scan_fwd(x, delta, delta_bias, softplus, lam, A, B, C, D=None, z=None, h0=None, x_prev=None,
+                      B_prev=None, out=None, h_last=None, stream=None, workspace=None, check=False):
+    """Forward scan with the exponential-trapezoidal rule.  lam: [batch, dim, L]
+    in x's dtype; x_prev [batch, dim] and B_prev [batch, 16]: the input before
+    t = 0 (the previous call's last x and B).  Returns (out, h_last)."""
+    if x.device.type != "cuda":
+        raise ValueError("ssm_trap_scan_fwd needs CUDA tensors")
+    dev = x.device
+    batch, dim, L = x.shape
+    code = _act_code(x)
+    act = x.dtype
+    f32 = torch.float32
+    ptrs = dict(
+        x=_ptr(x, dtype=act, device=dev, name="x"),
+        delta=_ptr(delta, dtype=act, device=dev, shape=x.shape, name="delta"),
+        lam=_ptr(lam, dtype=act, device=dev, shape=x.shape, name="lam"),
+        z=_ptr(z, dtype=act, device=dev, shape=x.shape, name="z"),
+        B=_ptr(B, dtype=act, device=dev, shape=(batch, DSTATE, L), name="B"),
+        C=_ptr(C, dtype=act, device=dev, shape=(batch, DSTATE, L), name="C"),
+        A=_ptr(A, dtype=f32, device=dev, shape=(dim, DSTATE), name="A"),
+        D=_ptr(D, dtype=f32, device=dev, shape=(dim,), name="D"),
+        delta_bias=_ptr(delta_bias, dtype=f32, device=dev, shape=(dim,), name="delta_bias"),
+        h0=_ptr(h0, dtype=f32, device=dev, shape=(batch, dim, DSTATE), name="h0"),
+        x_prev=_ptr(x_prev, dtype=act, device=dev, shape=(batch, dim), name="x_prev"),
+        B_prev=_ptr(B_prev, dtype=act, device=dev, shape=(batch, DSTATE), name="B_prev"),
+    )
+    if out is None:
+        out = torch.empty_like(x)
+    if h_last is None:
+        h_last = torch.empty((batch, dim, DSTATE), dtype=f32, device=dev)
+    po = _ptr(out, dtype=act, device=dev, shape=x.shape, name="out")
+    ph = _ptr(h_last, dtype=f32, device=dev, shape=(batch, dim, DSTATE), name="h_last")
+    dims = Dims(batch, L, dim, DSTATE, code)
+    if workspace is None:
+        workspace = torch.empty(ssm_scan_fwd_workspace_size(batch, L, dim, dev), dtype=torch.uint8,
+                                device=dev)
+    pw = _ptr(workspace, dtype=torch.uint8, device=dev, name="workspace")
+    sp = _stream_ptr(stream, dev)
+    with torch.cuda.device(dev):
+        rc = get_lib().ssm_trap_scan_fwd(ptrs["x"], ptrs["delta"], ptrs["delta_bias"], int(bool(softplus)),
+                                         ptrs["lam"], ptrs["A"], ptrs["B"], ptrs["C"], ptrs["D"], ptrs["z"],
+                                         ptrs["h0"], ptrs["x_prev"], ptrs["B_prev"], po, ph, pw, workspace.numel(),
+                                         ctypes.byref(dims), sp)
+        _check(rc)
+        if check:
+            _check(get_lib().ssm_scan_fwd_status(pw, sp))
+    return out, h_last
+
+
+def ssm_trap_scan_step(state, x, delta, delta_bias, softplus, lam, A, B, C, D=None, z=None, x_prev=None,
+                       B_prev=None, out=None, stream=None):
+    """One trapezoidal decode step; ``state`` is updated in place.  lam:
+    [batch, dim]; x_prev [batch, dim], B_prev [batch, 16]: the previous token's."""
+    if x.device.type != "cuda":
+        raise ValueError("ssm_trap_scan_step needs CUDA tensors")
+    dev = x.device
+    batch, dim = x.shape
+    code = _act_code(x)
+    act = x.dtype
+    f32 = torch.float32
+    args = [_ptr(state, dtype=f32, device=dev, shape=(batch, dim, DSTATE), name="state"),
+            _ptr(x, dtype=act, device=dev, name="x"),
+            _ptr(delta, dtype=act, device=dev, shape=x.shape, name="delta"),
+            _ptr(delta_bias, dtype=f32, device=dev, shape=(dim,), name="delta_bias"), int(bool(softplus)),
+            _ptr(lam, dtype=act, device=dev, shape=x.shape, name="lam"),
+            _ptr(A, dtype=f32, device=dev, shape=(dim, DSTATE), name="A"),
+            _ptr(B, dtype=act, device=dev, shape=(batch, DSTATE), name="B"),
+            _ptr(C, dtype=act, device=dev, shape=(batch, DSTATE), name="C"),
+            _ptr(D, dtype=f32, device=dev, shape=(dim,), name="D"),
+            _ptr(z, dtype=act, device=dev, shape=x.shape, name="z"),
+            _ptr(x_prev, dtype=act, device=dev, shape=x.shape, name="x_prev"),
+            _ptr(B_prev, dtype=act, device=dev, shape=(batch, DSTATE), name="B_prev")]
+    if out is None:
+        out = torch.empty_like(x)
+    args.append(_ptr(out, dtype=act, device=dev, shape=x.shape, name="out"))
+    dims = Dims(batch, 1, dim, DSTATE, code)
+    with torch.cuda.device(dev):
+        rc = get_lib().ssm_trap_scan_step(*args, ctypes.byref(dims), _stream_ptr(stream, dev))
+    _check(rc)
+    return out
+
+
 def ssm_scan_step(state, x, delta, delta_bias, softplus, A, B, C, D=None, z=None, out=None,
                   stream=None):
     """One recurrent decode step; ``state`` ([batch, dim, 16] float32) is
@@ -333,5 +420,5 @@ def ssm_scan_step(state, x, delta, delta_bias, softplus, A, B, C, D=None, z=None
 
 
 __all__ = ["ssm_scan_fwd", "ssm_scan_fwd_workspace_size", "ssm_scan_fwd_status", "ssm_scan_step",
-           "ssm_conv_scan_fwd", "ssm_conv_scan_step",
+           "ssm_conv_scan_fwd", "ssm_conv_scan_step", "ssm_trap_scan_fwd", "ssm_trap_scan_step",
            "ssm_strerror", "ssm_version", "SSMError", "Dims", "LIB_PATH", "get_lib"]

@@ -67,6 +67,10 @@ struct FwdParams {
     const float *conv_w;        // [dim][conv_k]
     const float *conv_bias;     // [dim] or NULL
     const void *conv_state;     // [batch][dim][conv_k - 1] raw inputs before t = 0, or NULL
+    // The exponential-trapezoidal rule (lam != NULL): lam [batch][dim][L] mixes
+    // the interval's two ends; x_prev [batch][dim] and B_prev [batch][16] are
+    // the input before t = 0 (zero unless both are given).
+    const void *lam, *x_prev, *B_prev;
 };
 constexpr int kChained = 0, kSummary = 1, kFromStart = 2;
 
@@ -74,52 +78,62 @@ constexpr int kChained = 0, kSummary = 1, kFromStart = 2;
 // tensors with [1][32][TC] boxes and the 64-byte swizzle (the same XOR layout
 // as swz()), B and C as [batch][16][L] with [1][16][TC] boxes.
 struct TmaMaps {
-    CUtensorMap x, delta, z, B, C, out;
+    CUtensorMap x, delta, z, B, C, out, lam;
 };
 
 constexpr int kPairs = 4;                    // warp triples per CTA (one per SM sub-partition)
 constexpr int kFwdThreads = 96 * kPairs;     // warps 0..3 scan, 4..7 stage + prepare, 8..11 finish
 constexpr int kRowBytes = 64;  // bytes of one channel row of a chunk
 constexpr int kPieces = kRowBytes / 16;
-constexpr int kStages = 3;     // staged chunks per pair (post-processing, next, loading)
-constexpr int kBCPitch = 36;   // floats per time row of widened B|C (32 used)
+constexpr int kBCPitch = 36;   // floats per time row of widened B|C (32 used; float 32 holds C.B with TRAP)
 
 // Shared memory of one warp triple.  Stages hold raw chunks (x, delta, z
-// tiles and the B, C rows); bcf and ur are double-buffered per chunk parity.
-// bcf and ur carry one spare step row so that the scan warp's step-ahead
-// preparation can run unconditionally on a chunk's last step.
-template <typename T>
+// tiles, the B, C rows and, with TRAP, the lambda tile); bcf, ur and g are
+// double-buffered per chunk parity.  bcf, ur and g carry one spare step row
+// so that the scan warp's step-ahead preparation can run unconditionally on a
+// chunk's last step.  TRAP keeps two stages instead of three to make room for
+// its lambda tile and g table.
+template <typename T, bool TRAP = false>
 struct FwdSmem {
     static constexpr int kTC = kRowBytes / Act<T>::kBytes;          // timesteps per chunk
     static constexpr int kTileBytes = 32 * kRowBytes;               // one [32 ch][TC] tile
-    static constexpr int kStageBytes = 3 * kTileBytes + 2 * kNState * kRowBytes;
+    static constexpr int kStages = TRAP ? 2 : 3;                    // staged chunks per pair
+    static constexpr int kBCRawOff = 3 * kTileBytes;                // raw B|C rows in a stage
+    static constexpr int kLamOff = kBCRawOff + 2 * kNState * kRowBytes;
+    static constexpr int kStageBytes = kLamOff + (TRAP ? kTileBytes : 0);
     static constexpr int kBCFBytes = (kTC + 1) * kBCPitch * 4;      // widened B|C, time-major
     static constexpr int kURBytes = (kTC + 1) * 32 * 8;             // float2 (u, r) per [t][lane]
+    static constexpr int kGBytes = TRAP ? (kTC + 1) * 32 * 4 : 0;   // float g per [t][lane] (TRAP)
     static constexpr int kBCFOff = kStages * kStageBytes;
     static constexpr int kUROff = kBCFOff + 2 * kBCFBytes;
-    static constexpr int kDescOff = kUROff + 2 * kURBytes;          // ring of 4 chunk descriptors
-    static constexpr int kBarOff = kDescOff + 4 * 64;               // mbarriers ready[2], done[2], posted[2], full[3]
-    static constexpr int kPairBytes = (kBarOff + 9 * 8 + 1023) / 1024 * 1024;
+    static constexpr int kGOff = kUROff + 2 * kURBytes;
+    static constexpr int kDescOff = kGOff + 2 * kGBytes;            // ring of 4 chunk descriptors
+    static constexpr int kBarOff = kDescOff + 4 * 64;               // ready[2], done[2], posted[2], full[kStages]
+    static constexpr int kPairBytes = (kBarOff + (6 + kStages) * 8 + 1023) / 1024 * 1024;
     static constexpr int kTotal = kPairs * kPairBytes + 1024;       // + slack to align the base to 1 KB
 };
+static_assert(FwdSmem<bf16raw, true>::kTotal <= 227 * 1024, "shared memory of the trapezoidal kernel");
+static_assert(FwdSmem<bf16raw, false>::kTotal <= 227 * 1024, "shared memory of the kernel");
 
 __device__ __forceinline__ int swz(int row, int pc) { return pc ^ ((row >> 1) & 3); }
 
 // ---- staging one chunk [t0, t0 + TC) of a warp's 32 channels element by element
 // (rows that are not 16-byte aligned, L * size % 16 != 0, cannot use TMA)
-template <typename T>
+template <typename T, bool TRAP = false>
 __device__ __forceinline__ void load_chunk_sync(const FwdParams &p, uint8_t *stage, int64_t b,
                                                 int64_t d0, int64_t t0, int lane) {
     using AT = Act<T>;
+    using SM = FwdSmem<T, TRAP>;
     using W = typename std::conditional<AT::kBytes == 2, uint16_t, uint32_t>::type;
-    constexpr int PP = AT::kPerPiece, TC = FwdSmem<T>::kTC;
+    constexpr int PP = AT::kPerPiece, TC = SM::kTC;
     const int64_t L = p.seqlen;
-    const void *const srcs[3] = {p.x, p.delta, p.z};
+    const void *const srcs[4] = {p.x, p.delta, p.z, TRAP ? p.lam : nullptr};
+    const int offs[4] = {0, SM::kTileBytes, 2 * SM::kTileBytes, SM::kLamOff};
 #pragma unroll
-    for (int k = 0; k < 3; ++k) {
+    for (int k = 0; k < 4; ++k) {
         if (srcs[k] == nullptr) continue;
         const W *base = static_cast<const W *>(srcs[k]);
-        uint8_t *tile = stage + k * FwdSmem<T>::kTileBytes;
+        uint8_t *tile = stage + offs[k];
         for (int row = 0; row < 32; ++row) {
             const int64_t d = d0 + row;
             for (int col = lane; col < TC; col += 32) {
@@ -135,7 +149,7 @@ __device__ __forceinline__ void load_chunk_sync(const FwdParams &p, uint8_t *sta
         for (int col = lane; col < TC; col += 32) {
             const int64_t t = t0 + col;
             const W v = t < L ? base[(b * kNState + (j & 15)) * L + t] : W(0);
-            *reinterpret_cast<W *>(stage + 3 * FwdSmem<T>::kTileBytes + j * kRowBytes + col * AT::kBytes) = v;
+            *reinterpret_cast<W *>(stage + SM::kBCRawOff + j * kRowBytes + col * AT::kBytes) = v;
         }
     }
 }
@@ -143,24 +157,37 @@ __device__ __forceinline__ void load_chunk_sync(const FwdParams &p, uint8_t *sta
 // Widen the chunk's B and C to float32, time-major: bcf[t][0..15] = B[.][t],
 // bcf[t][16..31] = C[.][t].  Lanes take consecutive t so each 16-byte store
 // of a quarter-warp lands in a distinct bank group (pitch 36 floats).
-template <typename T>
+// With TRAP the B half is shifted down one row (row t holds B of step t-1,
+// row TC the chunk's last B; the caller fills row 0's B half), and float 32
+// of row t holds C_t . B_t.
+template <typename T, bool TRAP = false>
 __device__ __forceinline__ void widen_bc(const uint8_t *raw, float *bcf, int lane) {
     using AT = Act<T>;
     using W = typename std::conditional<AT::kBytes == 2, uint16_t, uint32_t>::type;
     constexpr int TC = FwdSmem<T>::kTC;
+    auto rd = [&](int j, int t) {
+        const W w = reinterpret_cast<const W *>(raw + j * kRowBytes)[t];
+        if constexpr (AT::kBytes == 2)
+            return __uint_as_float(static_cast<uint32_t>(w) << 16);
+        else
+            return __uint_as_float(w);
+    };
 #pragma unroll
     for (int item = lane; item < TC * 8; item += 32) {
         const int t = item % TC, jg = item / TC;
         float v[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const W w = reinterpret_cast<const W *>(raw + (jg * 4 + q) * kRowBytes)[t];
-            if constexpr (AT::kBytes == 2)
-                v[q] = __uint_as_float(static_cast<uint32_t>(w) << 16);
-            else
-                v[q] = __uint_as_float(w);
+        for (int q = 0; q < 4; ++q) v[q] = rd(jg * 4 + q, t);
+        const int row = (TRAP && jg < 4) ? t + 1 : t;
+        *reinterpret_cast<float4 *>(bcf + row * kBCPitch + jg * 4) = make_float4(v[0], v[1], v[2], v[3]);
+    }
+    if constexpr (TRAP) {
+        if (lane < TC) {
+            float cb = 0.0f;
+#pragma unroll
+            for (int n = 0; n < kNState; ++n) cb = fmaf(rd(kNState + n, lane), rd(n, lane), cb);
+            bcf[lane * kBCPitch + 32] = cb;
         }
-        *reinterpret_cast<float4 *>(bcf + t * kBCPitch + jg * 4) = make_float4(v[0], v[1], v[2], v[3]);
     }
 }
 
@@ -203,9 +230,18 @@ __device__ __forceinline__ void conv_halo(const FwdParams &p, int64_t b, int64_t
 // inputs before it (halo, updated to this chunk's last three) give the
 // convolution, whose output replaces the raw row in the stage (in the
 // activation dtype, for the post warp's D skip) and feeds u = dt x in float32.
-template <typename T, bool S4D, bool CONV>
+//
+// With TRAP (the exponential-trapezoidal rule), ur gets (s_t, r_t) and g gets
+// g_t, where g_t = lam_t dt_t x_t weights the interval's end and
+// s_t = g_{t-1} + (1 - lam_t) dt_t x_{t-1} its start.  The scan then carries
+// h~_t = h_t - g_t B_t, for which h~_t = Abar_t (h~_{t-1} + s_t B_{t-1}): the
+// same work per state as the Euler rule.  x_last and g_last hold the step
+// before the chunk (updated to the chunk's last step).
+template <typename T, bool S4D, bool CONV, bool TRAP = false>
 __device__ __forceinline__ void chunk_prepass(uint8_t *stage, float2 *ur, int row,
-                                              const ChanConst &cc, bool softplus, float (&halo)[3]) {
+                                              const ChanConst &cc, bool softplus, float (&halo)[3],
+                                              float *garr = nullptr, float *x_last = nullptr,
+                                              float *g_last = nullptr) {
     using AT = Act<T>;
     constexpr bool kAccurate = AT::kBytes == 4;
     constexpr int PP = AT::kPerPiece, TC = FwdSmem<T>::kTC, NP = TC / 2;
@@ -289,12 +325,61 @@ __device__ __forceinline__ void chunk_prepass(uint8_t *stage, float2 *ur, int ro
 #pragma unroll
         for (int k = 0; k < NP; ++k) E[k] = make_float2(ex2_approx(E[k].x), ex2_approx(E[k].y));
     }
+    if constexpr (TRAP) {
+        const uint8_t *lr = stage + FwdSmem<T, true>::kLamOff + row * kRowBytes;
+        uint4 lv[kPieces];
 #pragma unroll
-    for (int k = 0; k < NP; ++k) {
-        const float2 U = __fmul2_rn(V[k], make_float2(XC[2 * k], XC[2 * k + 1]));
-        ur[(2 * k) * 32 + row] = make_float2(U.x, E[k].x);
-        ur[(2 * k + 1) * 32 + row] = make_float2(U.y, E[k].y);
+        for (int pc = 0; pc < kPieces; ++pc) lv[pc] = *reinterpret_cast<const uint4 *>(lr + (swz(row, pc) << 4));
+        float xp = *x_last, gp = *g_last;
+#pragma unroll
+        for (int k = 0; k < NP; ++k) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int t = 2 * k + e;
+                const float dt = e ? V[k].y : V[k].x;
+                const float lam = AT::piece(lv[t / PP], t % PP);
+                const float g = lam * dt * XC[t];
+                const float sv = fmaf((1.0f - lam) * dt, xp, gp);
+                ur[t * 32 + row] = make_float2(sv, e ? E[k].y : E[k].x);
+                garr[t * 32 + row] = g;
+                xp = XC[t];
+                gp = g;
+            }
+        }
+        *x_last = xp;
+        *g_last = gp;
+    } else {
+#pragma unroll
+        for (int k = 0; k < NP; ++k) {
+            const float2 U = __fmul2_rn(V[k], make_float2(XC[2 * k], XC[2 * k + 1]));
+            ur[(2 * k) * 32 + row] = make_float2(U.x, E[k].x);
+            ur[(2 * k + 1) * 32 + row] = make_float2(U.y, E[k].y);
+        }
     }
+}
+
+// The trapezoidal rule's history at a segment start t0 (one lane): the input
+// x_{t0-1}, its end weight g_{t0-1} = lam dt x, and (lanes 0..15) B_{t0-1}[lane]
+// into row 0 of the widened table; from x_prev and B_prev at t0 = 0.
+template <typename T>
+__device__ __forceinline__ void trap_history(const FwdParams &p, int64_t b, int64_t d, int64_t t0, int lane,
+                                             const ChanConst &cc, float *bcf, float *x_last, float *g_last) {
+    using AT = Act<T>;
+    const int64_t chan = b * p.dim + d;
+    const bool prev = p.x_prev && p.B_prev;
+    if (t0 == 0) {
+        *x_last = prev ? AT::load(p.x_prev, chan) : 0.0f;
+        *g_last = 0.0f;
+        if (lane < kNState) bcf[lane] = prev ? AT::load(p.B_prev, b * kNState + lane) : 0.0f;
+        return;
+    }
+    const int64_t i = chan * p.seqlen + t0 - 1;
+    const float xv = AT::load(p.x, i);
+    float v = AT::load(p.delta, i) + cc.biasx2.x;
+    if (p.softplus) v = AT::kBytes == 4 ? softplus_accurate(v) : softplus_fast(v);
+    *x_last = xv;
+    *g_last = AT::load(p.lam, i) * v * xv;
+    if (lane < kNState) bcf[lane] = AT::load(p.B, (b * kNState + lane) * p.seqlen + t0 - 1);
 }
 
 // ---- phase 2: the recurrence ---------------------------------------------------
@@ -302,11 +387,15 @@ __device__ __forceinline__ void chunk_prepass(uint8_t *stage, float2 *ur, int ro
 // pairs, c = C pairs.
 struct StepOps {
     float2 a[8], ub[8], c[8];
+    float gcb;  // TRAP: g_t (C_t . B_t), the readout of the interval's end term
 };
 
-template <bool S4D, bool READOUT = true>
+// With TRAP, ur holds (s_t, r_t) and row t's B half holds B_{t-1}, so ub is
+// s_t B_{t-1}; gcb comes from the g table and float 32 of the row.
+template <bool S4D, bool READOUT = true, bool TRAP = false>
 __device__ __forceinline__ void prepare_step(const float *bcf, const float2 *ur, int t, int row,
-                                             const float (&a2)[kNState], StepOps &s) {
+                                             const float (&a2)[kNState], StepOps &s, const float *garr = nullptr) {
+    if constexpr (TRAP && READOUT) s.gcb = garr[t * 32 + row] * bcf[t * kBCPitch + 32];
     const float2 ut_rt = ur[t * 32 + row];
     const float4 *p = reinterpret_cast<const float4 *>(bcf + t * kBCPitch);
     const float2 U2 = make_float2(ut_rt.x, ut_rt.x);
@@ -346,11 +435,14 @@ __device__ __forceinline__ void prepare_step(const float *bcf, const float2 *ur,
 // as float `lane` of row t of ur, over (u, r) pairs the warp has already read.  Full chunks run a branch-free body (the preparation of the
 // step after the chunk reads the spare table row); only the last, partial
 // chunk of a sequence tests the step index.
-template <bool S4D, bool FULL>
+// With TRAP the carried state is h~ (see chunk_prepass): h~ = Abar (h~ + s B_{t-1})
+// and y = C . h~ + g (C . B).
+template <bool S4D, bool FULL, bool TRAP = false>
 __device__ __forceinline__ void chunk_core(const float *bcf, float2 *ur, int row, int nvalid,
-                                           const float (&a2)[kNState], float2 (&h)[8]) {
+                                           const float (&a2)[kNState], float2 (&h)[8],
+                                           const float *garr = nullptr) {
     StepOps nxt;
-    prepare_step<S4D>(bcf, ur, 0, row, a2, nxt);
+    prepare_step<S4D, true, TRAP>(bcf, ur, 0, row, a2, nxt, garr);
 #pragma unroll 1
     for (int t0 = 0; t0 < nvalid; t0 += 8) {
 #pragma unroll
@@ -358,11 +450,14 @@ __device__ __forceinline__ void chunk_core(const float *bcf, float2 *ur, int row
             const int t = t0 + i;
             if (!FULL && t >= nvalid) break;
             const StepOps cur = nxt;
-            if (FULL || t + 1 < nvalid) prepare_step<S4D>(bcf, ur, t + 1, row, a2, nxt);
-            float2 ya = make_float2(0.0f, 0.0f), yb = make_float2(0.0f, 0.0f);
+            if (FULL || t + 1 < nvalid) prepare_step<S4D, true, TRAP>(bcf, ur, t + 1, row, a2, nxt, garr);
+            float2 ya = make_float2(TRAP ? cur.gcb : 0.0f, 0.0f), yb = make_float2(0.0f, 0.0f);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                h[j] = __ffma2_rn(cur.a[j], h[j], cur.ub[j]);
+                if constexpr (TRAP)
+                    h[j] = __fmul2_rn(cur.a[j], __fadd2_rn(h[j], cur.ub[j]));
+                else
+                    h[j] = __ffma2_rn(cur.a[j], h[j], cur.ub[j]);
                 if (j & 1) yb = __ffma2_rn(cur.c[j], h[j], yb);
                 else ya = __ffma2_rn(cur.c[j], h[j], ya);
             }
@@ -376,7 +471,7 @@ __device__ __forceinline__ void chunk_core(const float *bcf, float2 *ur, int row
 // the running product of the per-step decays P_n = prod_t Abar_{t,n} in place
 // of the readout (so P carries the rounding of the decays the sequential scan
 // applies).  No y is produced.
-template <bool S4D, bool FULL>
+template <bool S4D, bool FULL, bool TRAP = false>
 __device__ __forceinline__ void chunk_summary(const float *bcf, const float2 *ur, int row, int nvalid,
                                               const float (&a2)[kNState], float2 (&h)[8], float2 (&P)[8]) {
     StepOps nxt;
@@ -391,7 +486,10 @@ __device__ __forceinline__ void chunk_summary(const float *bcf, const float2 *ur
             if (FULL || t + 1 < nvalid) prepare_step<S4D, false>(bcf, ur, t + 1, row, a2, nxt);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                h[j] = __ffma2_rn(cur.a[j], h[j], cur.ub[j]);
+                if constexpr (TRAP)
+                    h[j] = __fmul2_rn(cur.a[j], __fadd2_rn(h[j], cur.ub[j]));
+                else
+                    h[j] = __ffma2_rn(cur.a[j], h[j], cur.ub[j]);
                 P[j] = __fmul2_rn(cur.a[j], P[j]);
             }
         }
@@ -697,7 +795,7 @@ struct ChunkCursor {
 // sub-partition.  Two instances run back to back: the S4D one takes groups
 // whose A rows are all S4D-structured and marks the scratch when it meets
 // another group; the general one then takes those.
-template <typename T, bool VEC, bool S4D, bool CONV>
+template <typename T, bool VEC, bool S4D, bool CONV, bool TRAP>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     scan_fwd_kernel(const FwdParams p, const FwdScratch sc, const __grid_constant__ TmaMaps tm) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -707,8 +805,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // rather than generic accesses, which cost twice the data-pipe passes on a
     // warp-uniform read.
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    using SM = FwdSmem<T>;
+    using SM = FwdSmem<T, TRAP>;
     constexpr int TC = SM::kTC;
+    constexpr int kStages = SM::kStages;
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int pair = warp & (kPairs - 1);
@@ -722,6 +821,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     auto stage_of = [&](int64_t j) { return ps + (j % kStages) * SM::kStageBytes; };
     auto bcf_of = [&](int64_t j) { return reinterpret_cast<float *>(ps + SM::kBCFOff + (j & 1) * SM::kBCFBytes); };
     auto ur_of = [&](int64_t j) { return reinterpret_cast<float2 *>(ps + SM::kUROff + (j & 1) * SM::kURBytes); };
+    auto g_of = [&](int64_t j) { return reinterpret_cast<float *>(ps + SM::kGOff + (j & 1) * SM::kGBytes); };
     auto parity = [](int64_t j, int n) { return static_cast<uint32_t>((j / n) & 1); };
 
     if (threadIdx.x < kPairs) {
@@ -737,7 +837,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     if (role == 1) {
         // ------------------------------------------------------------------ prep
         ChunkCursor<T, S4D> cur(p);
-        const uint32_t stage_tx = (p.z ? 3u : 2u) * SM::kTileBytes + 2u * kNState * kRowBytes;
+        const uint32_t stage_tx = (p.z ? 3u : 2u) * SM::kTileBytes + 2u * kNState * kRowBytes +
+                                  (TRAP ? static_cast<uint32_t>(SM::kTileBytes) : 0u);
         // TMA loads issued and waited for, in chunk order: every issued load is
         // waited for before the warp leaves, also when it gives up early
         int64_t n_issued = 0, n_waited = 0;
@@ -753,24 +854,28 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     tma_load_3d(st, &tm.x, t0, d0, b, bar);
                     tma_load_3d(st + SM::kTileBytes, &tm.delta, t0, d0, b, bar);
                     if (p.z) tma_load_3d(st + 2 * SM::kTileBytes, &tm.z, t0, d0, b, bar);
-                    tma_load_3d(st + 3 * SM::kTileBytes, &tm.B, t0, 0, b, bar);
-                    tma_load_3d(st + 3 * SM::kTileBytes + kNState * kRowBytes, &tm.C, t0, 0, b, bar);
+                    tma_load_3d(st + SM::kBCRawOff, &tm.B, t0, 0, b, bar);
+                    tma_load_3d(st + SM::kBCRawOff + kNState * kRowBytes, &tm.C, t0, 0, b, bar);
+                    if (TRAP) tma_load_3d(st + SM::kLamOff, &tm.lam, t0, d0, b, bar);
                 }
                 n_issued = j + 1;
             } else {
-                load_chunk_sync<T>(p, st, dsc.b, dsc.d0, dsc.t0, lane);
+                load_chunk_sync<T, TRAP>(p, st, dsc.b, dsc.d0, dsc.t0, lane);
             }
         };
         const bool softplus = p.softplus != 0;
         ChanConst cc;
         int64_t cc_d0 = -1;
         float halo[3] = {0.0f, 0.0f, 0.0f};  // convolution inputs before the chunk (CONV)
+        float x_last = 0.0f, g_last = 0.0f;  // the step before the chunk (TRAP)
         ChunkDesc dnext = cur.next(p, sc, counter, lane);
         issue(dnext, 0);
         for (int64_t j = 0;; ++j) {
             const ChunkDesc dj = dnext;
-            // chunk j+1 goes to the stage that chunk j-2 used: wait until it is posted
-            if (j >= 2 && !mbar_wait(posted + (j & 1), parity(j - 2, 2), sc.error)) break;
+            // chunk j+1 goes to the stage that chunk j+1-kStages used: wait until it is posted
+            if (j >= kStages - 1 &&
+                !mbar_wait(posted + ((j + 1 - kStages) & 1), parity(j + 1 - kStages, 2), sc.error))
+                break;
             if (!(dj.flags & kStop)) {
                 dnext = cur.next(p, sc, counter, lane);
                 issue(dnext, j + 1);
@@ -780,17 +885,28 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 }
                 __syncwarp();
                 uint8_t *st = stage_of(j);
-                widen_bc<T>(st + 3 * SM::kTileBytes, bcf_of(j), lane);
+                widen_bc<T, TRAP>(st + SM::kBCRawOff, bcf_of(j), lane);
                 if (dj.d0 != cc_d0) {  // the channel constants change only with the group
                     const int64_t d = dj.d0 + lane;
                     cc = chan_const(p, d < p.dim ? d : p.dim - 1);
                     cc_d0 = dj.d0;
                 }
+                if constexpr (TRAP) {
+                    // row 0's B half: B of the step before the chunk
+                    if (dj.flags & kFirst) {
+                        const int64_t d = dj.d0 + lane;
+                        trap_history<T>(p, dj.b, d < p.dim ? d : p.dim - 1, dj.t0, lane, cc, bcf_of(j), &x_last,
+                                        &g_last);
+                    } else if (lane < kNState) {
+                        bcf_of(j)[lane] = bcf_of(j - 1)[TC * kBCPitch + lane];
+                    }
+                }
                 if (CONV && (dj.flags & kFirst)) {
                     const int64_t d = dj.d0 + lane;
                     conv_halo<T>(p, dj.b, d < p.dim ? d : p.dim - 1, dj.t0, halo);
                 }
-                chunk_prepass<T, S4D, CONV>(st, ur_of(j), lane, cc, softplus, halo);
+                chunk_prepass<T, S4D, CONV, TRAP>(st, ur_of(j), lane, cc, softplus, halo, g_of(j), &x_last,
+                                                  &g_last);
             }
             if (lane == 0) ring[j & 3] = dj;
             __syncwarp();
@@ -893,13 +1009,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             }
             if (p.mode == kSummary) {
                 if (dk.nvalid == TC)
-                    chunk_summary<S4D, true>(bcf_of(k), ur_of(k), lane, TC, a2, h, P);
+                    chunk_summary<S4D, true, TRAP>(bcf_of(k), ur_of(k), lane, TC, a2, h, P);
                 else
-                    chunk_summary<S4D, false>(bcf_of(k), ur_of(k), lane, dk.nvalid, a2, h, P);
+                    chunk_summary<S4D, false, TRAP>(bcf_of(k), ur_of(k), lane, dk.nvalid, a2, h, P);
             } else if (dk.nvalid == TC) {
-                chunk_core<S4D, true>(bcf_of(k), ur_of(k), lane, TC, a2, h);
+                chunk_core<S4D, true, TRAP>(bcf_of(k), ur_of(k), lane, TC, a2, h, g_of(k));
             } else {
-                chunk_core<S4D, false>(bcf_of(k), ur_of(k), lane, dk.nvalid, a2, h);
+                chunk_core<S4D, false, TRAP>(bcf_of(k), ur_of(k), lane, dk.nvalid, a2, h, g_of(k));
             }
             if (dk.flags & kLast) {
                 if (p.mode == kSummary) {
@@ -923,9 +1039,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     }
                 } else if (active && p.h_last) {
                     float4 *hr = reinterpret_cast<float4 *>(p.h_last + (dk.b * p.dim + d) * kNState);
+                    float2 hv[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) hv[j] = h[j];
+                    if constexpr (TRAP) {
+                        // h = h~ + g B of the sequence's last step (row nvalid's B half holds B_{L-1})
+                        const float g = g_of(k)[(dk.nvalid - 1) * 32 + lane];
+                        const float *bl = bcf_of(k) + dk.nvalid * kBCPitch;
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) hv[j] = __ffma2_rn(make_float2(g, g), make_float2(bl[2 * j], bl[2 * j + 1]), hv[j]);
+                    }
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
-                        hr[q] = make_float4(h[2 * q].x, h[2 * q].y, h[2 * q + 1].x, h[2 * q + 1].y);
+                        hr[q] = make_float4(hv[2 * q].x, hv[2 * q].y, hv[2 * q + 1].x, hv[2 * q + 1].y);
                 }
             }
             __syncwarp();

@@ -28,6 +28,9 @@ struct StepParams {
     const float *conv_w;        // [dim][conv_k]
     const float *conv_bias;     // [dim] or NULL
     void *conv_state;           // [batch][dim][conv_k - 1] raw inputs, oldest first; read and shifted
+    // the exponential-trapezoidal rule: lam [batch][dim]; the previous token's
+    // x_prev [batch][dim] and B_prev [batch][16] (no previous input unless both)
+    const void *lam, *x_prev, *B_prev;
 };
 
 constexpr int kStepThreads = 256;
@@ -48,7 +51,8 @@ __device__ __forceinline__ float4 load4(const void *p, int64_t i) {
 // SMALL: every channel index fits in 32 bits, so (b, d) come from a 32-bit division.
 // CONV: the token first passes the convolution window (every lane of a
 // channel computes it; the first lane shifts the stored window).
-template <typename T, bool SMALL, bool CONV>
+// TRAP: h = Abar (h + (1 - lam) dt x_prev B_prev) + lam dt x B.
+template <typename T, bool SMALL, bool CONV, bool TRAP = false>
 __global__ void __launch_bounds__(kStepThreads) scan_step_kernel(const StepParams p) {
     using AT = Act<T>;
     constexpr bool kAccurate = AT::kBytes == 4;
@@ -99,10 +103,22 @@ __global__ void __launch_bounds__(kStepThreads) scan_step_kernel(const StepParam
     const float u = dt * xf;
     const float e = kLog2e * dt;
 
-    h.x = ex2_approx(a.x * e) * h.x + u * Bv.x;
-    h.y = ex2_approx(a.y * e) * h.y + u * Bv.y;
-    h.z = ex2_approx(a.z * e) * h.z + u * Bv.z;
-    h.w = ex2_approx(a.w * e) * h.w + u * Bv.w;
+    if constexpr (TRAP) {
+        const float lam = AT::load(p.lam, c);
+        const bool prev = p.x_prev && p.B_prev;
+        const float f = prev ? (1.0f - lam) * dt * AT::load(p.x_prev, c) : 0.0f;
+        const float4 Bp = prev ? load4<T>(p.B_prev, bn) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        const float g = lam * u;
+        h.x = ex2_approx(a.x * e) * fmaf(f, Bp.x, h.x) + g * Bv.x;
+        h.y = ex2_approx(a.y * e) * fmaf(f, Bp.y, h.y) + g * Bv.y;
+        h.z = ex2_approx(a.z * e) * fmaf(f, Bp.z, h.z) + g * Bv.z;
+        h.w = ex2_approx(a.w * e) * fmaf(f, Bp.w, h.w) + g * Bv.w;
+    } else {
+        h.x = ex2_approx(a.x * e) * h.x + u * Bv.x;
+        h.y = ex2_approx(a.y * e) * h.y + u * Bv.y;
+        h.z = ex2_approx(a.z * e) * h.z + u * Bv.z;
+        h.w = ex2_approx(a.w * e) * h.w + u * Bv.w;
+    }
     float y = (Cv.x * h.x + Cv.y * h.y) + (Cv.z * h.z + Cv.w * h.w);
     y += __shfl_xor_sync(0xffffffffu, y, 1);
     y += __shfl_xor_sync(0xffffffffu, y, 2);

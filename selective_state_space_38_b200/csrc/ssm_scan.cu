@@ -87,6 +87,7 @@ bool make_maps(const FwdParams &p, TmaMaps *tm) {
               encode3d(&tm->B, dt, es, p.B, L, kNState, Bt, tc, kNState, CU_TENSOR_MAP_SWIZZLE_NONE) &&
               encode3d(&tm->C, dt, es, p.C, L, kNState, Bt, tc, kNState, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (ok && p.z) ok = encode3d(&tm->z, dt, es, p.z, L, D, Bt, tc, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+    if (ok && p.lam) ok = encode3d(&tm->lam, dt, es, p.lam, L, D, Bt, tc, 32, CU_TENSOR_MAP_SWIZZLE_64B);
     return ok;
 }
 
@@ -112,29 +113,29 @@ int64_t parallel_segments(const FwdParams &p, int sms, int64_t *seg_steps) {
 
 // Persistent launch: one CTA of kPairs warp triples per SM (or fewer when there
 // are fewer items); the S4D instance, then the general one.
-template <typename T, bool VEC, bool CONV>
+template <typename T, bool VEC, bool CONV, bool TRAP>
 int launch_pass(const FwdParams &p, const FwdScratch &sc, const TmaMaps &tm, int sms, cudaStream_t stream) {
     const int64_t groups = ((p.dim + 31) / 32) * p.batch;
     const int64_t items = groups * ((p.seqlen + p.seg_steps - 1) / p.seg_steps);
     const int64_t want = (items + kPairs - 1) / kPairs;
     const int64_t ctas = want < sms ? want : sms;
-    const int smem = FwdSmem<T>::kTotal;
-    scan_fwd_kernel<T, VEC, true, CONV><<<static_cast<unsigned>(ctas), kFwdThreads, smem, stream>>>(p, sc, tm);
-    scan_fwd_kernel<T, VEC, false, CONV><<<static_cast<unsigned>(ctas), kFwdThreads, smem, stream>>>(p, sc, tm);
+    const int smem = FwdSmem<T, TRAP>::kTotal;
+    scan_fwd_kernel<T, VEC, true, CONV, TRAP><<<static_cast<unsigned>(ctas), kFwdThreads, smem, stream>>>(p, sc, tm);
+    scan_fwd_kernel<T, VEC, false, CONV, TRAP><<<static_cast<unsigned>(ctas), kFwdThreads, smem, stream>>>(p, sc, tm);
     return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
 // The kernels of one forward call on zeroed scratch: one chained pass, or the
 // summary pass, the segment combine and the second pass of the time-parallel
 // schedule (the queue is re-armed between the passes).
-template <typename T, bool VEC, bool CONV>
+template <typename T, bool VEC, bool CONV, bool TRAP>
 int launch_fwd_kernels(FwdParams p, void *scratch, int64_t segs, int sms, cudaStream_t stream) {
     const int64_t groups = ((p.dim + 31) / 32) * p.batch;
-    const int smem = FwdSmem<T>::kTotal;
-    if (cudaFuncSetAttribute(scan_fwd_kernel<T, VEC, true, CONV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess ||
-        cudaFuncSetAttribute(scan_fwd_kernel<T, VEC, false, CONV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
+    const int smem = FwdSmem<T, TRAP>::kTotal;
+    if (cudaFuncSetAttribute(scan_fwd_kernel<T, VEC, true, CONV, TRAP>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+        cudaFuncSetAttribute(scan_fwd_kernel<T, VEC, false, CONV, TRAP>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return SSM_ERR_CUDA;
     TmaMaps tm;
     memset(&tm, 0, sizeof tm);
@@ -144,11 +145,11 @@ int launch_fwd_kernels(FwdParams p, void *scratch, int64_t segs, int sms, cudaSt
         p.mode = kChained;
         p.pass = 0;
         p.seg_steps = kSegSteps;
-        return launch_pass<T, VEC, CONV>(p, sc, tm, sms, stream);
+        return launch_pass<T, VEC, CONV, TRAP>(p, sc, tm, sms, stream);
     }
     p.mode = kSummary;
     p.pass = 0;
-    int rc = launch_pass<T, VEC, CONV>(p, sc, tm, sms, stream);
+    int rc = launch_pass<T, VEC, CONV, TRAP>(p, sc, tm, sms, stream);
     if (rc != SSM_OK) return rc;
     const int64_t threads = groups * 32;
     segment_combine_kernel<<<static_cast<unsigned>((threads + 127) / 128), 128, 0, stream>>>(p, sc);
@@ -156,7 +157,7 @@ int launch_fwd_kernels(FwdParams p, void *scratch, int64_t segs, int sms, cudaSt
     // first pass stays set for the status query
     p.mode = kFromStart;
     p.pass = 1;
-    return launch_pass<T, VEC, CONV>(p, sc, tm, sms, stream);
+    return launch_pass<T, VEC, CONV, TRAP>(p, sc, tm, sms, stream);
 }
 
 // SMs of the current device (the schedule, and so the workspace size, depend on it)
@@ -177,13 +178,13 @@ size_t fwd_workspace_bytes(const FwdParams &p, int sms) {
 }
 
 // One forward call on the caller's workspace: zero its flag words, then the kernels.
-template <typename T, bool VEC, bool CONV>
+template <typename T, bool VEC, bool CONV, bool TRAP = false>
 int launch_fwd(FwdParams p, void *ws, size_t ws_bytes, int sms, bool force_chained, cudaStream_t stream) {
     const int64_t groups = ((p.dim + 31) / 32) * p.batch;
     const int64_t segs = force_chained ? 0 : parallel_segments(p, sms, &p.seg_steps);
     if (ws_bytes < fwd_scratch_bytes(groups, segs)) return SSM_ERR_INVALID_ARG;
     if (cudaMemsetAsync(ws, 0, fwd_scratch_flag_bytes(groups), stream) != cudaSuccess) return SSM_ERR_CUDA;
-    return launch_fwd_kernels<T, VEC, CONV>(p, ws, segs, sms, stream);
+    return launch_fwd_kernels<T, VEC, CONV, TRAP>(p, ws, segs, sms, stream);
 }
 
 // The convolution in front of the scan, when a forward call has one.
@@ -195,15 +196,22 @@ struct ConvArgs {
     void *state_out;     // [batch][dim][k-1] activation dtype, or NULL; may be `state`
 };
 
-template <typename T, bool CONV>
+// The exponential-trapezoidal rule, when a forward call or step uses it.
+struct TrapArgs {
+    const void *lam;     // [batch][dim][seqlen] (forward) or [batch][dim] (step), activation dtype
+    const void *x_prev;  // [batch][dim] activation dtype, or NULL
+    const void *B_prev;  // [batch][dstate] activation dtype, or NULL
+};
+
+template <typename T, bool CONV, bool TRAP = false>
 int launch_step(const StepParams &p, cudaStream_t stream) {
     const int64_t threads = p.batch * p.dim * 4;
     const int64_t blocks = (threads + kStepThreads - 1) / kStepThreads;
     if (blocks > INT_MAX) return SSM_ERR_UNSUPPORTED;
     if (p.batch * p.dim < (int64_t(1) << 31))
-        scan_step_kernel<T, true, CONV><<<static_cast<unsigned>(blocks), kStepThreads, 0, stream>>>(p);
+        scan_step_kernel<T, true, CONV, TRAP><<<static_cast<unsigned>(blocks), kStepThreads, 0, stream>>>(p);
     else
-        scan_step_kernel<T, false, CONV><<<static_cast<unsigned>(blocks), kStepThreads, 0, stream>>>(p);
+        scan_step_kernel<T, false, CONV, TRAP><<<static_cast<unsigned>(blocks), kStepThreads, 0, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
@@ -212,20 +220,21 @@ int launch_step(const StepParams &p, cudaStream_t stream) {
 // overlap anything.
 int validate_step(float *state, const void *x, const void *delta, const float *delta_bias, int softplus,
                   const float *A, const void *B, const void *C, const float *D, const void *z, void *out,
-                  const ConvArgs *conv, const ssm_dims_t *dims, StepParams *p) {
+                  const ConvArgs *conv, const ssm_dims_t *dims, StepParams *p, const TrapArgs *trap = nullptr) {
     if (!dims) return SSM_ERR_INVALID_ARG;
     const int64_t batch = dims->batch, dim = dims->dim, N = dims->dstate;
     if (!state || !x || !delta || !A || !B || !C || !out) return SSM_ERR_INVALID_ARG;
     if (conv && (!conv->w || (conv->k > 1 && !conv->state_out))) return SSM_ERR_INVALID_ARG;
+    if (trap && !trap->lam) return SSM_ERR_INVALID_ARG;
     if (!dims_ok(batch, 1, dim) || N < 1) return SSM_ERR_INVALID_ARG;
     if (N != kNState) return SSM_ERR_UNSUPPORTED;
     if (dims->act_dtype != SSM_F32 && dims->act_dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
     if (conv && (conv->k < 1 || conv->k > 4)) return SSM_ERR_UNSUPPORTED;
     const size_t es = dims->act_dtype == SSM_F32 ? 4 : 2;
     // state, A, B and C are read (and the state written) as 16-byte vectors per lane
-    for (const void *ptr : {(const void *)state, (const void *)A, B, C})
-        if (!aligned16(ptr)) return SSM_ERR_MISALIGNED;
-    for (const void *ptr : {x, delta, z, (const void *)out})
+    for (const void *ptr : {(const void *)state, (const void *)A, B, C, trap ? trap->B_prev : nullptr})
+        if (ptr && !aligned16(ptr)) return SSM_ERR_MISALIGNED;
+    for (const void *ptr : {x, delta, z, (const void *)out, trap ? trap->lam : nullptr, trap ? trap->x_prev : nullptr})
         if (ptr && reinterpret_cast<uintptr_t>(ptr) % es != 0) return SSM_ERR_MISALIGNED;
     for (const void *ptr : {(const void *)delta_bias, (const void *)D})
         if (ptr && !aligned4(ptr)) return SSM_ERR_MISALIGNED;
@@ -241,7 +250,9 @@ int validate_step(float *state, const void *x, const void *delta, const float *d
                         {A, static_cast<size_t>(dim) * N * 4}, {D, D ? static_cast<size_t>(dim) * 4 : 0},
                         {delta_bias, delta_bias ? static_cast<size_t>(dim) * 4 : 0},
                         {conv ? conv->w : nullptr, conv ? static_cast<size_t>(dim) * conv->k * 4 : 0},
-                        {conv && conv->bias ? conv->bias : nullptr, static_cast<size_t>(dim) * 4}};
+                        {conv && conv->bias ? conv->bias : nullptr, static_cast<size_t>(dim) * 4},
+                        {trap ? trap->lam : nullptr, nch * es}, {trap ? trap->x_prev : nullptr, nch * es},
+                        {trap ? trap->B_prev : nullptr, static_cast<size_t>(batch) * N * es}};
     const Span outs[] = {{out, nch * es}, {state, nch * N * 4},
                          {conv && conv->k > 1 ? conv->state_out : nullptr, conv ? nch * (conv->k - 1) * es : 0}};
     for (int o = 0; o < 3; ++o) {
@@ -261,6 +272,11 @@ int validate_step(float *state, const void *x, const void *delta, const float *d
         p->conv_bias = conv->bias;
         p->conv_state = conv->state_out;
     }
+    if (trap) {
+        p->lam = trap->lam;
+        p->x_prev = trap->x_prev;
+        p->B_prev = trap->B_prev;
+    }
     return SSM_OK;
 }
 
@@ -272,11 +288,12 @@ int validate_step(float *state, const void *x, const void *delta, const float *d
 int validate_fwd(const void *x, const void *delta, const float *delta_bias, int softplus, const float *A,
                  const void *B, const void *C, const float *D, const void *z, const float *h0, void *out,
                  float *h_last, const void *ws, size_t ws_bytes, const ConvArgs *conv, const ssm_dims_t *dims,
-                 FwdParams *p, size_t *es_out) {
+                 FwdParams *p, size_t *es_out, const TrapArgs *trap = nullptr) {
     if (!dims) return SSM_ERR_INVALID_ARG;
     const int64_t batch = dims->batch, L = dims->seqlen, dim = dims->dim, N = dims->dstate;
     if (!x || !delta || !A || !B || !C || !out) return SSM_ERR_INVALID_ARG;
     if (conv && !conv->w) return SSM_ERR_INVALID_ARG;
+    if (trap && !trap->lam) return SSM_ERR_INVALID_ARG;
     if (!dims_ok(batch, L, dim) || N < 1) return SSM_ERR_INVALID_ARG;
     if (N != kNState) return SSM_ERR_UNSUPPORTED;
     if (dims->act_dtype != SSM_F32 && dims->act_dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
@@ -287,10 +304,13 @@ int validate_fwd(const void *x, const void *delta, const float *delta_bias, int 
     if (groups * ((L + 255) / 256) > static_cast<int64_t>(UINT32_MAX) / 2) return SSM_ERR_UNSUPPORTED;
     const size_t es = dims->act_dtype == SSM_F32 ? 4 : 2;
     for (const void *ptr : {x, delta, (const void *)A, B, C, z, (const void *)h0, (const void *)out,
-                            (const void *)h_last, ws})
+                            (const void *)h_last, ws, trap ? trap->lam : nullptr})
         if (ptr && !aligned16(ptr)) return SSM_ERR_MISALIGNED;
     for (const void *ptr : {(const void *)delta_bias, (const void *)D})
         if (ptr && !aligned4(ptr)) return SSM_ERR_MISALIGNED;
+    if (trap)
+        for (const void *ptr : {trap->x_prev, trap->B_prev})
+            if (ptr && reinterpret_cast<uintptr_t>(ptr) % es != 0) return SSM_ERR_MISALIGNED;
     if (conv) {
         for (const void *ptr : {(const void *)conv->w, (const void *)conv->bias})
             if (ptr && !aligned4(ptr)) return SSM_ERR_MISALIGNED;
@@ -307,7 +327,10 @@ int validate_fwd(const void *x, const void *delta, const float *delta_bias, int 
                         {delta_bias, delta_bias ? static_cast<size_t>(dim) * 4 : 0}, {h0, h0 ? st : 0},
                         {conv ? conv->w : nullptr, conv ? static_cast<size_t>(dim) * conv->k * 4 : 0},
                         {conv && conv->bias ? conv->bias : nullptr, static_cast<size_t>(dim) * 4},
-                        {conv ? conv->state : nullptr, cst}};
+                        {conv ? conv->state : nullptr, cst},
+                        {trap ? trap->lam : nullptr, tok * es},
+                        {trap ? trap->x_prev : nullptr, static_cast<size_t>(batch) * dim * es},
+                        {trap ? trap->B_prev : nullptr, static_cast<size_t>(batch) * N * es}};
     const Span outs[] = {{out, tok * es}, {h_last, h_last ? st : 0}, {ws, ws ? ws_bytes : 0},
                          {conv ? conv->state_out : nullptr, cst}};
     const void *alias_of[] = {nullptr, h0, nullptr, conv ? conv->state : nullptr};  // allowed exact alias
@@ -335,6 +358,11 @@ int validate_fwd(const void *x, const void *delta, const float *delta_bias, int 
         p->conv_w = conv->w;
         p->conv_bias = conv->bias;
         p->conv_state = conv->state;
+    }
+    if (trap) {
+        p->lam = trap->lam;
+        p->x_prev = trap->x_prev;
+        p->B_prev = trap->B_prev;
     }
     *es_out = es;
     return SSM_OK;
@@ -365,6 +393,11 @@ int dispatch_fwd(const FwdParams &p, size_t es, int act_dtype, void *ws, size_t 
         }
         return rc;
     }
+    if (p.lam)
+        return bf ? (vec ? launch_fwd<bf16raw, true, false, true>(p, ws, ws_bytes, sms, force_chained, s)
+                         : launch_fwd<bf16raw, false, false, true>(p, ws, ws_bytes, sms, force_chained, s))
+                  : (vec ? launch_fwd<float, true, false, true>(p, ws, ws_bytes, sms, force_chained, s)
+                         : launch_fwd<float, false, false, true>(p, ws, ws_bytes, sms, force_chained, s));
     return bf ? (vec ? launch_fwd<bf16raw, true, false>(p, ws, ws_bytes, sms, force_chained, s)
                      : launch_fwd<bf16raw, false, false>(p, ws, ws_bytes, sms, force_chained, s))
               : (vec ? launch_fwd<float, true, false>(p, ws, ws_bytes, sms, force_chained, s)
@@ -457,6 +490,33 @@ int ssm_conv_scan_fwd(const void *x, const float *conv_w, const float *conv_bias
     if (rc != SSM_OK) return rc;
     return dispatch_fwd(p, es, dims->act_dtype, workspace, workspace_bytes, false, conv_state_out,
                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+int ssm_trap_scan_fwd(const void *x, const void *delta, const float *delta_bias, int softplus, const void *lam,
+                      const float *A, const void *B, const void *C, const float *D, const void *z, const float *h0,
+                      const void *x_prev, const void *B_prev, void *out, float *h_last, void *workspace,
+                      size_t workspace_bytes, const ssm_dims_t *dims, ssm_stream_t stream) {
+    if (!workspace) return SSM_ERR_INVALID_ARG;
+    const TrapArgs trap{lam, x_prev, B_prev};
+    FwdParams p;
+    size_t es = 0;
+    const int rc = validate_fwd(x, delta, delta_bias, softplus, A, B, C, D, z, h0, out, h_last, workspace,
+                                workspace_bytes, nullptr, dims, &p, &es, &trap);
+    if (rc != SSM_OK) return rc;
+    return dispatch_fwd(p, es, dims->act_dtype, workspace, workspace_bytes, false, nullptr,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+int ssm_trap_scan_step(float *state, const void *x, const void *delta, const float *delta_bias, int softplus,
+                       const void *lam, const float *A, const void *B, const void *C, const float *D, const void *z,
+                       const void *x_prev, const void *B_prev, void *out, const ssm_dims_t *dims,
+                       ssm_stream_t stream) {
+    const TrapArgs trap{lam, x_prev, B_prev};
+    StepParams p;
+    const int rc = validate_step(state, x, delta, delta_bias, softplus, A, B, C, D, z, out, nullptr, dims, &p, &trap);
+    if (rc != SSM_OK) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return dims->act_dtype == SSM_BF16 ? launch_step<bf16raw, false, true>(p, s) : launch_step<float, false, true>(p, s);
 }
 
 int ssm_conv_scan_step(void *conv_state, float *state, const void *x, const float *conv_w,

@@ -207,3 +207,34 @@ def test_conv_entries_reject_bad_arguments(lib):
     assert step(cs=_p(0)) == 1                            # window over the state
     assert step(cs=_p(1)) == 1                            # window over x
     assert step(B=ctypes.c_void_p(0x14000004)) == 3
+
+
+def test_trap_entries_reject_bad_arguments(lib):
+    """The trapezoidal entries share the forward and step checks; lam is
+    required, and lam, x_prev and B_prev are inputs that no output may overlap."""
+    import selective_state_space_38_b200 as m
+
+    def fwd(**over):
+        a = dict(x=_p(1), delta=_p(2), bias=None, sp=1, lam=_p(13), A=_p(3), B=_p(4), C=_p(5), D=None, z=_p(6),
+                 h0=None, xp=None, bp=None, out=_p(7), hl=None, ws=_p(9), wsb=WS, dims=_dims(m))
+        a.update(over)
+        return lib.ssm_trap_scan_fwd(a["x"], a["delta"], a["bias"], a["sp"], a["lam"], a["A"], a["B"], a["C"],
+                                     a["D"], a["z"], a["h0"], a["xp"], a["bp"], a["out"], a["hl"], a["ws"],
+                                     a["wsb"], a["dims"], None)
+    assert fwd(lam=None) == 1
+    assert fwd(lam=ctypes.c_void_p(0x1D000008)) == 3
+    assert fwd(xp=ctypes.c_void_p(0x1E000001)) == 3
+    assert fwd(out=_p(13)) == 1
+    assert fwd(hl=_p(14), xp=ctypes.c_void_p(0x1E000000 + 0x20)) == 1  # h_last over x_prev
+    assert fwd(ws=None) == 1
+
+    def step(**over):
+        a = dict(st=_p(0), x=_p(1), delta=_p(2), bias=None, sp=1, lam=_p(13), A=_p(3), B=_p(4), C=_p(5), D=None,
+                 z=None, xp=_p(14), bp=_p(15), out=_p(7), dims=_dims(m))
+        a.update(over)
+        return lib.ssm_trap_scan_step(a["st"], a["x"], a["delta"], a["bias"], a["sp"], a["lam"], a["A"], a["B"],
+                                      a["C"], a["D"], a["z"], a["xp"], a["bp"], a["out"], a["dims"], None)
+    assert step(lam=None) == 1
+    assert step(bp=ctypes.c_void_p(0x1F000004)) == 3  # B_prev is read as vectors
+    assert step(out=_p(14)) == 1
+    assert step(st=_p(15)) == 1

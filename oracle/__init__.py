@@ -68,6 +68,9 @@ class Oracle:
         lib.ssm_ref_trap_fwd.restype = I
         lib.ssm_ref_trap_step.argtypes = [P, P, P, P, I, P, P, P, P, P, P, P, P, I, L, L, L, P, I]
         lib.ssm_ref_trap_step.restype = I
+        lib.ssm_ref_bwd.argtypes = [P, P, P, I, P, P, P, P, P, P, P, P, I, L, L, L, L,
+                                    P, P, P, P, P, P, P, P, P, I]
+        lib.ssm_ref_bwd.restype = I
         self._lib = lib
 
     # -- marshalling helpers ---------------------------------------------
@@ -272,6 +275,33 @@ class Oracle:
         return out
 
 
+    # -- the backward pass ---------------------------------------------------
+    def bwd(self, x, delta, delta_bias, softplus, A, B, C, D, z, h0, dout, dh_last=None, threads=0):
+        """Derivatives of a loss L through the forward scan, given dout =
+        dL/dout (stored activations, like x) and dh_last = dL/dh_last (float32
+        [b,d,N] or None).  Returns a dict of float64 arrays: dx, ddelta, dz
+        (None without z) [b,d,L]; dB, dC [b,N,L]; dA [d,N]; dD, dbias [d];
+        dh0 [b,d,N]."""
+        code = self._dtype_code(x)
+        x, delta, B, C, z, dout = (self._act(t, code) for t in (x, delta, B, C, z, dout))
+        A, D, delta_bias, h0, dh_last = (self._f32(t) for t in (A, D, delta_bias, h0, dh_last))
+        batch, dim, L = x.shape
+        N = A.shape[1]
+        r = dict(dx=np.empty((batch, dim, L)), ddelta=np.empty((batch, dim, L)),
+                 dz=np.empty((batch, dim, L)) if z is not None else None,
+                 dB=np.empty((batch, N, L)), dC=np.empty((batch, N, L)), dA=np.empty((dim, N)),
+                 dD=np.empty(dim), dbias=np.empty(dim), dh0=np.empty((batch, dim, N)))
+        rc = self._lib.ssm_ref_bwd(
+            self._ptr(x), self._ptr(delta), self._ptr(delta_bias), int(bool(softplus)), self._ptr(A),
+            self._ptr(B), self._ptr(C), self._ptr(D), self._ptr(z), self._ptr(h0), self._ptr(dout),
+            self._ptr(dh_last), code, batch, L, dim, N,
+            *(self._ptr(r[k]) for k in ("dx", "ddelta", "dz", "dB", "dC", "dA", "dD", "dbias", "dh0")),
+            int(threads))
+        if rc != 0:
+            raise ValueError("oracle rejected the arguments")
+        return r
+
+
 def load(path: str | None = None) -> Oracle:
     """Build (if needed) and load the oracle library; cached per process."""
     global _lib
@@ -312,3 +342,7 @@ def trap_fwd(*args, **kw):
 
 def trap_step(*args, **kw):
     return load().trap_step(*args, **kw)
+
+
+def bwd(*args, **kw):
+    return load().bwd(*args, **kw)

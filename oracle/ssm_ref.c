@@ -516,3 +516,177 @@ int ssm_ref_trap_step(double *state, const void *x, const void *delta, const flo
     }
     return 0;
 }
+
+/* ---------------------------------------------------------------------------
+ * Backward pass of the scan (reverse-mode derivatives of ssm_ref_fwd).
+ *
+ * Gu & Dao, "Mamba", Appendix D "Hardware-aware Algorithm For Selective
+ * SSMs", paragraph "Memory": the backward pass does not store the
+ * intermediate states but recomputes them.  What it computes is fixed by the
+ * forward definition: given dout = dL/dout and dh_last = dL/dh_last (NULL =
+ * 0), the derivatives of L with respect to every input.  Written out for one
+ * channel, with dy_t = dout_t silu(z_t) and the adjoint
+ * g_t = dL/dh_t = C_t dy_t + Abar_{t+1} g_{t+1} (g_{L-1} = C_{L-1} dy_{L-1} + dh_last):
+ *
+ *   dz_t      = dout_t y_t silu'(z_t),  silu'(z) = s (1 + z (1 - s)), s = sigmoid(z)
+ *   dD        = sum_t dy_t x_t
+ *   dC[n,t]   = sum_d dy_t h_t[n]
+ *   dB[n,t]   = sum_d g_t[n] dt_t x_t
+ *   dx_t      = D dy_t + sum_n g_t[n] dt_t B[n,t]
+ *   ddt_t     = sum_n g_t[n] (A[n] Abar_t[n] h_{t-1}[n] + B[n,t] x_t)
+ *   dA[n]     = sum_{b,t} g_t[n] dt_t Abar_t[n] h_{t-1}[n]
+ *   ddelta_t  = ddt_t sigmoid(v_t) (softplus) or ddt_t;   dbias = sum_{b,t} ddelta_t
+ *   dh0       = Abar_0 g_0
+ *
+ * Outputs (all double): dx, ddelta, dz [batch][dim][seqlen] (dz only when z
+ * is given), dB, dC [batch][dstate][seqlen], dA [dim][dstate], dD, dbias
+ * [dim], dh0 [batch][dim][dstate].  Any output pointer may be NULL.
+ */
+static double sigmoid_ref(double v)
+{
+    return 1.0 / (1.0 + exp(-v));
+}
+
+static void bwd_channel(const ref_args *a, int64_t b, int64_t d, const void *dout, const float *dh_last,
+                        double *hs, double *dx, double *ddelta, double *dz, double *dB, double *dC,
+                        double *dA, double *dD, double *dbias, double *dh0)
+{
+    const int64_t L = a->seqlen, N = a->dstate, Dm = a->dim;
+    const int64_t chan = b * Dm + d;
+    /* forward, keeping every state: hs[(t + 1) * N + n] = h_t[n], hs[n] = h_{-1}[n] */
+    for (int64_t n = 0; n < N; n++)
+        hs[n] = a->h0 ? (double)a->h0[chan * N + n] : 0.0;
+    for (int64_t t = 0; t < L; t++) {
+        double v = load_act(a->delta, chan * L + t, a->dtype);
+        if (a->delta_bias)
+            v += (double)a->delta_bias[d];
+        const double dt = a->softplus ? softplus_ref(v) : v;
+        const double xt = load_act(a->x, chan * L + t, a->dtype);
+        for (int64_t n = 0; n < N; n++) {
+            const double abar = exp(dt * (double)a->A[d * N + n]);
+            hs[(t + 1) * N + n] = abar * hs[t * N + n] + dt * load_act(a->B, (b * N + n) * L + t, a->dtype) * xt;
+        }
+    }
+    double g[REF_MAX_DSTATE], gnext_decayed[REF_MAX_DSTATE];
+    for (int64_t n = 0; n < N; n++)
+        gnext_decayed[n] = dh_last ? (double)dh_last[chan * N + n] : 0.0;
+    double dDacc = 0.0, dbacc = 0.0;
+    for (int64_t t = L - 1; t >= 0; t--) {
+        double v = load_act(a->delta, chan * L + t, a->dtype);
+        if (a->delta_bias)
+            v += (double)a->delta_bias[d];
+        const double dt = a->softplus ? softplus_ref(v) : v;
+        const double xt = load_act(a->x, chan * L + t, a->dtype);
+        const double *ht = hs + (t + 1) * N, *hp = hs + t * N;
+        double y = 0.0;
+        for (int64_t n = 0; n < N; n++)
+            y += load_act(a->C, (b * N + n) * L + t, a->dtype) * ht[n];
+        if (a->D)
+            y += (double)a->D[d] * xt;
+        const double go = load_act(dout, chan * L + t, a->dtype);
+        double dy = go;
+        if (a->z) {
+            const double zt = load_act(a->z, chan * L + t, a->dtype);
+            const double s = sigmoid_ref(zt);
+            dy = go * zt * s;
+            if (dz)
+                dz[chan * L + t] = go * y * s * (1.0 + zt * (1.0 - s));
+        }
+        double dxt = a->D ? (double)a->D[d] * dy : 0.0;
+        dDacc += dy * xt;
+        double ddt = 0.0;
+        for (int64_t n = 0; n < N; n++) {
+            const double Cn = load_act(a->C, (b * N + n) * L + t, a->dtype);
+            const double Bn = load_act(a->B, (b * N + n) * L + t, a->dtype);
+            const double An = (double)a->A[d * N + n];
+            const double abar = exp(dt * An);
+            g[n] = Cn * dy + gnext_decayed[n];
+            if (dC)
+                dC[(b * N + n) * L + t] += dy * ht[n];
+            if (dB)
+                dB[(b * N + n) * L + t] += g[n] * dt * xt;
+            dxt += g[n] * dt * Bn;
+            ddt += g[n] * (An * abar * hp[n] + Bn * xt);
+            if (dA)
+                dA[d * N + n] += g[n] * dt * abar * hp[n];
+            gnext_decayed[n] = abar * g[n];
+        }
+        const double ddel = a->softplus ? ddt * sigmoid_ref(v) : ddt;
+        dbacc += ddel;
+        if (dx)
+            dx[chan * L + t] = dxt;
+        if (ddelta)
+            ddelta[chan * L + t] = ddel;
+    }
+    if (dh0)
+        for (int64_t n = 0; n < N; n++)
+            dh0[chan * N + n] = gnext_decayed[n];
+    if (dD)
+        dD[d] += dDacc;
+    if (dbias)
+        dbias[d] += dbacc;
+}
+
+/* The backward pass over every channel (OpenMP over channels).  The sums
+ * over channels (dB, dC, dA, dD, dbias) are taken per thread and then added
+ * thread by thread, in double precision.  Returns 0, 1 on bad sizes, 2 when
+ * out of memory. */
+int ssm_ref_bwd(const void *x, const void *delta, const float *delta_bias, int softplus,
+                const float *A, const void *B, const void *C, const float *D,
+                const void *z, const float *h0, const void *dout, const float *dh_last, int dtype,
+                int64_t batch, int64_t seqlen, int64_t dim, int64_t dstate,
+                double *dx, double *ddelta, double *dz, double *dB, double *dC,
+                double *dA, double *dD, double *dbias, double *dh0, int nthreads)
+{
+    if (check_dims(batch, seqlen, dim, dstate) || !x || !delta || !A || !B || !C || !dout)
+        return 1;
+    const ref_args a = {x, delta, delta_bias, softplus, A, B, C, D, z, h0, dtype,
+                        batch, seqlen, dim, dstate};
+    const size_t nbc = (size_t)(batch * dstate * seqlen), na = (size_t)(dim * dstate), nd = (size_t)dim;
+    const size_t part = 2 * nbc + na + 2 * nd;  /* one thread's dB, dC, dA, dD, dbias */
+    set_threads(nthreads);
+    int nt = 1;
+#ifdef _OPENMP
+    nt = omp_get_max_threads();
+#endif
+    double *acc = (double *)calloc((size_t)nt * part, sizeof(double));
+    if (!acc)
+        return 2;
+    int bad = 0;
+#pragma omp parallel
+    {
+        int tid = 0;
+#ifdef _OPENMP
+        tid = omp_get_thread_num();
+#endif
+        double *mine = acc + (size_t)tid * part;
+        double *hs = (double *)malloc((size_t)(seqlen + 1) * (size_t)dstate * sizeof(double));
+        if (!hs) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t c = 0; c < batch * dim; c++)
+                bwd_channel(&a, c / dim, c % dim, dout, dh_last, hs, dx, ddelta, dz, mine, mine + nbc,
+                            mine + 2 * nbc, mine + 2 * nbc + na, mine + 2 * nbc + na + nd, dh0);
+            free(hs);
+        }
+    }
+    if (!bad) {
+        double *outs[5] = {dB, dC, dA, dD, dbias};
+        const size_t offs[5] = {0, nbc, 2 * nbc, 2 * nbc + na, 2 * nbc + na + nd};
+        const size_t lens[5] = {nbc, nbc, na, nd, nd};
+        for (int k = 0; k < 5; k++) {
+            if (!outs[k])
+                continue;
+            for (size_t i = 0; i < lens[k]; i++) {
+                double sum = 0.0;
+                for (int th = 0; th < nt; th++)
+                    sum += acc[(size_t)th * part + offs[k] + i];
+                outs[k][i] = sum;
+            }
+        }
+    }
+    free(acc);
+    return bad ? 2 : 0;
+}

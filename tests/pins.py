@@ -601,6 +601,76 @@ def pin_trap_split_and_step(orc):
     _close(state, hl, rtol=1e-13, what="trap step state")
 
 
+# ---------------------------------------------------------------------------
+# The backward pass (reverse-mode derivatives of the forward scan).
+
+def _bwd(orc, c, dout, dh_last=None, **over):
+    a = dict(c)
+    a.update(over)
+    return orc.bwd(a["x"], a["delta"], a["delta_bias"], a["softplus"], a["A"], a["B"], a["C"], a["D"],
+                   a["z"], a["h0"], dout, dh_last)
+
+
+def pin_bwd_finite_differences(orc):
+    """Every derivative against central differences of the forward oracle:
+    the loss is L = sum(dout * out) + sum(dh_last * h_last); each input element
+    is moved by +-2^-12 (as far as float32 storage allows; the quotient uses
+    the stored values), so the derivative is pinned to ~1e-7 by the forward
+    definition alone."""
+    for softplus, zgate in ((True, True), (False, False)):
+        c = _rand_case(100 + softplus, b=2, d=3, n=4, L=6, z=zgate)
+        c["softplus"] = softplus
+        if not softplus:
+            c["delta"] = _f32(np.abs(c["delta"]) * 0.3)
+        r = _rng(101)
+        dout = _f32(r.standard_normal(c["x"].shape))
+        dhl = _f32(r.standard_normal(c["h0"].shape))
+        g = _bwd(orc, c, dout, dhl)
+
+        def loss(cc):
+            out, hl = _call(orc, cc)
+            return float((dout.astype(np.float64) * out).sum() + (dhl.astype(np.float64) * hl).sum())
+
+        names = [("x", "dx"), ("delta", "ddelta"), ("B", "dB"), ("C", "dC"), ("A", "dA"), ("D", "dD"),
+                 ("delta_bias", "dbias"), ("h0", "dh0")] + ([("z", "dz")] if zgate else [])
+        for key, gk in names:
+            base = c[key]
+            fd = np.empty(base.shape)
+            for idx in np.ndindex(base.shape):
+                up, dn = base.copy(), base.copy()
+                up[idx] = np.float32(float(base[idx]) + 2.0 ** -12)
+                dn[idx] = np.float32(float(base[idx]) - 2.0 ** -12)
+                fd[idx] = (loss(dict(c, **{key: up})) - loss(dict(c, **{key: dn}))) / \
+                    (float(up[idx]) - float(dn[idx]))
+            _close(g[gk], fd, rtol=2e-5, atol=2e-6, what=f"d{key} (softplus={softplus})")
+
+
+def pin_bwd_split(orc):
+    """The chain rule across a split: the backward of [m, L) gives dh0, which
+    is the dh_last of [0, m); the two halves' derivatives are the full ones
+    (the sums over time of dA, dD, dbias add up)."""
+    c = _rand_case(110, b=2, d=3, n=4, L=13)
+    r = _rng(111)
+    dout = _f32(r.standard_normal(c["x"].shape))
+    dhl = _f32(r.standard_normal(c["h0"].shape))
+    full = _bwd(orc, c, dout, dhl)
+    seq = ("x", "delta", "z", "B", "C")
+    for m in (1, 5, 12):
+        first = {k: (np.ascontiguousarray(v[..., :m]) if k in seq else v) for k, v in c.items()}
+        second = {k: (np.ascontiguousarray(v[..., m:]) if k in seq else v) for k, v in c.items()}
+        _, h_mid = _call(orc, first)
+        second["h0"] = _f32(h_mid)  # the state between the halves, rounded to float32 storage
+        g2 = _bwd(orc, second, np.ascontiguousarray(dout[..., m:]), dhl)
+        g1 = _bwd(orc, first, np.ascontiguousarray(dout[..., :m]), _f32(g2["dh0"]))
+        for k in ("dx", "ddelta", "dz"):
+            _close(np.concatenate([g1[k], g2[k]], -1), full[k], rtol=1e-5, atol=1e-6, what=f"split {k} m={m}")
+        for k in ("dB", "dC"):
+            _close(np.concatenate([g1[k], g2[k]], -1), full[k], rtol=1e-5, atol=1e-6, what=f"split {k} m={m}")
+        for k in ("dA", "dD", "dbias"):
+            _close(g1[k] + g2[k], full[k], rtol=1e-5, atol=1e-6, what=f"split {k} m={m}")
+        _close(g1["dh0"], full["dh0"], rtol=1e-5, atol=1e-6, what=f"split dh0 m={m}")
+
+
 ALL_PINS = [
     pin_single_step_closed_form,
     pin_hand_values,
@@ -623,4 +693,6 @@ ALL_PINS = [
     pin_trap_second_order,
     pin_trap_convolution_mode,
     pin_trap_split_and_step,
+    pin_bwd_finite_differences,
+    pin_bwd_split,
 ]

@@ -62,6 +62,19 @@ MUTANTS = [
      "const double xp = 0.0;"),
     ("trap step mixes by 1 - lambda twice", "hl[n] = alpha * h[n] + (1.0 - lt) * dt * alpha * vprev[n] + lt * dt * vt;",
      "hl[n] = alpha * h[n] + (1.0 - lt) * dt * alpha * vprev[n] + (1.0 - lt) * dt * vt;"),
+    # the backward pass
+    ("bwd silu derivative wrong", "dz[chan * L + t] = go * y * s * (1.0 + zt * (1.0 - s));",
+     "dz[chan * L + t] = go * y * s * (1.0 + zt * s);"),
+    ("bwd adjoint not decayed", "            gnext_decayed[n] = abar * g[n];", "            gnext_decayed[n] = g[n];"),
+    ("bwd dB without dt", "dB[(b * N + n) * L + t] += g[n] * dt * xt;", "dB[(b * N + n) * L + t] += g[n] * xt;"),
+    ("bwd ddt drops the decay term", "ddt += g[n] * (An * abar * hp[n] + Bn * xt);", "ddt += g[n] * (Bn * xt);"),
+    ("bwd dA uses h_t", "dA[d * N + n] += g[n] * dt * abar * hp[n];", "dA[d * N + n] += g[n] * dt * abar * ht[n];"),
+    ("bwd softplus derivative dropped", "const double ddel = a->softplus ? ddt * sigmoid_ref(v) : ddt;",
+     "const double ddel = ddt;"),
+    ("bwd dx drops the skip", "double dxt = a->D ? (double)a->D[d] * dy : 0.0;", "double dxt = 0.0;"),
+    ("bwd dC uses h_{t-1}", "dC[(b * N + n) * L + t] += dy * ht[n];", "dC[(b * N + n) * L + t] += dy * hp[n];"),
+    ("bwd dh_last ignored", "gnext_decayed[n] = dh_last ? (double)dh_last[chan * N + n] : 0.0;",
+     "gnext_decayed[n] = 0.0;"),
     ("trap step drops the previous token", "hl[n] = alpha * h[n] + (1.0 - lt) * dt * alpha * vprev[n] + lt * dt * vt;",
      "hl[n] = alpha * h[n] + lt * dt * vt;"),
 ]

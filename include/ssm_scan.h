@@ -237,6 +237,45 @@ int ssm_trap_scan_step(float *state, const void *x, const void *delta, const flo
                        void *out, const ssm_dims_t *dims, ssm_stream_t stream);
 
 /*
+ * Workspace bytes that ssm_scan_bwd needs for the shape `dims`: the states at
+ * the start of every 128-step chunk (64 B per channel and chunk) and one
+ * partial dB, dC per block of 32 channels (batch * 2 * dstate * seqlen * 4 B
+ * each).  Returns SSM_OK and writes *bytes, or an SSM_ERR_* code.
+ */
+int ssm_scan_bwd_workspace_size(const ssm_dims_t *dims, size_t *bytes);
+
+/*
+ * Backward pass of ssm_scan_fwd: the derivatives of a loss L with respect to
+ * every input, given dout = dL/dout and dh_last = dL/dh_last.  As Appendix D
+ * "Memory" describes, the intermediate states are not stored by the forward
+ * pass: the call stores the state at the start of every 128-step chunk and
+ * recomputes the chunk's states from it while it runs the adjoint recurrence
+ *   g_t = C_t dy_t + Abar_{t+1} g_{t+1},  dy_t = dout_t silu(z_t)
+ * backwards through the chunk.
+ *
+ *   x .. h0        the forward call's inputs (as for ssm_scan_fwd)
+ *   dout           required [batch][dim][seqlen], activation dtype
+ *   dh_last        optional [batch][dim][dstate] float32 (NULL = 0)
+ *   dx, ddelta     required [batch][dim][seqlen], activation dtype
+ *   dz             [batch][dim][seqlen], activation dtype; required when z is given
+ *   dB, dC         required [batch][dstate][seqlen] float32 (sums over channels)
+ *   dA             required [dim][dstate] float32 (sum over batch and time)
+ *   dD, dbias      optional [dim] float32 (NULL: not computed)
+ *   dh0            optional [batch][dim][dstate] float32 (NULL: not written)
+ *   workspace      at least ssm_scan_bwd_workspace_size bytes, 16-byte aligned
+ * Alignment: 16 bytes for every pointer except delta_bias, D, dD, dbias (4).
+ * No output may overlap an input or another output.  dB and dC are summed in
+ * a fixed order; dA, dD and dbias are summed over the batch with float atomics
+ * (their last bits may differ between calls).  Returns SSM_OK or an SSM_ERR_* code.
+ */
+int ssm_scan_bwd(const void *x, const void *delta, const float *delta_bias, int softplus,
+                 const float *A, const void *B, const void *C, const float *D, const void *z,
+                 const float *h0, const void *dout, const float *dh_last,
+                 void *dx, void *ddelta, void *dz, float *dB, float *dC, float *dA, float *dD,
+                 float *dbias, float *dh0, void *workspace, size_t workspace_bytes,
+                 const ssm_dims_t *dims, ssm_stream_t stream);
+
+/*
  * ssm_scan_fwd without a workspace.  The pages have no counterpart: this
  * entry point exists for callers that cannot allocate any device memory while
  * they run the scan, not even a workspace (code running inside an allocator or

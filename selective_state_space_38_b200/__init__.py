@@ -60,6 +60,10 @@ def _load():
     lib.ssm_trap_scan_fwd.restype = I
     lib.ssm_trap_scan_step.argtypes = [P, P, P, P, I, P, P, P, P, P, P, P, P, P, DP, P]
     lib.ssm_trap_scan_step.restype = I
+    lib.ssm_scan_bwd_workspace_size.argtypes = [DP, ctypes.POINTER(S)]
+    lib.ssm_scan_bwd_workspace_size.restype = I
+    lib.ssm_scan_bwd.argtypes = [P, P, P, I, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, DP, P]
+    lib.ssm_scan_bwd.restype = I
     lib.ssm_scan_step.argtypes = [P, P, P, P, I, P, P, P, P, P, P, DP, P]
     lib.ssm_scan_step.restype = I
     lib.ssm_strerror.argtypes = [I]
@@ -82,7 +86,7 @@ def get_lib():
 
 EXPORTS = ("ssm_scan_fwd_workspace_size", "ssm_scan_fwd", "ssm_scan_fwd_status", "ssm_scan_step",
            "ssm_conv_scan_fwd", "ssm_conv_scan_step", "ssm_trap_scan_fwd", "ssm_trap_scan_step",
-           "ssm_scan_fwd_noalloc", "ssm_debug_fwd_flag_timeout",
+           "ssm_scan_bwd_workspace_size", "ssm_scan_bwd", "ssm_scan_fwd_noalloc", "ssm_debug_fwd_flag_timeout",
            "ssm_strerror", "ssm_version")
 
 
@@ -387,6 +391,50 @@ def ssm_trap_scan_step(state, x, delta, delta_bias, softplus, lam, A, B, C, D=No
     return out
 
 
+def ssm_scan_bwd(x, delta, delta_bias, softplus, A, B, C, D, z, h0, dout, dh_last=None, stream=None,
+                 workspace=None):
+    """Backward pass of ssm_scan_fwd.  Returns a dict: dx, ddelta, dz (None
+    without z) in x's dtype [batch, dim, L]; dB, dC float32 [batch, 16, L];
+    dA float32 [dim, 16]; dD, dbias float32 [dim]; dh0 float32 [batch, dim, 16]."""
+    if x.device.type != "cuda":
+        raise ValueError("ssm_scan_bwd needs CUDA tensors")
+    dev = x.device
+    batch, dim, L = x.shape
+    code = _act_code(x)
+    act = x.dtype
+    f32 = torch.float32
+    ins = [_ptr(x, dtype=act, device=dev, name="x"),
+           _ptr(delta, dtype=act, device=dev, shape=x.shape, name="delta"),
+           _ptr(delta_bias, dtype=f32, device=dev, shape=(dim,), name="delta_bias"), int(bool(softplus)),
+           _ptr(A, dtype=f32, device=dev, shape=(dim, DSTATE), name="A"),
+           _ptr(B, dtype=act, device=dev, shape=(batch, DSTATE, L), name="B"),
+           _ptr(C, dtype=act, device=dev, shape=(batch, DSTATE, L), name="C"),
+           _ptr(D, dtype=f32, device=dev, shape=(dim,), name="D"),
+           _ptr(z, dtype=act, device=dev, shape=x.shape, name="z"),
+           _ptr(h0, dtype=f32, device=dev, shape=(batch, dim, DSTATE), name="h0"),
+           _ptr(dout, dtype=act, device=dev, shape=x.shape, name="dout"),
+           _ptr(dh_last, dtype=f32, device=dev, shape=(batch, dim, DSTATE), name="dh_last")]
+    g = dict(dx=torch.empty_like(x), ddelta=torch.empty_like(x), dz=torch.empty_like(x) if z is not None else None,
+             dB=torch.empty((batch, DSTATE, L), dtype=f32, device=dev),
+             dC=torch.empty((batch, DSTATE, L), dtype=f32, device=dev),
+             dA=torch.empty((dim, DSTATE), dtype=f32, device=dev), dD=torch.empty(dim, dtype=f32, device=dev),
+             dbias=torch.empty(dim, dtype=f32, device=dev),
+             dh0=torch.empty((batch, dim, DSTATE), dtype=f32, device=dev))
+    dims = Dims(batch, L, dim, DSTATE, code)
+    if workspace is None:
+        n = ctypes.c_size_t(0)
+        _check(get_lib().ssm_scan_bwd_workspace_size(ctypes.byref(dims), ctypes.byref(n)))
+        workspace = torch.empty(int(n.value), dtype=torch.uint8, device=dev)
+    outs = [None if g[k] is None else g[k].data_ptr()
+            for k in ("dx", "ddelta", "dz", "dB", "dC", "dA", "dD", "dbias", "dh0")]
+    pw = _ptr(workspace, dtype=torch.uint8, device=dev, name="workspace")
+    with torch.cuda.device(dev):
+        rc = get_lib().ssm_scan_bwd(*ins, *outs, pw, workspace.numel(), ctypes.byref(dims),
+                                    _stream_ptr(stream, dev))
+    _check(rc)
+    return g
+
+
 def ssm_scan_step(state, x, delta, delta_bias, softplus, A, B, C, D=None, z=None, out=None,
                   stream=None):
     """One recurrent decode step; ``state`` ([batch, dim, 16] float32) is
@@ -420,5 +468,5 @@ def ssm_scan_step(state, x, delta, delta_bias, softplus, A, B, C, D=None, z=None
 
 
 __all__ = ["ssm_scan_fwd", "ssm_scan_fwd_workspace_size", "ssm_scan_fwd_status", "ssm_scan_step",
-           "ssm_conv_scan_fwd", "ssm_conv_scan_step", "ssm_trap_scan_fwd", "ssm_trap_scan_step",
+           "ssm_conv_scan_fwd", "ssm_conv_scan_step", "ssm_trap_scan_fwd", "ssm_trap_scan_step", "ssm_scan_bwd",
            "ssm_strerror", "ssm_version", "SSMError", "Dims", "LIB_PATH", "get_lib"]

@@ -19,6 +19,7 @@
 #include "common.cuh"
 #include "scan_fwd.cuh"
 #include "scan_step.cuh"
+#include "scan_bwd.cuh"
 
 namespace {
 
@@ -404,6 +405,34 @@ int dispatch_fwd(const FwdParams &p, size_t es, int act_dtype, void *ws, size_t 
                      : launch_fwd<float, false, false>(p, ws, ws_bytes, sms, force_chained, s));
 }
 
+// Workspace of the backward pass: the chunk checkpoints, then the blocks'
+// partial dB, dC (256-byte aligned pieces).
+size_t bwd_ckpt_bytes(int64_t batch, int64_t L, int64_t dim) {
+    return (static_cast<size_t>(batch) * dim * bwd_chunks(L) * kNState * 4 + 255) / 256 * 256;
+}
+size_t bwd_workspace_bytes(int64_t batch, int64_t L, int64_t dim) {
+    return bwd_ckpt_bytes(batch, L, dim) + static_cast<size_t>(bwd_blocks(dim)) * batch * 2 * kNState * L * 4;
+}
+
+template <typename T>
+int launch_bwd(BwdParams p, cudaStream_t s) {
+    const int smem = static_cast<int>(sizeof(BwdSmem));
+    if (cudaFuncSetAttribute(scan_bwd_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    if (p.dA && cudaMemsetAsync(p.dA, 0, static_cast<size_t>(p.dim) * kNState * 4, s) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    if (p.dD && cudaMemsetAsync(p.dD, 0, static_cast<size_t>(p.dim) * 4, s) != cudaSuccess) return SSM_ERR_CUDA;
+    if (p.dbias && cudaMemsetAsync(p.dbias, 0, static_cast<size_t>(p.dim) * 4, s) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    const int64_t nch = p.batch * p.dim;
+    scan_bwd_ckpt_kernel<T><<<static_cast<unsigned>((nch + 3) / 4), 128, 0, s>>>(p);
+    const dim3 grid(static_cast<unsigned>(bwd_blocks(p.dim)), static_cast<unsigned>(p.batch));
+    scan_bwd_kernel<T><<<grid, kBwdWarps * 32, smem, s>>>(p);
+    const int64_t n = p.batch * 2 * kNState * p.seqlen;
+    scan_bwd_reduce_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(p);
+    return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -517,6 +546,70 @@ int ssm_trap_scan_step(float *state, const void *x, const void *delta, const flo
     if (rc != SSM_OK) return rc;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return dims->act_dtype == SSM_BF16 ? launch_step<bf16raw, false, true>(p, s) : launch_step<float, false, true>(p, s);
+}
+
+int ssm_scan_bwd_workspace_size(const ssm_dims_t *dims, size_t *bytes) {
+    if (!dims || !bytes) return SSM_ERR_INVALID_ARG;
+    if (!dims_ok(dims->batch, dims->seqlen, dims->dim) || dims->dstate < 1) return SSM_ERR_INVALID_ARG;
+    if (dims->dstate != kNState) return SSM_ERR_UNSUPPORTED;
+    *bytes = bwd_workspace_bytes(dims->batch, dims->seqlen, dims->dim);
+    return SSM_OK;
+}
+
+int ssm_scan_bwd(const void *x, const void *delta, const float *delta_bias, int softplus, const float *A,
+                 const void *B, const void *C, const float *D, const void *z, const float *h0, const void *dout,
+                 const float *dh_last, void *dx, void *ddelta, void *dz, float *dB, float *dC, float *dA,
+                 float *dD, float *dbias, float *dh0, void *workspace, size_t workspace_bytes,
+                 const ssm_dims_t *dims, ssm_stream_t stream) {
+    if (!dims) return SSM_ERR_INVALID_ARG;
+    const int64_t batch = dims->batch, L = dims->seqlen, dim = dims->dim, N = dims->dstate;
+    if (!x || !delta || !A || !B || !C || !dout || !dx || !ddelta || !dB || !dC || !dA || !workspace)
+        return SSM_ERR_INVALID_ARG;
+    if (z && !dz) return SSM_ERR_INVALID_ARG;
+    if (!dims_ok(batch, L, dim) || N < 1) return SSM_ERR_INVALID_ARG;
+    if (N != kNState) return SSM_ERR_UNSUPPORTED;
+    if (dims->act_dtype != SSM_F32 && dims->act_dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
+    if (batch > 65535 || bwd_blocks(dim) > INT32_MAX) return SSM_ERR_UNSUPPORTED;  // grid.y holds the batch
+    const size_t es = dims->act_dtype == SSM_F32 ? 4 : 2;
+    for (const void *ptr : {x, delta, (const void *)A, B, C, z, (const void *)h0, dout, (const void *)dx,
+                            (const void *)ddelta, (const void *)(z ? dz : nullptr), (const void *)dB,
+                            (const void *)dC, (const void *)dA, (const void *)dh_last, (const void *)dh0,
+                            (const void *)workspace})
+        if (ptr && !aligned16(ptr)) return SSM_ERR_MISALIGNED;
+    for (const void *ptr : {(const void *)delta_bias, (const void *)D, (const void *)dD, (const void *)dbias})
+        if (ptr && !aligned4(ptr)) return SSM_ERR_MISALIGNED;
+    if (workspace_bytes < bwd_workspace_bytes(batch, L, dim)) return SSM_ERR_INVALID_ARG;
+
+    const size_t tok = static_cast<size_t>(batch) * dim * L, bn = static_cast<size_t>(batch) * N * L;
+    const size_t st = static_cast<size_t>(batch) * dim * N * 4;
+    const Span ins[] = {{x, tok * es}, {delta, tok * es}, {z, z ? tok * es : 0}, {B, bn * es}, {C, bn * es},
+                        {A, static_cast<size_t>(dim) * N * 4}, {D, D ? static_cast<size_t>(dim) * 4 : 0},
+                        {delta_bias, delta_bias ? static_cast<size_t>(dim) * 4 : 0}, {h0, h0 ? st : 0},
+                        {dout, tok * es}, {dh_last, dh_last ? st : 0}};
+    const Span outs[] = {{dx, tok * es}, {ddelta, tok * es}, {z ? dz : nullptr, tok * es}, {dB, bn * 4},
+                         {dC, bn * 4}, {dA, static_cast<size_t>(dim) * N * 4},
+                         {dD, dD ? static_cast<size_t>(dim) * 4 : 0},
+                         {dbias, dbias ? static_cast<size_t>(dim) * 4 : 0}, {dh0, dh0 ? st : 0},
+                         {workspace, workspace_bytes}};
+    constexpr int kOuts = sizeof(outs) / sizeof(outs[0]);
+    for (int o = 0; o < kOuts; ++o) {
+        for (const Span &in : ins)
+            if (overlap(outs[o], in)) return SSM_ERR_INVALID_ARG;
+        for (int q = o + 1; q < kOuts; ++q)
+            if (overlap(outs[o], outs[q])) return SSM_ERR_INVALID_ARG;
+    }
+
+    BwdParams p;
+    memset(&p, 0, sizeof p);
+    p.x = x; p.delta = delta; p.z = z; p.B = B; p.C = C; p.dout = dout;
+    p.delta_bias = delta_bias; p.A = A; p.D = D; p.h0 = h0; p.dh_last = dh_last;
+    p.dx = dx; p.ddelta = ddelta; p.dz = z ? dz : nullptr;
+    p.dA = dA; p.dD = dD; p.dbias = dbias; p.dh0 = dh0; p.dB = dB; p.dC = dC;
+    p.ckpt = static_cast<float *>(workspace);
+    p.part = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + bwd_ckpt_bytes(batch, L, dim));
+    p.batch = batch; p.seqlen = L; p.dim = dim; p.softplus = softplus ? 1 : 0;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return dims->act_dtype == SSM_BF16 ? launch_bwd<bf16raw>(p, s) : launch_bwd<float>(p, s);
 }
 
 int ssm_conv_scan_step(void *conv_state, float *state, const void *x, const float *conv_w,

@@ -4,6 +4,9 @@ parity criteria used throughout the GPU tests.
 Tolerances (float outputs compared with the float64 oracle run on the same
 stored inputs):
   float32 activations: |gpu - ref| <= 1e-4 * (1 + |ref|) element-wise.
+  float32 backward pass ("f32bwd"): |gpu - ref| <= 1e-3 (|ref| + rms(ref)):
+    the derivatives run two more recurrences (the recomputed states and the
+    adjoint) and the sums over channels and time add up to 2^16 float32 terms.
   bfloat16 activations: |gpu - ref| <= 2e-2 * |ref| + 1e-3 * rms(ref)
     element-wise (2% relative, with an absolute floor of 0.1% of the tensor's
     RMS for values that cancel to near zero), and ||gpu - ref||_2 / ||ref||_2
@@ -40,6 +43,8 @@ def check(got, ref, dtype, what=""):
     rms = float(np.sqrt(np.mean(ref * ref))) if ref.size else 0.0
     if dtype == "f32":
         lim = 1e-4 * (1.0 + np.abs(ref))
+    elif dtype == "f32bwd":
+        lim = 1e-3 * (np.abs(ref) + rms)
     else:
         lim = 2e-2 * np.abs(ref) + 1e-3 * rms
     bad = err > lim
@@ -50,6 +55,6 @@ def check(got, ref, dtype, what=""):
         i = tuple(np.argwhere(bad)[0])
         raise AssertionError(f"{what}: {int(bad.sum())} elements out of tolerance; first at {i}: "
                              f"gpu={got[i]!r} ref={ref[i]!r}; {stats}")
-    if dtype != "f32":
+    if dtype not in ("f32", "f32bwd"):
         assert nl2 <= 5e-3, f"{what}: normalised L2 error {nl2:.3e} > 5e-3; {stats}"
     return stats

@@ -238,3 +238,34 @@ def test_trap_entries_reject_bad_arguments(lib):
     assert step(bp=ctypes.c_void_p(0x1F000004)) == 3  # B_prev is read as vectors
     assert step(out=_p(14)) == 1
     assert step(st=_p(15)) == 1
+
+
+def test_bwd_rejects_bad_arguments(lib):
+    """The backward entry: required inputs and outputs, dz with z, alignment,
+    a large enough workspace, and no output over an input or another output."""
+    import selective_state_space_38_b200 as m
+    need = ctypes.c_size_t(0)
+    assert lib.ssm_scan_bwd_workspace_size(_dims(m), ctypes.byref(need)) == 0
+    chunks, blocks = -(-64 // 128), -(-128 // 32)
+    assert need.value == (2 * 128 * chunks * 16 * 4 + 255) // 256 * 256 + blocks * 2 * 2 * 16 * 64 * 4
+
+    def bwd(**over):
+        a = dict(x=_p(1), delta=_p(2), bias=None, sp=1, A=_p(3), B=_p(4), C=_p(5), D=None, z=_p(6), h0=None,
+                 dout=_p(16), dhl=None, dx=_p(17), ddelta=_p(18), dz=_p(19), dB=_p(20), dC=_p(21), dA=_p(22),
+                 dD=None, dbias=None, dh0=None, ws=_p(23), wsb=need.value, dims=_dims(m))
+        a.update(over)
+        return lib.ssm_scan_bwd(a["x"], a["delta"], a["bias"], a["sp"], a["A"], a["B"], a["C"], a["D"], a["z"],
+                                a["h0"], a["dout"], a["dhl"], a["dx"], a["ddelta"], a["dz"], a["dB"], a["dC"],
+                                a["dA"], a["dD"], a["dbias"], a["dh0"], a["ws"], a["wsb"], a["dims"], None)
+    assert bwd(dout=None) == 1
+    assert bwd(dx=None) == 1
+    assert bwd(dA=None) == 1
+    assert bwd(dz=None) == 1                       # z is given, so dz is required
+    assert bwd(ws=None) == 1
+    assert bwd(wsb=need.value - 1) == 1
+    assert bwd(dims=_dims(m, N=8)) == 2
+    assert bwd(dx=ctypes.c_void_p(0x11000008)) == 3
+    assert bwd(dD=ctypes.c_void_p(0x1A000002)) == 3
+    assert bwd(dx=_p(1)) == 1                      # dx over x
+    assert bwd(dB=_p(17)) == 1                     # dB over dx
+    assert bwd(ws=_p(16)) == 1                     # workspace over dout

@@ -130,7 +130,12 @@ __global__ void __launch_bounds__(128) scan_bwd_ckpt_kernel(const BwdParams p) {
     for (int n = 0; n < kNState; ++n) hc[n] = p.h0 ? p.h0[chan * kNState + n] : 0.0f;
     const int64_t chunks = bwd_chunks(L);
     for (int64_t c = 0; c < chunks; ++c) {
-        if (lane < kNState) p.ckpt[(chan * chunks + c) * kNState + lane] = hc[lane];
+        {
+            float mine = 0.0f;  // hc[lane], without indexing registers by a runtime value
+#pragma unroll
+            for (int n = 0; n < kNState; ++n) mine = lane == n ? hc[n] : mine;
+            if (lane < kNState) p.ckpt[(chan * chunks + c) * kNState + lane] = mine;
+        }
         // this lane's steps: fold into (s, e) from a zero state
         float e[kNState], s = 0.0f;
 #pragma unroll
@@ -423,7 +428,12 @@ __global__ void __launch_bounds__(kBwdWarps * 32) scan_bwd_kernel(const BwdParam
                 dDl += __shfl_xor_sync(0xffffffffu, dDl, off);
                 dbl += __shfl_xor_sync(0xffffffffu, dbl, off);
             }
-            if (lane < kNState) sumA[ch][lane] += dAl[lane];
+            {
+                float mine = 0.0f;
+#pragma unroll
+                for (int n = 0; n < kNState; ++n) mine = lane == n ? dAl[n] : mine;
+                if (lane < kNState) sumA[ch][lane] += mine;
+            }
             if (lane == 0) {
                 sumD[ch] += dDl;
                 sumBias[ch] += dbl;

@@ -20,6 +20,7 @@ this project), on bounded samples of the same workload.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import os
@@ -394,6 +395,77 @@ def bench_e2e(args, device, world, inp):
     return dict(ms=ms, h2d=h2d, d2h=d2h, steps=steps)
 
 
+def _next_rows_inputs(device):
+    """The Mamba-2.8B layer workload on the device, plus the extra inputs of
+    the widened rows: width-4 convolution taps, lambda ~ U(0, 1), dout ~ N(0, 1)."""
+    import torch
+    c = workloads.CONFIGS[FWD_CFG]
+    inp = workloads.make_inputs(FWD_CFG)
+    t = {k: _to_dev(v, device) for k, v in inp.items() if isinstance(v, np.ndarray)}
+    g = torch.Generator(device=device)
+    g.manual_seed(22)
+    t["conv_w"] = torch.randn((c.dim, 4), generator=g, device=device) * 0.5
+    t["conv_bias"] = torch.randn(c.dim, generator=g, device=device) * 0.2
+    t["lam"] = torch.rand(t["x"].shape, generator=g, device=device).to(torch.bfloat16)
+    t["dout"] = torch.randn(t["x"].shape, generator=g, device=device).to(torch.bfloat16)
+    return c, t
+
+
+def bench_next_rows(args, device, hbm_peak, only=None):
+    """Event-timed sub-lines of the widened rows on the Mamba-2.8B layer shape:
+    the convolution fused in front of the scan, the exponential-trapezoidal
+    scan, and the backward pass.  Bytes are each call's compulsory traffic."""
+    import torch
+    import selective_state_space_38_b200 as ssm
+    c, t = _next_rows_inputs(device)
+    tok = c.batch * c.seqlen * c.dim
+    bc = 2 * c.batch * c.dstate * c.seqlen
+    base = fwd_bytes(FWD_CFG)
+    out = torch.empty_like(t["x"])
+    hl = torch.empty((c.batch, c.dim, c.dstate), dtype=torch.float32, device=device)
+    ws = torch.empty(ssm.ssm_scan_fwd_workspace_size(c.batch, c.seqlen, c.dim, device), dtype=torch.uint8,
+                     device=device)
+    cs_out = torch.empty((c.batch, c.dim, 3), dtype=torch.bfloat16, device=device)
+    dims = ssm.Dims(c.batch, c.seqlen, c.dim, c.dstate, ssm.SSM_BF16)
+    nbw = ctypes.c_size_t(0)
+    ssm.get_lib().ssm_scan_bwd_workspace_size(ctypes.byref(dims), ctypes.byref(nbw))
+    wsb = torch.empty(int(nbw.value), dtype=torch.uint8, device=device)
+    rows = {
+        "conv_scan_fwd": (lambda: ssm.ssm_conv_scan_fwd(
+            t["x"], t["conv_w"], t["conv_bias"], None, t["delta"], t["delta_bias"], True, t["A"], t["B"], t["C"],
+            t["D"], t["z"], None, out=out, h_last=hl, conv_state_out=cs_out, workspace=ws),
+            base + c.dim * 5 * 4 + c.batch * c.dim * 3 * 2, "causal conv (width 4) + silu fused in front of the scan"),
+        "trap_scan_fwd": (lambda: ssm.ssm_trap_scan_fwd(
+            t["x"], t["delta"], t["delta_bias"], True, t["lam"], t["A"], t["B"], t["C"], t["D"], t["z"], None,
+            out=out, h_last=hl, workspace=ws),
+            base + tok * 2, "exponential-trapezoidal scan (lambda per token and channel)"),
+        "scan_bwd": (lambda: ssm.ssm_scan_bwd(
+            t["x"], t["delta"], t["delta_bias"], True, t["A"], t["B"], t["C"], t["D"], t["z"], None, t["dout"],
+            None, workspace=wsb),
+            tok * 2 * 7 + bc * 2 + bc * 4 + c.dim * c.dstate * 8 + c.dim * 16 + c.batch * c.dim * c.dstate * 4,
+            "backward pass: read x, delta, z, dout, B, C; write dx, ddelta, dz, dB, dC, dA, dD, dbias, dh0"),
+    }
+    res = {}
+    for name, (fn, nbytes, what) in rows.items():
+        if only and name != only:
+            continue
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize(device)
+        n = 20 if name != "scan_bwd" else 10
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        for a, b in ev:
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize(device)
+        ms = statistics.mean([a.elapsed_time(b) for a, b in ev])
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        res[name] = {"workload": f"{c.name}: {what}", "ms": round(ms, 5), "value": round(gbs, 2), "unit": "GB/s",
+                     "frac": round(gbs / hbm_peak, 4), "algorithmic_bytes_per_launch": nbytes, "steps": n}
+    return res
+
+
 def _device_tokens(c, n, gen, device):
     """n decode token sets drawn on the device with the decode config's
     distributions (x, z, B, C ~ N(0,1), delta ~ N(0, 0.1^2)), rounded to bf16."""
@@ -484,6 +556,10 @@ def run_gpu(args):
         print(json.dumps({"only": "step", "ms_per_step": round(dec["ms"], 5), "value": round(dec["gbs"], 2),
                           "unit": "GB/s", "ms_per_step_flushed": round(dec["ms_flushed"], 5)}), flush=True)
         return 0
+    if args.only in ("conv_scan_fwd", "trap_scan_fwd", "scan_bwd"):
+        r = bench_next_rows(args, device, hbm_peak, only=args.only)
+        print(json.dumps({"only": args.only, **r[args.only]}), flush=True)
+        return 0
     if args.only == "fwd":
         f = bench_fwd(args, device, world, cfg=args.config)
         nb = fwd_bytes(args.config)
@@ -519,6 +595,7 @@ def run_gpu(args):
                              "pipes": _pipes(f"scan_fwd_cfg{cfg}")}
             launches += g["kernels_per_call"] * (steps + 3)
         launches += dec["launches"]
+        nxt = bench_next_rows(args, device, hbm_peak)
 
     if rank == 0:
         cpu_val, cpu_s, cpu_ch, cores = cpu_oracle_rate(FWD_CFG, target_s=float(
@@ -548,6 +625,7 @@ def run_gpu(args):
                              "sample": f"{cpu_ch} channels (full L) of the same workload, "
                                        f"{cpu_s:.1f} s of float64 oracle time"},
             "other_configs": subs,
+            "next_rows": nxt,
             "decode": {"workload": workloads.CONFIGS[DECODE_CFG].name,
                        "ms_per_step": round(dec["ms"], 5), "value": round(dec["gbs"], 2),
                        "unit": "GB/s", "pct_of_hbm_peak": round(100 * dec["gbs"] / hbm_peak, 2),
@@ -580,7 +658,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     # profiler runs: only the forward-scan or only the decode-step timing loop
-    ap.add_argument("--only", default=None, choices=["fwd", "step"])
+    ap.add_argument("--only", default=None, choices=["fwd", "step", "conv_scan_fwd", "trap_scan_fwd", "scan_bwd"])
     ap.add_argument("--config", type=int, default=FWD_CFG, choices=[0, 1, 2, 3],
                     help="forward config of --only fwd")
     args = ap.parse_args()

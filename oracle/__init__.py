@@ -71,6 +71,8 @@ class Oracle:
         lib.ssm_ref_bwd.argtypes = [P, P, P, I, P, P, P, P, P, P, P, P, I, L, L, L, L,
                                     P, P, P, P, P, P, P, P, P, I]
         lib.ssm_ref_bwd.restype = I
+        lib.ssm_ref_ssd_fwd.argtypes = [P, P, P, I, P, P, P, P, P, I, L, L, L, L, L, L, P, P, I]
+        lib.ssm_ref_ssd_fwd.restype = I
         self._lib = lib
 
     # -- marshalling helpers ---------------------------------------------
@@ -302,6 +304,26 @@ class Oracle:
         return r
 
 
+    # -- Mamba-2 SSD (scalar-times-identity transition) ------------------------
+    def ssd_fwd(self, x, dt, dt_bias, softplus, A, B, C, D, h0, threads=0):
+        """x [b,L,H,P], dt [b,L,H], B and C [b,L,G,N] stored activations; A, dt_bias,
+        D [H]; h0 [b,H,P,N] float32 or None.  Returns (y [b,L,H,P], h_last
+        [b,H,P,N]), float64."""
+        code = self._dtype_code(x)
+        x, dt, B, C = (self._act(t, code) for t in (x, dt, B, C))
+        A, dt_bias, D, h0 = (self._f32(t) for t in (A, dt_bias, D, h0))
+        batch, L, H, P = x.shape
+        G, N = B.shape[2], B.shape[3]
+        y = np.empty((batch, L, H, P), np.float64)
+        hl = np.empty((batch, H, P, N), np.float64)
+        rc = self._lib.ssm_ref_ssd_fwd(self._ptr(x), self._ptr(dt), self._ptr(dt_bias), int(bool(softplus)),
+                                       self._ptr(A), self._ptr(B), self._ptr(C), self._ptr(D), self._ptr(h0), code,
+                                       batch, L, H, P, G, N, self._ptr(y), self._ptr(hl), int(threads))
+        if rc != 0:
+            raise ValueError("oracle rejected the arguments")
+        return y, hl
+
+
 def load(path: str | None = None) -> Oracle:
     """Build (if needed) and load the oracle library; cached per process."""
     global _lib
@@ -346,3 +368,7 @@ def trap_step(*args, **kw):
 
 def bwd(*args, **kw):
     return load().bwd(*args, **kw)
+
+
+def ssd_fwd(*args, **kw):
+    return load().ssd_fwd(*args, **kw)

@@ -690,3 +690,72 @@ int ssm_ref_bwd(const void *x, const void *delta, const float *delta_bias, int s
     free(acc);
     return bad ? 2 : 0;
 }
+
+/* ---------------------------------------------------------------------------
+ * Mamba-2 state space duality (SSD): scalar-times-identity state transition.
+ *
+ * "A Secret Weapon For mamba paper" (the Mamba-2 abstract: SSMs and attention
+ * are connected through structured semiseparable matrices) and the "Mamba3"
+ * posts (Mamba-2 reduced the state transition matrix to a scalar times the
+ * identity).  The pages print no formula; the plain reading, per batch b and
+ * head h with head dimension P and state dimension N, is
+ *
+ *   dt_t   = softplus(dt[b,t,h] + dt_bias[h])          (dt + dt_bias without softplus)
+ *   a_t    = exp(dt_t A[h])                            one scalar per (b, t, h)
+ *   H_t    = a_t H_{t-1} + (dt_t x_t) B_t^T            H: P x N, H_{-1} = h0 (or 0)
+ *   y_t    = H_t C_t + D[h] x_t                        (y_t[p] = sum_n H_t[p,n] C_t[n] + D x_t[p])
+ *
+ * with B_t, C_t shared by the heads of a group (G groups, H / G heads each).
+ * Storage (time-major, as Mamba-2 layers hold it): x, y [batch][L][H][P];
+ * dt [batch][L][H]; B, C [batch][L][G][N] (activation dtype, dt too);
+ * A, dt_bias, D [H] float32; h0, h_last [batch][H][P][N] (float32 in, double out).
+ */
+int ssm_ref_ssd_fwd(const void *x, const void *dt, const float *dt_bias, int softplus, const float *A,
+                    const void *B, const void *C, const float *D, const float *h0, int dtype,
+                    int64_t batch, int64_t seqlen, int64_t heads, int64_t hdim, int64_t groups, int64_t dstate,
+                    double *y, double *h_last, int nthreads)
+{
+    if (batch <= 0 || seqlen <= 0 || heads <= 0 || hdim <= 0 || groups <= 0 || dstate <= 0 ||
+        heads % groups != 0 || !x || !dt || !A || !B || !C || !y)
+        return 1;
+    set_threads(nthreads);
+    const int64_t L = seqlen, Hh = heads, P = hdim, G = groups, N = dstate;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < batch * Hh; bh++) {
+        const int64_t b = bh / Hh, h = bh % Hh, g = h / (Hh / G);
+        double *S = (double *)malloc((size_t)(P * N) * sizeof(double));
+        if (!S) {
+#pragma omp atomic write
+            bad = 1;
+            continue;
+        }
+        for (int64_t i = 0; i < P * N; i++)
+            S[i] = h0 ? (double)h0[(b * Hh + h) * P * N + i] : 0.0;
+        for (int64_t t = 0; t < L; t++) {
+            double v = load_act(dt, (b * L + t) * Hh + h, dtype);
+            if (dt_bias)
+                v += (double)dt_bias[h];
+            const double dtt = softplus ? softplus_ref(v) : v;
+            const double at = exp(dtt * (double)A[h]);
+            for (int64_t p = 0; p < P; p++) {
+                const double xp = load_act(x, ((b * L + t) * Hh + h) * P + p, dtype);
+                double yp = 0.0;
+                for (int64_t n = 0; n < N; n++) {
+                    const double Bn = load_act(B, ((b * L + t) * G + g) * N + n, dtype);
+                    const double Cn = load_act(C, ((b * L + t) * G + g) * N + n, dtype);
+                    S[p * N + n] = at * S[p * N + n] + dtt * xp * Bn;
+                    yp += S[p * N + n] * Cn;
+                }
+                if (D)
+                    yp += (double)D[h] * xp;
+                y[((b * L + t) * Hh + h) * P + p] = yp;
+            }
+        }
+        if (h_last)
+            for (int64_t i = 0; i < P * N; i++)
+                h_last[(b * Hh + h) * P * N + i] = S[i];
+        free(S);
+    }
+    return bad ? 2 : 0;
+}

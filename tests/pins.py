@@ -671,6 +671,81 @@ def pin_bwd_split(orc):
         _close(g1["dh0"], full["dh0"], rtol=1e-5, atol=1e-6, what=f"split dh0 m={m}")
 
 
+# ---------------------------------------------------------------------------
+# Mamba-2 SSD: scalar-times-identity transition, multi-dimensional heads.
+
+def _ssd_case(seed, b=2, L=9, H=4, P=3, G=2, N=5, h0=True):
+    r = _rng(seed)
+    return dict(x=_f32(r.standard_normal((b, L, H, P))), dt=_f32(r.standard_normal((b, L, H)) * 0.5),
+                dt_bias=_f32(r.standard_normal(H) * 0.3), softplus=True, A=_f32(-r.uniform(0.2, 2.0, H)),
+                B=_f32(r.standard_normal((b, L, G, N))), C=_f32(r.standard_normal((b, L, G, N))),
+                D=_f32(r.standard_normal(H)), h0=_f32(r.standard_normal((b, H, P, N))) if h0 else None)
+
+
+def _ssd(orc, c, **over):
+    a = dict(c)
+    a.update(over)
+    return orc.ssd_fwd(a["x"], a["dt"], a["dt_bias"], a["softplus"], a["A"], a["B"], a["C"], a["D"], a["h0"])
+
+
+def pin_ssd_semiseparable_form(orc):
+    """The attention-like dual: y = M x + D x with the lower-triangular
+    (semiseparable) matrix M[t, s] = (C_t . B_s) exp(A sum_{r=s+1..t} dt_r) dt_s,
+    plus the h0 term C_t . (exp(A sum_{r<=t} dt_r) h0); built with numpy einsum
+    and cumulative sums, no recurrence."""
+    c = _ssd_case(120)
+    y, hl = _ssd(orc, c)
+    b, L, H, P = c["x"].shape
+    G, N = c["B"].shape[2:]
+    dt = np.logaddexp(0.0, c["dt"].astype(np.float64) + c["dt_bias"][None, None, :])   # [b,L,H]
+    cum = np.cumsum(dt * c["A"][None, None, :], axis=1)                                  # [b,L,H]
+    grp = np.arange(H) // (H // G)
+    Bh = c["B"].astype(np.float64)[:, :, grp, :]                                         # [b,L,H,N]
+    Ch = c["C"].astype(np.float64)[:, :, grp, :]
+    CB = np.einsum("bthn,bshn->bhts", Ch, Bh)
+    dec = np.exp(cum.transpose(0, 2, 1)[:, :, :, None] - cum.transpose(0, 2, 1)[:, :, None, :])  # [b,H,t,s]
+    mask = np.tril(np.ones((L, L)))[None, None]
+    M = CB * dec * mask * dt.transpose(0, 2, 1)[:, :, None, :]
+    want = np.einsum("bhts,bshp->bthp", M, c["x"].astype(np.float64))
+    want += c["D"].astype(np.float64)[None, None, :, None] * c["x"].astype(np.float64)
+    h0 = c["h0"].astype(np.float64)
+    want += np.einsum("bthn,bhpn,bth->bthp", Ch, h0, np.exp(cum))
+    _close(y, want, rtol=1e-11, atol=1e-12, what="ssd semiseparable form")
+    hw = np.einsum("bhs,bshp,bshn->bhpn", (np.exp(cum[:, -1:, :] - cum) * dt).transpose(0, 2, 1),
+                   c["x"].astype(np.float64), Bh) + np.exp(cum[:, -1, :])[:, :, None, None] * h0
+    _close(hl, hw, rtol=1e-11, atol=1e-12, what="ssd semiseparable h_last")
+
+
+def pin_ssd_reduces_to_s6(orc):
+    """P = N = 1, one head: the SSD recurrence is the selective scan of one
+    channel with a one-dimensional state (the S6 oracle, no gate)."""
+    c = _ssd_case(121, b=2, L=11, H=1, P=1, G=1, N=1)
+    y, hl = _ssd(orc, c)
+    s6 = dict(x=np.ascontiguousarray(c["x"][:, :, 0, 0][:, None, :]), delta=np.ascontiguousarray(c["dt"][:, :, 0][:, None, :]),
+              z=None, B=np.ascontiguousarray(c["B"][:, :, 0, 0][:, None, :]), C=np.ascontiguousarray(c["C"][:, :, 0, 0][:, None, :]),
+              A=_f32(c["A"].reshape(1, 1)), D=c["D"], delta_bias=c["dt_bias"],
+              h0=_f32(c["h0"].reshape(2, 1, 1)), softplus=True)
+    o2, h2 = _call(orc, s6)
+    _close(y[:, :, 0, 0], o2[:, 0, :], rtol=1e-13, atol=1e-14, what="ssd vs s6 out")
+    _close(hl.reshape(2, 1), h2.reshape(2, 1), rtol=1e-13, atol=1e-14, what="ssd vs s6 state")
+
+
+def pin_ssd_split(orc):
+    """Two calls continue one when h_last is carried."""
+    c = _ssd_case(122, L=14)
+    y, hl = _ssd(orc, c)
+    for m in (1, 7, 13):
+        first = dict(c, x=np.ascontiguousarray(c["x"][:, :m]), dt=np.ascontiguousarray(c["dt"][:, :m]),
+                     B=np.ascontiguousarray(c["B"][:, :m]), C=np.ascontiguousarray(c["C"][:, :m]))
+        y1, h1 = _ssd(orc, first)
+        second = dict(c, x=np.ascontiguousarray(c["x"][:, m:]), dt=np.ascontiguousarray(c["dt"][:, m:]),
+                      B=np.ascontiguousarray(c["B"][:, m:]), C=np.ascontiguousarray(c["C"][:, m:]), h0=_f32(h1))
+        y2, h2 = _ssd(orc, second)
+        _close(y1, y[:, :m], rtol=1e-12, what=f"ssd split m={m} first")
+        _close(y2, y[:, m:], rtol=2e-5, atol=2e-5, what=f"ssd split m={m} second")
+        _close(h2, hl, rtol=2e-5, atol=2e-5, what=f"ssd split m={m} state")
+
+
 ALL_PINS = [
     pin_single_step_closed_form,
     pin_hand_values,
@@ -695,4 +770,7 @@ ALL_PINS = [
     pin_trap_split_and_step,
     pin_bwd_finite_differences,
     pin_bwd_split,
+    pin_ssd_semiseparable_form,
+    pin_ssd_reduces_to_s6,
+    pin_ssd_split,
 ]

@@ -75,6 +75,16 @@ MUTANTS = [
     ("bwd dC uses h_{t-1}", "dC[(b * N + n) * L + t] += dy * ht[n];", "dC[(b * N + n) * L + t] += dy * hp[n];"),
     ("bwd dh_last ignored", "gnext_decayed[n] = dh_last ? (double)dh_last[chan * N + n] : 0.0;",
      "gnext_decayed[n] = 0.0;"),
+    # Mamba-2 SSD
+    ("ssd decay applied after the input", "S[p * N + n] = at * S[p * N + n] + dtt * xp * Bn;",
+     "S[p * N + n] = at * (S[p * N + n] + dtt * xp * Bn);"),
+    ("ssd input without dt", "S[p * N + n] = at * S[p * N + n] + dtt * xp * Bn;",
+     "S[p * N + n] = at * S[p * N + n] + xp * Bn;"),
+    ("ssd wrong group of B and C", "const int64_t b = bh / Hh, h = bh % Hh, g = h / (Hh / G);",
+     "const int64_t b = bh / Hh, h = bh % Hh, g = h % G;"),
+    ("ssd readout dropped", "                    yp += S[p * N + n] * Cn;\n",
+     "                    yp += 0.0;\n"),
+    ("ssd skip dropped", "                    yp += (double)D[h] * xp;", "                    yp += 0.0;"),
     ("trap step drops the previous token", "hl[n] = alpha * h[n] + (1.0 - lt) * dt * alpha * vprev[n] + lt * dt * vt;",
      "hl[n] = alpha * h[n] + lt * dt * vt;"),
 ]

@@ -445,6 +445,24 @@ def bench_next_rows(args, device, hbm_peak, only=None):
             tok * 2 * 7 + bc * 2 + bc * 4 + c.dim * c.dstate * 8 + c.dim * 16 + c.batch * c.dim * c.dstate * 4,
             "backward pass: read x, delta, z, dout, B, C; write dx, ddelta, dz, dB, dC, dA, dD, dbias, dh0"),
     }
+    # Mamba-2 SSD on a 2.7B-like layer: 4 x 4096, 80 heads of 64, one group of B and C, state 128
+    sb, sl, sh, sp_, sg, sn = 4, 4096, 80, 64, 1, 128
+    g = torch.Generator(device=device)
+    g.manual_seed(23)
+    sx = torch.randn((sb, sl, sh, sp_), generator=g, device=device).to(torch.bfloat16)
+    sdt = (torch.randn((sb, sl, sh), generator=g, device=device) * 0.1).to(torch.bfloat16)
+    sB = torch.randn((sb, sl, sg, sn), generator=g, device=device).to(torch.bfloat16)
+    sC = torch.randn((sb, sl, sg, sn), generator=g, device=device).to(torch.bfloat16)
+    sA = -(torch.rand(sh, generator=g, device=device) * 15 + 1)
+    sbias = torch.full((sh,), -4.0, device=device)
+    sD = torch.ones(sh, device=device)
+    sy = torch.empty_like(sx)
+    shl = torch.empty((sb, sh, sp_, sn), dtype=torch.float32, device=device)
+    sws = torch.empty(256, dtype=torch.uint8, device=device)
+    rows["ssd_fwd"] = (lambda: ssm.ssm_ssd_fwd(sx, sdt, sbias, True, sA, sB, sC, sD, None, y=sy, h_last=shl,
+                                                workspace=sws),
+                       2 * sx.numel() * 2 + sdt.numel() * 2 + 2 * sB.numel() * 2 + sh * 12 + shl.numel() * 4,
+                       "Mamba-2 SSD (tensor cores), 2.7B-like layer 4 x 4096, 80 heads x 64, state 128")
     res = {}
     for name, (fn, nbytes, what) in rows.items():
         if only and name != only:
@@ -461,7 +479,8 @@ def bench_next_rows(args, device, hbm_peak, only=None):
         torch.cuda.synchronize(device)
         ms = statistics.mean([a.elapsed_time(b) for a, b in ev])
         gbs = nbytes / (ms * 1e-3) / 1e9
-        res[name] = {"workload": f"{c.name}: {what}", "ms": round(ms, 5), "value": round(gbs, 2), "unit": "GB/s",
+        res[name] = {"workload": what if name == "ssd_fwd" else f"{c.name}: {what}", "ms": round(ms, 5),
+                     "value": round(gbs, 2), "unit": "GB/s",
                      "frac": round(gbs / hbm_peak, 4), "algorithmic_bytes_per_launch": nbytes, "steps": n}
     return res
 
@@ -556,7 +575,7 @@ def run_gpu(args):
         print(json.dumps({"only": "step", "ms_per_step": round(dec["ms"], 5), "value": round(dec["gbs"], 2),
                           "unit": "GB/s", "ms_per_step_flushed": round(dec["ms_flushed"], 5)}), flush=True)
         return 0
-    if args.only in ("conv_scan_fwd", "trap_scan_fwd", "scan_bwd"):
+    if args.only in ("conv_scan_fwd", "trap_scan_fwd", "scan_bwd", "ssd_fwd"):
         r = bench_next_rows(args, device, hbm_peak, only=args.only)
         print(json.dumps({"only": args.only, **r[args.only]}), flush=True)
         return 0
@@ -658,7 +677,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     # profiler runs: only the forward-scan or only the decode-step timing loop
-    ap.add_argument("--only", default=None, choices=["fwd", "step", "conv_scan_fwd", "trap_scan_fwd", "scan_bwd"])
+    ap.add_argument("--only", default=None, choices=["fwd", "step", "conv_scan_fwd", "trap_scan_fwd", "scan_bwd",
+                                                        "ssd_fwd"])
     ap.add_argument("--config", type=int, default=FWD_CFG, choices=[0, 1, 2, 3],
                     help="forward config of --only fwd")
     args = ap.parse_args()

@@ -72,6 +72,17 @@ typedef struct {
     int32_t act_dtype; /* ssm_dtype_t */
 } ssm_dims_t;
 
+/* Sizes of a Mamba-2 SSD call (ssm_ssd_fwd). */
+typedef struct {
+    int64_t batch;     /* sequences, >= 1 */
+    int64_t seqlen;    /* L, >= 1 */
+    int64_t heads;     /* H, >= 1, a multiple of groups */
+    int64_t headdim;   /* P per head; 64 is supported */
+    int64_t groups;    /* G groups of heads sharing B and C */
+    int64_t dstate;    /* N; 128 is supported */
+    int32_t act_dtype; /* ssm_dtype_t; SSM_BF16 is supported */
+} ssm_ssd_dims_t;
+
 enum {
     SSM_OK = 0,
     SSM_ERR_INVALID_ARG = 1, /* NULL required pointer, a dimension < 1, overlapping buffers, or a too small workspace */
@@ -274,6 +285,34 @@ int ssm_scan_bwd(const void *x, const void *delta, const float *delta_bias, int 
                  void *dx, void *ddelta, void *dz, float *dB, float *dC, float *dA, float *dD,
                  float *dbias, float *dh0, void *workspace, size_t workspace_bytes,
                  const ssm_dims_t *dims, ssm_stream_t stream);
+
+/*
+ * Mamba-2 state space duality (SSD) forward: a scalar-times-identity state
+ * transition per head (the "Mamba3" posts: Mamba-2 reduced the transition to
+ * a scalar times the identity; the Mamba-2 abstract: SSMs and attention meet
+ * in structured semiseparable matrices).  Per batch b and head h:
+ *
+ *   dt_t = softplus(dt[b,t,h] + dt_bias[h])   (dt + dt_bias when softplus == 0)
+ *   H_t  = exp(dt_t A[h]) H_{t-1} + (dt_t x_t) B_t^T      H: headdim x dstate
+ *   y_t  = H_t C_t + D[h] x_t
+ *
+ * computed chunk by chunk (128 steps) as dense products on the tensor cores.
+ *
+ *   x, y           [batch][seqlen][heads][headdim] bf16, 16-byte aligned
+ *   dt             [batch][seqlen][heads] bf16
+ *   B, C           [batch][seqlen][groups][dstate] bf16, 16-byte aligned
+ *                  (heads h*G/H .. share group h / (heads / groups))
+ *   A, dt_bias, D  [heads] float32 (dt_bias and D optional)
+ *   h0, h_last     optional [batch][heads][headdim][dstate] float32
+ *   workspace      at least 256 bytes (the bounded-wait error word that
+ *                  ssm_scan_fwd_status reads)
+ * Returns SSM_OK or an SSM_ERR_* code (SSM_ERR_UNSUPPORTED unless headdim 64,
+ * dstate 128, bf16).
+ */
+int ssm_ssd_fwd(const void *x, const void *dt, const float *dt_bias, int softplus, const float *A,
+                const void *B, const void *C, const float *D, const float *h0, void *y, float *h_last,
+                void *workspace, size_t workspace_bytes, const ssm_ssd_dims_t *dims,
+                ssm_stream_t stream);
 
 /*
  * ssm_scan_fwd without a workspace.  The pages have no counterpart: this

@@ -29,6 +29,12 @@ class SSMError(RuntimeError):
         self.code = code
 
 
+class SsdDims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("heads", ctypes.c_int64),
+                ("headdim", ctypes.c_int64), ("groups", ctypes.c_int64), ("dstate", ctypes.c_int64),
+                ("act_dtype", ctypes.c_int32)]
+
+
 class Dims(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("dim", ctypes.c_int64),
                 ("dstate", ctypes.c_int64), ("act_dtype", ctypes.c_int32)]
@@ -64,6 +70,8 @@ def _load():
     lib.ssm_scan_bwd_workspace_size.restype = I
     lib.ssm_scan_bwd.argtypes = [P, P, P, I, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, DP, P]
     lib.ssm_scan_bwd.restype = I
+    lib.ssm_ssd_fwd.argtypes = [P, P, P, I, P, P, P, P, P, P, P, P, S, ctypes.POINTER(SsdDims), P]
+    lib.ssm_ssd_fwd.restype = I
     lib.ssm_scan_step.argtypes = [P, P, P, P, I, P, P, P, P, P, P, DP, P]
     lib.ssm_scan_step.restype = I
     lib.ssm_strerror.argtypes = [I]
@@ -86,7 +94,8 @@ def get_lib():
 
 EXPORTS = ("ssm_scan_fwd_workspace_size", "ssm_scan_fwd", "ssm_scan_fwd_status", "ssm_scan_step",
            "ssm_conv_scan_fwd", "ssm_conv_scan_step", "ssm_trap_scan_fwd", "ssm_trap_scan_step",
-           "ssm_scan_bwd_workspace_size", "ssm_scan_bwd", "ssm_scan_fwd_noalloc", "ssm_debug_fwd_flag_timeout",
+           "ssm_scan_bwd_workspace_size", "ssm_scan_bwd", "ssm_ssd_fwd", "ssm_scan_fwd_noalloc",
+           "ssm_debug_fwd_flag_timeout",
            "ssm_strerror", "ssm_version")
 
 
@@ -435,6 +444,44 @@ def ssm_scan_bwd(x, delta, delta_bias, softplus, A, B, C, D, z, h0, dout, dh_las
     return g
 
 
+def ssm_ssd_fwd(x, dt, dt_bias, softplus, A, B, C, D=None, h0=None, y=None, h_last=None, stream=None,
+                workspace=None, check=False):
+    """Mamba-2 SSD forward on the tensor cores.  x [batch, L, heads, 64],
+    dt [batch, L, heads], B, C [batch, L, groups, 128] bf16; A, dt_bias, D
+    [heads] float32; h0 [batch, heads, 64, 128] float32.  Returns (y, h_last)."""
+    if x.device.type != "cuda":
+        raise ValueError("ssm_ssd_fwd needs CUDA tensors")
+    dev = x.device
+    batch, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    act = torch.bfloat16
+    f32 = torch.float32
+    args = [_ptr(x, dtype=act, device=dev, name="x"),
+            _ptr(dt, dtype=act, device=dev, shape=(batch, L, H), name="dt"),
+            _ptr(dt_bias, dtype=f32, device=dev, shape=(H,), name="dt_bias"), int(bool(softplus)),
+            _ptr(A, dtype=f32, device=dev, shape=(H,), name="A"),
+            _ptr(B, dtype=act, device=dev, shape=(batch, L, G, N), name="B"),
+            _ptr(C, dtype=act, device=dev, shape=(batch, L, G, N), name="C"),
+            _ptr(D, dtype=f32, device=dev, shape=(H,), name="D"),
+            _ptr(h0, dtype=f32, device=dev, shape=(batch, H, P, N), name="h0")]
+    if y is None:
+        y = torch.empty_like(x)
+    if h_last is None:
+        h_last = torch.empty((batch, H, P, N), dtype=f32, device=dev)
+    args += [_ptr(y, dtype=act, device=dev, shape=x.shape, name="y"),
+             _ptr(h_last, dtype=f32, device=dev, shape=(batch, H, P, N), name="h_last")]
+    if workspace is None:
+        workspace = torch.empty(256, dtype=torch.uint8, device=dev)
+    pw = _ptr(workspace, dtype=torch.uint8, device=dev, name="workspace")
+    dims = SsdDims(batch, L, H, P, G, N, SSM_BF16)
+    sp = _stream_ptr(stream, dev)
+    with torch.cuda.device(dev):
+        _check(get_lib().ssm_ssd_fwd(*args, pw, workspace.numel(), ctypes.byref(dims), sp))
+        if check:
+            _check(get_lib().ssm_scan_fwd_status(pw, sp))
+    return y, h_last
+
+
 def ssm_scan_step(state, x, delta, delta_bias, softplus, A, B, C, D=None, z=None, out=None,
                   stream=None):
     """One recurrent decode step; ``state`` ([batch, dim, 16] float32) is
@@ -469,4 +516,4 @@ def ssm_scan_step(state, x, delta, delta_bias, softplus, A, B, C, D=None, z=None
 
 __all__ = ["ssm_scan_fwd", "ssm_scan_fwd_workspace_size", "ssm_scan_fwd_status", "ssm_scan_step",
            "ssm_conv_scan_fwd", "ssm_conv_scan_step", "ssm_trap_scan_fwd", "ssm_trap_scan_step", "ssm_scan_bwd",
-           "ssm_strerror", "ssm_version", "SSMError", "Dims", "LIB_PATH", "get_lib"]
+           "ssm_ssd_fwd", "SsdDims", "ssm_strerror", "ssm_version", "SSMError", "Dims", "LIB_PATH", "get_lib"]

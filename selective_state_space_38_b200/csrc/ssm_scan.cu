@@ -21,6 +21,7 @@
 #include "scan_step.cuh"
 #include "scan_bwd.cuh"
 #include "scan_fwd_lat.cuh"
+#include "ssd_fwd.cuh"
 
 namespace {
 
@@ -636,6 +637,48 @@ int ssm_scan_bwd(const void *x, const void *delta, const float *delta_bias, int 
     p.batch = batch; p.seqlen = L; p.dim = dim; p.softplus = softplus ? 1 : 0;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return dims->act_dtype == SSM_BF16 ? launch_bwd<bf16raw>(p, s) : launch_bwd<float>(p, s);
+}
+
+int ssm_ssd_fwd(const void *x, const void *dt, const float *dt_bias, int softplus, const float *A, const void *B,
+                const void *C, const float *D, const float *h0, void *y, float *h_last, void *workspace,
+                size_t workspace_bytes, const ssm_ssd_dims_t *dims, ssm_stream_t stream) {
+    if (!dims || !x || !dt || !A || !B || !C || !y || !workspace) return SSM_ERR_INVALID_ARG;
+    const int64_t batch = dims->batch, L = dims->seqlen, H = dims->heads, P = dims->headdim, G = dims->groups,
+                  N = dims->dstate;
+    if (batch < 1 || L < 1 || H < 1 || P < 1 || G < 1 || N < 1 || H % G != 0) return SSM_ERR_INVALID_ARG;
+    if (P != kSsdP || N != kSsdN || dims->act_dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
+    if (batch * H > INT32_MAX || L > INT32_MAX) return SSM_ERR_UNSUPPORTED;
+    if (workspace_bytes < 256) return SSM_ERR_INVALID_ARG;
+    for (const void *ptr : {x, B, C, (const void *)y, (const void *)h0, (const void *)h_last, (const void *)workspace})
+        if (ptr && !aligned16(ptr)) return SSM_ERR_MISALIGNED;
+    for (const void *ptr : {(const void *)dt_bias, (const void *)A, (const void *)D})
+        if (ptr && !aligned4(ptr)) return SSM_ERR_MISALIGNED;
+    if (reinterpret_cast<uintptr_t>(dt) % 2 != 0) return SSM_ERR_MISALIGNED;
+    const size_t tok = static_cast<size_t>(batch) * L * H * P * 2, bc = static_cast<size_t>(batch) * L * G * N * 2;
+    const size_t st = static_cast<size_t>(batch) * H * P * N * 4;
+    const Span ins[] = {{x, tok}, {dt, static_cast<size_t>(batch) * L * H * 2}, {B, bc}, {C, bc},
+                        {A, static_cast<size_t>(H) * 4}, {dt_bias, dt_bias ? static_cast<size_t>(H) * 4 : 0},
+                        {D, D ? static_cast<size_t>(H) * 4 : 0}, {h0, h0 ? st : 0}};
+    const Span outs[] = {{y, tok}, {h_last, h_last ? st : 0}, {workspace, workspace_bytes}};
+    for (int o = 0; o < 3; ++o) {
+        for (const Span &in : ins)
+            if (overlap(outs[o], in)) return SSM_ERR_INVALID_ARG;
+        for (int q = o + 1; q < 3; ++q)
+            if (overlap(outs[o], outs[q])) return SSM_ERR_INVALID_ARG;
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(workspace, 0, 256, s) != cudaSuccess) return SSM_ERR_CUDA;
+    SsdParams prm;
+    prm.x = x; prm.dt = dt; prm.B = B; prm.C = C;
+    prm.dt_bias = dt_bias; prm.A = A; prm.D = D; prm.h0 = h0;
+    prm.y = y; prm.h_last = h_last;
+    prm.error = fwd_scratch_view(workspace, 0).error;
+    prm.batch = batch; prm.seqlen = L; prm.heads = H; prm.groups = G; prm.softplus = softplus ? 1 : 0;
+    const int smem = SsdSmem::kTotal;
+    if (cudaFuncSetAttribute(ssd_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    ssd_fwd_kernel<<<static_cast<unsigned>(batch * H), 128, smem, s>>>(prm);
+    return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
 int ssm_conv_scan_step(void *conv_state, float *state, const void *x, const float *conv_w,

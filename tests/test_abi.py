@@ -269,3 +269,27 @@ def test_bwd_rejects_bad_arguments(lib):
     assert bwd(dx=_p(1)) == 1                      # dx over x
     assert bwd(dB=_p(17)) == 1                     # dB over dx
     assert bwd(ws=_p(16)) == 1                     # workspace over dout
+
+
+def test_ssd_rejects_bad_arguments(lib):
+    """The SSD entry: head dim 64, state 128, bf16; heads a multiple of groups;
+    alignment; outputs disjoint from inputs."""
+    import selective_state_space_38_b200 as m
+
+    def ssd(**over):
+        a = dict(x=_p(1), dt=_p(2), bias=None, sp=1, A=_p(3), B=_p(4), C=_p(5), D=None, h0=None, y=_p(7),
+                 hl=None, ws=_p(9), wsb=256, dims=ctypes.byref(m.SsdDims(2, 256, 8, 64, 2, 128, 1)))
+        a.update(over)
+        return lib.ssm_ssd_fwd(a["x"], a["dt"], a["bias"], a["sp"], a["A"], a["B"], a["C"], a["D"], a["h0"],
+                               a["y"], a["hl"], a["ws"], a["wsb"], a["dims"], None)
+    assert ssd(x=None) == 1
+    assert ssd(ws=None) == 1
+    assert ssd(wsb=100) == 1
+    assert ssd(dims=ctypes.byref(m.SsdDims(2, 256, 8, 64, 3, 128, 1))) == 1   # 8 heads, 3 groups
+    assert ssd(dims=ctypes.byref(m.SsdDims(2, 256, 8, 32, 2, 128, 1))) == 2   # head dim
+    assert ssd(dims=ctypes.byref(m.SsdDims(2, 256, 8, 64, 2, 64, 1))) == 2    # state dim
+    assert ssd(dims=ctypes.byref(m.SsdDims(2, 256, 8, 64, 2, 128, 0))) == 2   # float32
+    assert ssd(x=ctypes.c_void_p(0x11000008)) == 3
+    assert ssd(dt=ctypes.c_void_p(0x12000001)) == 3
+    assert ssd(y=_p(1)) == 1
+    assert ssd(hl=_p(4)) == 1

@@ -77,11 +77,19 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // ---- step size, gate ----------------------------------------------------------
-// softplus(v) = ln(1 + e^v).  Fast form for bf16 activations: two MUFU ops,
-// identity above 15 (the remainder e^-v < 3.1e-7 is below float resolution of v).
+// softplus(v) = ln(1 + e^v) from e = e^v.  For e < 1/16 the log1p series
+// e (1 - e/2 + e^2/3 - e^3/4) (truncation below e^4/5 < 3.1e-6 relative):
+// there 1 + e would lose the low bits of e and lg2.approx's absolute error
+// would become a large relative error of a small step size.  Otherwise
+// lg2(1 + e) ln 2, whose argument is >= 1.0625 (relative error ~3e-6).
+__device__ __forceinline__ float softplus_from_exp(float e) {
+    const float series = e * fmaf(-e, fmaf(-e, fmaf(-e, 0.25f, 1.0f / 3.0f), 0.5f), 1.0f);
+    return e < 0.0625f ? series : lg2_approx(1.0f + e) * kLn2;
+}
+// Fast form for bf16 activations: two MUFU ops, identity above 15 (the
+// remainder e^-v < 3.1e-7 is below float resolution of v).
 __device__ __forceinline__ float softplus_fast(float v) {
-    const float e = ex2_approx(v * kLog2e);
-    const float s = lg2_approx(1.0f + e) * kLn2;
+    const float s = softplus_from_exp(ex2_approx(fminf(v, 126.0f) * kLog2e));
     return v > 15.0f ? v : s;
 }
 // Accurate form for float32 activations.

@@ -91,19 +91,20 @@ constexpr int kBCPitch = 36;   // floats per time row of widened B|C (32 used; f
 // tiles, the B, C rows and, with TRAP, the lambda tile); bcf, ur and g are
 // double-buffered per chunk parity.  bcf, ur and g carry one spare step row
 // so that the scan warp's step-ahead preparation can run unconditionally on a
-// chunk's last step.  TRAP keeps two stages instead of three to make room for
-// its lambda tile and g table.
-template <typename T, bool TRAP = false>
+// chunk's last step.  The g table holds one float per step and lane: with
+// TRAP the end weight g_t, with CONV the skip term D xc_t.  TRAP and CONV keep
+// two stages instead of three to make room for it (and TRAP's lambda tile).
+template <typename T, bool TRAP = false, bool CONV = false>
 struct FwdSmem {
     static constexpr int kTC = kRowBytes / Act<T>::kBytes;          // timesteps per chunk
     static constexpr int kTileBytes = 32 * kRowBytes;               // one [32 ch][TC] tile
-    static constexpr int kStages = TRAP ? 2 : 3;                    // staged chunks per pair
+    static constexpr int kStages = (TRAP || CONV) ? 2 : 3;          // staged chunks per pair
     static constexpr int kBCRawOff = 3 * kTileBytes;                // raw B|C rows in a stage
     static constexpr int kLamOff = kBCRawOff + 2 * kNState * kRowBytes;
     static constexpr int kStageBytes = kLamOff + (TRAP ? kTileBytes : 0);
     static constexpr int kBCFBytes = (kTC + 1) * kBCPitch * 4;      // widened B|C, time-major
     static constexpr int kURBytes = (kTC + 1) * 32 * 8;             // float2 (u, r) per [t][lane]
-    static constexpr int kGBytes = TRAP ? (kTC + 1) * 32 * 4 : 0;   // float g per [t][lane] (TRAP)
+    static constexpr int kGBytes = (TRAP || CONV) ? (kTC + 1) * 32 * 4 : 0;  // float per [t][lane]
     static constexpr int kBCFOff = kStages * kStageBytes;
     static constexpr int kUROff = kBCFOff + 2 * kBCFBytes;
     static constexpr int kGOff = kUROff + 2 * kURBytes;
@@ -113,6 +114,7 @@ struct FwdSmem {
     static constexpr int kTotal = kPairs * kPairBytes + 1024;       // + slack to align the base to 1 KB
 };
 static_assert(FwdSmem<bf16raw, true>::kTotal <= 227 * 1024, "shared memory of the trapezoidal kernel");
+static_assert(FwdSmem<bf16raw, false, true>::kTotal <= 227 * 1024, "shared memory of the convolution kernel");
 static_assert(FwdSmem<bf16raw, false>::kTotal <= 227 * 1024, "shared memory of the kernel");
 
 __device__ __forceinline__ int swz(int row, int pc) { return pc ^ ((row >> 1) & 3); }
@@ -228,8 +230,8 @@ __device__ __forceinline__ void conv_halo(const FwdParams &p, int64_t b, int64_t
 // special-function op is covered by the other pairs' work.
 // With CONV, x first becomes silu(conv(x)): the lane's raw row and the three
 // inputs before it (halo, updated to this chunk's last three) give the
-// convolution, whose output replaces the raw row in the stage (in the
-// activation dtype, for the post warp's D skip) and feeds u = dt x in float32.
+// convolution, whose output feeds u = dt x and, as the skip term D xc written
+// to the g table, the post warp's output, both in float32.
 //
 // With TRAP (the exponential-trapezoidal rule), ur gets (s_t, r_t) and g gets
 // g_t, where g_t = lam_t dt_t x_t weights the interval's end and
@@ -271,20 +273,7 @@ __device__ __forceinline__ void chunk_prepass(uint8_t *stage, float2 *ur, int ro
 #pragma unroll
             for (int k = 0; k < 4; ++k) acc = fmaf(cc.cw[k], raw[t + k], acc);
             XC[t] = kAccurate ? acc * (1.0f / (1.0f + expf(-acc))) : silu_fast(acc);
-        }
-#pragma unroll
-        for (int pc = 0; pc < kPieces; ++pc) {
-            uint4 pk;
-            if constexpr (AT::kBytes == 2) {
-                const int t = pc * PP;
-                pk = make_uint4(pack_bf16x2(XC[t], XC[t + 1]), pack_bf16x2(XC[t + 2], XC[t + 3]),
-                                pack_bf16x2(XC[t + 4], XC[t + 5]), pack_bf16x2(XC[t + 6], XC[t + 7]));
-            } else {
-                const int t = pc * PP;
-                pk = make_uint4(__float_as_uint(XC[t]), __float_as_uint(XC[t + 1]), __float_as_uint(XC[t + 2]),
-                                __float_as_uint(XC[t + 3]));
-            }
-            *reinterpret_cast<uint4 *>(xr + (swz(row, pc) << 4)) = pk;
+            garr[t * 32 + row] = cc.Dx2.x * XC[t];
         }
     }
     float2 V[NP], E[NP];
@@ -298,8 +287,8 @@ __device__ __forceinline__ void chunk_prepass(uint8_t *stage, float2 *ur, int ro
 #pragma unroll
             for (int k = 0; k < NP; ++k) V[k] = make_float2(softplus_accurate(V[k].x), softplus_accurate(V[k].y));
         } else {
-            // ln(1 + e^v) = lg2(1 + 2^(v log2 e)) ln 2; the exponent is clamped so the
-            // sum stays finite, and max(., v) restores dt = v for large v
+            // e = 2^(v log2 e) (exponent clamped so 1 + e stays finite), then
+            // softplus_from_exp; max(., v) restores dt = v for large v
 #pragma unroll
             for (int k = 0; k < NP; ++k) {
                 E[k] = __fmul2_rn(V[k], make_float2(kLog2e, kLog2e));
@@ -308,14 +297,10 @@ __device__ __forceinline__ void chunk_prepass(uint8_t *stage, float2 *ur, int ro
 #pragma unroll
             for (int k = 0; k < NP; ++k) E[k] = make_float2(ex2_approx(E[k].x), ex2_approx(E[k].y));
 #pragma unroll
-            for (int k = 0; k < NP; ++k) E[k] = __fadd2_rn(E[k], make_float2(1.0f, 1.0f));
+            for (int k = 0; k < NP; ++k)
+                E[k] = make_float2(softplus_from_exp(E[k].x), softplus_from_exp(E[k].y));
 #pragma unroll
-            for (int k = 0; k < NP; ++k) E[k] = make_float2(lg2_approx(E[k].x), lg2_approx(E[k].y));
-#pragma unroll
-            for (int k = 0; k < NP; ++k) {
-                E[k] = __fmul2_rn(E[k], make_float2(kLn2, kLn2));
-                V[k] = make_float2(fmaxf(E[k].x, V[k].x), fmaxf(E[k].y, V[k].y));
-            }
+            for (int k = 0; k < NP; ++k) V[k] = make_float2(fmaxf(E[k].x, V[k].x), fmaxf(E[k].y, V[k].y));
         }
     }
     // V holds dt; E becomes r (S4D) or dt
@@ -500,9 +485,10 @@ __device__ __forceinline__ void chunk_summary(const float *bcf, const float2 *ur
 // out_t = (y_t + D x_t) silu(z_t), written over the lane's own x row of the
 // stage (already consumed); stage by stage over step pairs as in phase 1.
 // y_t is float `lane` of row t of ur.
-template <typename T>
+// With CONV the skip term comes from the g table (D xc, float32) instead of D x.
+template <typename T, bool CONV = false>
 __device__ __forceinline__ void chunk_postpass(uint8_t *stage, const float2 *ur, int row,
-                                               const ChanConst &cc, bool has_z) {
+                                               const ChanConst &cc, bool has_z, const float *garr = nullptr) {
     using AT = Act<T>;
     constexpr bool kAccurate = AT::kBytes == 4;
     constexpr int PP = AT::kPerPiece, TC = FwdSmem<T>::kTC, NP = TC / 2;
@@ -519,9 +505,12 @@ __device__ __forceinline__ void chunk_postpass(uint8_t *stage, const float2 *ur,
 #pragma unroll
     for (int k = 0; k < NP; ++k) {
         const int pc = (2 * k) / PP, i = (2 * k) % PP;
-        const float2 X = make_float2(AT::piece(xv[pc], i), AT::piece(xv[pc], i + 1));
-        O[k] = __ffma2_rn(X, cc.Dx2, make_float2(reinterpret_cast<const float *>(ur + (2 * k) * 32)[row],
-                                                 reinterpret_cast<const float *>(ur + (2 * k + 1) * 32)[row]));
+        const float2 Y = make_float2(reinterpret_cast<const float *>(ur + (2 * k) * 32)[row],
+                                     reinterpret_cast<const float *>(ur + (2 * k + 1) * 32)[row]);
+        if constexpr (CONV)
+            O[k] = __fadd2_rn(Y, make_float2(garr[(2 * k) * 32 + row], garr[(2 * k + 1) * 32 + row]));
+        else
+            O[k] = __ffma2_rn(make_float2(AT::piece(xv[pc], i), AT::piece(xv[pc], i + 1)), cc.Dx2, Y);
     }
     if (has_z) {
         float2 Z[NP], E[NP];
@@ -805,7 +794,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // rather than generic accesses, which cost twice the data-pipe passes on a
     // warp-uniform read.
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    using SM = FwdSmem<T, TRAP>;
+    using SM = FwdSmem<T, TRAP, CONV>;
     constexpr int TC = SM::kTC;
     constexpr int kStages = SM::kStages;
     const int lane = threadIdx.x & 31;
@@ -935,7 +924,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 cc = chan_const(p, d < p.dim ? d : p.dim - 1);
                 cc_d0 = dj.d0;
             }
-            chunk_postpass<T>(st, ur_of(j), lane, cc, has_z);
+            chunk_postpass<T, CONV>(st, ur_of(j), lane, cc, has_z, g_of(j));
             if constexpr (VEC) {
                 fence_proxy_async_smem();
                 __syncwarp();

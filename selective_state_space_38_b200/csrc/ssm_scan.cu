@@ -122,7 +122,7 @@ int launch_pass(const FwdParams &p, const FwdScratch &sc, const TmaMaps &tm, int
     const int64_t items = groups * ((p.seqlen + p.seg_steps - 1) / p.seg_steps);
     const int64_t want = (items + kPairs - 1) / kPairs;
     const int64_t ctas = want < sms ? want : sms;
-    const int smem = FwdSmem<T, TRAP>::kTotal;
+    const int smem = FwdSmem<T, TRAP, CONV>::kTotal;
     scan_fwd_kernel<T, VEC, true, CONV, TRAP><<<static_cast<unsigned>(ctas), kFwdThreads, smem, stream>>>(p, sc, tm);
     scan_fwd_kernel<T, VEC, false, CONV, TRAP><<<static_cast<unsigned>(ctas), kFwdThreads, smem, stream>>>(p, sc, tm);
     return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
@@ -134,7 +134,7 @@ int launch_pass(const FwdParams &p, const FwdScratch &sc, const TmaMaps &tm, int
 template <typename T, bool VEC, bool CONV, bool TRAP>
 int launch_fwd_kernels(FwdParams p, void *scratch, int64_t segs, int sms, cudaStream_t stream) {
     const int64_t groups = ((p.dim + 31) / 32) * p.batch;
-    const int smem = FwdSmem<T, TRAP>::kTotal;
+    const int smem = FwdSmem<T, TRAP, CONV>::kTotal;
     if (cudaFuncSetAttribute(scan_fwd_kernel<T, VEC, true, CONV, TRAP>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
         cudaFuncSetAttribute(scan_fwd_kernel<T, VEC, false, CONV, TRAP>,

@@ -33,7 +33,7 @@ def _gpu(inp, h0=None, conv_state=None, in_place=False):
     t = {k: to_dev(v) for k, v in inp.items() if isinstance(v, np.ndarray)}
     cs = to_dev(conv_state) if conv_state is not None else t.get("conv_state")
     out, hl, cso = ssm.ssm_conv_scan_fwd(
-        t["x"], t["conv_w"], t["conv_bias"], cs, t["delta"], t["delta_bias"], True, t["A"], t["B"], t["C"],
+        t["x"], t["conv_w"], t.get("conv_bias"), cs, t["delta"], t["delta_bias"], True, t["A"], t["B"], t["C"],
         t["D"], t["z"], to_dev(h0) if h0 is not None else t.get("h0"),
         conv_state_out=cs if (in_place and cs is not None) else None, check=True)
     torch.cuda.synchronize()

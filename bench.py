@@ -467,9 +467,13 @@ def bench_next_rows(args, device, hbm_peak, only=None):
     for name, (fn, nbytes, what) in rows.items():
         if only and name != only:
             continue
-        for _ in range(3):
-            fn()
-        torch.cuda.synchronize(device)
+        try:
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize(device)
+        except ssm.SSMError as exc:  # a refused call is reported in its row, not fatal to the line
+            res[name] = {"workload": what, "error": str(exc)}
+            continue
         n = 20 if name != "scan_bwd" else 10
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
         for a, b in ev:

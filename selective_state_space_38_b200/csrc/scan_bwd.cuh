@@ -285,7 +285,10 @@ __global__ void __launch_bounds__(kBwdWarps * 32) scan_bwd_kernel(const BwdParam
             // exclusive: the maps of the lanes before this one
             float h[kNState];
             {
-                const float sx = lane ? __shfl_up_sync(0xffffffffu, s, 1) : 0.0f;
+                // every lane takes part in the shuffle (a full-mask shuffle that a lane
+                // skips waits for it forever); lane 0 then discards the value
+                const float sxv = __shfl_up_sync(0xffffffffu, s, 1);
+                const float sx = lane ? sxv : 0.0f;
                 float ex[kNState], P[kNState];
 #pragma unroll
                 for (int n = 0; n < kNState; ++n) {
@@ -360,7 +363,8 @@ __global__ void __launch_bounds__(kBwdWarps * 32) scan_bwd_kernel(const BwdParam
             }
             float G[kNState];  // decayed adjoint entering this lane's last step from the right
             {
-                const float sx = lane < 31 ? __shfl_down_sync(0xffffffffu, s, 1) : 0.0f;
+                const float sxv = __shfl_down_sync(0xffffffffu, s, 1);  // every lane takes part
+                const float sx = lane < 31 ? sxv : 0.0f;
                 float fx[kNState], P[kNState];
 #pragma unroll
                 for (int n = 0; n < kNState; ++n) {

@@ -20,7 +20,6 @@
 #include "scan_fwd.cuh"
 #include "scan_step.cuh"
 #include "scan_bwd.cuh"
-#include "scan_fwd_lat.cuh"
 #include "ssd_fwd.cuh"
 
 namespace {
@@ -371,24 +370,6 @@ int validate_fwd(const void *x, const void *delta, const float *delta_bias, int 
     return SSM_OK;
 }
 
-// Whether a plain forward call takes the lanes-across-time kernel (one warp
-// per channel, warp-shuffle scans inside 128-step chunks) instead of the
-// two-pass segment schedule.  Both serve shapes whose channel groups are too
-// few for one chain per SM sub-partition.
-bool use_lat_schedule(const FwdParams &p, int sms) {
-    (void)p;
-    (void)sms;
-    return false;
-}
-
-template <typename T>
-int launch_fwd_lat(const FwdParams &p, cudaStream_t s) {
-    const dim3 grid(static_cast<unsigned>((p.dim + kLatWarps - 1) / kLatWarps), static_cast<unsigned>(p.batch));
-    if (p.batch > 65535) return SSM_ERR_UNSUPPORTED;
-    scan_fwd_lat_kernel<T><<<grid, kLatWarps * 32, 0, s>>>(p);
-    return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
-}
-
 // The forward call on a validated shape and a workspace of ws_bytes; then,
 // for a call with a convolution, the new convolution state.
 int dispatch_fwd(const FwdParams &p, size_t es, int act_dtype, void *ws, size_t ws_bytes, bool force_chained,
@@ -397,13 +378,6 @@ int dispatch_fwd(const FwdParams &p, size_t es, int act_dtype, void *ws, size_t 
     if (current_sms(&sms) != SSM_OK) return SSM_ERR_CUDA;
     const bool vec = (static_cast<size_t>(p.seqlen) * es) % 16 == 0;
     const bool bf = act_dtype == SSM_BF16;
-    if (!p.conv_k && !p.lam && !force_chained && use_lat_schedule(p, sms)) {
-        // the workspace's error word must still read as success
-        const int64_t groups = ((p.dim + 31) / 32) * p.batch;
-        if (ws_bytes < fwd_scratch_flag_bytes(groups)) return SSM_ERR_INVALID_ARG;
-        if (cudaMemsetAsync(ws, 0, fwd_scratch_flag_bytes(groups), s) != cudaSuccess) return SSM_ERR_CUDA;
-        return bf ? launch_fwd_lat<bf16raw>(p, s) : launch_fwd_lat<float>(p, s);
-    }
     int rc;
     if (p.conv_k) {
         rc = bf ? (vec ? launch_fwd<bf16raw, true, true>(p, ws, ws_bytes, sms, force_chained, s)

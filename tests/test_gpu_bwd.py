@@ -80,3 +80,13 @@ def test_mamba130m_layer_shape(orc):
     inp["dout"] = workloads.f32_to_bf16_bits(rng.standard_normal(inp["x"].shape).astype(np.float32))
     inp["dh_last"] = None
     _run(orc, inp, "mamba-130m layer")
+
+
+def test_mamba2p8b_layer_shape(orc):
+    """The Mamba-2.8B mixer-layer shape (4 x 4096 x 5120, bf16) in full: every
+    derivative of every channel, and dB, dC summed over all 5120 channels."""
+    inp = workloads.make_inputs(2)
+    rng = np.random.default_rng(2001)
+    inp["dout"] = workloads.f32_to_bf16_bits(rng.standard_normal(inp["x"].shape).astype(np.float32))
+    inp["dh_last"] = None
+    _run(orc, inp, "mamba-2.8b layer")

@@ -483,9 +483,11 @@ def bench_next_rows(args, device, hbm_peak, only=None):
         torch.cuda.synchronize(device)
         ms = statistics.mean([a.elapsed_time(b) for a, b in ev])
         gbs = nbytes / (ms * 1e-3) / 1e9
+        key = {"ssd_fwd": "ssd_fwd_layer", "scan_bwd": "scan_bwd_cfg2"}.get(name, f"{name}_cfg2")
         res[name] = {"workload": what if name == "ssd_fwd" else f"{c.name}: {what}", "ms": round(ms, 5),
                      "value": round(gbs, 2), "unit": "GB/s",
-                     "frac": round(gbs / hbm_peak, 4), "algorithmic_bytes_per_launch": nbytes, "steps": n}
+                     "frac": round(gbs / hbm_peak, 4), "algorithmic_bytes_per_launch": nbytes, "steps": n,
+                     "traffic": (_profiled(key) or {}).get("dram_bytes_per_launch"), "pipes": _pipes(key)}
     return res
 
 

@@ -857,17 +857,24 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         int64_t cc_d0 = -1;
         float halo[3] = {0.0f, 0.0f, 0.0f};  // convolution inputs before the chunk (CONV)
         float x_last = 0.0f, g_last = 0.0f;  // the step before the chunk (TRAP)
+        // Buffer reuse.  The u/r, B|C and g tables of chunk j are those chunk j - 2
+        // used, and the post warp reads chunk j - 2's outputs from them: chunk j is
+        // prepared once chunk j - 2 is posted.  The stage of chunk j + 1 is the one
+        // chunk j + 1 - kStages used.  With three stages that is chunk j - 2 too, so
+        // its load is issued before chunk j is prepared; with two stages it is chunk
+        // j - 1, whose post ends after chunk j could be prepared, so the load is
+        // issued once chunk j has been handed over (waiting for chunk j - 1 first
+        // would keep the prep warp idle while the scan warp runs chunk j - 1).
         ChunkDesc dnext = cur.next(p, sc, counter, lane);
         issue(dnext, 0);
         for (int64_t j = 0;; ++j) {
             const ChunkDesc dj = dnext;
-            // chunk j+1 goes to the stage that chunk j+1-kStages used: wait until it is posted
-            if (j >= kStages - 1 &&
-                !mbar_wait(posted + ((j + 1 - kStages) & 1), parity(j + 1 - kStages, 2), sc.error))
-                break;
+            if (j >= 2 && !mbar_wait(posted + (j & 1), parity(j - 2, 2), sc.error)) break;
             if (!(dj.flags & kStop)) {
-                dnext = cur.next(p, sc, counter, lane);
-                issue(dnext, j + 1);
+                if (kStages == 3) {
+                    dnext = cur.next(p, sc, counter, lane);
+                    issue(dnext, j + 1);
+                }
                 if constexpr (VEC) {
                     if (!mbar_wait(full + (j % kStages), parity(j, kStages), sc.error)) break;
                     n_waited = j + 1;
@@ -901,6 +908,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             __syncwarp();
             mbar_arrive(ready + (j & 1));
             if (dj.flags & kStop) break;
+            if (kStages == 2) {
+                if (j >= 1 && !mbar_wait(posted + ((j - 1) & 1), parity(j - 1, 2), sc.error)) break;
+                dnext = cur.next(p, sc, counter, lane);
+                issue(dnext, j + 1);
+            }
         }
         // loads still in flight after a wait gave up (none on the normal path)
         for (int64_t j = n_waited; j < n_issued; ++j) mbar_drain(full + (j % kStages), parity(j, kStages), sc.error);

@@ -11,18 +11,23 @@
 // the chunk,
 //   Y_diag = (C B^T o L) X,      L[i, j] = exp(cs_i - cs_j) dt_j (j <= i)
 //   Y_off  = diag(exp(cs)) C S_in^T
-//   S_out  = exp(cs_{Q-1}) S_in + (B o w)^T X,   w_j = exp(cs_{Q-1} - cs_j) dt_j
-// One CTA owns one (batch, head) sequence and walks its chunks; the state
-// S^T (N x P float32) stays in registers, one row per thread.  Per chunk:
-//   MMA1 G = C B^T (128 x 128 x 128) and MMA3 Yo = C S_in^T (128 x 64 x 128),
-//   then the epilogue forms L o G and B o w, then
-//   MMA2 Yd = (L o G) X (128 x 64 x 128) and MMA4 ST = (B o w)^T X (128 x 64 x 128).
-// Operands are bf16 in shared memory in the 128-byte-swizzled canonical
-// layouts; the ones that are products (L o G, B o w, S) are split into a bf16
-// high and low part (two MMAs each), so they keep about 16 bits.  One thread
-// issues the MMAs; tcgen05.commit arrives on an mbarrier that all warps wait
-// on (bounded); each thread then reads its TMEM lane with tcgen05.ld.
+//   S_out  = exp(cs_{Q-1}) S_in + B^T (w o X),   w_j = exp(cs_{Q-1} - cs_j) dt_j
+// One CTA owns one (batch, head) sequence and walks its chunks; the state S
+// (P x N float32) stays in registers, spread over the 256 threads.  Per chunk:
+//   MMA1 G = C B^T (128 x 128 x 128) and MMA3 Yo = C S_in^T (128 x 64 x 128);
+//   epilogue 1 forms L o G from G in tensor memory and writes it back there as
+//   bf16 (the A operand of MMA2), and w o X into shared memory;
+//   MMA2 Yd = (L o G) X (128 x 64 x 128) and MMA4 ST = B^T (w o X) (128 x 64 x 128);
+//   epilogue 2 writes y and updates the state.
+// Operands are bf16 in the 128-byte-swizzled canonical layouts; the ones that
+// are products (L o G, w o X, S) are split into a bf16 high part and a low part
+// (two MMAs each), so they keep about 16 bits.  C, B and X arrive by TMA into
+// one of two buffers, the next chunk's while this one is computed.  One thread
+// issues the MMAs; tcgen05.commit arrives on an mbarrier that every thread
+// waits on (bounded); each thread reads its TMEM lane with tcgen05.ld.
 #pragma once
+
+#include <cuda.h>
 
 #include "common.cuh"
 
@@ -31,10 +36,17 @@ namespace ssm {
 constexpr int kSsdQ = 128;  // chunk length
 constexpr int kSsdP = 64;   // head dimension
 constexpr int kSsdN = 128;  // state dimension
+constexpr int kSsdThreads = 256;
 constexpr uint32_t kSsdWaitLimit = 1u << 24;
 
+// TMA maps, rank 4 with the innermost dimension first: x [P][H][L][batch],
+// B and C [N][G][L][batch]; every box is 64 elements x 1 x 128 steps x 1.
+struct SsdMaps {
+    CUtensorMap x, B, C;
+};
+
 struct SsdParams {
-    const void *x, *dt, *B, *C;  // x [b][L][H][P], dt [b][L][H], B, C [b][L][G][N] (bf16)
+    const void *dt;              // [b][L][H] bf16
     const float *dt_bias, *A, *D, *h0;
     void *y;                     // [b][L][H][P] bf16
     float *h_last;               // [b][H][P][N]
@@ -43,19 +55,18 @@ struct SsdParams {
     int softplus;
 };
 
-// Shared memory (1024-byte aligned pieces; every operand tile is [rows][64] bf16
-// with 128-byte rows and the 128-byte swizzle).
+// Shared memory (1024-byte aligned pieces; every operand tile is [128 rows][64]
+// bf16 with 128-byte rows and the 128-byte swizzle).
 struct SsdSmem {
-    static constexpr int kTile = 128 * 128;          // one [128][64] bf16 tile
-    static constexpr int kC = 0;                     // C  [t][n]: 2 tiles (n < 64, n >= 64)
-    static constexpr int kB = kC + 2 * kTile;        // B  [t][n], then B o w (high part) in place
-    static constexpr int kBWlo = kB + 2 * kTile;     // B o w (low part)
-    static constexpr int kX = kBWlo + 2 * kTile;     // X  [t][p]: 1 tile
-    static constexpr int kMhi = kX + kTile;          // L o G [i][j] high: 2 tiles (j < 64, j >= 64)
-    static constexpr int kMlo = kMhi + 2 * kTile;    // low
-    static constexpr int kS = kMlo + 2 * kTile;      // S [p][n] high and low: 2 x 2 tiles of [64][64]
-    static constexpr int kCs = kS + 4 * 64 * 128;    // cs[128], dt[128], warp sums[4]
-    static constexpr int kBar = kCs + 3 * 128 * 4;
+    static constexpr int kTile = 128 * 128;        // one tile, 16 KB
+    static constexpr int kInC = 0;                 // C [t][n]: 2 tiles (n < 64, n >= 64)
+    static constexpr int kInB = 2 * kTile;         // B [t][n]: 2 tiles
+    static constexpr int kInX = 4 * kTile;         // X [t][p]: 1 tile
+    static constexpr int kInBytes = 5 * kTile;     // one input buffer (two of them)
+    static constexpr int kXw = 2 * kInBytes;       // w o X [t][p]: high tile, low tile
+    static constexpr int kS = kXw + 2 * kTile;     // S^T [n][p]: high tile, low tile
+    static constexpr int kCs = kS + 2 * kTile;     // cs[128], dt[128], warp sums[4]
+    static constexpr int kBar = kCs + 1088;        // load[2], mma[2], TMEM base
     static constexpr int kTotal = kBar + 64 + 1024;  // + alignment slack
 };
 static_assert(SsdSmem::kTotal <= 227 * 1024, "shared memory of the SSD kernel");
@@ -79,11 +90,23 @@ __host__ __device__ constexpr uint32_t ssd_idesc(int M, int N, int a_mn, int b_m
            (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// D (TMEM) (+)= A (shared memory) B (shared memory)
 __device__ __forceinline__ void ssd_mma(uint32_t d_tmem, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc) {
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(d_tmem),
         "l"(da), "l"(db), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+        : "memory");
+}
+
+// D (TMEM) (+)= A (TMEM: lane = row, two bf16 per column, lower index in the
+// low half) B (shared memory)
+__device__ __forceinline__ void ssd_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t db, uint32_t idesc,
+                                           uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(db), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
         : "memory");
 }
 
@@ -105,47 +128,87 @@ __device__ __forceinline__ void ssd_ld16(uint32_t taddr, float (&v)[16]) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 16 consecutive 32-bit columns of this thread's TMEM lane from registers
+__device__ __forceinline__ void ssd_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
+// 4-D tiled TMA load of a box at (c0, c1, c2, c3); completion as bytes on the mbarrier.
+__device__ __forceinline__ void tma_load_4d(void *dst, const void *tmap, int c0, int c1, int c2, int c3,
+                                            uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
+        "[%6];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ bool ssd_try(uint32_t addr, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Bounded wait for a phase of an mbarrier; gives up early once another wait
+// of the launch has given up (the error word is non-zero).
 __device__ __forceinline__ bool ssd_wait(uint64_t *bar, uint32_t parity, uint32_t *error) {
     const uint32_t addr = smem_u32(bar);
     for (uint32_t n = 0; n < kSsdWaitLimit; ++n) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(done)
-            : "r"(addr), "r"(parity)
-            : "memory");
-        if (done) return true;
+        if (ssd_try(addr, parity)) return true;
+        if ((n & 1023u) == 1023u && *reinterpret_cast<volatile uint32_t *>(error) != 0) return false;
     }
     atomicOr(error, 2u);
     return false;
 }
-
-__device__ __forceinline__ void split_bf16(float v, uint16_t &hi, uint16_t &lo) {
-    const uint32_t h = pack_bf16x2(v, 0.0f) & 0xffffu;
-    hi = static_cast<uint16_t>(h);
-    const float rest = v - __uint_as_float(h << 16);
-    lo = static_cast<uint16_t>(pack_bf16x2(rest, 0.0f) & 0xffffu);
+// The same wait before the CTA may exit with a load or an MMA in flight: it does
+// not stop early on the error word.
+__device__ __forceinline__ void ssd_drain(uint64_t *bar, uint32_t parity, uint32_t *error) {
+    const uint32_t addr = smem_u32(bar);
+    for (uint32_t n = 0; n < kSsdWaitLimit; ++n)
+        if (ssd_try(addr, parity)) return;
+    atomicOr(error, 2u);
 }
 
-// grid: batch * heads CTAs; block: 128 threads (thread i = TMEM lane i).
-__global__ void __launch_bounds__(128, 1) ssd_fwd_kernel(const SsdParams p) {
+// v = hi + lo with hi = bf16(v) and lo = bf16(v - hi), for two values at once:
+// the high parts and the low parts as bf16 pairs (first value in the low half).
+__device__ __forceinline__ void split_pair(float a, float b, uint32_t &hi, uint32_t &lo) {
+    hi = pack_bf16x2(a, b);
+    lo = pack_bf16x2(a - __uint_as_float(hi << 16), b - __uint_as_float(hi & 0xffff0000u));
+}
+
+// grid: batch * heads CTAs; block: 256 threads.  Thread (quad, half, lane) owns
+// row 32 quad + lane of every [128][..] tile (its TMEM lane) and the half
+// `half` of that row's columns.
+__global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams p, const __grid_constant__ SsdMaps tm) {
     extern __shared__ __align__(1024) uint8_t ssd_smem_raw[];
     uint8_t *sm = ssd_smem_raw + ((1024u - (smem_u32(ssd_smem_raw) & 1023u)) & 1023u);
     using S = SsdSmem;
     float *cs = reinterpret_cast<float *>(sm + S::kCs);
     float *dts = cs + 128;
     float *wsum = dts + 128;
-    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + S::kBar);  // [0] C-stage MMAs, [1] X-stage MMAs
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + S::kBar + 16);
+    uint64_t *lbar = reinterpret_cast<uint64_t *>(sm + S::kBar);  // [2] input buffer landed
+    uint64_t *mbar = lbar + 2;                                    // [0] MMA1/3 done, [1] MMA2/4 done
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(mbar + 2);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;
+    const int row = quad * 32 + lane;
     const int64_t b = blockIdx.x / p.heads, h = blockIdx.x % p.heads;
     const int64_t g = h / (p.heads / p.groups);
-    const int64_t L = p.seqlen, H = p.heads, G = p.groups;
+    const int64_t L = p.seqlen, H = p.heads;
     const float Ah = p.A[h], bias = p.dt_bias ? p.dt_bias[h] : 0.0f, Dh = p.D ? p.D[h] : 0.0f;
+    const int64_t chunks = (L + kSsdQ - 1) / kSsdQ;
 
     if (tid == 0) {
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(bar)));
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(bar + 1)));
+        for (int i = 0; i < 4; ++i) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(lbar + i)));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) {
@@ -156,188 +219,238 @@ __global__ void __launch_bounds__(128, 1) ssd_fwd_kernel(const SsdParams p) {
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tbase = *reinterpret_cast<volatile uint32_t *>(tslot);
+    // TMEM columns: G then L o G (128), Yd (64), Yo (64), ST (64)
     const uint32_t tG = tbase, tYd = tbase + 128, tYo = tbase + 192, tST = tbase + 256;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
 
-    // this thread's row n of the carried state S^T (64 values over p)
-    float st[kSsdP];
+    // the inputs of chunk c into buffer c & 1 (one thread)
+    auto load = [&](int64_t c) {
+        uint8_t *in = sm + (c & 1) * S::kInBytes;
+        uint64_t *bar = lbar + (c & 1);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive_expect_tx(bar, S::kInBytes);
+        const int t0 = static_cast<int>(c * kSsdQ), bi = static_cast<int>(b), gi = static_cast<int>(g);
+        tma_load_4d(in + S::kInC, &tm.C, 0, gi, t0, bi, bar);
+        tma_load_4d(in + S::kInC + S::kTile, &tm.C, 64, gi, t0, bi, bar);
+        tma_load_4d(in + S::kInB, &tm.B, 0, gi, t0, bi, bar);
+        tma_load_4d(in + S::kInB + S::kTile, &tm.B, 64, gi, t0, bi, bar);
+        tma_load_4d(in + S::kInX, &tm.x, 0, static_cast<int>(h), t0, bi, bar);
+    };
+    // raw dt of step t (zero past the end)
+    auto load_dt = [&](int64_t t) -> float {
+        return t < L ? Act<bf16raw>::load(p.dt, (b * L + t) * H + h) : 0.0f;
+    };
+
+    // this thread's share of the state: S[p][n] for n = row, p in [32 half, 32 half + 32)
+    float st[32];
 #pragma unroll
-    for (int q = 0; q < kSsdP; ++q) st[q] = p.h0 ? p.h0[((b * H + h) * kSsdP + q) * kSsdN + tid] : 0.0f;
+    for (int q = 0; q < 32; ++q)
+        st[q] = p.h0 ? p.h0[((b * H + h) * kSsdP + 32 * half + q) * kSsdN + row] : 0.0f;
+    // S^T [n][p] as bf16 high and low tiles (the B operand of MMA3, N = p contiguous)
+    auto write_state = [&]() {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) split_pair(st[8 * k + 2 * e], st[8 * k + 2 * e + 1], hi[e], lo[e]);
+            const uint32_t o = ssd_sw128(row, 32 * half + 8 * k);
+            *reinterpret_cast<uint4 *>(sm + S::kS + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4 *>(sm + S::kS + S::kTile + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+    };
 
-    const uint32_t a_c = smem_u32(sm + S::kC), a_b = smem_u32(sm + S::kB), a_bwlo = smem_u32(sm + S::kBWlo);
-    const uint32_t a_x = smem_u32(sm + S::kX), a_mhi = smem_u32(sm + S::kMhi), a_mlo = smem_u32(sm + S::kMlo);
-    const uint32_t a_s = smem_u32(sm + S::kS);
-    const int64_t chunks = (L + kSsdQ - 1) / kSsdQ;
+    int64_t loads_issued = 0, loads_waited = 0;
+    uint64_t *mma_pending = nullptr;  // the commit barrier of MMAs not yet seen complete
+    uint32_t mma_parity = 0;
+    if (tid == 0) load(0);
+    loads_issued = 1;
+    float dt_raw = tid < kSsdQ ? load_dt(tid) : 0.0f;
+    write_state();
+
+    const uint32_t a_s = smem_u32(sm + S::kS), a_xw = smem_u32(sm + S::kXw);
     bool ok = true;
-    for (int64_t c = 0; c < chunks && ok; ++c) {
+    for (int64_t c = 0; c < chunks; ++c) {
         const int64_t t0 = c * kSsdQ;
-        __syncthreads();
-        // ---- stage C, B ([t][n], 16-byte pieces), X ([t][p]) and dt; zero past L
-        const uint16_t *Bg = static_cast<const uint16_t *>(p.B), *Cg = static_cast<const uint16_t *>(p.C);
-        const uint16_t *Xg = static_cast<const uint16_t *>(p.x);
-        for (int i = tid; i < 128 * 16; i += 128) {  // 128 rows x 16 pieces of 8 elements
-            const int r = i / 16, pc = i % 16;
-            const int64_t t = t0 + r;
-            uint4 vb = make_uint4(0, 0, 0, 0), vc = vb;
-            if (t < L) {
-                const int64_t off = ((b * L + t) * G + g) * kSsdN + pc * 8;
-                vb = *reinterpret_cast<const uint4 *>(Bg + off);
-                vc = *reinterpret_cast<const uint4 *>(Cg + off);
-            }
-            const uint32_t o = (pc / 8) * S::kTile + ssd_sw128(r, (pc % 8) * 8);
-            *reinterpret_cast<uint4 *>(sm + S::kB + o) = vb;
-            *reinterpret_cast<uint4 *>(sm + S::kC + o) = vc;
-        }
-        for (int i = tid; i < 128 * 8; i += 128) {
-            const int r = i / 8, pc = i % 8;
-            const int64_t t = t0 + r;
-            uint4 vx = make_uint4(0, 0, 0, 0);
-            if (t < L) vx = *reinterpret_cast<const uint4 *>(Xg + ((b * L + t) * H + h) * kSsdP + pc * 8);
-            *reinterpret_cast<uint4 *>(sm + S::kX + ssd_sw128(r, pc * 8)) = vx;
-        }
-        // the carried state as bf16 high/low S[p][n] (K-major for C S^T: rows p, K = n)
-        for (int q = 0; q < kSsdP; ++q) {
-            uint16_t hi, lo;
-            split_bf16(st[q], hi, lo);
-            const uint32_t o = (tid / 64) * (64 * 128) + ssd_sw128(q, tid % 64);
-            *reinterpret_cast<uint16_t *>(sm + S::kS + o) = hi;
-            *reinterpret_cast<uint16_t *>(sm + S::kS + 2 * 64 * 128 + o) = lo;
-        }
-        // dt and the running sum cs of dt A over the chunk
-        {
-            const int64_t t = t0 + tid;
-            float dtv = 0.0f;
-            if (t < L) {
-                const float v = Act<bf16raw>::load(p.dt, (b * L + t) * H + h) + bias;
+        uint8_t *in = sm + (c & 1) * S::kInBytes;
+        const uint32_t a_c = smem_u32(in + S::kInC), a_b = smem_u32(in + S::kInB), a_x = smem_u32(in + S::kInX);
+        // ---- dt and the running sum cs of dt A over the chunk (threads 0..127)
+        float s = 0.0f, dtv = 0.0f;
+        if (tid < kSsdQ) {
+            if (t0 + tid < L) {
+                const float v = dt_raw + bias;
                 dtv = p.softplus ? softplus_fast(v) : v;
             }
-            float s = dtv * Ah;
+            s = dtv * Ah;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
                 const float o = __shfl_up_sync(0xffffffffu, s, off);
                 if (lane >= off) s += o;
             }
             if (lane == 31) wsum[warp] = s;
-            dts[tid] = dtv;
-            __syncthreads();
+            if (c + 1 < chunks) dt_raw = load_dt(t0 + kSsdQ + tid);  // the next chunk's, in flight meanwhile
+        }
+        // the next chunk's inputs go to the other buffer, whose last readers (chunk
+        // c - 1's MMAs and epilogue) have finished
+        if (tid == 0 && c + 1 < chunks) load(c + 1);
+        if (c + 1 < chunks) loads_issued = c + 2;
+        __syncthreads();
+        if (tid < kSsdQ) {
             for (int w = 0; w < warp; ++w) s += wsum[w];
             cs[tid] = s;
+            dts[tid] = dtv;
         }
+        // S^T visible to the tensor core, cs to every thread
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-        __syncthreads();
+        if (!__syncthreads_and(ssd_wait(lbar + (c & 1), static_cast<uint32_t>((c >> 1) & 1), p.error))) {
+            ok = false;
+            break;
+        }
+        loads_waited = c + 1;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         // ---- MMA1: G = C B^T; MMA3: Yo = C S^T (high, then low accumulated)
         if (tid == 0) {
-            constexpr uint32_t i1 = ssd_idesc(128, 128, 0, 0), i3 = ssd_idesc(128, 64, 0, 0);
-            for (int s = 0; s < 8; ++s) {
-                const uint32_t ko = (s / 4) * S::kTile + (s % 4) * 32;
-                ssd_mma(tG, ssd_desc(a_c + ko, 16, 1024), ssd_desc(a_b + ko, 16, 1024), i1, s > 0);
+            constexpr uint32_t i1 = ssd_idesc(128, 128, 0, 0), i3 = ssd_idesc(128, 64, 0, 1);
+            for (int k = 0; k < 8; ++k) {
+                const uint32_t ko = (k / 4) * S::kTile + (k % 4) * 32;
+                ssd_mma(tG, ssd_desc(a_c + ko, 16, 1024), ssd_desc(a_b + ko, 16, 1024), i1, k > 0);
             }
             for (int part = 0; part < 2; ++part)
-                for (int s = 0; s < 8; ++s) {
-                    const uint32_t ka = (s / 4) * S::kTile + (s % 4) * 32;
-                    const uint32_t kb = part * (2 * 64 * 128) + (s / 4) * (64 * 128) + (s % 4) * 32;
-                    ssd_mma(tYo, ssd_desc(a_c + ka, 16, 1024), ssd_desc(a_s + kb, 16, 1024), i3, part > 0 || s > 0);
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t ka = (k / 4) * S::kTile + (k % 4) * 32;
+                    ssd_mma(tYo, ssd_desc(a_c + ka, 16, 1024),
+                            ssd_desc(a_s + part * S::kTile + 2048 * k, S::kTile, 1024), i3, part > 0 || k > 0);
                 }
-            ssd_commit(bar);
+            ssd_commit(mbar);
         }
-        // every thread takes the same branch: a wait that gave up ends the walk
-        if (!__syncthreads_and(ssd_wait(bar, static_cast<uint32_t>(c & 1), p.error))) {
+        mma_pending = mbar;
+        if (!__syncthreads_and(ssd_wait(mbar, mma_parity, p.error))) {
             ok = false;
             break;
         }
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        // ---- epilogue 1: row i of L o G (high/low); row j of B o w (high in place, low)
         const float total = cs[kSsdQ - 1];
+        float dx[32];  // D x of this thread's row and column half, kept for epilogue 2
         {
-            const int i = tid;
+            // ---- epilogue 1a: row i of L o G, columns j in [64 half, 64 half + 64), 32
+            // at a time: read their G, then write the high parts to the first 16 and
+            // the low parts to the last 16 of the same 32 TMEM columns (two bf16 each)
+            const int i = row;
             const float csi = cs[i];
-            for (int j0 = 0; j0 < kSsdQ; j0 += 16) {
-                float v[16];
-                ssd_ld16(tG + lane_off + j0, v);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int j = j0 + e;
-                    const float m = j <= i ? v[e] * __expf(csi - cs[j]) * dts[j] : 0.0f;
-                    uint16_t hi, lo;
-                    split_bf16(m, hi, lo);
-                    const uint32_t o = (j / 64) * S::kTile + ssd_sw128(i, j % 64);
-                    *reinterpret_cast<uint16_t *>(sm + S::kMhi + o) = hi;
-                    *reinterpret_cast<uint16_t *>(sm + S::kMlo + o) = lo;
+            for (int jp = 0; jp < 2; ++jp) {
+                const uint32_t col = tG + lane_off + 64 * half + 32 * jp;
+                float v[32];
+                {
+                    float v0[16], v1[16];
+                    ssd_ld16(col, v0);
+                    ssd_ld16(col + 16, v1);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) v[e] = v0[e], v[16 + e] = v1[e];
                 }
+                uint32_t mh[16], ml[16];
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    const int j = 64 * half + 32 * jp + e;
+                    const float m0 = j <= i ? v[e] * __expf(csi - cs[j]) * dts[j] : 0.0f;
+                    const float m1 = j + 1 <= i ? v[e + 1] * __expf(csi - cs[j + 1]) * dts[j + 1] : 0.0f;
+                    split_pair(m0, m1, mh[e / 2], ml[e / 2]);
+                }
+                ssd_st16(col, mh);
+                ssd_st16(col + 16, ml);
             }
-            const int jr = tid;
-            const float w = __expf(total - cs[jr]) * dts[jr];
-            for (int n = 0; n < kSsdN; ++n) {
-                const uint32_t o = (n / 64) * S::kTile + ssd_sw128(jr, n % 64);
-                const float bv = __uint_as_float(static_cast<uint32_t>(*reinterpret_cast<uint16_t *>(sm + S::kB + o)) << 16);
-                uint16_t hi, lo;
-                split_bf16(bv * w, hi, lo);
-                *reinterpret_cast<uint16_t *>(sm + S::kB + o) = hi;
-                *reinterpret_cast<uint16_t *>(sm + S::kBWlo + o) = lo;
+            // ---- epilogue 1b: row t of w o X (high and low tiles) and D x, p in [32 half, 32 half + 32)
+            const int t = row;
+            const float w = __expf(total - cs[t]) * dts[t];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t o = ssd_sw128(t, 32 * half + 8 * k);
+                const uint4 xv = *reinterpret_cast<const uint4 *>(in + S::kInX + o);
+                const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float x0 = __uint_as_float(xw[e] << 16), x1 = __uint_as_float(xw[e] & 0xffff0000u);
+                    dx[8 * k + 2 * e] = Dh * x0;
+                    dx[8 * k + 2 * e + 1] = Dh * x1;
+                    split_pair(w * x0, w * x1, hi[e], lo[e]);
+                }
+                *reinterpret_cast<uint4 *>(sm + S::kXw + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4 *>(sm + S::kXw + S::kTile + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
             }
         }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
         __syncthreads();
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        // ---- MMA2: Yd = (L o G) X; MMA4: ST = (B o w)^T X (each high + low)
+        // ---- MMA2: Yd = (L o G) X, A from TMEM; MMA4: ST = B^T (w o X); each high + low
         if (tid == 0) {
             constexpr uint32_t i2 = ssd_idesc(128, 64, 0, 1), i4 = ssd_idesc(128, 64, 1, 1);
             for (int part = 0; part < 2; ++part)
-                for (int s = 0; s < 8; ++s) {
-                    const uint32_t ka = (s / 4) * S::kTile + (s % 4) * 32;
-                    ssd_mma(tYd, ssd_desc((part ? a_mlo : a_mhi) + ka, 16, 1024), ssd_desc(a_x + 2048 * s, S::kTile, 1024),
-                            i2, part > 0 || s > 0);
+                for (int k = 0; k < 8; ++k) {
+                    // K step k covers j in [16 k, 16 k + 16): column half k / 4, 32-column
+                    // block (k % 4) / 2, high or low 16 columns, 8 columns per 16 j
+                    const uint32_t acol = 64 * (k / 4) + 32 * ((k % 4) / 2) + 16 * part + 8 * (k % 2);
+                    ssd_mma_ts(tYd, tG + acol, ssd_desc(a_x + 2048 * k, S::kTile, 1024), i2, part > 0 || k > 0);
                 }
             for (int part = 0; part < 2; ++part)
-                for (int s = 0; s < 8; ++s)
-                    ssd_mma(tST, ssd_desc((part ? a_bwlo : a_b) + 2048 * s, S::kTile, 1024),
-                            ssd_desc(a_x + 2048 * s, S::kTile, 1024), i4, part > 0 || s > 0);
-            ssd_commit(bar + 1);
+                for (int k = 0; k < 8; ++k)
+                    ssd_mma(tST, ssd_desc(a_b + 2048 * k, S::kTile, 1024),
+                            ssd_desc(a_xw + part * S::kTile + 2048 * k, S::kTile, 1024), i4, part > 0 || k > 0);
+            ssd_commit(mbar + 1);
         }
-        if (!__syncthreads_and(ssd_wait(bar + 1, static_cast<uint32_t>(c & 1), p.error))) {
+        mma_pending = mbar + 1;
+        if (!__syncthreads_and(ssd_wait(mbar + 1, mma_parity, p.error))) {
             ok = false;
             break;
         }
+        mma_pending = nullptr;
+        mma_parity ^= 1u;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        // ---- epilogue 2: y row i; state row n
+        // ---- epilogue 2: y row i, p in [32 half, 32 half + 32); state row n, same p
         {
-            const int i = tid;
+            const int i = row;
             const int64_t t = t0 + i;
             const float ecs = __expf(cs[i]);
             uint16_t *yg = static_cast<uint16_t *>(p.y);
-            for (int q0 = 0; q0 < kSsdP; q0 += 16) {
+#pragma unroll
+            for (int q0 = 0; q0 < 32; q0 += 16) {
                 float yd[16], yo[16];
-                ssd_ld16(tYd + lane_off + q0, yd);
-                ssd_ld16(tYo + lane_off + q0, yo);
+                ssd_ld16(tYd + lane_off + 32 * half + q0, yd);
+                ssd_ld16(tYo + lane_off + 32 * half + q0, yo);
                 uint32_t pk[8];
 #pragma unroll
-                for (int e = 0; e < 16; e += 2) {
-                    const float x0 = __uint_as_float(static_cast<uint32_t>(*reinterpret_cast<uint16_t *>(sm + S::kX + ssd_sw128(i, q0 + e))) << 16);
-                    const float x1 = __uint_as_float(static_cast<uint32_t>(*reinterpret_cast<uint16_t *>(sm + S::kX + ssd_sw128(i, q0 + e + 1))) << 16);
-                    pk[e / 2] = pack_bf16x2(fmaf(ecs, yo[e], yd[e]) + Dh * x0, fmaf(ecs, yo[e + 1], yd[e + 1]) + Dh * x1);
-                }
+                for (int e = 0; e < 16; e += 2)
+                    pk[e / 2] = pack_bf16x2(fmaf(ecs, yo[e], yd[e]) + dx[q0 + e],
+                                            fmaf(ecs, yo[e + 1], yd[e + 1]) + dx[q0 + e + 1]);
                 if (t < L) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(yg + ((b * L + t) * H + h) * kSsdP + q0);
+                    uint4 *dst = reinterpret_cast<uint4 *>(yg + ((b * L + t) * H + h) * kSsdP + 32 * half + q0);
                     dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                     dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
                 }
             }
             const float et = __expf(total);
-            for (int q0 = 0; q0 < kSsdP; q0 += 16) {
+#pragma unroll
+            for (int q0 = 0; q0 < 32; q0 += 16) {
                 float v[16];
-                ssd_ld16(tST + lane_off + q0, v);
+                ssd_ld16(tST + lane_off + 32 * half + q0, v);
 #pragma unroll
                 for (int e = 0; e < 16; ++e) st[q0 + e] = fmaf(et, st[q0 + e], v[e]);
             }
+            write_state();
         }
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     }
+    // a wait that gave up leaves no load or MMA running when the CTA ends
+    if (!ok && tid == 0) {
+        if (mma_pending) ssd_drain(mma_pending, mma_parity, p.error);
+        for (int64_t c = loads_waited; c < loads_issued; ++c)
+            ssd_drain(lbar + (c & 1), static_cast<uint32_t>((c >> 1) & 1), p.error);
+    }
     if (p.h_last && ok) {
 #pragma unroll
-        for (int q = 0; q < kSsdP; ++q) p.h_last[((b * H + h) * kSsdP + q) * kSsdN + tid] = st[q];
+        for (int q = 0; q < 32; ++q) p.h_last[((b * H + h) * kSsdP + 32 * half + q) * kSsdN + row] = st[q];
     }
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");

@@ -77,6 +77,19 @@ bool encode3d(CUtensorMap *m, CUtensorMapDataType dt, size_t es, const void *bas
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A rank-4 [d3][d2][d1][d0] tensor (d0 contiguous) with a [1][box2][1][box0] box.
+bool encode4d(CUtensorMap *m, CUtensorMapDataType dt, size_t es, const void *base, uint64_t d0, uint64_t d1,
+              uint64_t d2, uint64_t d3, uint32_t box0, uint32_t box2, CUtensorMapSwizzle sw) {
+    auto fn = tensor_map_encoder();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {d0, d1, d2, d3};
+    const cuuint64_t strides[3] = {d0 * es, d0 * d1 * es, d0 * d1 * d2 * es};
+    const cuuint32_t box[4] = {box0, 1, box2, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(m, dt, 4, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <typename T>
 bool make_maps(const FwdParams &p, TmaMaps *tm) {
     const CUtensorMapDataType dt = Act<T>::kBytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
@@ -621,7 +634,11 @@ int ssm_ssd_fwd(const void *x, const void *dt, const float *dt_bias, int softplu
                   N = dims->dstate;
     if (batch < 1 || L < 1 || H < 1 || P < 1 || G < 1 || N < 1 || H % G != 0) return SSM_ERR_INVALID_ARG;
     if (P != kSsdP || N != kSsdN || dims->act_dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
-    if (batch * H > INT32_MAX || L > INT32_MAX) return SSM_ERR_UNSUPPORTED;
+    // grid.x holds batch * heads; TMA coordinates and strides are 32-bit and 40-bit
+    if (batch * H > INT32_MAX || L > INT32_MAX - kSsdQ ||
+        static_cast<double>(batch) * L * H * P * 2 >= static_cast<double>(1ull << 40) ||
+        static_cast<double>(batch) * L * G * N * 2 >= static_cast<double>(1ull << 40))
+        return SSM_ERR_UNSUPPORTED;
     if (workspace_bytes < 256) return SSM_ERR_INVALID_ARG;
     for (const void *ptr : {x, B, C, (const void *)y, (const void *)h0, (const void *)h_last, (const void *)workspace})
         if (ptr && !aligned16(ptr)) return SSM_ERR_MISALIGNED;
@@ -643,15 +660,23 @@ int ssm_ssd_fwd(const void *x, const void *dt, const float *dt_bias, int softplu
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(workspace, 0, 256, s) != cudaSuccess) return SSM_ERR_CUDA;
     SsdParams prm;
-    prm.x = x; prm.dt = dt; prm.B = B; prm.C = C;
+    prm.dt = dt;
     prm.dt_bias = dt_bias; prm.A = A; prm.D = D; prm.h0 = h0;
     prm.y = y; prm.h_last = h_last;
     prm.error = fwd_scratch_view(workspace, 0).error;
     prm.batch = batch; prm.seqlen = L; prm.heads = H; prm.groups = G; prm.softplus = softplus ? 1 : 0;
+    SsdMaps tm;
+    constexpr CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    constexpr CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+    const uint64_t ub = static_cast<uint64_t>(batch), uL = static_cast<uint64_t>(L);
+    if (!encode4d(&tm.x, bf, 2, x, kSsdP, static_cast<uint64_t>(H), uL, ub, 64, kSsdQ, sw) ||
+        !encode4d(&tm.B, bf, 2, B, kSsdN, static_cast<uint64_t>(G), uL, ub, 64, kSsdQ, sw) ||
+        !encode4d(&tm.C, bf, 2, C, kSsdN, static_cast<uint64_t>(G), uL, ub, 64, kSsdQ, sw))
+        return SSM_ERR_CUDA;
     const int smem = SsdSmem::kTotal;
     if (cudaFuncSetAttribute(ssd_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return SSM_ERR_CUDA;
-    ssd_fwd_kernel<<<static_cast<unsigned>(batch * H), 128, smem, s>>>(prm);
+    ssd_fwd_kernel<<<static_cast<unsigned>(batch * H), kSsdThreads, smem, s>>>(prm, tm);
     return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 

@@ -249,9 +249,8 @@ int ssm_trap_scan_step(float *state, const void *x, const void *delta, const flo
 
 /*
  * Workspace bytes that ssm_scan_bwd needs for the shape `dims`: the states at
- * the start of every 128-step chunk (64 B per channel and chunk) and one
- * partial dB, dC per block of 32 channels (batch * 2 * dstate * seqlen * 4 B
- * each).  Returns SSM_OK and writes *bytes, or an SSM_ERR_* code.
+ * the start of every 32-step segment (64 B per channel and segment, i.e. 2 B
+ * per channel and step).  Returns SSM_OK and writes *bytes, or an SSM_ERR_* code.
  */
 int ssm_scan_bwd_workspace_size(const ssm_dims_t *dims, size_t *bytes);
 
@@ -259,8 +258,8 @@ int ssm_scan_bwd_workspace_size(const ssm_dims_t *dims, size_t *bytes);
  * Backward pass of ssm_scan_fwd: the derivatives of a loss L with respect to
  * every input, given dout = dL/dout and dh_last = dL/dh_last.  As Appendix D
  * "Memory" describes, the intermediate states are not stored by the forward
- * pass: the call stores the state at the start of every 128-step chunk and
- * recomputes the chunk's states from it while it runs the adjoint recurrence
+ * pass: the call stores the state at the start of every 32-step segment and
+ * recomputes the segment's states from it while it runs the adjoint recurrence
  *   g_t = C_t dy_t + Abar_{t+1} g_{t+1},  dy_t = dout_t silu(z_t)
  * backwards through the chunk.
  *
@@ -275,9 +274,9 @@ int ssm_scan_bwd_workspace_size(const ssm_dims_t *dims, size_t *bytes);
  *   dh0            optional [batch][dim][dstate] float32 (NULL: not written)
  *   workspace      at least ssm_scan_bwd_workspace_size bytes, 16-byte aligned
  * Alignment: 16 bytes for every pointer except delta_bias, D, dD, dbias (4).
- * No output may overlap an input or another output.  dB and dC are summed in
- * a fixed order; dA, dD and dbias are summed over the batch with float atomics
- * (their last bits may differ between calls).  Returns SSM_OK or an SSM_ERR_* code.
+ * No output may overlap an input or another output.  dB and dC (sums over
+ * channels) and dA, dD, dbias (sums over the batch) are added with float
+ * atomics, so their last bits may differ between calls.  Returns SSM_OK or an SSM_ERR_* code.
  */
 int ssm_scan_bwd(const void *x, const void *delta, const float *delta_bias, int softplus,
                  const float *A, const void *B, const void *C, const float *D, const void *z,

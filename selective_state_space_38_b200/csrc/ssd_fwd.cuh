@@ -65,8 +65,8 @@ struct SsdSmem {
     static constexpr int kInBytes = 5 * kTile;     // one input buffer (two of them)
     static constexpr int kXw = 2 * kInBytes;       // w o X [t][p]: high tile, low tile
     static constexpr int kS = kXw + 2 * kTile;     // S^T [n][p]: high tile, low tile
-    static constexpr int kCs = kS + 2 * kTile;     // cs[128], dt[128], warp sums[4]
-    static constexpr int kBar = kCs + 1088;        // load[2], mma[2], TMEM base
+    static constexpr int kCs = kS + 2 * kTile;     // cs[128], dt[128], F[128], warp sums[4]
+    static constexpr int kBar = kCs + 1600;        // load[2], mma[2], TMEM base
     static constexpr int kTotal = kBar + 64 + 1024;  // + alignment slack
 };
 static_assert(SsdSmem::kTotal <= 227 * 1024, "shared memory of the SSD kernel");
@@ -194,7 +194,8 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
     using S = SsdSmem;
     float *cs = reinterpret_cast<float *>(sm + S::kCs);
     float *dts = cs + 128;
-    float *wsum = dts + 128;
+    float *Fs = dts + 128;  // F_j = exp(-cs_j) dt_j, when every |cs| of the chunk is at most 80
+    float *wsum = Fs + 128;
     uint64_t *lbar = reinterpret_cast<uint64_t *>(sm + S::kBar);  // [2] input buffer landed
     uint64_t *mbar = lbar + 2;                                    // [0] MMA1/3 done, [1] MMA2/4 done
     uint32_t *tslot = reinterpret_cast<uint32_t *>(mbar + 2);
@@ -298,7 +299,10 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
             for (int w = 0; w < warp; ++w) s += wsum[w];
             cs[tid] = s;
             dts[tid] = dtv;
+            Fs[tid] = __expf(-s) * dtv;
         }
+        // exp(cs_i - cs_j) = exp(cs_i) exp(-cs_j) without overflow when every |cs| <= 80
+        const bool factored = __syncthreads_and(tid >= kSsdQ || fabsf(s) <= 80.0f) != 0;
         // S^T visible to the tensor core, cs to every thread
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -310,16 +314,22 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         // ---- MMA1: G = C B^T; MMA3: Yo = C S^T (high, then low accumulated)
         if (tid == 0) {
+            // a descriptor of base + off is the base's plus off / 16 (no carry: every
+            // shared-memory address is below 2^18)
             constexpr uint32_t i1 = ssd_idesc(128, 128, 0, 0), i3 = ssd_idesc(128, 64, 0, 1);
+            const uint64_t dC = ssd_desc(a_c, 16, 1024), dB = ssd_desc(a_b, 16, 1024);
+            const uint64_t dS = ssd_desc(a_s, S::kTile, 1024);
+#pragma unroll
             for (int k = 0; k < 8; ++k) {
-                const uint32_t ko = (k / 4) * S::kTile + (k % 4) * 32;
-                ssd_mma(tG, ssd_desc(a_c + ko, 16, 1024), ssd_desc(a_b + ko, 16, 1024), i1, k > 0);
+                const uint32_t ko = ((k / 4) * S::kTile + (k % 4) * 32) >> 4;
+                ssd_mma(tG, dC + ko, dB + ko, i1, k > 0);
             }
+#pragma unroll
             for (int part = 0; part < 2; ++part)
+#pragma unroll
                 for (int k = 0; k < 8; ++k) {
-                    const uint32_t ka = (k / 4) * S::kTile + (k % 4) * 32;
-                    ssd_mma(tYo, ssd_desc(a_c + ka, 16, 1024),
-                            ssd_desc(a_s + part * S::kTile + 2048 * k, S::kTile, 1024), i3, part > 0 || k > 0);
+                    const uint32_t ka = ((k / 4) * S::kTile + (k % 4) * 32) >> 4;
+                    ssd_mma(tYo, dC + ka, dS + ((part * S::kTile + 2048 * k) >> 4), i3, part > 0 || k > 0);
                 }
             ssd_commit(mbar);
         }
@@ -336,7 +346,7 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
             // at a time: read their G, then write the high parts to the first 16 and
             // the low parts to the last 16 of the same 32 TMEM columns (two bf16 each)
             const int i = row;
-            const float csi = cs[i];
+            const float csi = cs[i], Ei = __expf(csi);
 #pragma unroll
             for (int jp = 0; jp < 2; ++jp) {
                 const uint32_t col = tG + lane_off + 64 * half + 32 * jp;
@@ -349,12 +359,27 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
                     for (int e = 0; e < 16; ++e) v[e] = v0[e], v[16 + e] = v1[e];
                 }
                 uint32_t mh[16], ml[16];
+                const int j0 = 64 * half + 32 * jp;
+                if (factored) {
+                    const float4 *F4 = reinterpret_cast<const float4 *>(Fs + j0);
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const int j = 64 * half + 32 * jp + e;
-                    const float m0 = j <= i ? v[e] * __expf(csi - cs[j]) * dts[j] : 0.0f;
-                    const float m1 = j + 1 <= i ? v[e + 1] * __expf(csi - cs[j + 1]) * dts[j + 1] : 0.0f;
-                    split_pair(m0, m1, mh[e / 2], ml[e / 2]);
+                    for (int e = 0; e < 32; e += 4) {
+                        const float4 f = F4[e / 4];
+                        const float m0 = j0 + e <= i ? v[e] * (Ei * f.x) : 0.0f;
+                        const float m1 = j0 + e + 1 <= i ? v[e + 1] * (Ei * f.y) : 0.0f;
+                        const float m2 = j0 + e + 2 <= i ? v[e + 2] * (Ei * f.z) : 0.0f;
+                        const float m3 = j0 + e + 3 <= i ? v[e + 3] * (Ei * f.w) : 0.0f;
+                        split_pair(m0, m1, mh[e / 2], ml[e / 2]);
+                        split_pair(m2, m3, mh[e / 2 + 1], ml[e / 2 + 1]);
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        const int j = j0 + e;
+                        const float m0 = j <= i ? v[e] * __expf(csi - cs[j]) * dts[j] : 0.0f;
+                        const float m1 = j + 1 <= i ? v[e + 1] * __expf(csi - cs[j + 1]) * dts[j + 1] : 0.0f;
+                        split_pair(m0, m1, mh[e / 2], ml[e / 2]);
+                    }
                 }
                 ssd_st16(col, mh);
                 ssd_st16(col + 16, ml);
@@ -387,17 +412,23 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
         // ---- MMA2: Yd = (L o G) X, A from TMEM; MMA4: ST = B^T (w o X); each high + low
         if (tid == 0) {
             constexpr uint32_t i2 = ssd_idesc(128, 64, 0, 1), i4 = ssd_idesc(128, 64, 1, 1);
+            const uint64_t dX = ssd_desc(a_x, S::kTile, 1024), dBt = ssd_desc(a_b, S::kTile, 1024);
+            const uint64_t dXw = ssd_desc(a_xw, S::kTile, 1024);
+#pragma unroll
             for (int part = 0; part < 2; ++part)
+#pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     // K step k covers j in [16 k, 16 k + 16): column half k / 4, 32-column
                     // block (k % 4) / 2, high or low 16 columns, 8 columns per 16 j
                     const uint32_t acol = 64 * (k / 4) + 32 * ((k % 4) / 2) + 16 * part + 8 * (k % 2);
-                    ssd_mma_ts(tYd, tG + acol, ssd_desc(a_x + 2048 * k, S::kTile, 1024), i2, part > 0 || k > 0);
+                    ssd_mma_ts(tYd, tG + acol, dX + ((2048 * k) >> 4), i2, part > 0 || k > 0);
                 }
+#pragma unroll
             for (int part = 0; part < 2; ++part)
+#pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    ssd_mma(tST, ssd_desc(a_b + 2048 * k, S::kTile, 1024),
-                            ssd_desc(a_xw + part * S::kTile + 2048 * k, S::kTile, 1024), i4, part > 0 || k > 0);
+                    ssd_mma(tST, dBt + ((2048 * k) >> 4), dXw + ((part * S::kTile + 2048 * k) >> 4), i4,
+                            part > 0 || k > 0);
             ssd_commit(mbar + 1);
         }
         mma_pending = mbar + 1;

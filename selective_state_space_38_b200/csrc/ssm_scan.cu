@@ -419,13 +419,10 @@ int dispatch_fwd(const FwdParams &p, size_t es, int act_dtype, void *ws, size_t 
                      : launch_fwd<float, false, false>(p, ws, ws_bytes, sms, force_chained, s));
 }
 
-// Workspace of the backward pass: the chunk checkpoints, then the blocks'
-// partial dB, dC (256-byte aligned pieces).
-size_t bwd_ckpt_bytes(int64_t batch, int64_t L, int64_t dim) {
-    return (static_cast<size_t>(batch) * dim * bwd_chunks(L) * kNState * 4 + 255) / 256 * 256;
-}
+// Workspace of the backward pass: the states at every segment start (64 B per
+// channel and segment of 32 steps), rounded up to 256 bytes.
 size_t bwd_workspace_bytes(int64_t batch, int64_t L, int64_t dim) {
-    return bwd_ckpt_bytes(batch, L, dim) + static_cast<size_t>(bwd_blocks(dim)) * batch * 2 * kNState * L * 4;
+    return (static_cast<size_t>(batch) * dim * bwd_segments(L) * kNState * 4 + 255) / 256 * 256;
 }
 
 template <typename T>
@@ -433,17 +430,16 @@ int launch_bwd(BwdParams p, cudaStream_t s) {
     const int smem = static_cast<int>(sizeof(BwdSmem));
     if (cudaFuncSetAttribute(scan_bwd_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return SSM_ERR_CUDA;
-    if (p.dA && cudaMemsetAsync(p.dA, 0, static_cast<size_t>(p.dim) * kNState * 4, s) != cudaSuccess)
+    const size_t bn = static_cast<size_t>(p.batch) * kNState * p.seqlen * 4;
+    if (cudaMemsetAsync(p.dA, 0, static_cast<size_t>(p.dim) * kNState * 4, s) != cudaSuccess ||
+        cudaMemsetAsync(p.dB, 0, bn, s) != cudaSuccess || cudaMemsetAsync(p.dC, 0, bn, s) != cudaSuccess)
         return SSM_ERR_CUDA;
     if (p.dD && cudaMemsetAsync(p.dD, 0, static_cast<size_t>(p.dim) * 4, s) != cudaSuccess) return SSM_ERR_CUDA;
     if (p.dbias && cudaMemsetAsync(p.dbias, 0, static_cast<size_t>(p.dim) * 4, s) != cudaSuccess)
         return SSM_ERR_CUDA;
-    const int64_t nch = p.batch * p.dim;
-    scan_bwd_ckpt_kernel<T><<<static_cast<unsigned>((nch + 3) / 4), 128, 0, s>>>(p);
-    const dim3 grid(static_cast<unsigned>(bwd_blocks(p.dim)), static_cast<unsigned>(p.batch));
-    scan_bwd_kernel<T><<<grid, kBwdWarps * 32, smem, s>>>(p);
-    const int64_t n = p.batch * 2 * kNState * p.seqlen;
-    scan_bwd_reduce_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(p);
+    const int64_t groups = bwd_groups(p.batch, p.dim);
+    scan_bwd_ckpt_kernel<T><<<static_cast<unsigned>((groups + 3) / 4), 128, 0, s>>>(p);
+    scan_bwd_kernel<T><<<static_cast<unsigned>(groups), 32, smem, s>>>(p);
     return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
@@ -583,7 +579,7 @@ int ssm_scan_bwd(const void *x, const void *delta, const float *delta_bias, int 
     if (!dims_ok(batch, L, dim) || N < 1) return SSM_ERR_INVALID_ARG;
     if (N != kNState) return SSM_ERR_UNSUPPORTED;
     if (dims->act_dtype != SSM_F32 && dims->act_dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
-    if (batch > 65535 || bwd_blocks(dim) > INT32_MAX) return SSM_ERR_UNSUPPORTED;  // grid.y holds the batch
+    if (bwd_groups(batch, dim) > INT32_MAX) return SSM_ERR_UNSUPPORTED;  // grid.x holds the groups
     const size_t es = dims->act_dtype == SSM_F32 ? 4 : 2;
     for (const void *ptr : {x, delta, (const void *)A, B, C, z, (const void *)h0, dout, (const void *)dx,
                             (const void *)ddelta, (const void *)(z ? dz : nullptr), (const void *)dB,
@@ -620,7 +616,6 @@ int ssm_scan_bwd(const void *x, const void *delta, const float *delta_bias, int 
     p.dx = dx; p.ddelta = ddelta; p.dz = z ? dz : nullptr;
     p.dA = dA; p.dD = dD; p.dbias = dbias; p.dh0 = dh0; p.dB = dB; p.dC = dC;
     p.ckpt = static_cast<float *>(workspace);
-    p.part = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + bwd_ckpt_bytes(batch, L, dim));
     p.batch = batch; p.seqlen = L; p.dim = dim; p.softplus = softplus ? 1 : 0;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return dims->act_dtype == SSM_BF16 ? launch_bwd<bf16raw>(p, s) : launch_bwd<float>(p, s);

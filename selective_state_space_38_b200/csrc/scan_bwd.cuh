@@ -48,23 +48,23 @@ __device__ __forceinline__ float bwd_softplus(float v) {
     return Act<T>::kBytes == 4 ? softplus_accurate(v) : softplus_fast(v);
 }
 
-// exp(A[d, n] dt) for the 16 states.  all_s4d (warp-uniform): every lane's row
-// has the S4D-real structure A[d, n] = (n + 1) A[d, 0], and the decays are the
-// powers of r = exp(A[d, 0] dt) (one MUFU op and a multiplication tree);
-// otherwise sixteen MUFU ops.
-__device__ __forceinline__ void bwd_decay(const float (&a2)[kNState], bool all_s4d, float dt,
-                                          float (&out)[kNState]) {
+// exp(A[d, n] dt) for the 16 states, as pairs (states 2j, 2j + 1).  all_s4d
+// (warp-uniform): every lane's row has the S4D-real structure
+// A[d, n] = (n + 1) A[d, 0], and the decays are the powers of r = exp(A[d, 0] dt)
+// (one MUFU op and a multiplication tree); otherwise sixteen MUFU ops.
+__device__ __forceinline__ void bwd_decay(const float (&a2)[kNState], bool all_s4d, float dt, float2 (&out)[8]) {
     if (all_s4d) {
         const float r = ex2_approx(a2[0] * dt);
         const float r2 = r * r, r4 = r2 * r2, r8 = r4 * r4;
-        out[0] = r; out[1] = r2; out[2] = r2 * r; out[3] = r4;
+        out[0] = make_float2(r, r2);
+        out[1] = __fmul2_rn(out[0], make_float2(r2, r2));  // r^3, r^4
+        out[2] = __fmul2_rn(out[0], make_float2(r4, r4));  // r^5, r^6
+        out[3] = __fmul2_rn(out[1], make_float2(r4, r4));  // r^7, r^8
 #pragma unroll
-        for (int n = 4; n < 8; ++n) out[n] = out[n - 4] * r4;
-#pragma unroll
-        for (int n = 8; n < 16; ++n) out[n] = out[n - 8] * r8;
+        for (int j = 4; j < 8; ++j) out[j] = __fmul2_rn(out[j - 4], make_float2(r8, r8));
     } else {
 #pragma unroll
-        for (int n = 0; n < kNState; ++n) out[n] = ex2_approx(a2[n] * dt);
+        for (int j = 0; j < 8; ++j) out[j] = make_float2(ex2_approx(a2[2 * j] * dt), ex2_approx(a2[2 * j + 1] * dt));
     }
 }
 
@@ -122,109 +122,136 @@ __device__ __forceinline__ void bwd_store16(void *base, int64_t row_off, int64_t
     }
 }
 
-// Warp transpose-reduce: every lane holds 32 values; afterwards lane k holds
-// the sum over the warp's lanes of value k.  Five butterfly levels; at the
-// level of mask m a lane keeps the half of its values selected by (lane & m)
-// and receives the partner's copy of that half.
-__device__ __forceinline__ float warp_transpose_sum32(const float (&v)[32], int lane) {
-    float w16[16], w8[8], w4[4], w2[2];
+
+// Warp transpose-reduce: every lane holds 32 values (16 pairs); afterwards lane
+// k holds the sum over the warp's lanes of value k.  Five butterfly levels; at
+// the level of mask m a lane keeps the half of its values selected by
+// (lane & m) and receives the partner's copy of that half.
+__device__ __forceinline__ float warp_transpose_sum32(const float2 (&v)[16], int lane) {
+    float2 w8[8], w4[4], w2[2];
+    float2 w1;
     {
         const bool up = lane & 16;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float send = up ? v[i] : v[i + 16], keep = up ? v[i + 16] : v[i];
-            w16[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+        for (int i = 0; i < 8; ++i) {
+            const float2 send = up ? v[i] : v[i + 8], keep = up ? v[i + 8] : v[i];
+            w8[i] = __fadd2_rn(keep, make_float2(__shfl_xor_sync(0xffffffffu, send.x, 16),
+                                                 __shfl_xor_sync(0xffffffffu, send.y, 16)));
         }
     }
     {
         const bool up = lane & 8;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float send = up ? w16[i] : w16[i + 8], keep = up ? w16[i + 8] : w16[i];
-            w8[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+        for (int i = 0; i < 4; ++i) {
+            const float2 send = up ? w8[i] : w8[i + 4], keep = up ? w8[i + 4] : w8[i];
+            w4[i] = __fadd2_rn(keep, make_float2(__shfl_xor_sync(0xffffffffu, send.x, 8),
+                                                 __shfl_xor_sync(0xffffffffu, send.y, 8)));
         }
     }
     {
         const bool up = lane & 4;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float send = up ? w8[i] : w8[i + 4], keep = up ? w8[i + 4] : w8[i];
-            w4[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+        for (int i = 0; i < 2; ++i) {
+            const float2 send = up ? w4[i] : w4[i + 2], keep = up ? w4[i + 2] : w4[i];
+            w2[i] = __fadd2_rn(keep, make_float2(__shfl_xor_sync(0xffffffffu, send.x, 4),
+                                                 __shfl_xor_sync(0xffffffffu, send.y, 4)));
         }
     }
     {
         const bool up = lane & 2;
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const float send = up ? w4[i] : w4[i + 2], keep = up ? w4[i + 2] : w4[i];
-            w2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-        }
+        const float2 send = up ? w2[0] : w2[1], keep = up ? w2[1] : w2[0];
+        w1 = __fadd2_rn(keep, make_float2(__shfl_xor_sync(0xffffffffu, send.x, 2),
+                                          __shfl_xor_sync(0xffffffffu, send.y, 2)));
     }
     const bool up = lane & 1;
-    const float send = up ? w2[0] : w2[1], keep = up ? w2[1] : w2[0];
+    const float send = up ? w1.x : w1.y, keep = up ? w1.y : w1.x;
     return keep + __shfl_xor_sync(0xffffffffu, send, 1);
 }
 
 // B (n < 16) and C (16 <= n < 32) of a sub-chunk's steps, widened: row k holds
 // the 32 values of step t0 + k (zero past L).  Lane j loads row j of B or C.
 template <typename T>
-__device__ __forceinline__ void bwd_stage_bc(const BwdParams &p, int64_t b, int64_t t0, bool vec, int lane,
-                                             float *bc) {
-    float v[kBwdSub];
+__device__ __forceinline__ void bwd_load_bc(const BwdParams &p, int64_t b, int64_t t0, bool vec, int lane,
+                                            float (&v)[kBwdSub]) {
     const void *src = lane < kNState ? p.B : p.C;
     bwd_load16<T>(src, (b * kNState + (lane & (kNState - 1))) * p.seqlen, t0, p.seqlen, vec, v);
+}
+__device__ __forceinline__ void bwd_put_bc(float *bc, int lane, const float (&v)[kBwdSub]) {
 #pragma unroll
     for (int k = 0; k < kBwdSub; ++k) bc[k * 32 + lane] = v[k];
 }
 
-// B and C of step k from the staged rows (warp-uniform 16-byte reads)
-__device__ __forceinline__ void bwd_bc_row(const float *bc, int k, float (&Bv)[kNState], float (&Cv)[kNState]) {
+// B and C of step k from the staged rows (warp-uniform 16-byte reads), as pairs
+__device__ __forceinline__ void bwd_b_row(const float *bc, int k, float2 (&B2)[8]) {
     const float4 *r = reinterpret_cast<const float4 *>(bc + k * 32);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-        const float4 b = r[q], c = r[4 + q];
-        Bv[4 * q] = b.x; Bv[4 * q + 1] = b.y; Bv[4 * q + 2] = b.z; Bv[4 * q + 3] = b.w;
-        Cv[4 * q] = c.x; Cv[4 * q + 1] = c.y; Cv[4 * q + 2] = c.z; Cv[4 * q + 3] = c.w;
+        const float4 b = r[q];
+        B2[2 * q] = make_float2(b.x, b.y);
+        B2[2 * q + 1] = make_float2(b.z, b.w);
+    }
+}
+__device__ __forceinline__ void bwd_c_row(const float *bc, int k, float2 (&C2)[8]) {
+    const float4 *r = reinterpret_cast<const float4 *>(bc + k * 32 + kNState);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float4 c = r[q];
+        C2[2 * q] = make_float2(c.x, c.y);
+        C2[2 * q + 1] = make_float2(c.z, c.w);
     }
 }
 
-// One step of the forward recurrence: h = exp(A dt) h + dt x B.
-__device__ __forceinline__ void bwd_fwd_step(float (&h)[kNState], const float (&a2)[kNState], bool all_s4d,
-                                             float dt, float x, const float *bc, int k) {
-    float a[kNState], Bv[kNState], Cv[kNState];
-    bwd_decay(a2, all_s4d, dt, a);
-    bwd_bc_row(bc, k, Bv, Cv);
-    const float u = dt * x;
-#pragma unroll
-    for (int n = 0; n < kNState; ++n) h[n] = fmaf(a[n], h[n], u * Bv[n]);
+// Four consecutive floats added to global memory without a returned value
+// (the address 16-byte aligned).
+__device__ __forceinline__ void red_add_v4(float *p, float a, float b, float c, float d) {
+    asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
 }
 
-// Per-lane constants of a channel: A row (and A log2 e), S4D structure, bias, D.
+// Per-lane constants of a channel: A row (A log2 e for the decays, A as pairs),
+// S4D structure of the whole warp, bias, D.
 struct BwdChan {
-    float a2[kNState], An[kNState];
+    float a2[kNState];
+    float2 An2[8];
     bool all_s4d;
     float bias, Dd;
 };
 __device__ __forceinline__ BwdChan bwd_chan(const BwdParams &p, int64_t dc) {
     BwdChan c;
+    float An[kNState];
     const float4 *ar = reinterpret_cast<const float4 *>(p.A + dc * kNState);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         const float4 v = __ldg(ar + q);
-        c.An[4 * q] = v.x; c.An[4 * q + 1] = v.y; c.An[4 * q + 2] = v.z; c.An[4 * q + 3] = v.w;
+        An[4 * q] = v.x; An[4 * q + 1] = v.y; An[4 * q + 2] = v.z; An[4 * q + 3] = v.w;
     }
 #pragma unroll
-    for (int n = 0; n < kNState; ++n) c.a2[n] = c.An[n] * kLog2e;
-    c.all_s4d = __all_sync(0xffffffffu, bwd_row_is_s4d(c.An));
+    for (int n = 0; n < kNState; ++n) c.a2[n] = An[n] * kLog2e;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) c.An2[j] = make_float2(An[2 * j], An[2 * j + 1]);
+    c.all_s4d = __all_sync(0xffffffffu, bwd_row_is_s4d(An));
     c.bias = p.delta_bias ? p.delta_bias[dc] : 0.0f;
     c.Dd = p.D ? p.D[dc] : 0.0f;
     return c;
 }
 
+// One step of the forward recurrence: h = exp(A dt) h + dt x B (pairs of states).
+__device__ __forceinline__ void bwd_fwd_step(float2 (&h)[8], const BwdChan &cc, float dt, float x, const float *bc,
+                                             int k) {
+    float2 a[8], B2[8];
+    bwd_decay(cc.a2, cc.all_s4d, dt, a);
+    bwd_b_row(bc, k, B2);
+    const float u = dt * x;
+    const float2 u2 = make_float2(u, u);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) h[j] = __ffma2_rn(a[j], h[j], __fmul2_rn(u2, B2[j]));
+}
+
 // ---- checkpoints: the state at the start of every segment -------------------------
 // One warp per group of 32 channels of one sequence (four groups per CTA, each
 // on its own); the forward recurrence over the whole sequence, with the state
-// written at every segment start.
+// written at every segment start.  The next sub-chunk's inputs are loaded
+// while the current one is computed.
 template <typename T>
 __global__ void __launch_bounds__(128) scan_bwd_ckpt_kernel(const BwdParams p) {
     __shared__ __align__(16) float bc_all[4][kBwdSub * 32];
@@ -239,37 +266,48 @@ __global__ void __launch_bounds__(128) scan_bwd_ckpt_kernel(const BwdParams p) {
     const bool vec = (L * Act<T>::kBytes) % 16 == 0;
     const BwdChan cc = bwd_chan(p, dc);
     float *bc = bc_all[warp];
-    float h[kNState];
+    float2 h[8];
     if (p.h0) {
         const float4 *src = reinterpret_cast<const float4 *>(p.h0 + chan * kNState);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             const float4 v = __ldg(src + q);
-            h[4 * q] = v.x; h[4 * q + 1] = v.y; h[4 * q + 2] = v.z; h[4 * q + 3] = v.w;
+            h[2 * q] = make_float2(v.x, v.y);
+            h[2 * q + 1] = make_float2(v.z, v.w);
         }
     } else {
 #pragma unroll
-        for (int n = 0; n < kNState; ++n) h[n] = 0.0f;
+        for (int j = 0; j < 8; ++j) h[j] = make_float2(0.0f, 0.0f);
     }
+    float xv[kBwdSub], dv[kBwdSub], bv[kBwdSub];
+    bwd_load16<T>(p.x, chan * L, 0, L, vec, xv);
+    bwd_load16<T>(p.delta, chan * L, 0, L, vec, dv);
+    bwd_load_bc<T>(p, b, 0, vec, lane, bv);
     for (int64_t t0 = 0; t0 < L; t0 += kBwdSub) {
         if (t0 % kBwdSeg == 0 && active) {
             float4 *dst = reinterpret_cast<float4 *>(p.ckpt + (chan * segs + t0 / kBwdSeg) * kNState);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) dst[q] = make_float4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
+            for (int q = 0; q < 4; ++q)
+                dst[q] = make_float4(h[2 * q].x, h[2 * q].y, h[2 * q + 1].x, h[2 * q + 1].y);
         }
-        float xv[kBwdSub], dv[kBwdSub];
-        bwd_load16<T>(p.x, chan * L, t0, L, vec, xv);
-        bwd_load16<T>(p.delta, chan * L, t0, L, vec, dv);
         __syncwarp();  // the previous sub-chunk's reads of bc are done
-        bwd_stage_bc<T>(p, b, t0, vec, lane, bc);
+        bwd_put_bc(bc, lane, bv);
         __syncwarp();
+        float xn[kBwdSub], dn[kBwdSub];
+        if (t0 + kBwdSub < L) {  // the next sub-chunk's inputs, in flight during this one
+            bwd_load16<T>(p.x, chan * L, t0 + kBwdSub, L, vec, xn);
+            bwd_load16<T>(p.delta, chan * L, t0 + kBwdSub, L, vec, dn);
+            bwd_load_bc<T>(p, b, t0 + kBwdSub, vec, lane, bv);
+        }
 #pragma unroll
         for (int k = 0; k < kBwdSub; ++k) {
             if (t0 + k >= L) break;  // warp-uniform
             const float v = dv[k] + cc.bias;
             const float dt = p.softplus ? bwd_softplus<T>(v) : v;
-            bwd_fwd_step(h, cc.a2, cc.all_s4d, dt, xv[k], bc, k);
+            bwd_fwd_step(h, cc, dt, xv[k], bc, k);
         }
+#pragma unroll
+        for (int k = 0; k < kBwdSub; ++k) xv[k] = xn[k], dv[k] = dn[k];
     }
 }
 
@@ -278,43 +316,28 @@ struct BwdSmem {
     float hs[kBwdSub + 1][4][32][4];  // h_{t0-1} .. h_{t0+15} of the sub-chunk, per quarter and lane
     float bc[kBwdSub * 32];           // B|C of the sub-chunk's steps
     float io[4][kBwdSub][32];         // x, delta, z, dout per step and lane; then dx, ddelta, dz and
-                                      // this lane's dB|dC sum in their places
+                                      // the warp's dB|dC sums of the step in their places
 };
 
-__device__ __forceinline__ void bwd_put_state(BwdSmem &sm, int k, int lane, const float (&h)[kNState]) {
+__device__ __forceinline__ void bwd_put_state(BwdSmem &sm, int k, int lane, const float2 (&h)[8]) {
 #pragma unroll
     for (int q = 0; q < 4; ++q)
-        *reinterpret_cast<float4 *>(sm.hs[k][q][lane]) = make_float4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
+        *reinterpret_cast<float4 *>(sm.hs[k][q][lane]) =
+            make_float4(h[2 * q].x, h[2 * q].y, h[2 * q + 1].x, h[2 * q + 1].y);
 }
-__device__ __forceinline__ void bwd_get_state(const BwdSmem &sm, int k, int lane, float (&h)[kNState]) {
+__device__ __forceinline__ void bwd_get_state(const BwdSmem &sm, int k, int lane, float2 (&h)[8]) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         const float4 v = *reinterpret_cast<const float4 *>(sm.hs[k][q][lane]);
-        h[4 * q] = v.x; h[4 * q + 1] = v.y; h[4 * q + 2] = v.z; h[4 * q + 3] = v.w;
+        h[2 * q] = make_float2(v.x, v.y);
+        h[2 * q + 1] = make_float2(v.z, v.w);
     }
-}
-
-// The lane's per-step scalars of step k of the staged sub-chunk.
-struct BwdStep {
-    float x, dt, sg, z, go;
-};
-template <typename T>
-__device__ __forceinline__ BwdStep bwd_step_in(const BwdParams &p, const BwdSmem &sm, const BwdChan &cc, int k,
-                                               int lane) {
-    BwdStep s;
-    s.x = sm.io[0][k][lane];
-    const float v = sm.io[1][k][lane] + cc.bias;
-    s.dt = p.softplus ? bwd_softplus<T>(v) : v;
-    s.sg = p.softplus ? 1.0f / (1.0f + __expf(-v)) : 1.0f;  // d dt / d v
-    s.z = sm.io[2][k][lane];
-    s.go = sm.io[3][k][lane];
-    return s;
 }
 
 // ---- the backward pass over one group of 32 channels of one sequence -------------
 // grid: one warp (CTA) per group.
 template <typename T>
-__global__ void __launch_bounds__(32) scan_bwd_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(32, 1) scan_bwd_kernel(const BwdParams p) {
     using AT = Act<T>;
     constexpr bool kAccurate = AT::kBytes == 4;
     extern __shared__ __align__(16) uint8_t bwd_smem_raw[];
@@ -329,48 +352,49 @@ __global__ void __launch_bounds__(32) scan_bwd_kernel(const BwdParams p) {
     const bool vec = (L * AT::kBytes) % 16 == 0;
     const BwdChan cc = bwd_chan(p, dc);
 
-    float G[kNState], dA[kNState];  // decayed adjoint entering the current step from the right; dA sum
+    // G: the decayed adjoint entering the current step from the right; dA: its sum
+    float2 G[8], dA[8];
 #pragma unroll
-    for (int n = 0; n < kNState; ++n) {
-        G[n] = p.dh_last ? p.dh_last[chan * kNState + n] : 0.0f;
-        dA[n] = 0.0f;
+    for (int j = 0; j < 8; ++j) {
+        G[j] = p.dh_last ? make_float2(p.dh_last[chan * kNState + 2 * j], p.dh_last[chan * kNState + 2 * j + 1])
+                         : make_float2(0.0f, 0.0f);
+        dA[j] = make_float2(0.0f, 0.0f);
     }
     float dDs = 0.0f, dbs = 0.0f;
 
     // stage the inputs and B|C of the sub-chunk starting at t0 (all four inputs,
     // or only x and delta for a pass that recomputes states)
     auto stage = [&](int64_t t0, bool all) {
-        __syncwarp();  // the previous users of io and bc are done
-        float v[kBwdSub];
+        float v[kBwdSub], w[kBwdSub];
         bwd_load16<T>(p.x, row, t0, L, vec, v);
+        bwd_load16<T>(p.delta, row, t0, L, vec, w);
+        float bv[kBwdSub];
+        bwd_load_bc<T>(p, b, t0, vec, lane, bv);
+        __syncwarp();  // the previous users of io and bc are done
 #pragma unroll
-        for (int k = 0; k < kBwdSub; ++k) sm.io[0][k][lane] = v[k];
-        bwd_load16<T>(p.delta, row, t0, L, vec, v);
-#pragma unroll
-        for (int k = 0; k < kBwdSub; ++k) sm.io[1][k][lane] = v[k];
+        for (int k = 0; k < kBwdSub; ++k) sm.io[0][k][lane] = v[k], sm.io[1][k][lane] = w[k];
+        bwd_put_bc(sm.bc, lane, bv);
         if (all) {
-            if (p.z) {
-                bwd_load16<T>(p.z, row, t0, L, vec, v);
+            if (p.z) bwd_load16<T>(p.z, row, t0, L, vec, v);
+            bwd_load16<T>(p.dout, row, t0, L, vec, w);
 #pragma unroll
-                for (int k = 0; k < kBwdSub; ++k) sm.io[2][k][lane] = v[k];
+            for (int k = 0; k < kBwdSub; ++k) {
+                if (p.z) sm.io[2][k][lane] = v[k];
+                sm.io[3][k][lane] = w[k];
             }
-            bwd_load16<T>(p.dout, row, t0, L, vec, v);
-#pragma unroll
-            for (int k = 0; k < kBwdSub; ++k) sm.io[3][k][lane] = v[k];
         }
-        bwd_stage_bc<T>(p, b, t0, vec, lane, sm.bc);
         __syncwarp();
     };
     // the forward recurrence over the staged sub-chunk from h (steps below L);
     // with keep, the states before and after every step go to sm.hs
-    auto forward = [&](int64_t t0, float (&h)[kNState], bool keep) {
+    auto forward = [&](int64_t t0, float2 (&h)[8], bool keep) {
         if (keep) bwd_put_state(sm, 0, lane, h);
-#pragma unroll
+#pragma unroll 4
         for (int k = 0; k < kBwdSub; ++k) {
             if (t0 + k < L) {  // warp-uniform
                 const float v = sm.io[1][k][lane] + cc.bias;
                 const float dt = p.softplus ? bwd_softplus<T>(v) : v;
-                bwd_fwd_step(h, cc.a2, cc.all_s4d, dt, sm.io[0][k][lane], sm.bc, k);
+                bwd_fwd_step(h, cc, dt, sm.io[0][k][lane], sm.bc, k);
             }
             if (keep) bwd_put_state(sm, k + 1, lane, h);
         }
@@ -379,49 +403,57 @@ __global__ void __launch_bounds__(32) scan_bwd_kernel(const BwdParams p) {
     // the adjoint over the staged sub-chunk, its steps from the last to the first,
     // with the states in sm.hs; then its outputs
     auto backward = [&](int64_t t0) {
-#pragma unroll 1
+#pragma unroll 2
         for (int k = kBwdSub - 1; k >= 0; --k) {
             if (t0 + k >= L) continue;  // warp-uniform
-            const BwdStep s = bwd_step_in<T>(p, sm, cc, k, lane);
-            float a[kNState], Bv[kNState], Cv[kNState], hn[kNState];
-            bwd_decay(cc.a2, cc.all_s4d, s.dt, a);
-            bwd_bc_row(sm.bc, k, Bv, Cv);
+            const float x = sm.io[0][k][lane];
+            const float v = sm.io[1][k][lane] + cc.bias;
+            const float dt = p.softplus ? bwd_softplus<T>(v) : v;
+            const float sg = p.softplus ? 1.0f / (1.0f + __expf(-v)) : 1.0f;  // d dt / d v
+            float2 a[8], B2[8], C2[8], hn[8];
+            bwd_decay(cc.a2, cc.all_s4d, dt, a);
+            bwd_b_row(sm.bc, k, B2);
+            bwd_c_row(sm.bc, k, C2);
             bwd_get_state(sm, k + 1, lane, hn);  // h_t
-            float y = cc.Dd * s.x;
+            float2 y2 = make_float2(cc.Dd * x, 0.0f);
 #pragma unroll
-            for (int n = 0; n < kNState; ++n) y = fmaf(Cv[n], hn[n], y);
-            float dy = s.go, dzv = 0.0f;
+            for (int j = 0; j < 8; ++j) y2 = __ffma2_rn(C2[j], hn[j], y2);
+            const float y = y2.x + y2.y, go = sm.io[3][k][lane];
+            float dy = go, dzv = 0.0f;
             if (p.z) {
-                const float sz = kAccurate ? 1.0f / (1.0f + expf(-s.z)) : rcp_approx(1.0f + ex2_approx(-s.z * kLog2e));
-                dy = s.go * s.z * sz;
-                dzv = s.go * y * sz * fmaf(s.z, 1.0f - sz, 1.0f);
+                const float zz = sm.io[2][k][lane];
+                const float sz = kAccurate ? 1.0f / (1.0f + expf(-zz)) : rcp_approx(1.0f + ex2_approx(-zz * kLog2e));
+                dy = go * zz * sz;
+                dzv = go * y * sz * fmaf(zz, 1.0f - sz, 1.0f);
             }
-            float vals[32];  // this lane's dB (n < 16) and dC (n >= 16) terms of the step
-            float g[kNState];
+            float2 vals[16];  // this lane's dB (values 0..15) and dC (16..31) terms of the step
+            float2 g[8];
+            const float2 dy2 = make_float2(dy, dy), dya2 = make_float2(act * dy, act * dy);
 #pragma unroll
-            for (int n = 0; n < kNState; ++n) {
-                g[n] = fmaf(Cv[n], dy, G[n]);
-                vals[kNState + n] = act * dy * hn[n];
+            for (int j = 0; j < 8; ++j) {
+                g[j] = __ffma2_rn(C2[j], dy2, G[j]);
+                vals[8 + j] = __fmul2_rn(dya2, hn[j]);
             }
-            float hp[kNState];
+            float2 hp[8];
             bwd_get_state(sm, k, lane, hp);  // h_{t-1}
-            const float dtx = s.dt * s.x;
-            float dxs = 0.0f, ddt = 0.0f;
+            const float dtxa = act * dt * x;
+            const float2 dtx2 = make_float2(dtxa, dtxa), x2 = make_float2(x, x), dt2 = make_float2(dt, dt);
+            float2 dxs2 = make_float2(0.0f, 0.0f), ddt2 = make_float2(0.0f, 0.0f);
 #pragma unroll
-            for (int n = 0; n < kNState; ++n) {
-                vals[n] = act * g[n] * dtx;
-                dxs = fmaf(g[n], Bv[n], dxs);
-                const float ah = a[n] * hp[n];
-                ddt = fmaf(g[n], fmaf(cc.An[n], ah, Bv[n] * s.x), ddt);
-                dA[n] = fmaf(g[n] * s.dt, ah, dA[n]);
-                G[n] = a[n] * g[n];
+            for (int j = 0; j < 8; ++j) {
+                vals[j] = __fmul2_rn(g[j], dtx2);
+                dxs2 = __ffma2_rn(g[j], B2[j], dxs2);
+                const float2 ah = __fmul2_rn(a[j], hp[j]);
+                ddt2 = __ffma2_rn(g[j], __ffma2_rn(cc.An2[j], ah, __fmul2_rn(B2[j], x2)), ddt2);
+                dA[j] = __ffma2_rn(__fmul2_rn(g[j], dt2), ah, dA[j]);
+                G[j] = __fmul2_rn(a[j], g[j]);
             }
-            const float dd = ddt * s.sg;
-            dDs = fmaf(dy, s.x, dDs);
+            const float dd = (ddt2.x + ddt2.y) * sg;
+            dDs = fmaf(dy, x, dDs);
             dbs += dd;
-            sm.io[0][k][lane] = fmaf(cc.Dd, dy, s.dt * dxs);  // dx
-            sm.io[1][k][lane] = dd;                            // ddelta
-            sm.io[2][k][lane] = dzv;                           // dz
+            sm.io[0][k][lane] = fmaf(cc.Dd, dy, dt * (dxs2.x + dxs2.y));  // dx
+            sm.io[1][k][lane] = dd;                                     // ddelta
+            sm.io[2][k][lane] = dzv;                                    // dz
             sm.io[3][k][lane] = warp_transpose_sum32(vals, lane);
         }
         __syncwarp();
@@ -444,9 +476,8 @@ __global__ void __launch_bounds__(32) scan_bwd_kernel(const BwdParams p) {
         if (L % 4 == 0 && t0 + kBwdSub <= L) {
 #pragma unroll
             for (int q = 0; q < kBwdSub / 4; ++q)
-                atomicAdd(reinterpret_cast<float4 *>(dst) + q,
-                          make_float4(sm.io[3][4 * q][lane], sm.io[3][4 * q + 1][lane], sm.io[3][4 * q + 2][lane],
-                                      sm.io[3][4 * q + 3][lane]));
+                red_add_v4(dst + 4 * q, sm.io[3][4 * q][lane], sm.io[3][4 * q + 1][lane], sm.io[3][4 * q + 2][lane],
+                           sm.io[3][4 * q + 3][lane]);
         } else {
             for (int k = 0; k < kBwdSub; ++k)
                 if (t0 + k < L) atomicAdd(dst + k, sm.io[3][k][lane]);
@@ -455,39 +486,47 @@ __global__ void __launch_bounds__(32) scan_bwd_kernel(const BwdParams p) {
 
     for (int64_t s = segs - 1; s >= 0; --s) {
         const int64_t ts = s * kBwdSeg;
-        float hck[kNState], h[kNState];
+        float2 hck[8], h[8];
         {
             const float4 *src = reinterpret_cast<const float4 *>(p.ckpt + (chan * segs + s) * kNState);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const float4 v = src[q];
-                hck[4 * q] = v.x; hck[4 * q + 1] = v.y; hck[4 * q + 2] = v.z; hck[4 * q + 3] = v.w;
+                hck[2 * q] = make_float2(v.x, v.y);
+                hck[2 * q + 1] = make_float2(v.z, v.w);
             }
         }
-        if (ts + kBwdSub < L) {
-            // the segment's second sub-chunk: its start state from the first, then back through it
+        // passes over the segment: with a second sub-chunk, (0) the first one forward
+        // only, for the second one's start state, (1) the second one forward and back;
+        // then (2) the first one forward from the checkpoint and back.  One call site
+        // each keeps the kernel's code small.
+        const bool two = ts + kBwdSub < L;
+#pragma unroll 1
+        for (int q = two ? 0 : 2; q < 3; ++q) {
+            if (q != 1) {
 #pragma unroll
-            for (int n = 0; n < kNState; ++n) h[n] = hck[n];
-            stage(ts, false);
-            forward(ts, h, false);
-            stage(ts + kBwdSub, true);
-            forward(ts + kBwdSub, h, true);
-            backward(ts + kBwdSub);
+                for (int j = 0; j < 8; ++j) h[j] = hck[j];
+            }
+            const int64_t t0 = q == 1 ? ts + kBwdSub : ts;
+            stage(t0, q != 0);
+            forward(t0, h, q != 0);
+            if (q != 0) backward(t0);
         }
-#pragma unroll
-        for (int n = 0; n < kNState; ++n) h[n] = hck[n];
-        stage(ts, true);
-        forward(ts, h, true);
-        backward(ts);
     }
     // dh0 = Abar_0 g_0, the adjoint carried out of the first step; sums over time
     if (active) {
         if (p.dh0) {
 #pragma unroll
-            for (int n = 0; n < kNState; ++n) p.dh0[chan * kNState + n] = G[n];
+            for (int j = 0; j < 8; ++j) {
+                p.dh0[chan * kNState + 2 * j] = G[j].x;
+                p.dh0[chan * kNState + 2 * j + 1] = G[j].y;
+            }
         }
 #pragma unroll
-        for (int n = 0; n < kNState; ++n) atomicAdd(p.dA + dc * kNState + n, dA[n]);
+        for (int j = 0; j < 8; ++j) {
+            atomicAdd(p.dA + dc * kNState + 2 * j, dA[j].x);
+            atomicAdd(p.dA + dc * kNState + 2 * j + 1, dA[j].y);
+        }
         if (p.dD) atomicAdd(p.dD + dc, dDs);
         if (p.dbias) atomicAdd(p.dbias + dc, dbs);
     }

@@ -439,7 +439,7 @@ int launch_bwd(BwdParams p, cudaStream_t s) {
         return SSM_ERR_CUDA;
     const int64_t groups = bwd_groups(p.batch, p.dim);
     scan_bwd_ckpt_kernel<T><<<static_cast<unsigned>((groups + 3) / 4), 128, 0, s>>>(p);
-    scan_bwd_kernel<T><<<static_cast<unsigned>(groups), 32, smem, s>>>(p);
+    scan_bwd_kernel<T><<<static_cast<unsigned>(bwd_groups16(p.batch, p.dim)), 32, smem, s>>>(p);
     return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
@@ -579,7 +579,7 @@ int ssm_scan_bwd(const void *x, const void *delta, const float *delta_bias, int 
     if (!dims_ok(batch, L, dim) || N < 1) return SSM_ERR_INVALID_ARG;
     if (N != kNState) return SSM_ERR_UNSUPPORTED;
     if (dims->act_dtype != SSM_F32 && dims->act_dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
-    if (bwd_groups(batch, dim) > INT32_MAX) return SSM_ERR_UNSUPPORTED;  // grid.x holds the groups
+    if (bwd_groups16(batch, dim) > INT32_MAX) return SSM_ERR_UNSUPPORTED;  // grid.x holds the groups
     const size_t es = dims->act_dtype == SSM_F32 ? 4 : 2;
     for (const void *ptr : {x, delta, (const void *)A, B, C, z, (const void *)h0, dout, (const void *)dx,
                             (const void *)ddelta, (const void *)(z ? dz : nullptr), (const void *)dB,

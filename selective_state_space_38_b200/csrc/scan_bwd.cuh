@@ -12,14 +12,16 @@
 // backwards through them, carrying the decayed adjoint G = Abar_t g_t from
 // step to step.
 //
-// Work layout: channels across lanes, as in the forward scan.  A warp owns 32
-// consecutive channels of one sequence (lane = channel) and runs every step of
-// them in order, so each recurrence is one sequential chain per lane with its
-// 16 states in registers.  The sums over channels (dB, dC) are reduced across
-// the warp's lanes with a transpose-reduce of warp shuffles (after it, lane k
-// holds the warp's sum of value k) and added to the outputs with float
-// atomics, four steps per atomic.  Sums over time (dA, dD, dbias) stay in the
-// lane's registers until the end and are added with float atomics.
+// Work layout: channels across lanes, as in the forward scan, with a channel's
+// 16 states split over a pair of lanes.  A warp owns 16 consecutive channels of
+// one sequence; lane 2c + hf runs channel c's states 8 hf .. 8 hf + 7 through
+// every step in order, so each recurrence is a sequential chain in registers.
+// The sums over a channel's states (y, dx, ddelta) take one shuffle with the
+// other lane of the pair.  The sums over channels (dB, dC) are reduced across
+// the warp's lanes with a transpose-reduce of warp shuffles and added to the
+// outputs with vector float reductions, four steps each.  Sums over time (dA,
+// dD, dbias) stay in the lane's registers until the end and are added with
+// float atomics.
 #pragma once
 
 #include "common.cuh"
@@ -41,31 +43,10 @@ struct BwdParams {
 };
 
 __host__ __device__ inline int64_t bwd_segments(int64_t L) { return (L + kBwdSeg - 1) / kBwdSeg; }
-__host__ __device__ inline int64_t bwd_groups(int64_t batch, int64_t dim) { return batch * ((dim + 31) / 32); }
 
 template <typename T>
 __device__ __forceinline__ float bwd_softplus(float v) {
     return Act<T>::kBytes == 4 ? softplus_accurate(v) : softplus_fast(v);
-}
-
-// exp(A[d, n] dt) for the 16 states, as pairs (states 2j, 2j + 1).  all_s4d
-// (warp-uniform): every lane's row has the S4D-real structure
-// A[d, n] = (n + 1) A[d, 0], and the decays are the powers of r = exp(A[d, 0] dt)
-// (one MUFU op and a multiplication tree); otherwise sixteen MUFU ops.
-__device__ __forceinline__ void bwd_decay(const float (&a2)[kNState], bool all_s4d, float dt, float2 (&out)[8]) {
-    if (all_s4d) {
-        const float r = ex2_approx(a2[0] * dt);
-        const float r2 = r * r, r4 = r2 * r2, r8 = r4 * r4;
-        out[0] = make_float2(r, r2);
-        out[1] = __fmul2_rn(out[0], make_float2(r2, r2));  // r^3, r^4
-        out[2] = __fmul2_rn(out[0], make_float2(r4, r4));  // r^5, r^6
-        out[3] = __fmul2_rn(out[1], make_float2(r4, r4));  // r^7, r^8
-#pragma unroll
-        for (int j = 4; j < 8; ++j) out[j] = __fmul2_rn(out[j - 4], make_float2(r8, r8));
-    } else {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) out[j] = make_float2(ex2_approx(a2[2 * j] * dt), ex2_approx(a2[2 * j + 1] * dt));
-    }
 }
 
 // Whether A[d, :] has the S4D-real structure A[d, n] = (n + 1) A[d, 0] exactly.
@@ -123,51 +104,6 @@ __device__ __forceinline__ void bwd_store16(void *base, int64_t row_off, int64_t
 }
 
 
-// Warp transpose-reduce: every lane holds 32 values (16 pairs); afterwards lane
-// k holds the sum over the warp's lanes of value k.  Five butterfly levels; at
-// the level of mask m a lane keeps the half of its values selected by
-// (lane & m) and receives the partner's copy of that half.
-__device__ __forceinline__ float warp_transpose_sum32(const float2 (&v)[16], int lane) {
-    float2 w8[8], w4[4], w2[2];
-    float2 w1;
-    {
-        const bool up = lane & 16;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float2 send = up ? v[i] : v[i + 8], keep = up ? v[i + 8] : v[i];
-            w8[i] = __fadd2_rn(keep, make_float2(__shfl_xor_sync(0xffffffffu, send.x, 16),
-                                                 __shfl_xor_sync(0xffffffffu, send.y, 16)));
-        }
-    }
-    {
-        const bool up = lane & 8;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float2 send = up ? w8[i] : w8[i + 4], keep = up ? w8[i + 4] : w8[i];
-            w4[i] = __fadd2_rn(keep, make_float2(__shfl_xor_sync(0xffffffffu, send.x, 8),
-                                                 __shfl_xor_sync(0xffffffffu, send.y, 8)));
-        }
-    }
-    {
-        const bool up = lane & 4;
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const float2 send = up ? w4[i] : w4[i + 2], keep = up ? w4[i + 2] : w4[i];
-            w2[i] = __fadd2_rn(keep, make_float2(__shfl_xor_sync(0xffffffffu, send.x, 4),
-                                                 __shfl_xor_sync(0xffffffffu, send.y, 4)));
-        }
-    }
-    {
-        const bool up = lane & 2;
-        const float2 send = up ? w2[0] : w2[1], keep = up ? w2[1] : w2[0];
-        w1 = __fadd2_rn(keep, make_float2(__shfl_xor_sync(0xffffffffu, send.x, 2),
-                                          __shfl_xor_sync(0xffffffffu, send.y, 2)));
-    }
-    const bool up = lane & 1;
-    const float send = up ? w1.x : w1.y, keep = up ? w1.y : w1.x;
-    return keep + __shfl_xor_sync(0xffffffffu, send, 1);
-}
-
 // B (n < 16) and C (16 <= n < 32) of a sub-chunk's steps, widened: row k holds
 // the 32 values of step t0 + k (zero past L).  Lane j loads row j of B or C.
 template <typename T>
@@ -181,26 +117,6 @@ __device__ __forceinline__ void bwd_put_bc(float *bc, int lane, const float (&v)
     for (int k = 0; k < kBwdSub; ++k) bc[k * 32 + lane] = v[k];
 }
 
-// B and C of step k from the staged rows (warp-uniform 16-byte reads), as pairs
-__device__ __forceinline__ void bwd_b_row(const float *bc, int k, float2 (&B2)[8]) {
-    const float4 *r = reinterpret_cast<const float4 *>(bc + k * 32);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const float4 b = r[q];
-        B2[2 * q] = make_float2(b.x, b.y);
-        B2[2 * q + 1] = make_float2(b.z, b.w);
-    }
-}
-__device__ __forceinline__ void bwd_c_row(const float *bc, int k, float2 (&C2)[8]) {
-    const float4 *r = reinterpret_cast<const float4 *>(bc + k * 32 + kNState);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const float4 c = r[q];
-        C2[2 * q] = make_float2(c.x, c.y);
-        C2[2 * q + 1] = make_float2(c.z, c.w);
-    }
-}
-
 // Four consecutive floats added to global memory without a returned value
 // (the address 16-byte aligned).
 __device__ __forceinline__ void red_add_v4(float *p, float a, float b, float c, float d) {
@@ -208,109 +124,22 @@ __device__ __forceinline__ void red_add_v4(float *p, float a, float b, float c, 
                  : "memory");
 }
 
-// Per-lane constants of a channel: A row (A log2 e for the decays, A as pairs),
-// S4D structure of the whole warp, bias, D.
-struct BwdChan {
-    float a2[kNState];
-    float2 An2[8];
-    bool all_s4d;
-    float bias, Dd;
-};
-__device__ __forceinline__ BwdChan bwd_chan(const BwdParams &p, int64_t dc) {
-    BwdChan c;
-    float An[kNState];
-    const float4 *ar = reinterpret_cast<const float4 *>(p.A + dc * kNState);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const float4 v = __ldg(ar + q);
-        An[4 * q] = v.x; An[4 * q + 1] = v.y; An[4 * q + 2] = v.z; An[4 * q + 3] = v.w;
-    }
-#pragma unroll
-    for (int n = 0; n < kNState; ++n) c.a2[n] = An[n] * kLog2e;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) c.An2[j] = make_float2(An[2 * j], An[2 * j + 1]);
-    c.all_s4d = __all_sync(0xffffffffu, bwd_row_is_s4d(An));
-    c.bias = p.delta_bias ? p.delta_bias[dc] : 0.0f;
-    c.Dd = p.D ? p.D[dc] : 0.0f;
-    return c;
-}
-
-// One step of the forward recurrence: h = exp(A dt) h + dt x B (pairs of states).
-__device__ __forceinline__ void bwd_fwd_step(float2 (&h)[8], const BwdChan &cc, float dt, float x, const float *bc,
-                                             int k) {
-    float2 a[8], B2[8];
-    bwd_decay(cc.a2, cc.all_s4d, dt, a);
-    bwd_b_row(bc, k, B2);
-    const float u = dt * x;
-    const float2 u2 = make_float2(u, u);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) h[j] = __ffma2_rn(a[j], h[j], __fmul2_rn(u2, B2[j]));
-}
-
-// ---- checkpoints: the state at the start of every segment -------------------------
-// One warp per group of 32 channels of one sequence (four groups per CTA, each
-// on its own); the forward recurrence over the whole sequence, with the state
-// written at every segment start.  The next sub-chunk's inputs are loaded
-// while the current one is computed.
+// Sixteen consecutive activations as raw 16-byte pieces (the row offset 16-byte
+// aligned), and element k of them widened.
 template <typename T>
-__global__ void __launch_bounds__(128) scan_bwd_ckpt_kernel(const BwdParams p) {
-    __shared__ __align__(16) float bc_all[4][kBwdSub * 32];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t grp = static_cast<int64_t>(blockIdx.x) * 4 + warp;
-    if (grp >= bwd_groups(p.batch, p.dim)) return;  // warp-uniform
-    const int64_t tiles = (p.dim + 31) / 32;
-    const int64_t b = grp / tiles, d = (grp % tiles) * 32 + lane;
-    const bool active = d < p.dim;
-    const int64_t dc = active ? d : p.dim - 1;
-    const int64_t chan = b * p.dim + dc, L = p.seqlen, segs = bwd_segments(L);
-    const bool vec = (L * Act<T>::kBytes) % 16 == 0;
-    const BwdChan cc = bwd_chan(p, dc);
-    float *bc = bc_all[warp];
-    float2 h[8];
-    if (p.h0) {
-        const float4 *src = reinterpret_cast<const float4 *>(p.h0 + chan * kNState);
+struct Raw16 {
+    uint4 q[kBwdSub / Act<T>::kPerPiece];
+};
+template <typename T>
+__device__ __forceinline__ void raw_load16(const void *base, int64_t off, Raw16<T> &r) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(base) + off * Act<T>::kBytes);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float4 v = __ldg(src + q);
-            h[2 * q] = make_float2(v.x, v.y);
-            h[2 * q + 1] = make_float2(v.z, v.w);
-        }
-    } else {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) h[j] = make_float2(0.0f, 0.0f);
-    }
-    float xv[kBwdSub], dv[kBwdSub], bv[kBwdSub];
-    bwd_load16<T>(p.x, chan * L, 0, L, vec, xv);
-    bwd_load16<T>(p.delta, chan * L, 0, L, vec, dv);
-    bwd_load_bc<T>(p, b, 0, vec, lane, bv);
-    for (int64_t t0 = 0; t0 < L; t0 += kBwdSub) {
-        if (t0 % kBwdSeg == 0 && active) {
-            float4 *dst = reinterpret_cast<float4 *>(p.ckpt + (chan * segs + t0 / kBwdSeg) * kNState);
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                dst[q] = make_float4(h[2 * q].x, h[2 * q].y, h[2 * q + 1].x, h[2 * q + 1].y);
-        }
-        __syncwarp();  // the previous sub-chunk's reads of bc are done
-        bwd_put_bc(bc, lane, bv);
-        __syncwarp();
-        float xn[kBwdSub], dn[kBwdSub];
-        if (t0 + kBwdSub < L) {  // the next sub-chunk's inputs, in flight during this one
-            bwd_load16<T>(p.x, chan * L, t0 + kBwdSub, L, vec, xn);
-            bwd_load16<T>(p.delta, chan * L, t0 + kBwdSub, L, vec, dn);
-            bwd_load_bc<T>(p, b, t0 + kBwdSub, vec, lane, bv);
-        }
-#pragma unroll
-        for (int k = 0; k < kBwdSub; ++k) {
-            if (t0 + k >= L) break;  // warp-uniform
-            const float v = dv[k] + cc.bias;
-            const float dt = p.softplus ? bwd_softplus<T>(v) : v;
-            bwd_fwd_step(h, cc, dt, xv[k], bc, k);
-        }
-#pragma unroll
-        for (int k = 0; k < kBwdSub; ++k) xv[k] = xn[k], dv[k] = dn[k];
-    }
+    for (int i = 0; i < kBwdSub / Act<T>::kPerPiece; ++i) r.q[i] = __ldg(src + i);
 }
-
+template <typename T>
+__device__ __forceinline__ float raw_get(const Raw16<T> &r, int k) {
+    return Act<T>::piece(r.q[k / Act<T>::kPerPiece], k % Act<T>::kPerPiece);
+}
 
 // ---- the backward pass: 16 channels per warp, two lanes per channel --------------
 // Lane 2c + hf owns channel c of the warp's group and the states
@@ -635,6 +464,93 @@ __global__ void __launch_bounds__(32) scan_bwd_kernel(const BwdParams p) {
         if (!hf) {
             if (p.dD) atomicAdd(p.dD + dc, dDs);
             if (p.dbias) atomicAdd(p.dbias + dc, dbs);
+        }
+    }
+}
+
+// ---- checkpoints: the state at the start of every segment -------------------------
+// One warp per group of 16 channels of one sequence (two lanes per channel, as in
+// the backward kernel; four warps per CTA, each on its own): the forward
+// recurrence over the whole sequence, with the state written at every segment
+// start.  Each lane loads one row per sub-chunk (lane (c, 0) channel c's x,
+// lane (c, 1) its delta, lane j row j of B|C), two sub-chunks ahead.
+template <typename T>
+__global__ void __launch_bounds__(128) scan_bwd_ckpt_kernel(const BwdParams p) {
+    struct Warp {
+        float bc[kBwdSub * 32];
+        float io[2][kBwdSub][kBwdCh];
+    };
+    __shared__ __align__(16) Warp wsm[4];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, c = lane >> 1, hf = lane & 1;
+    const int64_t grp = static_cast<int64_t>(blockIdx.x) * 4 + warp;
+    if (grp >= bwd_groups16(p.batch, p.dim)) return;  // warp-uniform
+    const int64_t tiles = (p.dim + kBwdCh - 1) / kBwdCh;
+    const int64_t b = grp / tiles, d = (grp % tiles) * kBwdCh + c;
+    const bool active = d < p.dim;
+    const int64_t dc = active ? d : p.dim - 1;
+    const int64_t chan = b * p.dim + dc, L = p.seqlen, segs = bwd_segments(L), row = chan * L;
+    const bool vec = (L * Act<T>::kBytes) % 16 == 0;
+    const BwdHalf cc = bwd_half(p, dc, hf);
+    const int n0 = 8 * hf;
+    Warp &w = wsm[warp];
+    const void *mine = hf ? p.delta : p.x;
+    const void *bsrc = lane < kNState ? p.B : p.C;
+    const int64_t brow = (b * kNState + (lane & (kNState - 1))) * L;
+    float2 h[4];
+    if (p.h0) {
+        const float4 *src = reinterpret_cast<const float4 *>(p.h0 + chan * kNState + n0);
+        const float4 u = __ldg(src), v = __ldg(src + 1);
+        h[0] = make_float2(u.x, u.y); h[1] = make_float2(u.z, u.w);
+        h[2] = make_float2(v.x, v.y); h[3] = make_float2(v.z, v.w);
+    } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) h[j] = make_float2(0.0f, 0.0f);
+    }
+    // raw rows of the next two sub-chunks (aligned rows, whole sub-chunks only)
+    Raw16<T> r0, r1, q0, q1;
+    const bool raw_ok = vec;
+    auto fetch = [&](int64_t t0, Raw16<T> &rv, Raw16<T> &rb) {
+        if (raw_ok && t0 + kBwdSub <= L) {
+            raw_load16<T>(mine, row + t0, rv);
+            raw_load16<T>(bsrc, brow + t0, rb);
+        }
+    };
+    fetch(0, r0, q0);
+    fetch(kBwdSub, r1, q1);
+    for (int64_t t0 = 0; t0 < L; t0 += kBwdSub) {
+        if (t0 % kBwdSeg == 0 && active) {
+            float4 *dst = reinterpret_cast<float4 *>(p.ckpt + (chan * segs + t0 / kBwdSeg) * kNState + n0);
+            dst[0] = make_float4(h[0].x, h[0].y, h[1].x, h[1].y);
+            dst[1] = make_float4(h[2].x, h[2].y, h[3].x, h[3].y);
+        }
+        float v[kBwdSub], bv[kBwdSub];
+        if (raw_ok && t0 + kBwdSub <= L) {
+#pragma unroll
+            for (int k = 0; k < kBwdSub; ++k) v[k] = raw_get(r0, k), bv[k] = raw_get(q0, k);
+        } else {
+            bwd_load16<T>(mine, row, t0, L, vec, v);
+            bwd_load16<T>(bsrc, brow, t0, L, vec, bv);
+        }
+        r0 = r1;
+        q0 = q1;
+        fetch(t0 + 2 * kBwdSub, r1, q1);  // two sub-chunks ahead, in flight during this one
+        __syncwarp();  // the previous sub-chunk's reads are done
+#pragma unroll
+        for (int k = 0; k < kBwdSub; ++k) w.io[hf][k][c] = v[k];
+        bwd_put_bc(w.bc, lane, bv);
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < kBwdSub; ++k) {
+            if (t0 + k >= L) break;  // warp-uniform
+            const float vv = w.io[1][k][c] + cc.bias;
+            const float dt = p.softplus ? bwd_softplus<T>(vv) : vv;
+            const float u = dt * w.io[0][k][c];
+            float2 a[4], B2[4];
+            bwd_decay_half(cc, hf, dt, a);
+            bwd_get8(w.bc + k * 32 + n0, B2);
+            const float2 u2 = make_float2(u, u);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) h[j] = __ffma2_rn(a[j], h[j], __fmul2_rn(u2, B2[j]));
         }
     }
 }

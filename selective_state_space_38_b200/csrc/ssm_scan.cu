@@ -437,9 +437,9 @@ int launch_bwd(BwdParams p, cudaStream_t s) {
     if (p.dD && cudaMemsetAsync(p.dD, 0, static_cast<size_t>(p.dim) * 4, s) != cudaSuccess) return SSM_ERR_CUDA;
     if (p.dbias && cudaMemsetAsync(p.dbias, 0, static_cast<size_t>(p.dim) * 4, s) != cudaSuccess)
         return SSM_ERR_CUDA;
-    const int64_t groups = bwd_groups(p.batch, p.dim);
+    const int64_t groups = bwd_groups16(p.batch, p.dim);
     scan_bwd_ckpt_kernel<T><<<static_cast<unsigned>((groups + 3) / 4), 128, 0, s>>>(p);
-    scan_bwd_kernel<T><<<static_cast<unsigned>(bwd_groups16(p.batch, p.dim)), 32, smem, s>>>(p);
+    scan_bwd_kernel<T><<<static_cast<unsigned>(groups), 32, smem, s>>>(p);
     return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 

@@ -122,8 +122,8 @@ def _pipes(kernel_key):
     rec = _profiled(kernel_key)
     if rec is None:
         return None
-    keys = ("fma_pipe_pct", "xu_pipe_pct", "dram_throughput_pct", "issue_active_pct", "smem_pipe_pct",
-            "smem_bank_conflicts_ld", "smem_bank_conflicts_st")
+    keys = ("fma_pipe_pct", "xu_pipe_pct", "tensor_pipe_pct", "dram_throughput_pct", "issue_active_pct",
+            "smem_pipe_pct", "smem_bank_conflicts_ld", "smem_bank_conflicts_st")
     out = {k: rec[k] for k in keys if k in rec}
     out["source"] = "ncu, profiles/traffic.json"
     return out

@@ -108,9 +108,10 @@ struct FwdSmem {
     static constexpr int kBCFOff = kStages * kStageBytes;
     static constexpr int kUROff = kBCFOff + 2 * kBCFBytes;
     static constexpr int kGOff = kUROff + 2 * kURBytes;
-    static constexpr int kDescOff = kGOff + 2 * kGBytes;            // ring of 4 chunk descriptors
-    static constexpr int kBarOff = kDescOff + 4 * 64;               // ready[2], done[2], posted[2], full[kStages]
-    static constexpr int kPairBytes = (kBarOff + (6 + kStages) * 8 + 1023) / 1024 * 1024;
+    static constexpr int kDescOff = kGOff + 2 * kGBytes;            // ring of 8 chunk descriptors
+    static constexpr int kBarOff = kDescOff + 8 * 64;               // ready[2], done[4], posted[2], full[kStages],
+                                                                    // dready[4], then the load count
+    static constexpr int kPairBytes = (kBarOff + (12 + kStages) * 8 + 8 + 1023) / 1024 * 1024;
     static constexpr int kTotal = kPairs * kPairBytes + 1024;       // + slack to align the base to 1 KB
 };
 static_assert(FwdSmem<bf16raw, true>::kTotal <= 227 * 1024, "shared memory of the trapezoidal kernel");
@@ -118,6 +119,21 @@ static_assert(FwdSmem<bf16raw, false, true>::kTotal <= 227 * 1024, "shared memor
 static_assert(FwdSmem<bf16raw, false>::kTotal <= 227 * 1024, "shared memory of the kernel");
 
 __device__ __forceinline__ int swz(int row, int pc) { return pc ^ ((row >> 1) & 3); }
+
+// Row t (32 floats, one per channel of the group) of a chunk's y.  With
+// YS (three stages, loads issued by the post warp) y goes to the chunk's stage,
+// over the delta tile (steps 0..15) and the raw B|C rows (steps 16..31), which
+// the prep warp has consumed; the (u, r) table is then free once the scan is
+// done with it.  Otherwise y goes over the (u, r) table's row t (lanes 0..15's
+// pairs, already consumed), as the prep warp waits for the post warp anyway.
+template <bool YS>
+__device__ __forceinline__ float *y_row(uint8_t *stage, const float2 *ur, int t) {
+    constexpr int TB = 32 * kRowBytes;
+    if constexpr (YS)
+        return reinterpret_cast<float *>(stage + (t < 16 ? TB + t * 128 : 3 * TB + (t - 16) * 128));
+    else
+        return const_cast<float *>(reinterpret_cast<const float *>(ur + t * 32));
+}
 
 // ---- staging one chunk [t0, t0 + TC) of a warp's 32 channels element by element
 // (rows that are not 16-byte aligned, L * size % 16 != 0, cannot use TMA)
@@ -422,8 +438,8 @@ __device__ __forceinline__ void prepare_step(const float *bcf, const float2 *ur,
 // chunk of a sequence tests the step index.
 // With TRAP the carried state is h~ (see chunk_prepass): h~ = Abar (h~ + s B_{t-1})
 // and y = C . h~ + g (C . B).
-template <bool S4D, bool FULL, bool TRAP = false>
-__device__ __forceinline__ void chunk_core(const float *bcf, float2 *ur, int row, int nvalid,
+template <bool S4D, bool FULL, bool TRAP, bool YS>
+__device__ __forceinline__ void chunk_core(const float *bcf, const float2 *ur, uint8_t *stage, int row, int nvalid,
                                            const float (&a2)[kNState], float2 (&h)[8],
                                            const float *garr = nullptr) {
     StepOps nxt;
@@ -447,7 +463,7 @@ __device__ __forceinline__ void chunk_core(const float *bcf, float2 *ur, int row
                 else ya = __ffma2_rn(cur.c[j], h[j], ya);
             }
             const float2 ys = __fadd2_rn(ya, yb);
-            reinterpret_cast<float *>(ur + t * 32)[row] = ys.x + ys.y;  // dense: one wavefront
+            y_row<YS>(stage, ur, t)[row] = ys.x + ys.y;  // dense: one wavefront
         }
     }
 }
@@ -484,9 +500,9 @@ __device__ __forceinline__ void chunk_summary(const float *bcf, const float2 *ur
 // ---- phase 3: D skip, gate, output -----------------------------------------------
 // out_t = (y_t + D x_t) silu(z_t), written over the lane's own x row of the
 // stage (already consumed); stage by stage over step pairs as in phase 1.
-// y_t is float `lane` of row t of ur.
+// y_t is float `lane` of row t of the chunk's y (y_row).
 // With CONV the skip term comes from the g table (D xc, float32) instead of D x.
-template <typename T, bool CONV = false>
+template <typename T, bool CONV, bool YS>
 __device__ __forceinline__ void chunk_postpass(uint8_t *stage, const float2 *ur, int row,
                                                const ChanConst &cc, bool has_z, const float *garr = nullptr) {
     using AT = Act<T>;
@@ -505,8 +521,7 @@ __device__ __forceinline__ void chunk_postpass(uint8_t *stage, const float2 *ur,
 #pragma unroll
     for (int k = 0; k < NP; ++k) {
         const int pc = (2 * k) / PP, i = (2 * k) % PP;
-        const float2 Y = make_float2(reinterpret_cast<const float *>(ur + (2 * k) * 32)[row],
-                                     reinterpret_cast<const float *>(ur + (2 * k + 1) * 32)[row]);
+        const float2 Y = make_float2(y_row<YS>(stage, ur, 2 * k)[row], y_row<YS>(stage, ur, 2 * k + 1)[row]);
         if constexpr (CONV)
             O[k] = __fadd2_rn(Y, make_float2(garr[(2 * k) * 32 + row], garr[(2 * k + 1) * 32 + row]));
         else
@@ -636,6 +651,8 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar))
                  : "memory");
 }
+// one arrival by one thread (a barrier initialised with count 1)
+__device__ __forceinline__ void mbar_arrive1(uint64_t *bar) { mbar_arrive(bar); }
 // Wait for the completion of the phase with the given parity.  Returns false
 // when the wait gives up: after kBarLimit polls (the error word gets bit 1), or
 // early, once another wait of the launch has given up (the error word is
@@ -803,9 +820,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const int role = warp / kPairs;  // 0 scan, 1 prep, 2 post
     uint8_t *ps = smem + pair * SM::kPairBytes;
     uint64_t *ready = reinterpret_cast<uint64_t *>(ps + SM::kBarOff);
+    // done[4]: the scan warp may finish up to kStages chunks ahead of the post warp
+    // (the post warp issues the loads), so the barrier of chunk j is not reused
+    // before the post warp has waited on it
     uint64_t *done = ready + 2;
-    uint64_t *posted = ready + 4;
-    uint64_t *full = ready + 6;  // [kStages]: TMA bytes of a staged chunk have landed
+    uint64_t *posted = ready + 6;
+    uint64_t *full = ready + 8;  // [kStages]: TMA bytes of a staged chunk have landed
     ChunkDesc *ring = reinterpret_cast<ChunkDesc *>(ps + SM::kDescOff);
     auto stage_of = [&](int64_t j) { return ps + (j % kStages) * SM::kStageBytes; };
     auto bcf_of = [&](int64_t j) { return reinterpret_cast<float *>(ps + SM::kBCFOff + (j & 1) * SM::kBCFBytes); };
@@ -813,68 +833,101 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     auto g_of = [&](int64_t j) { return reinterpret_cast<float *>(ps + SM::kGOff + (j & 1) * SM::kGBytes); };
     auto parity = [](int64_t j, int n) { return static_cast<uint32_t>((j / n) & 1); };
 
+    uint64_t *dready = full + kStages;  // [4]: the descriptor of chunk j + kStages is in the ring
+    uint32_t *load_count = reinterpret_cast<uint32_t *>(dready + 4);  // loads the post warp issued, plus one
     if (threadIdx.x < kPairs) {
         uint64_t *r = reinterpret_cast<uint64_t *>(smem + threadIdx.x * SM::kPairBytes + SM::kBarOff);
-        for (int i = 0; i < 6; ++i) mbar_init(r + i, 32);
-        for (int i = 0; i < kStages; ++i) mbar_init(r + 6 + i, 1);
+        for (int i = 0; i < 8; ++i) mbar_init(r + i, 32);
+        for (int i = 0; i < kStages + 4; ++i) mbar_init(r + 8 + i, 1);
+        *reinterpret_cast<uint32_t *>(r + 12 + kStages) = 0;
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     __syncthreads();
     if (!S4D && *reinterpret_cast<volatile uint32_t *>(sc.general) == 0) return;
     uint32_t *counter = sc.counter + 2 * p.pass + (S4D ? 0 : 1);
+    const uint32_t stage_tx = (p.z ? 3u : 2u) * SM::kTileBytes + 2u * kNState * kRowBytes +
+                              (TRAP ? static_cast<uint32_t>(SM::kTileBytes) : 0u);
+    // stage chunk j: TMA (one lane, completion on full[j % kStages]) or element loads
+    auto load_stage = [&](const ChunkDesc &dsc, int64_t j) {
+        if (dsc.flags & kStop) return;
+        uint8_t *st = stage_of(j);
+        if constexpr (VEC) {
+            if (lane == 0) {
+                uint64_t *bar = full + (j % kStages);
+                mbar_arrive_expect_tx(bar, stage_tx);
+                const int t0 = static_cast<int>(dsc.t0), d0 = static_cast<int>(dsc.d0), b = static_cast<int>(dsc.b);
+                tma_load_3d(st, &tm.x, t0, d0, b, bar);
+                tma_load_3d(st + SM::kTileBytes, &tm.delta, t0, d0, b, bar);
+                if (p.z) tma_load_3d(st + 2 * SM::kTileBytes, &tm.z, t0, d0, b, bar);
+                tma_load_3d(st + SM::kBCRawOff, &tm.B, t0, 0, b, bar);
+                tma_load_3d(st + SM::kBCRawOff + kNState * kRowBytes, &tm.C, t0, 0, b, bar);
+                if (TRAP) tma_load_3d(st + SM::kLamOff, &tm.lam, t0, d0, b, bar);
+            }
+        } else {
+            load_chunk_sync<T, TRAP>(p, st, dsc.b, dsc.d0, dsc.t0, lane);
+        }
+    };
+    // Who loads the stages.  Three stages with TMA: the post warp, into the stage
+    // it has just posted (the prep warp keeps preparing).  Two stages: the prep
+    // warp, right after it hands a chunk over (a load issued by the post warp
+    // would land too late for the next chunk); element loads: the prep warp.
+    constexpr bool kPrepLoads = !VEC || kStages == 2;
+    // TMA loads the prep warp waited for and issued (for the drain at the end:
+    // every issued load completes before the CTA exits)
+    int64_t n_waited = 0, n_prep_issued = 0;
 
     if (role == 1) {
         // ------------------------------------------------------------------ prep
+        // Buffer reuse.  Chunk j's u/r, B|C and g tables are chunk j - 2's: chunk j is
+        // prepared once chunk j - 2's scan is done (and, when the prep warp loads the
+        // stages or the convolution's post warp reads the g table, once chunk j - 2
+        // is posted).  When the post warp loads, it loads chunk j + kStages into
+        // chunk j's stage as soon as it has posted chunk j, and the prep warp puts
+        // that chunk's descriptor in the ring kStages chunks ahead.
         ChunkCursor<T, S4D> cur(p);
-        const uint32_t stage_tx = (p.z ? 3u : 2u) * SM::kTileBytes + 2u * kNState * kRowBytes +
-                                  (TRAP ? static_cast<uint32_t>(SM::kTileBytes) : 0u);
-        // TMA loads issued and waited for, in chunk order: every issued load is
-        // waited for before the warp leaves, also when it gives up early
-        int64_t n_issued = 0, n_waited = 0;
-        // stage chunk j: TMA (one lane, completion on full[j % kStages]) or element loads
-        auto issue = [&](const ChunkDesc &dsc, int64_t j) {
-            if (dsc.flags & kStop) return;
-            uint8_t *st = stage_of(j);
-            if constexpr (VEC) {
-                if (lane == 0) {
-                    uint64_t *bar = full + (j % kStages);
-                    mbar_arrive_expect_tx(bar, stage_tx);
-                    const int t0 = static_cast<int>(dsc.t0), d0 = static_cast<int>(dsc.d0), b = static_cast<int>(dsc.b);
-                    tma_load_3d(st, &tm.x, t0, d0, b, bar);
-                    tma_load_3d(st + SM::kTileBytes, &tm.delta, t0, d0, b, bar);
-                    if (p.z) tma_load_3d(st + 2 * SM::kTileBytes, &tm.z, t0, d0, b, bar);
-                    tma_load_3d(st + SM::kBCRawOff, &tm.B, t0, 0, b, bar);
-                    tma_load_3d(st + SM::kBCRawOff + kNState * kRowBytes, &tm.C, t0, 0, b, bar);
-                    if (TRAP) tma_load_3d(st + SM::kLamOff, &tm.lam, t0, d0, b, bar);
-                }
-                n_issued = j + 1;
-            } else {
-                load_chunk_sync<T, TRAP>(p, st, dsc.b, dsc.d0, dsc.t0, lane);
-            }
-        };
         const bool softplus = p.softplus != 0;
         ChanConst cc;
         int64_t cc_d0 = -1;
         float halo[3] = {0.0f, 0.0f, 0.0f};  // convolution inputs before the chunk (CONV)
         float x_last = 0.0f, g_last = 0.0f;  // the step before the chunk (TRAP)
-        // Buffer reuse.  The u/r, B|C and g tables of chunk j are those chunk j - 2
-        // used, and the post warp reads chunk j - 2's outputs from them: chunk j is
-        // prepared once chunk j - 2 is posted.  The stage of chunk j + 1 is the one
-        // chunk j + 1 - kStages used.  With three stages that is chunk j - 2 too, so
-        // its load is issued before chunk j is prepared; with two stages it is chunk
-        // j - 1, whose post ends after chunk j could be prepared, so the load is
-        // issued once chunk j has been handed over (waiting for chunk j - 1 first
-        // would keep the prep warp idle while the scan warp runs chunk j - 1).
-        ChunkDesc dnext = cur.next(p, sc, counter, lane);
-        issue(dnext, 0);
+        bool stopped = false;
+        auto next_desc = [&]() {
+            ChunkDesc d;
+            d.flags = kStop;
+            if (!stopped) {
+                d = cur.next(p, sc, counter, lane);
+                stopped = (d.flags & kStop) != 0;
+            }
+            return d;
+        };
+        const int64_t ahead = kPrepLoads ? 1 : kStages;  // chunks loaded before the loop
+        for (int64_t j = 0; j < ahead; ++j) {
+            const ChunkDesc d = next_desc();
+            if (lane == 0) ring[j & 7] = d;
+            load_stage(d, j);
+            if (!(d.flags & kStop)) n_prep_issued = j + 1;
+        }
+        __syncwarp();
         for (int64_t j = 0;; ++j) {
-            const ChunkDesc dj = dnext;
-            if (j >= 2 && !mbar_wait(posted + (j & 1), parity(j - 2, 2), sc.error)) break;
-            if (!(dj.flags & kStop)) {
-                if (kStages == 3) {
-                    dnext = cur.next(p, sc, counter, lane);
-                    issue(dnext, j + 1);
+            const ChunkDesc dj = ring[j & 7];
+            if (j >= 2) {
+                if (!mbar_wait(done + ((j - 2) & 3), parity(j - 2, 4), sc.error)) break;
+                if ((CONV || kPrepLoads) && !mbar_wait(posted + (j & 1), parity(j - 2, 2), sc.error)) break;
+            }
+            if constexpr (!kPrepLoads) {
+                const ChunkDesc dn = next_desc();
+                if (lane == 0) {
+                    ring[(j + kStages) & 7] = dn;
+                    mbar_arrive1(dready + (j & 3));
                 }
+            } else if (kStages == 3 && !(dj.flags & kStop)) {
+                // the stage of chunk j + 1 is chunk j - 2's, posted above
+                const ChunkDesc dn = next_desc();
+                if (lane == 0) ring[(j + 1) & 7] = dn;
+                load_stage(dn, j + 1);
+                if (!(dn.flags & kStop)) n_prep_issued = j + 2;
+            }
+            if (!(dj.flags & kStop)) {
                 if constexpr (VEC) {
                     if (!mbar_wait(full + (j % kStages), parity(j, kStages), sc.error)) break;
                     n_waited = j + 1;
@@ -901,58 +954,68 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     const int64_t d = dj.d0 + lane;
                     conv_halo<T>(p, dj.b, d < p.dim ? d : p.dim - 1, dj.t0, halo);
                 }
-                chunk_prepass<T, S4D, CONV, TRAP>(st, ur_of(j), lane, cc, softplus, halo, g_of(j), &x_last,
+        chunk_prepass<T, S4D, CONV, TRAP>(st, ur_of(j), lane, cc, softplus, halo, g_of(j), &x_last,
                                                   &g_last);
             }
-            if (lane == 0) ring[j & 3] = dj;
             __syncwarp();
             mbar_arrive(ready + (j & 1));
             if (dj.flags & kStop) break;
-            if (kStages == 2) {
+            if (kPrepLoads && kStages == 2) {
+                // the stage of chunk j + 1 is chunk j - 1's: load once it is posted
                 if (j >= 1 && !mbar_wait(posted + ((j - 1) & 1), parity(j - 1, 2), sc.error)) break;
-                dnext = cur.next(p, sc, counter, lane);
-                issue(dnext, j + 1);
+                const ChunkDesc dn = next_desc();
+                if (lane == 0) ring[(j + 1) & 7] = dn;
+                load_stage(dn, j + 1);
+                if (!(dn.flags & kStop)) n_prep_issued = j + 2;
+                __syncwarp();
             }
         }
-        // loads still in flight after a wait gave up (none on the normal path)
-        for (int64_t j = n_waited; j < n_issued; ++j) mbar_drain(full + (j % kStages), parity(j, kStages), sc.error);
     } else if (role == 2) {
         // ------------------------------------------------------------------ post
         const bool has_z = p.z != nullptr;
         ChanConst cc;
         int64_t cc_d0 = -1;
+        uint32_t issued = 0;  // one past the last chunk this warp loaded
         for (int64_t j = 0;; ++j) {
-            if (!mbar_wait(done + (j & 1), parity(j, 2), sc.error)) break;
-            const ChunkDesc dj = ring[j & 3];
+            if (!mbar_wait(done + (j & 3), parity(j, 4), sc.error)) break;
+            const ChunkDesc dj = ring[j & 7];
             if (dj.flags & kStop) break;
             uint8_t *st = stage_of(j);
-            if (p.mode == kSummary) {  // the summary pass writes no output
-                __syncwarp();
-                mbar_arrive(posted + (j & 1));
-                continue;
-            }
-            if (dj.d0 != cc_d0) {
-                const int64_t d = dj.d0 + lane;
-                cc = chan_const(p, d < p.dim ? d : p.dim - 1);
-                cc_d0 = dj.d0;
-            }
-            chunk_postpass<T, CONV>(st, ur_of(j), lane, cc, has_z, g_of(j));
-            if constexpr (VEC) {
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_3d(&tm.out, static_cast<int>(dj.t0), static_cast<int>(dj.d0), static_cast<int>(dj.b), st);
-                    tma_store_commit();
-                    tma_store_wait_read();  // the stage is handed back for loading right after
+            if (p.mode != kSummary) {  // the summary pass writes no output
+                if (dj.d0 != cc_d0) {
+                    const int64_t d = dj.d0 + lane;
+                    cc = chan_const(p, d < p.dim ? d : p.dim - 1);
+                    cc_d0 = dj.d0;
                 }
-            } else {
-                __syncwarp();
-                store_chunk_sync<T>(p, st, dj.b, dj.d0, dj.t0, lane);
+                chunk_postpass<T, CONV, !kPrepLoads>(st, ur_of(j), lane, cc, has_z, g_of(j));
+                if constexpr (VEC) {
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_3d(&tm.out, static_cast<int>(dj.t0), static_cast<int>(dj.d0), static_cast<int>(dj.b),
+                                     st);
+                        tma_store_commit();
+                        tma_store_wait_read();  // the stage is loaded again right after
+                    }
+                } else {
+                    __syncwarp();
+                    store_chunk_sync<T>(p, st, dj.b, dj.d0, dj.t0, lane);
+                }
+            }
+            if constexpr (!kPrepLoads) {
+                // chunk j's stage is free: load chunk j + kStages into it
+                if (!mbar_wait(dready + (j & 3), parity(j, 4), sc.error)) break;
+                const ChunkDesc dn = ring[(j + kStages) & 7];
+                load_stage(dn, j + kStages);
+                if (!(dn.flags & kStop)) issued = static_cast<uint32_t>(j + kStages + 1);
             }
             __syncwarp();
             mbar_arrive(posted + (j & 1));
         }
-        if (VEC && lane == 0) tma_store_wait_all();
+        if (VEC && lane == 0) {
+            *load_count = issued;
+            tma_store_wait_all();
+        }
     } else {
         // ------------------------------------------------------------------ scan
         const int64_t segs = (p.seqlen + p.seg_steps - 1) / p.seg_steps;
@@ -964,9 +1027,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int n = 0; n < kNState; ++n) a2[n] = 0.0f;
         for (int64_t k = 0;; ++k) {
             if (!mbar_wait(ready + (k & 1), parity(k, 2), sc.error)) break;
-            const ChunkDesc dk = ring[k & 3];
+            const ChunkDesc dk = ring[k & 7];
             if (dk.flags & kStop) {
-                mbar_arrive(done + (k & 1));  // lets the post warp see the end
+                mbar_arrive(done + (k & 3));  // lets the post warp see the end
                 break;
             }
             const int64_t d = dk.d0 + lane;
@@ -1014,9 +1077,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 else
                     chunk_summary<S4D, false, TRAP>(bcf_of(k), ur_of(k), lane, dk.nvalid, a2, h, P);
             } else if (dk.nvalid == TC) {
-                chunk_core<S4D, true, TRAP>(bcf_of(k), ur_of(k), lane, TC, a2, h, g_of(k));
+                chunk_core<S4D, true, TRAP, !kPrepLoads>(bcf_of(k), ur_of(k), stage_of(k), lane, TC, a2, h, g_of(k));
             } else {
-                chunk_core<S4D, false, TRAP>(bcf_of(k), ur_of(k), lane, dk.nvalid, a2, h, g_of(k));
+                chunk_core<S4D, false, TRAP, !kPrepLoads>(bcf_of(k), ur_of(k), stage_of(k), lane, dk.nvalid, a2, h,
+                                                          g_of(k));
             }
             if (dk.flags & kLast) {
                 if (p.mode == kSummary) {
@@ -1056,7 +1120,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 }
             }
             __syncwarp();
-            mbar_arrive(done + (k & 1));
+            mbar_arrive(done + (k & 3));
+        }
+    }
+    // every TMA load still in flight after a wait gave up completes before the CTA
+    // exits (none on the normal path): the prep warp drains, in chunk order, the
+    // loads it has not waited for
+    if constexpr (VEC) {
+        __syncthreads();
+        if (role == 1 && lane == 0) {
+            const int64_t issued = n_prep_issued > static_cast<int64_t>(*load_count) ? n_prep_issued : *load_count;
+            for (int64_t j = n_waited; j < issued; ++j) mbar_drain(full + (j % kStages), parity(j, kStages), sc.error);
         }
     }
 }

@@ -197,8 +197,8 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
     float *Fs = dts + 128;  // F_j = exp(-cs_j) dt_j, when every |cs| of the chunk is at most 80
     float *wsum = Fs + 128;
     uint64_t *lbar = reinterpret_cast<uint64_t *>(sm + S::kBar);  // [2] input buffer landed
-    uint64_t *mbar = lbar + 2;                                    // [0] MMA1/3 done, [1] MMA2/4 done
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(mbar + 2);
+    uint64_t *mbar = lbar + 2;  // [0] MMA1 (G) done, [1] MMA2/4 (Yd, ST) done, [2] MMA3 (Yo) done
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(mbar + 3);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, half = warp >> 2;
     const int row = quad * 32 + lane;
@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
     const int64_t chunks = (L + kSsdQ - 1) / kSsdQ;
 
     if (tid == 0) {
-        for (int i = 0; i < 4; ++i) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(lbar + i)));
+        for (int i = 0; i < 5; ++i) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(lbar + i)));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) {
@@ -260,18 +260,46 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
         }
     };
 
+    // Chunks overlap on the tensor core: chunk c + 1's G = C B^T is issued as soon as
+    // chunk c's MMA2/4 have read L o G out of its TMEM columns, and runs during
+    // chunk c's epilogue 2; chunk c's Yo = C S^T is issued before its epilogue 1,
+    // which does not need it.  Each MMA group commits to its own mbarrier, one
+    // phase per chunk; the counts below let a walk that gives up drain them.
     int64_t loads_issued = 0, loads_waited = 0;
-    uint64_t *mma_pending = nullptr;  // the commit barrier of MMAs not yet seen complete
-    uint32_t mma_parity = 0;
+    uint32_t committed[3] = {0, 0, 0}, waited[3] = {0, 0, 0};
     if (tid == 0) load(0);
     loads_issued = 1;
     float dt_raw = tid < kSsdQ ? load_dt(tid) : 0.0f;
     write_state();
 
     const uint32_t a_s = smem_u32(sm + S::kS), a_xw = smem_u32(sm + S::kXw);
-    bool ok = true;
-    for (int64_t c = 0; c < chunks; ++c) {
+    // a descriptor of base + off is the base's plus off / 16 (no carry: every
+    // shared-memory address is below 2^18)
+    auto issue_g = [&](int64_t c) {  // MMA1: G = C B^T of chunk c
+        uint8_t *in = sm + (c & 1) * S::kInBytes;
+        constexpr uint32_t i1 = ssd_idesc(128, 128, 0, 0);
+        const uint64_t dC = ssd_desc(smem_u32(in + S::kInC), 16, 1024), dB = ssd_desc(smem_u32(in + S::kInB), 16, 1024);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const uint32_t ko = ((k / 4) * S::kTile + (k % 4) * 32) >> 4;
+            ssd_mma(tG, dC + ko, dB + ko, i1, k > 0);
+        }
+        ssd_commit(mbar);
+    };
+    // a bounded wait that every thread takes the same way, and its bookkeeping
+    auto wait_all = [&](uint64_t *bar, uint32_t parity) -> bool {
+        return __syncthreads_and(ssd_wait(bar, parity, p.error)) != 0;
+    };
+    bool ok = wait_all(lbar, 0u);
+    if (ok) {
+        loads_waited = 1;
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        if (tid == 0) issue_g(0);
+        committed[0] = 1;
+    }
+    for (int64_t c = 0; ok && c < chunks; ++c) {
         const int64_t t0 = c * kSsdQ;
+        const uint32_t ph = static_cast<uint32_t>(c & 1);
         uint8_t *in = sm + (c & 1) * S::kInBytes;
         const uint32_t a_c = smem_u32(in + S::kInC), a_b = smem_u32(in + S::kInB), a_x = smem_u32(in + S::kInX);
         // ---- dt and the running sum cs of dt A over the chunk (threads 0..127)
@@ -301,29 +329,16 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
             dts[tid] = dtv;
             Fs[tid] = __expf(-s) * dtv;
         }
-        // exp(cs_i - cs_j) = exp(cs_i) exp(-cs_j) without overflow when every |cs| <= 80
-        const bool factored = __syncthreads_and(tid >= kSsdQ || fabsf(s) <= 80.0f) != 0;
-        // S^T visible to the tensor core, cs to every thread
+        // exp(cs_i - cs_j) = exp(cs_i) exp(-cs_j) without overflow when every |cs| <= 80;
+        // the barrier also makes S^T (written by epilogue 2) visible to the tensor core
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-        if (!__syncthreads_and(ssd_wait(lbar + (c & 1), static_cast<uint32_t>((c >> 1) & 1), p.error))) {
-            ok = false;
-            break;
-        }
-        loads_waited = c + 1;
+        const bool factored = __syncthreads_and(tid >= kSsdQ || fabsf(s) <= 80.0f) != 0;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        // ---- MMA1: G = C B^T; MMA3: Yo = C S^T (high, then low accumulated)
+        // ---- MMA3: Yo = C S^T (high, then low accumulated); epilogue 2 needs it
         if (tid == 0) {
-            // a descriptor of base + off is the base's plus off / 16 (no carry: every
-            // shared-memory address is below 2^18)
-            constexpr uint32_t i1 = ssd_idesc(128, 128, 0, 0), i3 = ssd_idesc(128, 64, 0, 1);
-            const uint64_t dC = ssd_desc(a_c, 16, 1024), dB = ssd_desc(a_b, 16, 1024);
-            const uint64_t dS = ssd_desc(a_s, S::kTile, 1024);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint32_t ko = ((k / 4) * S::kTile + (k % 4) * 32) >> 4;
-                ssd_mma(tG, dC + ko, dB + ko, i1, k > 0);
-            }
+            constexpr uint32_t i3 = ssd_idesc(128, 64, 0, 1);
+            const uint64_t dC = ssd_desc(a_c, 16, 1024), dS = ssd_desc(a_s, S::kTile, 1024);
 #pragma unroll
             for (int part = 0; part < 2; ++part)
 #pragma unroll
@@ -331,13 +346,15 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
                     const uint32_t ka = ((k / 4) * S::kTile + (k % 4) * 32) >> 4;
                     ssd_mma(tYo, dC + ka, dS + ((part * S::kTile + 2048 * k) >> 4), i3, part > 0 || k > 0);
                 }
-            ssd_commit(mbar);
+            ssd_commit(mbar + 2);
         }
-        mma_pending = mbar;
-        if (!__syncthreads_and(ssd_wait(mbar, mma_parity, p.error))) {
+        committed[2] = static_cast<uint32_t>(c + 1);
+        // ---- G of this chunk (issued during the previous chunk's epilogue 2)
+        if (!wait_all(mbar, ph)) {
             ok = false;
             break;
         }
+        waited[0] = static_cast<uint32_t>(c + 1);
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         const float total = cs[kSsdQ - 1];
         float dx[32];  // D x of this thread's row and column half, kept for epilogue 2
@@ -431,14 +448,29 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
                             part > 0 || k > 0);
             ssd_commit(mbar + 1);
         }
-        mma_pending = mbar + 1;
-        if (!__syncthreads_and(ssd_wait(mbar + 1, mma_parity, p.error))) {
+        committed[1] = static_cast<uint32_t>(c + 1);
+        if (!wait_all(mbar + 1, ph)) {
             ok = false;
             break;
         }
-        mma_pending = nullptr;
-        mma_parity ^= 1u;
+        waited[1] = static_cast<uint32_t>(c + 1);
+        if (!wait_all(mbar + 2, ph)) {
+            ok = false;
+            break;
+        }
+        waited[2] = static_cast<uint32_t>(c + 1);
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        // ---- the next chunk's G: its inputs have landed and G's columns are read
+        if (c + 1 < chunks) {
+            if (!wait_all(lbar + ((c + 1) & 1), static_cast<uint32_t>(((c + 1) >> 1) & 1))) {
+                ok = false;
+                break;
+            }
+            loads_waited = c + 2;
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            if (tid == 0) issue_g(c + 1);
+            committed[0] = static_cast<uint32_t>(c + 2);
+        }
         // ---- epilogue 2: y row i, p in [32 half, 32 half + 32); state row n, same p
         {
             const int i = row;
@@ -475,7 +507,8 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
     }
     // a wait that gave up leaves no load or MMA running when the CTA ends
     if (!ok && tid == 0) {
-        if (mma_pending) ssd_drain(mma_pending, mma_parity, p.error);
+        for (int g = 0; g < 3; ++g)
+            for (uint32_t n = waited[g]; n < committed[g]; ++n) ssd_drain(mbar + g, n & 1u, p.error);
         for (int64_t c = loads_waited; c < loads_issued; ++c)
             ssd_drain(lbar + (c & 1), static_cast<uint32_t>((c >> 1) & 1), p.error);
     }

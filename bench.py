@@ -625,6 +625,9 @@ def run_gpu(args):
     if rank == 0:
         cpu_val, cpu_s, cpu_ch, cores = cpu_oracle_rate(FWD_CFG, target_s=float(
             os.environ.get("SSM_CPU_BASELINE_S", "10")))
+        # the oracle on one thread, on the Mamba-130M layer shape (a bounded channel sample)
+        one_val, one_s, one_ch, _ = cpu_oracle_rate(1, target_s=float(os.environ.get("SSM_CPU_ONE_S", "3")),
+                                                    threads=1)
         tok_ch = c.batch * c.seqlen * c.dim
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
@@ -633,6 +636,7 @@ def run_gpu(args):
             "data": "synthetic",
             "config": fwd_config(world),
             "pct_of_hbm_peak": round(100.0 * value / world / hbm_peak, 2),
+            "pct_of_hbm_spec_8tbs": round(100.0 * value / world / 8000.0, 2),
             "gtok_ch_per_s": round(world * tok_ch / (ms_step * 1e-3) / 1e9, 2),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": hbm_peak,
                          "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
@@ -648,7 +652,10 @@ def run_gpu(args):
             "cpu_baseline": {"value": round(cpu_val, 4), "unit": "GB/s", "cores": cores,
                              "kind": "oracle", "cpu": _cpu_model(),
                              "sample": f"{cpu_ch} channels (full L) of the same workload, "
-                                       f"{cpu_s:.1f} s of float64 oracle time"},
+                                       f"{cpu_s:.1f} s of float64 oracle time",
+                             "single_thread": {"value": round(one_val, 4), "unit": "GB/s", "cores": 1,
+                                               "workload": workloads.CONFIGS[1].name,
+                                               "sample": f"{one_ch} channels (full L), {one_s:.1f} s"}},
             "other_configs": subs,
             "next_rows": nxt,
             "decode": {"workload": workloads.CONFIGS[DECODE_CFG].name,

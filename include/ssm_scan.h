@@ -248,9 +248,12 @@ int ssm_trap_scan_step(float *state, const void *x, const void *delta, const flo
                        void *out, const ssm_dims_t *dims, ssm_stream_t stream);
 
 /*
- * Workspace bytes that ssm_scan_bwd needs for the shape `dims`: the states at
- * the start of every 32-step segment (64 B per channel and segment, i.e. 2 B
- * per channel and step).  Returns SSM_OK and writes *bytes, or an SSM_ERR_* code.
+ * Workspace bytes that ssm_scan_bwd needs for the shape `dims`: the scratch of
+ * the forward pass that stores the checkpoints (as ssm_scan_fwd_workspace_size
+ * gives it for 256 SMs; ssm_scan_fwd_status on the backward's workspace reads
+ * its error word), then the states at the start of every 32-step segment (64 B
+ * per channel and segment, i.e. 2 B per channel and step).  Needs no device.
+ * Returns SSM_OK and writes *bytes, or an SSM_ERR_* code.
  */
 int ssm_scan_bwd_workspace_size(const ssm_dims_t *dims, size_t *bytes);
 
@@ -258,8 +261,9 @@ int ssm_scan_bwd_workspace_size(const ssm_dims_t *dims, size_t *bytes);
  * Backward pass of ssm_scan_fwd: the derivatives of a loss L with respect to
  * every input, given dout = dL/dout and dh_last = dL/dh_last.  As Appendix D
  * "Memory" describes, the intermediate states are not stored by the forward
- * pass: the call stores the state at the start of every 32-step segment and
- * recomputes the segment's states from it while it runs the adjoint recurrence
+ * pass: the call first runs the forward scan without output, storing the state
+ * at the start of every 32-step segment, and recomputes each segment's states
+ * from it while it runs the adjoint recurrence
  *   g_t = C_t dy_t + Abar_{t+1} g_{t+1},  dy_t = dout_t silu(z_t)
  * backwards through the chunk.
  *

@@ -3,8 +3,9 @@
 // Gu & Dao, "Mamba", Appendix D "Hardware-aware Algorithm For Selective
 // SSMs", paragraph "Memory": the backward pass does not keep the intermediate
 // states; it recomputes them when the inputs are loaded into on-chip memory.
-// Here a first kernel stores only the state at the start of every segment of
-// kBwdSeg steps (a checkpoint, 64 B per channel and segment); the backward
+// Here the forward scan kernel, run without output, stores only the state at
+// the start of every segment of kBwdSeg steps (a checkpoint, 64 B per channel
+// and segment); the backward
 // kernel walks each channel's segments from the last to the first, recomputes
 // a segment's states 16 steps at a time into shared memory and runs the
 // adjoint recurrence
@@ -28,7 +29,7 @@
 
 namespace ssm {
 
-constexpr int kBwdSeg = 32;   // steps between checkpoints
+constexpr int kBwdSeg = kCkptSteps;  // steps between checkpoints (stored by the forward kernel)
 constexpr int kBwdSub = 16;   // steps recomputed and run backwards at a time
 
 struct BwdParams {
@@ -122,23 +123,6 @@ __device__ __forceinline__ void bwd_put_bc(float *bc, int lane, const float (&v)
 __device__ __forceinline__ void red_add_v4(float *p, float a, float b, float c, float d) {
     asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
                  : "memory");
-}
-
-// Sixteen consecutive activations as raw 16-byte pieces (the row offset 16-byte
-// aligned), and element k of them widened.
-template <typename T>
-struct Raw16 {
-    uint4 q[kBwdSub / Act<T>::kPerPiece];
-};
-template <typename T>
-__device__ __forceinline__ void raw_load16(const void *base, int64_t off, Raw16<T> &r) {
-    const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(base) + off * Act<T>::kBytes);
-#pragma unroll
-    for (int i = 0; i < kBwdSub / Act<T>::kPerPiece; ++i) r.q[i] = __ldg(src + i);
-}
-template <typename T>
-__device__ __forceinline__ float raw_get(const Raw16<T> &r, int k) {
-    return Act<T>::piece(r.q[k / Act<T>::kPerPiece], k % Act<T>::kPerPiece);
 }
 
 // ---- the backward pass: 16 channels per warp, two lanes per channel --------------
@@ -464,93 +448,6 @@ __global__ void __launch_bounds__(32) scan_bwd_kernel(const BwdParams p) {
         if (!hf) {
             if (p.dD) atomicAdd(p.dD + dc, dDs);
             if (p.dbias) atomicAdd(p.dbias + dc, dbs);
-        }
-    }
-}
-
-// ---- checkpoints: the state at the start of every segment -------------------------
-// One warp per group of 16 channels of one sequence (two lanes per channel, as in
-// the backward kernel; four warps per CTA, each on its own): the forward
-// recurrence over the whole sequence, with the state written at every segment
-// start.  Each lane loads one row per sub-chunk (lane (c, 0) channel c's x,
-// lane (c, 1) its delta, lane j row j of B|C), two sub-chunks ahead.
-template <typename T>
-__global__ void __launch_bounds__(128) scan_bwd_ckpt_kernel(const BwdParams p) {
-    struct Warp {
-        float bc[kBwdSub * 32];
-        float io[2][kBwdSub][kBwdCh];
-    };
-    __shared__ __align__(16) Warp wsm[4];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, c = lane >> 1, hf = lane & 1;
-    const int64_t grp = static_cast<int64_t>(blockIdx.x) * 4 + warp;
-    if (grp >= bwd_groups16(p.batch, p.dim)) return;  // warp-uniform
-    const int64_t tiles = (p.dim + kBwdCh - 1) / kBwdCh;
-    const int64_t b = grp / tiles, d = (grp % tiles) * kBwdCh + c;
-    const bool active = d < p.dim;
-    const int64_t dc = active ? d : p.dim - 1;
-    const int64_t chan = b * p.dim + dc, L = p.seqlen, segs = bwd_segments(L), row = chan * L;
-    const bool vec = (L * Act<T>::kBytes) % 16 == 0;
-    const BwdHalf cc = bwd_half(p, dc, hf);
-    const int n0 = 8 * hf;
-    Warp &w = wsm[warp];
-    const void *mine = hf ? p.delta : p.x;
-    const void *bsrc = lane < kNState ? p.B : p.C;
-    const int64_t brow = (b * kNState + (lane & (kNState - 1))) * L;
-    float2 h[4];
-    if (p.h0) {
-        const float4 *src = reinterpret_cast<const float4 *>(p.h0 + chan * kNState + n0);
-        const float4 u = __ldg(src), v = __ldg(src + 1);
-        h[0] = make_float2(u.x, u.y); h[1] = make_float2(u.z, u.w);
-        h[2] = make_float2(v.x, v.y); h[3] = make_float2(v.z, v.w);
-    } else {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) h[j] = make_float2(0.0f, 0.0f);
-    }
-    // raw rows of the next two sub-chunks (aligned rows, whole sub-chunks only)
-    Raw16<T> r0, r1, q0, q1;
-    const bool raw_ok = vec;
-    auto fetch = [&](int64_t t0, Raw16<T> &rv, Raw16<T> &rb) {
-        if (raw_ok && t0 + kBwdSub <= L) {
-            raw_load16<T>(mine, row + t0, rv);
-            raw_load16<T>(bsrc, brow + t0, rb);
-        }
-    };
-    fetch(0, r0, q0);
-    fetch(kBwdSub, r1, q1);
-    for (int64_t t0 = 0; t0 < L; t0 += kBwdSub) {
-        if (t0 % kBwdSeg == 0 && active) {
-            float4 *dst = reinterpret_cast<float4 *>(p.ckpt + (chan * segs + t0 / kBwdSeg) * kNState + n0);
-            dst[0] = make_float4(h[0].x, h[0].y, h[1].x, h[1].y);
-            dst[1] = make_float4(h[2].x, h[2].y, h[3].x, h[3].y);
-        }
-        float v[kBwdSub], bv[kBwdSub];
-        if (raw_ok && t0 + kBwdSub <= L) {
-#pragma unroll
-            for (int k = 0; k < kBwdSub; ++k) v[k] = raw_get(r0, k), bv[k] = raw_get(q0, k);
-        } else {
-            bwd_load16<T>(mine, row, t0, L, vec, v);
-            bwd_load16<T>(bsrc, brow, t0, L, vec, bv);
-        }
-        r0 = r1;
-        q0 = q1;
-        fetch(t0 + 2 * kBwdSub, r1, q1);  // two sub-chunks ahead, in flight during this one
-        __syncwarp();  // the previous sub-chunk's reads are done
-#pragma unroll
-        for (int k = 0; k < kBwdSub; ++k) w.io[hf][k][c] = v[k];
-        bwd_put_bc(w.bc, lane, bv);
-        __syncwarp();
-#pragma unroll
-        for (int k = 0; k < kBwdSub; ++k) {
-            if (t0 + k >= L) break;  // warp-uniform
-            const float vv = w.io[1][k][c] + cc.bias;
-            const float dt = p.softplus ? bwd_softplus<T>(vv) : vv;
-            const float u = dt * w.io[0][k][c];
-            float2 a[4], B2[4];
-            bwd_decay_half(cc, hf, dt, a);
-            bwd_get8(w.bc + k * 32 + n0, B2);
-            const float2 u2 = make_float2(u, u);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) h[j] = __ffma2_rn(a[j], h[j], __fmul2_rn(u2, B2[j]));
         }
     }
 }

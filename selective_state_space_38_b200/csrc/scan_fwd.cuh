@@ -39,11 +39,17 @@
 
 namespace ssm {
 
+constexpr int kCkptSteps = 32;  // spacing of the states a checkpoint pass stores
+
 struct FwdParams {
     const void *x, *delta, *z, *B, *C;
     const float *delta_bias, *A, *D, *h0;
-    void *out;
+    void *out;      // NULL: no output (a checkpoint pass)
     float *h_last;
+    // When set, the state at every kCkptSteps-th step of every channel:
+    // ckpt[(b * dim + d) * ckpt_segs + t / kCkptSteps][16], the state before step t.
+    float *ckpt;
+    int64_t ckpt_segs;
     int64_t batch, seqlen, dim;
     int softplus;
     // kChained: segments of a group run in order, each starting from its
@@ -981,7 +987,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             const ChunkDesc dj = ring[j & 7];
             if (dj.flags & kStop) break;
             uint8_t *st = stage_of(j);
-            if (p.mode != kSummary) {  // the summary pass writes no output
+            if (p.mode != kSummary && p.out) {  // the summary pass and a checkpoint pass write no output
                 if (dj.d0 != cc_d0) {
                     const int64_t d = dj.d0 + lane;
                     cc = chan_const(p, d < p.dim ? d : p.dim - 1);
@@ -1070,6 +1076,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     h[2 * q] = make_float2(v.x, v.y);
                     h[2 * q + 1] = make_float2(v.z, v.w);
                 }
+            }
+            if (p.ckpt && p.mode != kSummary && active && dk.t0 % kCkptSteps == 0) {
+                float4 *ck = reinterpret_cast<float4 *>(p.ckpt +
+                                                        ((dk.b * p.dim + d) * p.ckpt_segs + dk.t0 / kCkptSteps) * kNState);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) ck[q] = make_float4(h[2 * q].x, h[2 * q].y, h[2 * q + 1].x, h[2 * q + 1].y);
             }
             if (p.mode == kSummary) {
                 if (dk.nvalid == TC)

@@ -98,7 +98,7 @@ bool make_maps(const FwdParams &p, TmaMaps *tm) {
     const uint64_t L = p.seqlen, D = p.dim, Bt = p.batch;
     bool ok = encode3d(&tm->x, dt, es, p.x, L, D, Bt, tc, 32, CU_TENSOR_MAP_SWIZZLE_64B) &&
               encode3d(&tm->delta, dt, es, p.delta, L, D, Bt, tc, 32, CU_TENSOR_MAP_SWIZZLE_64B) &&
-              encode3d(&tm->out, dt, es, p.out, L, D, Bt, tc, 32, CU_TENSOR_MAP_SWIZZLE_64B) &&
+              (!p.out || encode3d(&tm->out, dt, es, p.out, L, D, Bt, tc, 32, CU_TENSOR_MAP_SWIZZLE_64B)) &&
               encode3d(&tm->B, dt, es, p.B, L, kNState, Bt, tc, kNState, CU_TENSOR_MAP_SWIZZLE_NONE) &&
               encode3d(&tm->C, dt, es, p.C, L, kNState, Bt, tc, kNState, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (ok && p.z) ok = encode3d(&tm->z, dt, es, p.z, L, D, Bt, tc, 32, CU_TENSOR_MAP_SWIZZLE_64B);
@@ -419,10 +419,26 @@ int dispatch_fwd(const FwdParams &p, size_t es, int act_dtype, void *ws, size_t 
                      : launch_fwd<float, false, false>(p, ws, ws_bytes, sms, force_chained, s));
 }
 
-// Workspace of the backward pass: the states at every segment start (64 B per
-// channel and segment of 32 steps), rounded up to 256 bytes.
+// Workspace of the backward pass: first the scratch of the forward pass that
+// stores the checkpoints (so ssm_scan_fwd_status reads its error word), then
+// the states at every segment start (64 B per channel and segment of 32 steps).
+FwdParams bwd_ckpt_params(int64_t batch, int64_t L, int64_t dim) {
+    FwdParams f;
+    memset(&f, 0, sizeof f);
+    f.batch = batch; f.seqlen = L; f.dim = dim;
+    f.seg_steps = kSegSteps;
+    f.spin_limit = kSpinLimit;
+    return f;
+}
+// The forward scratch grows with the SM count (more segments on the two-pass
+// schedule); it is sized for kBwdMaxSms, so the size needs no device.
+constexpr int kBwdMaxSms = 256;
+size_t bwd_fwd_scratch_bytes(int64_t batch, int64_t L, int64_t dim) {
+    return (fwd_workspace_bytes(bwd_ckpt_params(batch, L, dim), kBwdMaxSms) + 255) / 256 * 256;
+}
 size_t bwd_workspace_bytes(int64_t batch, int64_t L, int64_t dim) {
-    return (static_cast<size_t>(batch) * dim * bwd_segments(L) * kNState * 4 + 255) / 256 * 256;
+    return bwd_fwd_scratch_bytes(batch, L, dim) +
+           (static_cast<size_t>(batch) * dim * bwd_segments(L) * kNState * 4 + 255) / 256 * 256;
 }
 
 template <typename T>
@@ -438,7 +454,6 @@ int launch_bwd(BwdParams p, cudaStream_t s) {
     if (p.dbias && cudaMemsetAsync(p.dbias, 0, static_cast<size_t>(p.dim) * 4, s) != cudaSuccess)
         return SSM_ERR_CUDA;
     const int64_t groups = bwd_groups16(p.batch, p.dim);
-    scan_bwd_ckpt_kernel<T><<<static_cast<unsigned>((groups + 3) / 4), 128, 0, s>>>(p);
     scan_bwd_kernel<T><<<static_cast<unsigned>(groups), 32, smem, s>>>(p);
     return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
@@ -588,6 +603,10 @@ int ssm_scan_bwd(const void *x, const void *delta, const float *delta_bias, int 
         if (ptr && !aligned16(ptr)) return SSM_ERR_MISALIGNED;
     for (const void *ptr : {(const void *)delta_bias, (const void *)D, (const void *)dD, (const void *)dbias})
         if (ptr && !aligned4(ptr)) return SSM_ERR_MISALIGNED;
+    // the checkpoint pass is the forward kernel: its 32-bit limits apply
+    if (batch > INT32_MAX || L > INT32_MAX - 64 || dim > INT32_MAX - 64) return SSM_ERR_UNSUPPORTED;
+    if (((dim + 31) / 32) * batch * ((L + 255) / 256) > static_cast<int64_t>(UINT32_MAX) / 2)
+        return SSM_ERR_UNSUPPORTED;
     if (workspace_bytes < bwd_workspace_bytes(batch, L, dim)) return SSM_ERR_INVALID_ARG;
 
     const size_t tok = static_cast<size_t>(batch) * dim * L, bn = static_cast<size_t>(batch) * N * L;
@@ -615,9 +634,20 @@ int ssm_scan_bwd(const void *x, const void *delta, const float *delta_bias, int 
     p.delta_bias = delta_bias; p.A = A; p.D = D; p.h0 = h0; p.dh_last = dh_last;
     p.dx = dx; p.ddelta = ddelta; p.dz = z ? dz : nullptr;
     p.dA = dA; p.dD = dD; p.dbias = dbias; p.dh0 = dh0; p.dB = dB; p.dC = dC;
-    p.ckpt = static_cast<float *>(workspace);
+    const size_t fws = bwd_fwd_scratch_bytes(batch, L, dim);
+    p.ckpt = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + fws);
     p.batch = batch; p.seqlen = L; p.dim = dim; p.softplus = softplus ? 1 : 0;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // the checkpoints: the forward scan with no output, storing its state every
+    // 32 steps (its scratch at the start of the workspace)
+    FwdParams f = bwd_ckpt_params(batch, L, dim);
+    f.x = x; f.delta = delta; f.B = B; f.C = C;
+    f.delta_bias = delta_bias; f.A = A; f.h0 = h0;
+    f.softplus = p.softplus;
+    f.ckpt = p.ckpt;
+    f.ckpt_segs = bwd_segments(L);
+    const int rc = dispatch_fwd(f, es, dims->act_dtype, workspace, fws, false, nullptr, s);
+    if (rc != SSM_OK) return rc;
     return dims->act_dtype == SSM_BF16 ? launch_bwd<bf16raw>(p, s) : launch_bwd<float>(p, s);
 }
 

@@ -246,8 +246,12 @@ def test_bwd_rejects_bad_arguments(lib):
     import selective_state_space_38_b200 as m
     need = ctypes.c_size_t(0)
     assert lib.ssm_scan_bwd_workspace_size(_dims(m), ctypes.byref(need)) == 0
-    segments = -(-64 // 32)  # one 64-byte state per channel and 32-step segment
-    assert need.value == (2 * 128 * segments * 16 * 4 + 255) // 256 * 256
+    # the checkpoint pass's forward scratch (sized for 256 SMs), then one 64-byte
+    # state per channel and 32-step segment
+    fwd = ctypes.c_size_t(0)
+    assert lib.ssm_scan_fwd_workspace_size(_dims(m), 256, ctypes.byref(fwd)) == 0
+    segments = -(-64 // 32)
+    assert need.value == (fwd.value + 255) // 256 * 256 + (2 * 128 * segments * 16 * 4 + 255) // 256 * 256
 
     def bwd(**over):
         a = dict(x=_p(1), delta=_p(2), bias=None, sp=1, A=_p(3), B=_p(4), C=_p(5), D=None, z=_p(6), h0=None,

@@ -458,7 +458,7 @@ def bench_next_rows(args, device, hbm_peak, only=None):
     sD = torch.ones(sh, device=device)
     sy = torch.empty_like(sx)
     shl = torch.empty((sb, sh, sp_, sn), dtype=torch.float32, device=device)
-    sws = torch.empty(256, dtype=torch.uint8, device=device)
+    sws = torch.empty(ssm.ssm_ssd_fwd_workspace_size(sb, sh, device), dtype=torch.uint8, device=device)
     rows["ssd_fwd"] = (lambda: ssm.ssm_ssd_fwd(sx, sdt, sbias, True, sA, sB, sC, sD, None, y=sy, h_last=shl,
                                                 workspace=sws),
                        2 * sx.numel() * 2 + sdt.numel() * 2 + 2 * sB.numel() * 2 + sh * 12 + shl.numel() * 4,

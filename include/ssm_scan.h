@@ -308,10 +308,27 @@ int ssm_scan_bwd(const void *x, const void *delta, const float *delta_bias, int 
  *   A, dt_bias, D  [heads] float32 (dt_bias and D optional)
  *   h0, h_last     optional [batch][heads][headdim][dstate] float32
  *   workspace      at least 256 bytes (the bounded-wait error word that
- *                  ssm_scan_fwd_status reads)
+ *                  ssm_scan_fwd_status reads), 16-byte aligned, owned by the
+ *                  caller and not used by a concurrent call.  With
+ *                  ssm_ssd_fwd_workspace_size bytes or more, a call with more
+ *                  sequences (batch * heads) than SMs runs one CTA per SM over
+ *                  equal numbers of chunks: a sequence may be split between two
+ *                  CTAs, whose state passes through the workspace.  With less,
+ *                  every sequence gets its own CTA.  Results are the same
+ *                  either way, up to rounding order.
  * Returns SSM_OK or an SSM_ERR_* code (SSM_ERR_UNSUPPORTED unless headdim 64,
  * dstate 128, bf16).
  */
+/*
+ * Workspace bytes for ssm_ssd_fwd to balance the sequences over sm_count SMs
+ * (sm_count <= 0: the current device's): 256 when batch * heads is at most
+ * the SM count (nothing is split), else 2048 + 32768 bytes per SM, for at most
+ * 448 SMs (one hand-off flag and one headdim x dstate float32 state each).  Needs only dims.batch
+ * and dims.heads.  Returns SSM_OK, SSM_ERR_INVALID_ARG (NULL pointer, batch or
+ * heads < 1) or SSM_ERR_CUDA (no current device when sm_count <= 0).
+ */
+int ssm_ssd_fwd_workspace_size(const ssm_ssd_dims_t *dims, int sm_count, size_t *bytes);
+
 int ssm_ssd_fwd(const void *x, const void *dt, const float *dt_bias, int softplus, const float *A,
                 const void *B, const void *C, const float *D, const float *h0, void *y, float *h_last,
                 void *workspace, size_t workspace_bytes, const ssm_ssd_dims_t *dims,

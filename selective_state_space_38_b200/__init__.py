@@ -70,6 +70,8 @@ def _load():
     lib.ssm_scan_bwd_workspace_size.restype = I
     lib.ssm_scan_bwd.argtypes = [P, P, P, I, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, DP, P]
     lib.ssm_scan_bwd.restype = I
+    lib.ssm_ssd_fwd_workspace_size.argtypes = [ctypes.POINTER(SsdDims), I, ctypes.POINTER(S)]
+    lib.ssm_ssd_fwd_workspace_size.restype = I
     lib.ssm_ssd_fwd.argtypes = [P, P, P, I, P, P, P, P, P, P, P, P, S, ctypes.POINTER(SsdDims), P]
     lib.ssm_ssd_fwd.restype = I
     lib.ssm_scan_step.argtypes = [P, P, P, P, I, P, P, P, P, P, P, DP, P]
@@ -94,7 +96,8 @@ def get_lib():
 
 EXPORTS = ("ssm_scan_fwd_workspace_size", "ssm_scan_fwd", "ssm_scan_fwd_status", "ssm_scan_step",
            "ssm_conv_scan_fwd", "ssm_conv_scan_step", "ssm_trap_scan_fwd", "ssm_trap_scan_step",
-           "ssm_scan_bwd_workspace_size", "ssm_scan_bwd", "ssm_ssd_fwd", "ssm_scan_fwd_noalloc",
+           "ssm_scan_bwd_workspace_size", "ssm_scan_bwd", "ssm_ssd_fwd_workspace_size", "ssm_ssd_fwd",
+           "ssm_scan_fwd_noalloc",
            "ssm_debug_fwd_flag_timeout",
            "ssm_strerror", "ssm_version")
 
@@ -444,6 +447,19 @@ def ssm_scan_bwd(x, delta, delta_bias, softplus, A, B, C, D, z, h0, dout, dh_las
     return g
 
 
+def ssm_ssd_fwd_workspace_size(batch: int, heads: int, device=None, sm_count: int = 0) -> int:
+    """Workspace bytes with which ssm_ssd_fwd balances batch * heads sequences
+    over the device's SMs (``sm_count`` > 0 sizes it without a device)."""
+    dims = SsdDims(batch, 1, heads, 64, 1, 128, SSM_BF16)
+    out = ctypes.c_size_t(0)
+    if sm_count > 0:
+        _check(get_lib().ssm_ssd_fwd_workspace_size(ctypes.byref(dims), int(sm_count), ctypes.byref(out)))
+    else:
+        with torch.cuda.device(torch.device(device or "cuda")):
+            _check(get_lib().ssm_ssd_fwd_workspace_size(ctypes.byref(dims), 0, ctypes.byref(out)))
+    return int(out.value)
+
+
 def ssm_ssd_fwd(x, dt, dt_bias, softplus, A, B, C, D=None, h0=None, y=None, h_last=None, stream=None,
                 workspace=None, check=False):
     """Mamba-2 SSD forward on the tensor cores.  x [batch, L, heads, 64],
@@ -470,10 +486,10 @@ def ssm_ssd_fwd(x, dt, dt_bias, softplus, A, B, C, D=None, h0=None, y=None, h_la
         h_last = torch.empty((batch, H, P, N), dtype=f32, device=dev)
     args += [_ptr(y, dtype=act, device=dev, shape=x.shape, name="y"),
              _ptr(h_last, dtype=f32, device=dev, shape=(batch, H, P, N), name="h_last")]
-    if workspace is None:
-        workspace = torch.empty(256, dtype=torch.uint8, device=dev)
-    pw = _ptr(workspace, dtype=torch.uint8, device=dev, name="workspace")
     dims = SsdDims(batch, L, H, P, G, N, SSM_BF16)
+    if workspace is None:
+        workspace = torch.empty(ssm_ssd_fwd_workspace_size(batch, H, dev), dtype=torch.uint8, device=dev)
+    pw = _ptr(workspace, dtype=torch.uint8, device=dev, name="workspace")
     sp = _stream_ptr(stream, dev)
     with torch.cuda.device(dev):
         _check(get_lib().ssm_ssd_fwd(*args, pw, workspace.numel(), ctypes.byref(dims), sp))
@@ -516,4 +532,4 @@ def ssm_scan_step(state, x, delta, delta_bias, softplus, A, B, C, D=None, z=None
 
 __all__ = ["ssm_scan_fwd", "ssm_scan_fwd_workspace_size", "ssm_scan_fwd_status", "ssm_scan_step",
            "ssm_conv_scan_fwd", "ssm_conv_scan_step", "ssm_trap_scan_fwd", "ssm_trap_scan_step", "ssm_scan_bwd",
-           "ssm_ssd_fwd", "SsdDims", "ssm_strerror", "ssm_version", "SSMError", "Dims", "LIB_PATH", "get_lib"]
+           "ssm_ssd_fwd", "ssm_ssd_fwd_workspace_size", "SsdDims", "ssm_strerror", "ssm_version", "SSMError", "Dims", "LIB_PATH", "get_lib"]

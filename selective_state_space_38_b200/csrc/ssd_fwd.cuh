@@ -12,7 +12,9 @@
 //   Y_diag = (C B^T o L) X,      L[i, j] = exp(cs_i - cs_j) dt_j (j <= i)
 //   Y_off  = diag(exp(cs)) C S_in^T
 //   S_out  = exp(cs_{Q-1}) S_in + B^T (w o X),   w_j = exp(cs_{Q-1} - cs_j) dt_j
-// One CTA owns one (batch, head) sequence and walks its chunks; the state S
+// A CTA walks the chunks of whole sequences in order, and may begin with the
+// start of one more sequence and end with the rest of another, whose state
+// passes between the two CTAs through global memory (SsdRange); the state S
 // (P x N float32) stays in registers, spread over the 256 threads.  Per chunk:
 //   MMA1 G = C B^T (128 x 128 x 128) and MMA3 Yo = C S_in^T (128 x 64 x 128);
 //   epilogue 1 forms L o G from G in tensor memory and writes it back there as
@@ -38,6 +40,7 @@ constexpr int kSsdP = 64;   // head dimension
 constexpr int kSsdN = 128;  // state dimension
 constexpr int kSsdThreads = 256;
 constexpr uint32_t kSsdWaitLimit = 1u << 24;
+constexpr uint32_t kSsdFlagLimit = 1u << 20;  // polls of a hand-off flag, 64 ns apart at least
 
 // TMA maps, rank 4 with the innermost dimension first: x [P][H][L][batch],
 // B and C [N][G][L][batch]; every box is 64 elements x 1 x 128 steps x 1.
@@ -51,10 +54,81 @@ struct SsdParams {
     void *y;                     // [b][L][H][P] bf16
     float *h_last;               // [b][H][P][N]
     uint32_t *error;             // bounded-wait failure word
+    // Split sequences (all three set, or none): the CTAs' order of start (a
+    // counter), one flag and one P x N state per hand-off between two CTAs.
+    uint32_t *order, *flags;
+    float *slots;
     int64_t batch, seqlen, heads, groups;
+    int64_t units_per_cta;       // chunks a CTA walks (the chunk count of a sequence without splits)
     int softplus;
 };
 
+// The chunks a CTA walks.  The batch * heads sequences, chunk by chunk, form one
+// list of units; CTA k (in the order the CTAs start) owns units [k W, k W + W).
+// With W at least one sequence's chunk count, such a range is: the end of one
+// sequence (its "tail"), whole sequences, and the start of another (its
+// "head").  The CTA walks the head first, hands its state on to CTA k + 1, then
+// the whole sequences, and the tail last, from the state CTA k - 1 handed on
+// at the end of its own head, which it walked first: no CTA waits on one that
+// started after it.
+// One unit of a CTA's walk: its sequence (batch b, head h, group g) and chunk;
+// whether it starts a part, ends one, and whether that end is the hand-off.
+struct SsdUnit {
+    int64_t seq, c, b, h, g;
+    bool first, last, handoff;
+};
+
+struct SsdRange {
+    int64_t chunks;            // chunks per sequence
+    int64_t head, full, tail;  // units in each part (full: whole sequences x chunks)
+    int64_t head_seq, first_full, tail_seq, tail_chunk;
+    int64_t heads, per_group;
+    __device__ SsdRange(int64_t k, int64_t W, int64_t nseq, int64_t C, int64_t H, int64_t HG)
+        : chunks(C), heads(H), per_group(HG) {
+        const int64_t s0 = k * W, e0 = min(s0 + W, nseq * C);
+        tail_chunk = s0 % C;
+        tail_seq = s0 / C;
+        head = e0 % C;
+        head_seq = e0 / C;
+        first_full = tail_chunk == 0 ? tail_seq : tail_seq + 1;
+        full = (e0 / C - first_full) * C;
+        tail = tail_chunk == 0 ? 0 : C - tail_chunk;
+    }
+    __device__ int64_t units() const { return head + full + tail; }
+    __device__ void set(SsdUnit &x, int64_t u, int64_t seq, int64_t c, bool new_seq) const {
+        if (new_seq) {
+            x.b = seq / heads;
+            x.h = seq - x.b * heads;
+            x.g = x.h / per_group;
+        }
+        x.seq = seq;
+        x.c = c;
+        x.first = c == 0 || (tail > 0 && u == head + full);
+        x.last = c == chunks - 1 || u == head - 1;
+        x.handoff = u < head;
+    }
+    __device__ SsdUnit first_unit() const {
+        SsdUnit x;
+        if (head > 0) set(x, 0, head_seq, 0, true);
+        else if (full > 0) set(x, 0, first_full, 0, true);
+        else set(x, 0, tail_seq, tail_chunk, true);
+        return x;
+    }
+    // x (unit u) becomes unit u + 1, without a division unless the sequence changes
+    __device__ void advance(SsdUnit &x, int64_t u) const {
+        const int64_t v = u + 1;
+        if (v == head) {
+            if (full > 0) set(x, v, first_full, 0, true);
+            else set(x, v, tail_seq, tail_chunk, true);
+        } else if (v == head + full) {
+            set(x, v, tail_seq, tail_chunk, true);
+        } else if (x.c + 1 == chunks) {
+            set(x, v, x.seq + 1, 0, true);
+        } else {
+            set(x, v, x.seq, x.c + 1, false);
+        }
+    }
+};
 // Shared memory (1024-byte aligned pieces; every operand tile is [128 rows][64]
 // bf16 with 128-byte rows and the 128-byte swizzle).
 struct SsdSmem {
@@ -66,7 +140,7 @@ struct SsdSmem {
     static constexpr int kXw = 2 * kInBytes;       // w o X [t][p]: high tile, low tile
     static constexpr int kS = kXw + 2 * kTile;     // S^T [n][p]: high tile, low tile
     static constexpr int kCs = kS + 2 * kTile;     // cs[128], dt[128], F[128], warp sums[4]
-    static constexpr int kBar = kCs + 1600;        // load[2], mma[2], TMEM base
+    static constexpr int kBar = kCs + 1600;        // load[2], mma[3], TMEM base, CTA order
     static constexpr int kTotal = kBar + 64 + 1024;  // + alignment slack
 };
 static_assert(SsdSmem::kTotal <= 227 * 1024, "shared memory of the SSD kernel");
@@ -185,9 +259,9 @@ __device__ __forceinline__ void split_pair(float a, float b, uint32_t &hi, uint3
     lo = pack_bf16x2(a - __uint_as_float(hi << 16), b - __uint_as_float(hi & 0xffff0000u));
 }
 
-// grid: batch * heads CTAs; block: 256 threads.  Thread (quad, half, lane) owns
-// row 32 quad + lane of every [128][..] tile (its TMEM lane) and the half
-// `half` of that row's columns.
+// grid: one CTA per range of units (SsdRange); block: 256 threads.  Thread
+// (quad, half, lane) owns row 32 quad + lane of every [128][..] tile (its TMEM
+// lane) and the half `half` of that row's columns.
 __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams p, const __grid_constant__ SsdMaps tm) {
     extern __shared__ __align__(1024) uint8_t ssd_smem_raw[];
     uint8_t *sm = ssd_smem_raw + ((1024u - (smem_u32(ssd_smem_raw) & 1023u)) & 1023u);
@@ -199,18 +273,18 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
     uint64_t *lbar = reinterpret_cast<uint64_t *>(sm + S::kBar);  // [2] input buffer landed
     uint64_t *mbar = lbar + 2;  // [0] MMA1 (G) done, [1] MMA2/4 (Yd, ST) done, [2] MMA3 (Yo) done
     uint32_t *tslot = reinterpret_cast<uint32_t *>(mbar + 3);
+    uint32_t *korder = tslot + 1;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, half = warp >> 2;
     const int row = quad * 32 + lane;
-    const int64_t b = blockIdx.x / p.heads, h = blockIdx.x % p.heads;
-    const int64_t g = h / (p.heads / p.groups);
-    const int64_t L = p.seqlen, H = p.heads;
-    const float Ah = p.A[h], bias = p.dt_bias ? p.dt_bias[h] : 0.0f, Dh = p.D ? p.D[h] : 0.0f;
+    const int64_t L = p.seqlen, H = p.heads, per_group = p.heads / p.groups;
     const int64_t chunks = (L + kSsdQ - 1) / kSsdQ;
 
     if (tid == 0) {
         for (int i = 0; i < 5; ++i) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(lbar + i)));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        // with split sequences a CTA's range is its place in the order of start
+        *korder = p.order ? atomicAdd(p.order, 1u) : blockIdx.x;
     }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(tslot)));
@@ -220,33 +294,80 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tbase = *reinterpret_cast<volatile uint32_t *>(tslot);
+    const int64_t kcta = *reinterpret_cast<volatile uint32_t *>(korder);
+    const SsdRange rg(kcta, p.units_per_cta, p.batch * H, chunks, H, per_group);
+    const int64_t units = rg.units();
     // TMEM columns: G then L o G (128), Yd (64), Yo (64), ST (64)
     const uint32_t tG = tbase, tYd = tbase + 128, tYo = tbase + 192, tST = tbase + 256;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
 
-    // the inputs of chunk c into buffer c & 1 (one thread)
-    auto load = [&](int64_t c) {
-        uint8_t *in = sm + (c & 1) * S::kInBytes;
-        uint64_t *bar = lbar + (c & 1);
+    // the inputs of unit u (x) into buffer u & 1 (one thread)
+    auto load = [&](const SsdUnit &x, int64_t u) {
+        uint8_t *in = sm + (u & 1) * S::kInBytes;
+        uint64_t *bar = lbar + (u & 1);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         mbar_arrive_expect_tx(bar, S::kInBytes);
-        const int t0 = static_cast<int>(c * kSsdQ), bi = static_cast<int>(b), gi = static_cast<int>(g);
+        const int t0 = static_cast<int>(x.c * kSsdQ), bi = static_cast<int>(x.b), gi = static_cast<int>(x.g);
         tma_load_4d(in + S::kInC, &tm.C, 0, gi, t0, bi, bar);
         tma_load_4d(in + S::kInC + S::kTile, &tm.C, 64, gi, t0, bi, bar);
         tma_load_4d(in + S::kInB, &tm.B, 0, gi, t0, bi, bar);
         tma_load_4d(in + S::kInB + S::kTile, &tm.B, 64, gi, t0, bi, bar);
-        tma_load_4d(in + S::kInX, &tm.x, 0, static_cast<int>(h), t0, bi, bar);
+        tma_load_4d(in + S::kInX, &tm.x, 0, static_cast<int>(x.h), t0, bi, bar);
     };
-    // raw dt of step t (zero past the end)
-    auto load_dt = [&](int64_t t) -> float {
-        return t < L ? Act<bf16raw>::load(p.dt, (b * L + t) * H + h) : 0.0f;
+    // raw dt of this thread's step of unit x (zero past the end)
+    auto load_dt = [&](const SsdUnit &x) -> float {
+        const int64_t t = x.c * kSsdQ + tid;
+        return t < L ? Act<bf16raw>::load(p.dt, (x.b * L + t) * H + x.h) : 0.0f;
     };
 
     // this thread's share of the state: S[p][n] for n = row, p in [32 half, 32 half + 32)
     float st[32];
+    // the state a part starts from: h0 (or zero) at a sequence start, else the
+    // one the previous CTA handed on (a bounded wait on its flag)
+    auto begin_part = [&](int64_t seq, int64_t c) -> bool {
+        if (c == 0) {
 #pragma unroll
-    for (int q = 0; q < 32; ++q)
-        st[q] = p.h0 ? p.h0[((b * H + h) * kSsdP + 32 * half + q) * kSsdN + row] : 0.0f;
+            for (int q = 0; q < 32; ++q)
+                st[q] = p.h0 ? p.h0[(seq * kSsdP + 32 * half + q) * kSsdN + row] : 0.0f;
+            return true;
+        }
+        bool got = true;
+        if (tid == 0) {
+            got = false;
+            const uint32_t *flag = p.flags + (kcta - 1);
+            for (uint32_t n = 0; n < kSsdFlagLimit; ++n) {
+                if (ld_acquire(flag) != 0) {
+                    got = true;
+                    break;
+                }
+                if ((n & 255u) == 255u && *reinterpret_cast<volatile uint32_t *>(p.error) != 0) break;
+                __nanosleep(64);
+            }
+            if (!got && *reinterpret_cast<volatile uint32_t *>(p.error) == 0) atomicOr(p.error, 2u);
+        }
+        if (!__syncthreads_and(got)) return false;
+        const float *src = p.slots + (kcta - 1) * (kSsdP * kSsdN);
+#pragma unroll
+        for (int q = 0; q < 32; ++q) st[q] = __ldcg(src + (32 * half + q) * kSsdN + row);
+        return true;
+    };
+    // the state at the end of a part: h_last at a sequence end, else to this
+    // CTA's hand-off slot, then its flag (release)
+    auto end_part = [&](int64_t seq, bool handoff) {
+        if (handoff) {
+            float *dst = p.slots + kcta * (kSsdP * kSsdN);
+#pragma unroll
+            for (int q = 0; q < 32; ++q) dst[(32 * half + q) * kSsdN + row] = st[q];
+            __syncthreads();
+            if (tid == 0) {
+                __threadfence();
+                st_release(p.flags + kcta, 1u);
+            }
+        } else if (p.h_last) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) p.h_last[(seq * kSsdP + 32 * half + q) * kSsdN + row] = st[q];
+        }
+    };
     // S^T [n][p] as bf16 high and low tiles (the B operand of MMA3, N = p contiguous)
     auto write_state = [&]() {
 #pragma unroll
@@ -260,23 +381,31 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
         }
     };
 
-    // Chunks overlap on the tensor core: chunk c + 1's G = C B^T is issued as soon as
-    // chunk c's MMA2/4 have read L o G out of its TMEM columns, and runs during
-    // chunk c's epilogue 2; chunk c's Yo = C S^T is issued before its epilogue 1,
+    // Chunks overlap on the tensor core: unit u + 1's G = C B^T is issued as soon as
+    // unit u's MMA2/4 have read L o G out of its TMEM columns, and runs during
+    // unit u's epilogue 2; unit u's Yo = C S^T is issued before its epilogue 1,
     // which does not need it.  Each MMA group commits to its own mbarrier, one
-    // phase per chunk; the counts below let a walk that gives up drain them.
+    // phase per unit; the counts below let a walk that gives up drain them.
     int64_t loads_issued = 0, loads_waited = 0;
     uint32_t committed[3] = {0, 0, 0}, waited[3] = {0, 0, 0};
-    if (tid == 0) load(0);
-    loads_issued = 1;
-    float dt_raw = tid < kSsdQ ? load_dt(tid) : 0.0f;
-    write_state();
+    // the unit being computed and the next one
+    SsdUnit cur = rg.first_unit(), nxt = cur;
+    bool ok = units > 0;
+    if (ok) {
+        if (tid == 0) load(cur, 0);
+        loads_issued = 1;
+    }
+    float dt_raw = ok && tid < kSsdQ ? load_dt(cur) : 0.0f;
+    if (ok) {
+        ok = begin_part(cur.seq, cur.c);
+        write_state();
+    }
 
     const uint32_t a_s = smem_u32(sm + S::kS), a_xw = smem_u32(sm + S::kXw);
     // a descriptor of base + off is the base's plus off / 16 (no carry: every
     // shared-memory address is below 2^18)
-    auto issue_g = [&](int64_t c) {  // MMA1: G = C B^T of chunk c
-        uint8_t *in = sm + (c & 1) * S::kInBytes;
+    auto issue_g = [&](int64_t u) {  // MMA1: G = C B^T of unit u
+        uint8_t *in = sm + (u & 1) * S::kInBytes;
         constexpr uint32_t i1 = ssd_idesc(128, 128, 0, 0);
         const uint64_t dC = ssd_desc(smem_u32(in + S::kInC), 16, 1024), dB = ssd_desc(smem_u32(in + S::kInB), 16, 1024);
 #pragma unroll
@@ -290,17 +419,29 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
     auto wait_all = [&](uint64_t *bar, uint32_t parity) -> bool {
         return __syncthreads_and(ssd_wait(bar, parity, p.error)) != 0;
     };
-    bool ok = wait_all(lbar, 0u);
+    if (ok) ok = wait_all(lbar, 0u);
     if (ok) {
         loads_waited = 1;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         if (tid == 0) issue_g(0);
         committed[0] = 1;
     }
-    for (int64_t c = 0; ok && c < chunks; ++c) {
+    // the head's A, dt bias and D: those of the next unit are loaded a unit ahead
+    float Ah = p.A[cur.h], bias = p.dt_bias ? p.dt_bias[cur.h] : 0.0f, Dh = p.D ? p.D[cur.h] : 0.0f;
+    for (int64_t u = 0; ok && u < units; ++u) {
+        float nAh = Ah, nbias = bias, nDh = Dh;
+        if (u + 1 < units) {
+            rg.advance(nxt, u);
+            if (nxt.h != cur.h) {
+                nAh = p.A[nxt.h];
+                nbias = p.dt_bias ? p.dt_bias[nxt.h] : 0.0f;
+                nDh = p.D ? p.D[nxt.h] : 0.0f;
+            }
+        }
+        const int64_t b = cur.b, h = cur.h, c = cur.c;
         const int64_t t0 = c * kSsdQ;
-        const uint32_t ph = static_cast<uint32_t>(c & 1);
-        uint8_t *in = sm + (c & 1) * S::kInBytes;
+        const uint32_t ph = static_cast<uint32_t>(u & 1);
+        uint8_t *in = sm + (u & 1) * S::kInBytes;
         const uint32_t a_c = smem_u32(in + S::kInC), a_b = smem_u32(in + S::kInB), a_x = smem_u32(in + S::kInX);
         // ---- dt and the running sum cs of dt A over the chunk (threads 0..127)
         float s = 0.0f, dtv = 0.0f;
@@ -316,12 +457,12 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
                 if (lane >= off) s += o;
             }
             if (lane == 31) wsum[warp] = s;
-            if (c + 1 < chunks) dt_raw = load_dt(t0 + kSsdQ + tid);  // the next chunk's, in flight meanwhile
+            if (u + 1 < units) dt_raw = load_dt(nxt);  // the next unit's, in flight meanwhile
         }
         // the next chunk's inputs go to the other buffer, whose last readers (chunk
         // c - 1's MMAs and epilogue) have finished
-        if (tid == 0 && c + 1 < chunks) load(c + 1);
-        if (c + 1 < chunks) loads_issued = c + 2;
+        if (tid == 0 && u + 1 < units) load(nxt, u + 1);
+        if (u + 1 < units) loads_issued = u + 2;
         __syncthreads();
         if (tid < kSsdQ) {
             for (int w = 0; w < warp; ++w) s += wsum[w];
@@ -348,13 +489,13 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
                 }
             ssd_commit(mbar + 2);
         }
-        committed[2] = static_cast<uint32_t>(c + 1);
+        committed[2] = static_cast<uint32_t>(u + 1);
         // ---- G of this chunk (issued during the previous chunk's epilogue 2)
         if (!wait_all(mbar, ph)) {
             ok = false;
             break;
         }
-        waited[0] = static_cast<uint32_t>(c + 1);
+        waited[0] = static_cast<uint32_t>(u + 1);
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         const float total = cs[kSsdQ - 1];
         float dx[32];  // D x of this thread's row and column half, kept for epilogue 2
@@ -448,28 +589,28 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
                             part > 0 || k > 0);
             ssd_commit(mbar + 1);
         }
-        committed[1] = static_cast<uint32_t>(c + 1);
+        committed[1] = static_cast<uint32_t>(u + 1);
         if (!wait_all(mbar + 1, ph)) {
             ok = false;
             break;
         }
-        waited[1] = static_cast<uint32_t>(c + 1);
+        waited[1] = static_cast<uint32_t>(u + 1);
         if (!wait_all(mbar + 2, ph)) {
             ok = false;
             break;
         }
-        waited[2] = static_cast<uint32_t>(c + 1);
+        waited[2] = static_cast<uint32_t>(u + 1);
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         // ---- the next chunk's G: its inputs have landed and G's columns are read
-        if (c + 1 < chunks) {
-            if (!wait_all(lbar + ((c + 1) & 1), static_cast<uint32_t>(((c + 1) >> 1) & 1))) {
+        if (u + 1 < units) {
+            if (!wait_all(lbar + ((u + 1) & 1), static_cast<uint32_t>(((u + 1) >> 1) & 1))) {
                 ok = false;
                 break;
             }
-            loads_waited = c + 2;
+            loads_waited = u + 2;
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            if (tid == 0) issue_g(c + 1);
-            committed[0] = static_cast<uint32_t>(c + 2);
+            if (tid == 0) issue_g(u + 1);
+            committed[0] = static_cast<uint32_t>(u + 2);
         }
         // ---- epilogue 2: y row i, p in [32 half, 32 half + 32); state row n, same p
         {
@@ -501,8 +642,21 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
 #pragma unroll
                 for (int e = 0; e < 16; ++e) st[q0 + e] = fmaf(et, st[q0 + e], v[e]);
             }
+        }
+        // the end of a part (h_last, or the hand-off to the next CTA); the state the
+        // next unit starts from, as MMA3's operand
+        if (cur.last) end_part(cur.seq, cur.handoff);
+        if (u + 1 < units) {
+            if (nxt.first && !begin_part(nxt.seq, nxt.c)) {
+                ok = false;
+                break;
+            }
             write_state();
         }
+        cur = nxt;
+        Ah = nAh;
+        bias = nbias;
+        Dh = nDh;
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     }
     // a wait that gave up leaves no load or MMA running when the CTA ends
@@ -511,10 +665,6 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
             for (uint32_t n = waited[g]; n < committed[g]; ++n) ssd_drain(mbar + g, n & 1u, p.error);
         for (int64_t c = loads_waited; c < loads_issued; ++c)
             ssd_drain(lbar + (c & 1), static_cast<uint32_t>((c >> 1) & 1), p.error);
-    }
-    if (p.h_last && ok) {
-#pragma unroll
-        for (int q = 0; q < 32; ++q) p.h_last[((b * H + h) * kSsdP + 32 * half + q) * kSsdN + row] = st[q];
     }
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");

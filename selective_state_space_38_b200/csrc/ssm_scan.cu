@@ -4,6 +4,7 @@
 // fails a check launches nothing.  Kernels run asynchronously on the caller's
 // stream.
 
+#include <algorithm>
 #include <climits>
 #include <cstring>
 #include <cstddef>
@@ -651,6 +652,26 @@ int ssm_scan_bwd(const void *x, const void *delta, const float *delta_bias, int 
     return dims->act_dtype == SSM_BF16 ? launch_bwd<bf16raw>(p, s) : launch_bwd<float>(p, s);
 }
 
+// SSD workspace: bytes [0, 256) hold the CTA order counter (at 0) and the error
+// word (at 16) of every workspace layout; [256, 2048) one hand-off flag per CTA;
+// from 2048 one P x N float32 state per CTA.
+constexpr int64_t kSsdFlagOff = 256, kSsdSlotOff = 2048, kSsdMaxCtas = (kSsdSlotOff - kSsdFlagOff) / 4;
+constexpr int64_t kSsdSlotBytes = static_cast<int64_t>(kSsdP) * kSsdN * 4;
+
+// CTAs of a split launch on sms SMs (0: sequences are not split)
+static int64_t ssd_split_ctas(int64_t nseq, int sms) {
+    const int64_t cap = std::min<int64_t>(sms, kSsdMaxCtas);
+    return nseq > cap ? cap : 0;
+}
+
+int ssm_ssd_fwd_workspace_size(const ssm_ssd_dims_t *dims, int sm_count, size_t *bytes) {
+    if (!dims || !bytes || dims->batch < 1 || dims->heads < 1) return SSM_ERR_INVALID_ARG;
+    if (sm_count <= 0 && current_sms(&sm_count) != SSM_OK) return SSM_ERR_CUDA;
+    const int64_t ctas = ssd_split_ctas(dims->batch * dims->heads, sm_count);
+    *bytes = ctas ? static_cast<size_t>(kSsdSlotOff + ctas * kSsdSlotBytes) : 256;
+    return SSM_OK;
+}
+
 int ssm_ssd_fwd(const void *x, const void *dt, const float *dt_bias, int softplus, const float *A, const void *B,
                 const void *C, const float *D, const float *h0, void *y, float *h_last, void *workspace,
                 size_t workspace_bytes, const ssm_ssd_dims_t *dims, ssm_stream_t stream) {
@@ -682,9 +703,25 @@ int ssm_ssd_fwd(const void *x, const void *dt, const float *dt_bias, int softplu
         for (int q = o + 1; q < 3; ++q)
             if (overlap(outs[o], outs[q])) return SSM_ERR_INVALID_ARG;
     }
+    // more sequences than SMs: persistent CTAs over equal ranges of chunks, when
+    // the workspace holds the hand-offs; else one CTA per sequence
+    int sms = 0;
+    if (current_sms(&sms) != SSM_OK) return SSM_ERR_CUDA;
+    const int64_t nseq = batch * H, chunks = (L + kSsdQ - 1) / kSsdQ;
+    int64_t ctas = ssd_split_ctas(nseq, sms), per_cta = chunks;
+    if (ctas && workspace_bytes < static_cast<size_t>(kSsdSlotOff + ctas * kSsdSlotBytes)) ctas = 0;
+    if (ctas) {
+        per_cta = (nseq * chunks + ctas - 1) / ctas;  // at least chunks, as nseq > ctas
+        ctas = (nseq * chunks + per_cta - 1) / per_cta;
+    }
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (cudaMemsetAsync(workspace, 0, 256, s) != cudaSuccess) return SSM_ERR_CUDA;
+    if (cudaMemsetAsync(workspace, 0, ctas ? kSsdSlotOff : 256, s) != cudaSuccess) return SSM_ERR_CUDA;
+    uint8_t *wb = static_cast<uint8_t *>(workspace);
     SsdParams prm;
+    prm.order = ctas ? reinterpret_cast<uint32_t *>(wb) : nullptr;
+    prm.flags = ctas ? reinterpret_cast<uint32_t *>(wb + kSsdFlagOff) : nullptr;
+    prm.slots = ctas ? reinterpret_cast<float *>(wb + kSsdSlotOff) : nullptr;
+    prm.units_per_cta = per_cta;
     prm.dt = dt;
     prm.dt_bias = dt_bias; prm.A = A; prm.D = D; prm.h0 = h0;
     prm.y = y; prm.h_last = h_last;
@@ -701,7 +738,7 @@ int ssm_ssd_fwd(const void *x, const void *dt, const float *dt_bias, int softplu
     const int smem = SsdSmem::kTotal;
     if (cudaFuncSetAttribute(ssd_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return SSM_ERR_CUDA;
-    ssd_fwd_kernel<<<static_cast<unsigned>(batch * H), kSsdThreads, smem, s>>>(prm, tm);
+    ssd_fwd_kernel<<<static_cast<unsigned>(ctas ? ctas : nseq), kSsdThreads, smem, s>>>(prm, tm);
     return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 

@@ -297,3 +297,23 @@ def test_ssd_rejects_bad_arguments(lib):
     assert ssd(dt=ctypes.c_void_p(0x12000001)) == 3
     assert ssd(y=_p(1)) == 1
     assert ssd(hl=_p(4)) == 1
+
+
+def test_ssd_workspace_size(lib):
+    """Split sequences need 2048 bytes plus one 32 KB state per CTA (at most one
+    per SM, at most 448); without more sequences than SMs, 256 bytes."""
+    import selective_state_space_38_b200 as m
+    n = ctypes.c_size_t(0)
+
+    def size(batch, heads, sms):
+        assert lib.ssm_ssd_fwd_workspace_size(ctypes.byref(m.SsdDims(batch, 4096, heads, 64, 1, 128, 1)), sms,
+                                              ctypes.byref(n)) == 0
+        return n.value
+    assert size(4, 80, 148) == 2048 + 148 * 32768
+    assert size(1, 148, 148) == 256
+    assert size(1, 149, 148) == 2048 + 148 * 32768
+    assert size(4, 200, 1000) == 2048 + 448 * 32768
+    assert m.ssm_ssd_fwd_workspace_size(4, 80, sm_count=132) == 2048 + 132 * 32768
+    assert lib.ssm_ssd_fwd_workspace_size(None, 148, ctypes.byref(n)) == 1
+    assert lib.ssm_ssd_fwd_workspace_size(ctypes.byref(m.SsdDims(0, 1, 1, 64, 1, 128, 1)), 148,
+                                          ctypes.byref(n)) == 1

@@ -93,3 +93,24 @@ def test_softplus_off(orc):
     ry, rh = _ref(orc, inp, softplus=False)
     check(to_np64(y), ry, "bf16", "ssd softplus off y")
     check(to_np64(hl), rh, "bf16", "ssd softplus off h_last")
+
+
+@pytest.mark.parametrize("L", [100, 300])
+def test_split_sequences(orc, L):
+    """More sequences (3 x 64 heads) than SMs: with the sized workspace the CTAs
+    walk equal numbers of chunks and hand the state of a split sequence on
+    through the workspace (ragged last chunk at L = 300); with a 256-byte
+    workspace every sequence gets its own CTA.  Both against the oracle."""
+    import selective_state_space_38_b200 as ssm
+    inp = ssd_inputs(3, L, 64, 2, seed=20 + L, h0=True)
+    t = {k: to_dev(v) for k, v in inp.items() if isinstance(v, np.ndarray)}
+    ry, rh = _ref(orc, inp)
+    sized = ssm.ssm_ssd_fwd_workspace_size(3, 64, t["x"].device)
+    assert sized > 256
+    for nbytes in (sized, 256):
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=t["x"].device)
+        y, hl = ssm.ssm_ssd_fwd(t["x"], t["dt"], t["dt_bias"], True, t["A"], t["B"], t["C"], t["D"], t["h0"],
+                                workspace=ws, check=True)
+        torch.cuda.synchronize()
+        check(to_np64(y), ry, "bf16", f"ssd split y L={L} ws={nbytes}")
+        check(to_np64(hl), rh, "bf16", f"ssd split h_last L={L} ws={nbytes}")

@@ -74,7 +74,7 @@ struct SsdParams {
 // One unit of a CTA's walk: its sequence (batch b, head h, group g) and chunk;
 // whether it starts a part, ends one, and whether that end is the hand-off.
 struct SsdUnit {
-    int64_t seq, c, b, h, g;
+    int seq, c, b, h, g;  // below 2^31: batch * heads and the chunk count are checked on the host
     bool first, last, handoff;
 };
 
@@ -97,12 +97,13 @@ struct SsdRange {
     __device__ int64_t units() const { return head + full + tail; }
     __device__ void set(SsdUnit &x, int64_t u, int64_t seq, int64_t c, bool new_seq) const {
         if (new_seq) {
-            x.b = seq / heads;
-            x.h = seq - x.b * heads;
-            x.g = x.h / per_group;
+            const int64_t bb = seq / heads;
+            x.b = static_cast<int>(bb);
+            x.h = static_cast<int>(seq - bb * heads);
+            x.g = static_cast<int>(x.h / per_group);
         }
-        x.seq = seq;
-        x.c = c;
+        x.seq = static_cast<int>(seq);
+        x.c = static_cast<int>(c);
         x.first = c == 0 || (tail > 0 && u == head + full);
         x.last = c == chunks - 1 || u == head - 1;
         x.handoff = u < head;
@@ -140,7 +141,7 @@ struct SsdSmem {
     static constexpr int kXw = 2 * kInBytes;       // w o X [t][p]: high tile, low tile
     static constexpr int kS = kXw + 2 * kTile;     // S^T [n][p]: high tile, low tile
     static constexpr int kCs = kS + 2 * kTile;     // cs[128], dt[128], F[128], warp sums[4]
-    static constexpr int kBar = kCs + 1600;        // load[2], mma[3], TMEM base, CTA order
+    static constexpr int kBar = kCs + 1600;        // load[2], mma[5], TMEM base, CTA order (64 bytes)
     static constexpr int kTotal = kBar + 64 + 1024;  // + alignment slack
 };
 static_assert(SsdSmem::kTotal <= 227 * 1024, "shared memory of the SSD kernel");
@@ -271,8 +272,8 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
     float *Fs = dts + 128;  // F_j = exp(-cs_j) dt_j, when every |cs| of the chunk is at most 80
     float *wsum = Fs + 128;
     uint64_t *lbar = reinterpret_cast<uint64_t *>(sm + S::kBar);  // [2] input buffer landed
-    uint64_t *mbar = lbar + 2;  // [0] MMA1 (G) done, [1] MMA2/4 (Yd, ST) done, [2] MMA3 (Yo) done
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(mbar + 3);
+    uint64_t *mbar = lbar + 2;  // [0] MMA1 (G), [1] MMA2 high, [2] MMA3 (Yo), [3] MMA4 (ST), [4] MMA2 low done
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(mbar + 5);
     uint32_t *korder = tslot + 1;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, half = warp >> 2;
@@ -281,7 +282,7 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
     const int64_t chunks = (L + kSsdQ - 1) / kSsdQ;
 
     if (tid == 0) {
-        for (int i = 0; i < 5; ++i) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(lbar + i)));
+        for (int i = 0; i < 7; ++i) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(lbar + i)));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         // with split sequences a CTA's range is its place in the order of start
         *korder = p.order ? atomicAdd(p.order, 1u) : blockIdx.x;
@@ -297,8 +298,10 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
     const int64_t kcta = *reinterpret_cast<volatile uint32_t *>(korder);
     const SsdRange rg(kcta, p.units_per_cta, p.batch * H, chunks, H, per_group);
     const int64_t units = rg.units();
-    // TMEM columns: G then L o G (128), Yd (64), Yo (64), ST (64)
-    const uint32_t tG = tbase, tYd = tbase + 128, tYo = tbase + 192, tST = tbase + 256;
+    // TMEM columns: G then L o G (128); Yd (128: the products of the high and of
+    // the low part of L o G side by side); Yo (128: the same for S^T); ST (128:
+    // the same for w o X)
+    const uint32_t tG = tbase, tYd = tbase + 128, tYo = tbase + 256, tST = tbase + 384;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
 
     // the inputs of unit u (x) into buffer u & 1 (one thread)
@@ -387,18 +390,58 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
     // which does not need it.  Each MMA group commits to its own mbarrier, one
     // phase per unit; the counts below let a walk that gives up drain them.
     int64_t loads_issued = 0, loads_waited = 0;
-    uint32_t committed[3] = {0, 0, 0}, waited[3] = {0, 0, 0};
-    // the unit being computed and the next one
+    uint32_t committed[5] = {0, 0, 0, 0, 0}, waited[5] = {0, 0, 0, 0, 0};
+    // the running sums of unit x's chunk: first dt and the running sum within each
+    // warp (threads 0..127; the warp's total to wsum), then, after a barrier, the
+    // sums of the warps before it; cs, dt and F to their tables.  Returns whether
+    // this thread's |cs| is at most 80 (threads 128.. return true).
+    float s = 0.0f, dtv = 0.0f;
+    auto sums_in_warp = [&](const SsdUnit &x, float raw, float bias_x, float A_x) {
+        if (tid < kSsdQ) {
+            dtv = 0.0f;
+            if (static_cast<int64_t>(x.c) * kSsdQ + tid < L) {
+                const float v = raw + bias_x;
+                dtv = p.softplus ? softplus_fast(v) : v;
+            }
+            s = dtv * A_x;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float o = __shfl_up_sync(0xffffffffu, s, off);
+                if (lane >= off) s += o;
+            }
+            if (lane == 31) wsum[warp] = s;
+        }
+    };
+    auto sums_across_warps = [&]() -> bool {
+        if (tid >= kSsdQ) return true;
+        for (int w = 0; w < warp; ++w) s += wsum[w];
+        cs[tid] = s;
+        dts[tid] = dtv;
+        Fs[tid] = __expf(-s) * dtv;
+        return fabsf(s) <= 80.0f;
+    };
+
+    // Per unit u: cur is unit u, nxt unit u + 1, nn unit u + 2 (whose dt is loaded
+    // while u runs); the cs tables hold unit u's, and unit u + 1's are formed while
+    // u's MMA2 and MMA4 run (epilogue 2 keeps what it needs in registers).
     SsdUnit cur = rg.first_unit(), nxt = cur;
+    if (units > 1) rg.advance(nxt, 0);
     bool ok = units > 0;
     if (ok) {
         if (tid == 0) load(cur, 0);
         loads_issued = 1;
     }
+    // the head's A, dt bias and D (the next unit's are loaded a unit ahead)
+    float Ah = p.A[cur.h], bias = p.dt_bias ? p.dt_bias[cur.h] : 0.0f, Dh = p.D ? p.D[cur.h] : 0.0f;
     float dt_raw = ok && tid < kSsdQ ? load_dt(cur) : 0.0f;
+    bool factored = true;  // every |cs| of the unit's chunk at most 80: exp(cs_i - cs_j) = exp(cs_i) exp(-cs_j)
     if (ok) {
         ok = begin_part(cur.seq, cur.c);
         write_state();
+        sums_in_warp(cur, dt_raw, bias, Ah);
+        if (units > 1 && tid < kSsdQ) dt_raw = load_dt(nxt);
+        __syncthreads();
+        factored = __syncthreads_and(sums_across_warps()) != 0;
     }
 
     const uint32_t a_s = smem_u32(sm + S::kS), a_xw = smem_u32(sm + S::kXw);
@@ -426,67 +469,40 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
         if (tid == 0) issue_g(0);
         committed[0] = 1;
     }
-    // the head's A, dt bias and D: those of the next unit are loaded a unit ahead
-    float Ah = p.A[cur.h], bias = p.dt_bias ? p.dt_bias[cur.h] : 0.0f, Dh = p.D ? p.D[cur.h] : 0.0f;
     for (int64_t u = 0; ok && u < units; ++u) {
+        SsdUnit nn = nxt;
+        if (u + 2 < units) rg.advance(nn, u + 1);
         float nAh = Ah, nbias = bias, nDh = Dh;
-        if (u + 1 < units) {
-            rg.advance(nxt, u);
-            if (nxt.h != cur.h) {
-                nAh = p.A[nxt.h];
-                nbias = p.dt_bias ? p.dt_bias[nxt.h] : 0.0f;
-                nDh = p.D ? p.D[nxt.h] : 0.0f;
-            }
+        if (u + 1 < units && nxt.h != cur.h) {
+            nAh = p.A[nxt.h];
+            nbias = p.dt_bias ? p.dt_bias[nxt.h] : 0.0f;
+            nDh = p.D ? p.D[nxt.h] : 0.0f;
         }
         const int64_t b = cur.b, h = cur.h, c = cur.c;
         const int64_t t0 = c * kSsdQ;
         const uint32_t ph = static_cast<uint32_t>(u & 1);
         uint8_t *in = sm + (u & 1) * S::kInBytes;
         const uint32_t a_c = smem_u32(in + S::kInC), a_b = smem_u32(in + S::kInB), a_x = smem_u32(in + S::kInX);
-        // ---- dt and the running sum cs of dt A over the chunk (threads 0..127)
-        float s = 0.0f, dtv = 0.0f;
-        if (tid < kSsdQ) {
-            if (t0 + tid < L) {
-                const float v = dt_raw + bias;
-                dtv = p.softplus ? softplus_fast(v) : v;
-            }
-            s = dtv * Ah;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float o = __shfl_up_sync(0xffffffffu, s, off);
-                if (lane >= off) s += o;
-            }
-            if (lane == 31) wsum[warp] = s;
-            if (u + 1 < units) dt_raw = load_dt(nxt);  // the next unit's, in flight meanwhile
-        }
-        // the next chunk's inputs go to the other buffer, whose last readers (chunk
-        // c - 1's MMAs and epilogue) have finished
-        if (tid == 0 && u + 1 < units) load(nxt, u + 1);
+        // the next chunk's inputs go to the other buffer, whose last readers (the
+        // previous unit's MMAs and epilogue 1) have finished; a warp that has no
+        // other work here issues them
+        if (tid == kSsdThreads - 1 && u + 1 < units) load(nxt, u + 1);
         if (u + 1 < units) loads_issued = u + 2;
-        __syncthreads();
-        if (tid < kSsdQ) {
-            for (int w = 0; w < warp; ++w) s += wsum[w];
-            cs[tid] = s;
-            dts[tid] = dtv;
-            Fs[tid] = __expf(-s) * dtv;
-        }
-        // exp(cs_i - cs_j) = exp(cs_i) exp(-cs_j) without overflow when every |cs| <= 80;
-        // the barrier also makes S^T (written by epilogue 2) visible to the tensor core
+        // S^T (written at the end of the previous unit) visible to the tensor core
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-        const bool factored = __syncthreads_and(tid >= kSsdQ || fabsf(s) <= 80.0f) != 0;
+        __syncthreads();
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        // ---- MMA3: Yo = C S^T (high, then low accumulated); epilogue 2 needs it
+        // ---- MMA3: Yo = C [S^T high | S^T low] (N = 128: the low tile is the
+        // operand's second 64-column atom, one tile on); epilogue 2 needs it
         if (tid == 0) {
-            constexpr uint32_t i3 = ssd_idesc(128, 64, 0, 1);
+            constexpr uint32_t i3 = ssd_idesc(128, 128, 0, 1);
             const uint64_t dC = ssd_desc(a_c, 16, 1024), dS = ssd_desc(a_s, S::kTile, 1024);
 #pragma unroll
-            for (int part = 0; part < 2; ++part)
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const uint32_t ka = ((k / 4) * S::kTile + (k % 4) * 32) >> 4;
-                    ssd_mma(tYo, dC + ka, dS + ((part * S::kTile + 2048 * k) >> 4), i3, part > 0 || k > 0);
-                }
+            for (int k = 0; k < 8; ++k) {
+                const uint32_t ka = ((k / 4) * S::kTile + (k % 4) * 32) >> 4;
+                ssd_mma(tYo, dC + ka, dS + ((2048 * k) >> 4), i3, k > 0);
+            }
             ssd_commit(mbar + 2);
         }
         committed[2] = static_cast<uint32_t>(u + 1);
@@ -499,12 +515,14 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         const float total = cs[kSsdQ - 1];
         float dx[32];  // D x of this thread's row and column half, kept for epilogue 2
+        float ecs;     // exp(cs) of this thread's row, kept for epilogue 2
         {
             // ---- epilogue 1a: row i of L o G, columns j in [64 half, 64 half + 64), 32
             // at a time: read their G, then write the high parts to the first 16 and
             // the low parts to the last 16 of the same 32 TMEM columns (two bf16 each)
             const int i = row;
             const float csi = cs[i], Ei = __expf(csi);
+            ecs = Ei;
 #pragma unroll
             for (int jp = 0; jp < 2; ++jp) {
                 const uint32_t col = tG + lane_off + 64 * half + 32 * jp;
@@ -567,39 +585,57 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
         __syncthreads();
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        // ---- MMA2: Yd = (L o G) X, A from TMEM; MMA4: ST = B^T (w o X); each high + low
-        if (tid == 0) {
-            constexpr uint32_t i2 = ssd_idesc(128, 64, 0, 1), i4 = ssd_idesc(128, 64, 1, 1);
-            const uint64_t dX = ssd_desc(a_x, S::kTile, 1024), dBt = ssd_desc(a_b, S::kTile, 1024);
-            const uint64_t dXw = ssd_desc(a_xw, S::kTile, 1024);
+        // ---- MMA2: Yd = (L o G high) X | (L o G low) X, A from TMEM, by threads 0
+        // and 64; MMA4: ST = B^T [w o X high | w o X low] (N = 128), by thread 32:
+        // three threads issue at once
+        if (tid == 0 || tid == 64) {
+            const int part = tid >> 6;
+            constexpr uint32_t i2 = ssd_idesc(128, 64, 0, 1);
+            const uint64_t dX = ssd_desc(a_x, S::kTile, 1024);
 #pragma unroll
-            for (int part = 0; part < 2; ++part)
+            for (int k = 0; k < 8; ++k) {
+                // K step k covers j in [16 k, 16 k + 16): column half k / 4, 32-column
+                // block (k % 4) / 2, high or low 16 columns, 8 columns per 16 j
+                const uint32_t acol = 64 * (k / 4) + 32 * ((k % 4) / 2) + 16 * part + 8 * (k % 2);
+                ssd_mma_ts(tYd + 64 * part, tG + acol, dX + ((2048 * k) >> 4), i2, k > 0);
+            }
+            ssd_commit(mbar + (part ? 4 : 1));
+        } else if (tid == 32) {
+            constexpr uint32_t i4 = ssd_idesc(128, 128, 1, 1);
+            const uint64_t dBt = ssd_desc(a_b, S::kTile, 1024), dXw = ssd_desc(a_xw, S::kTile, 1024);
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    // K step k covers j in [16 k, 16 k + 16): column half k / 4, 32-column
-                    // block (k % 4) / 2, high or low 16 columns, 8 columns per 16 j
-                    const uint32_t acol = 64 * (k / 4) + 32 * ((k % 4) / 2) + 16 * part + 8 * (k % 2);
-                    ssd_mma_ts(tYd, tG + acol, dX + ((2048 * k) >> 4), i2, part > 0 || k > 0);
-                }
-#pragma unroll
-            for (int part = 0; part < 2; ++part)
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    ssd_mma(tST, dBt + ((2048 * k) >> 4), dXw + ((part * S::kTile + 2048 * k) >> 4), i4,
-                            part > 0 || k > 0);
-            ssd_commit(mbar + 1);
+            for (int k = 0; k < 8; ++k)
+                ssd_mma(tST, dBt + ((2048 * k) >> 4), dXw + ((2048 * k) >> 4), i4, k > 0);
+            ssd_commit(mbar + 3);
         }
-        committed[1] = static_cast<uint32_t>(u + 1);
+        committed[1] = committed[3] = committed[4] = static_cast<uint32_t>(u + 1);
+        // ---- meanwhile the next unit's running sums (its dt loaded a unit ago)
+        if (u + 1 < units) {
+            sums_in_warp(nxt, dt_raw, nbias, nAh);
+            if (u + 2 < units && tid < kSsdQ) dt_raw = load_dt(nn);
+        }
         if (!wait_all(mbar + 1, ph)) {
             ok = false;
             break;
         }
         waited[1] = static_cast<uint32_t>(u + 1);
-        if (!wait_all(mbar + 2, ph)) {
-            ok = false;
-            break;
+        // the tables are free: epilogue 1 has read them, epilogue 2 needs none
+        const bool fac_next = u + 1 < units ? sums_across_warps() : true;
+        bool factored_next = true;
+        {
+            // the other three MMA groups, and whether every |cs| of the next unit is
+            // at most 80, in one barrier (two more only when that is not so)
+            const bool w = ssd_wait(mbar + 4, ph, p.error) && ssd_wait(mbar + 3, ph, p.error) &&
+                           ssd_wait(mbar + 2, ph, p.error);
+            if (!__syncthreads_and(w && fac_next)) {
+                factored_next = __syncthreads_and(fac_next) != 0;
+                if (!__syncthreads_and(w)) {
+                    ok = false;
+                    break;
+                }
+            }
         }
-        waited[2] = static_cast<uint32_t>(u + 1);
+        waited[2] = waited[3] = waited[4] = static_cast<uint32_t>(u + 1);
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         // ---- the next chunk's G: its inputs have landed and G's columns are read
         if (u + 1 < units) {
@@ -616,13 +652,24 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
         {
             const int i = row;
             const int64_t t = t0 + i;
-            const float ecs = __expf(cs[i]);
             uint16_t *yg = static_cast<uint16_t *>(p.y);
 #pragma unroll
             for (int q0 = 0; q0 < 32; q0 += 16) {
                 float yd[16], yo[16];
-                ssd_ld16(tYd + lane_off + 32 * half + q0, yd);
-                ssd_ld16(tYo + lane_off + 32 * half + q0, yo);
+                {
+                    float lo[16];
+                    ssd_ld16(tYo + lane_off + 32 * half + q0, yo);
+                    ssd_ld16(tYo + 64 + lane_off + 32 * half + q0, lo);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) yo[e] += lo[e];
+                }
+                {
+                    float lo[16];
+                    ssd_ld16(tYd + lane_off + 32 * half + q0, yd);
+                    ssd_ld16(tYd + 64 + lane_off + 32 * half + q0, lo);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) yd[e] += lo[e];
+                }
                 uint32_t pk[8];
 #pragma unroll
                 for (int e = 0; e < 16; e += 2)
@@ -637,10 +684,11 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
             const float et = __expf(total);
 #pragma unroll
             for (int q0 = 0; q0 < 32; q0 += 16) {
-                float v[16];
+                float v[16], lo[16];
                 ssd_ld16(tST + lane_off + 32 * half + q0, v);
+                ssd_ld16(tST + 64 + lane_off + 32 * half + q0, lo);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) st[q0 + e] = fmaf(et, st[q0 + e], v[e]);
+                for (int e = 0; e < 16; ++e) st[q0 + e] = fmaf(et, st[q0 + e], v[e] + lo[e]);
             }
         }
         // the end of a part (h_last, or the hand-off to the next CTA); the state the
@@ -654,14 +702,16 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
             write_state();
         }
         cur = nxt;
+        nxt = nn;
         Ah = nAh;
         bias = nbias;
         Dh = nDh;
+        factored = factored_next;
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     }
     // a wait that gave up leaves no load or MMA running when the CTA ends
     if (!ok && tid == 0) {
-        for (int g = 0; g < 3; ++g)
+        for (int g = 0; g < 5; ++g)
             for (uint32_t n = waited[g]; n < committed[g]; ++n) ssd_drain(mbar + g, n & 1u, p.error);
         for (int64_t c = loads_waited; c < loads_issued; ++c)
             ssd_drain(lbar + (c & 1), static_cast<uint32_t>((c >> 1) & 1), p.error);

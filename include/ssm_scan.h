@@ -251,8 +251,8 @@ int ssm_trap_scan_step(float *state, const void *x, const void *delta, const flo
  * Workspace bytes that ssm_scan_bwd needs for the shape `dims`: the scratch of
  * the forward pass that stores the checkpoints (as ssm_scan_fwd_workspace_size
  * gives it for 256 SMs; ssm_scan_fwd_status on the backward's workspace reads
- * its error word), then the states at the start of every 32-step segment (64 B
- * per channel and segment, i.e. 2 B per channel and step).  Needs no device.
+ * its error word), then the states at the start of every 16-step segment (64 B
+ * per channel and segment, i.e. 4 B per channel and step).  Needs no device.
  * Returns SSM_OK and writes *bytes, or an SSM_ERR_* code.
  */
 int ssm_scan_bwd_workspace_size(const ssm_dims_t *dims, size_t *bytes);

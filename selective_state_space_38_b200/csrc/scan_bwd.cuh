@@ -5,10 +5,9 @@
 // states; it recomputes them when the inputs are loaded into on-chip memory.
 // Here the forward scan kernel, run without output, stores only the state at
 // the start of every segment of kBwdSeg steps (a checkpoint, 64 B per channel
-// and segment); the backward
-// kernel walks each channel's segments from the last to the first, recomputes
-// a segment's states 16 steps at a time into shared memory and runs the
-// adjoint recurrence
+// and segment); the backward kernel walks each channel's segments from the
+// last to the first, recomputes a segment's states from its checkpoint into
+// shared memory, kBwdSub steps at a time, and runs the adjoint recurrence
 //   g_t = C_t dy_t + Abar_{t+1} g_{t+1}
 // backwards through them, carrying the decayed adjoint G = Abar_t g_t from
 // step to step.
@@ -31,6 +30,7 @@ namespace ssm {
 
 constexpr int kBwdSeg = kCkptSteps;  // steps between checkpoints (stored by the forward kernel)
 constexpr int kBwdSub = 16;   // steps recomputed and run backwards at a time
+static_assert(kBwdSeg % kBwdSub == 0 && kBwdSeg <= 2 * kBwdSub, "one or two sub-chunks per segment");
 
 struct BwdParams {
     const void *x, *delta, *z, *B, *C, *dout;
@@ -418,7 +418,7 @@ __global__ void __launch_bounds__(32) scan_bwd_kernel(const BwdParams p) {
         // only, for the second one's start state, (1) the second one forward and back;
         // then (2) the first one forward from the checkpoint and back.  One call site
         // each keeps the kernel's code small.
-        const bool two = ts + kBwdSub < L;
+        const bool two = kBwdSeg > kBwdSub && ts + kBwdSub < L;
 #pragma unroll 1
         for (int q = two ? 0 : 2; q < 3; ++q) {
             if (q != 1) {

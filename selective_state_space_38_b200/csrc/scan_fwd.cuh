@@ -39,7 +39,7 @@
 
 namespace ssm {
 
-constexpr int kCkptSteps = 32;  // spacing of the states a checkpoint pass stores
+constexpr int kCkptSteps = 16;  // spacing of the states a checkpoint pass stores
 
 struct FwdParams {
     const void *x, *delta, *z, *B, *C;
@@ -474,6 +474,32 @@ __device__ __forceinline__ void chunk_core(const float *bcf, const float2 *ur, u
     }
 }
 
+// The state update alone, without the readout (no C, no y), for a launch with
+// no output: the backward entry's checkpoint pass.  With mid set, the state
+// before the chunk's step kCkptSteps goes there as well.
+template <bool S4D, bool FULL>
+__device__ __forceinline__ void chunk_states(const float *bcf, const float2 *ur, int row, int nvalid,
+                                             const float (&a2)[kNState], float2 (&h)[8], float4 *mid) {
+    StepOps nxt;
+    prepare_step<S4D, false>(bcf, ur, 0, row, a2, nxt);
+#pragma unroll 1
+    for (int t0 = 0; t0 < nvalid; t0 += 8) {
+        if (t0 == kCkptSteps && mid) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) mid[q] = make_float4(h[2 * q].x, h[2 * q].y, h[2 * q + 1].x, h[2 * q + 1].y);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int t = t0 + i;
+            if (!FULL && t >= nvalid) break;
+            const StepOps cur = nxt;
+            if (FULL || t + 1 < nvalid) prepare_step<S4D, false>(bcf, ur, t + 1, row, a2, nxt);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) h[j] = __ffma2_rn(cur.a[j], h[j], cur.ub[j]);
+        }
+    }
+}
+
 // The summary pass of the time-parallel schedule: the same state update, with
 // the running product of the per-step decays P_n = prod_t Abar_{t,n} in place
 // of the readout (so P carries the rounding of the decays the sequential scan
@@ -798,9 +824,10 @@ struct ChunkCursor {
 // sub-partition.  Two instances run back to back: the S4D one takes groups
 // whose A rows are all S4D-structured and marks the scratch when it meets
 // another group; the general one then takes those.
-template <typename T, bool VEC, bool S4D, bool CONV, bool TRAP>
+template <typename T, bool VEC, bool S4D, bool CONV, bool TRAP, bool STATES = false>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     scan_fwd_kernel(const FwdParams p, const FwdScratch sc, const __grid_constant__ TmaMaps tm) {
+    static_assert(!STATES || (!CONV && !TRAP), "the states-only instance is the plain scan's");
     extern __shared__ __align__(128) uint8_t smem_raw[];
     // 1 KB alignment keeps every tile on a whole period of the 64-byte swizzle.  The
     // offset is added to the shared-memory pointer itself (no round trip through an
@@ -1079,6 +1106,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     chunk_summary<S4D, true, TRAP>(bcf_of(k), ur_of(k), lane, TC, a2, h, P);
                 else
                     chunk_summary<S4D, false, TRAP>(bcf_of(k), ur_of(k), lane, dk.nvalid, a2, h, P);
+            } else if constexpr (STATES) {
+                // no output: the states alone, and the checkpoint inside the chunk
+                float4 *mid = nullptr;
+                if (TC > kCkptSteps && p.ckpt && active)
+                    mid = reinterpret_cast<float4 *>(
+                        p.ckpt + ((dk.b * p.dim + d) * p.ckpt_segs + dk.t0 / kCkptSteps + 1) * kNState);
+                if (dk.nvalid == TC)
+                    chunk_states<S4D, true>(bcf_of(k), ur_of(k), lane, TC, a2, h, mid);
+                else
+                    chunk_states<S4D, false>(bcf_of(k), ur_of(k), lane, dk.nvalid, a2, h, mid);
             } else if (dk.nvalid == TC) {
                 chunk_core<S4D, true, TRAP, !kPrepLoads>(bcf_of(k), ur_of(k), stage_of(k), lane, TC, a2, h, g_of(k));
             } else {

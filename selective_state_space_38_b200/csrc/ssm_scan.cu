@@ -129,28 +129,31 @@ int64_t parallel_segments(const FwdParams &p, int sms, int64_t *seg_steps) {
 
 // Persistent launch: one CTA of kPairs warp triples per SM (or fewer when there
 // are fewer items); the S4D instance, then the general one.
-template <typename T, bool VEC, bool CONV, bool TRAP>
+template <typename T, bool VEC, bool CONV, bool TRAP, bool STATES>
 int launch_pass(const FwdParams &p, const FwdScratch &sc, const TmaMaps &tm, int sms, cudaStream_t stream) {
     const int64_t groups = ((p.dim + 31) / 32) * p.batch;
     const int64_t items = groups * ((p.seqlen + p.seg_steps - 1) / p.seg_steps);
     const int64_t want = (items + kPairs - 1) / kPairs;
     const int64_t ctas = want < sms ? want : sms;
     const int smem = FwdSmem<T, TRAP, CONV>::kTotal;
-    scan_fwd_kernel<T, VEC, true, CONV, TRAP><<<static_cast<unsigned>(ctas), kFwdThreads, smem, stream>>>(p, sc, tm);
-    scan_fwd_kernel<T, VEC, false, CONV, TRAP><<<static_cast<unsigned>(ctas), kFwdThreads, smem, stream>>>(p, sc, tm);
+    scan_fwd_kernel<T, VEC, true, CONV, TRAP, STATES>
+        <<<static_cast<unsigned>(ctas), kFwdThreads, smem, stream>>>(p, sc, tm);
+    scan_fwd_kernel<T, VEC, false, CONV, TRAP, STATES>
+        <<<static_cast<unsigned>(ctas), kFwdThreads, smem, stream>>>(p, sc, tm);
     return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
 // The kernels of one forward call on zeroed scratch: one chained pass, or the
 // summary pass, the segment combine and the second pass of the time-parallel
-// schedule (the queue is re-armed between the passes).
-template <typename T, bool VEC, bool CONV, bool TRAP>
+// schedule (the queue is re-armed between the passes).  STATES: the instances
+// for a call with no output (the backward entry's checkpoint pass).
+template <typename T, bool VEC, bool CONV, bool TRAP, bool STATES>
 int launch_fwd_kernels(FwdParams p, void *scratch, int64_t segs, int sms, cudaStream_t stream) {
     const int64_t groups = ((p.dim + 31) / 32) * p.batch;
     const int smem = FwdSmem<T, TRAP, CONV>::kTotal;
-    if (cudaFuncSetAttribute(scan_fwd_kernel<T, VEC, true, CONV, TRAP>,
+    if (cudaFuncSetAttribute(scan_fwd_kernel<T, VEC, true, CONV, TRAP, STATES>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
-        cudaFuncSetAttribute(scan_fwd_kernel<T, VEC, false, CONV, TRAP>,
+        cudaFuncSetAttribute(scan_fwd_kernel<T, VEC, false, CONV, TRAP, STATES>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return SSM_ERR_CUDA;
     TmaMaps tm;
@@ -161,11 +164,11 @@ int launch_fwd_kernels(FwdParams p, void *scratch, int64_t segs, int sms, cudaSt
         p.mode = kChained;
         p.pass = 0;
         p.seg_steps = kSegSteps;
-        return launch_pass<T, VEC, CONV, TRAP>(p, sc, tm, sms, stream);
+        return launch_pass<T, VEC, CONV, TRAP, STATES>(p, sc, tm, sms, stream);
     }
     p.mode = kSummary;
     p.pass = 0;
-    int rc = launch_pass<T, VEC, CONV, TRAP>(p, sc, tm, sms, stream);
+    int rc = launch_pass<T, VEC, CONV, TRAP, STATES>(p, sc, tm, sms, stream);
     if (rc != SSM_OK) return rc;
     const int64_t threads = groups * 32;
     segment_combine_kernel<<<static_cast<unsigned>((threads + 127) / 128), 128, 0, stream>>>(p, sc);
@@ -173,7 +176,7 @@ int launch_fwd_kernels(FwdParams p, void *scratch, int64_t segs, int sms, cudaSt
     // first pass stays set for the status query
     p.mode = kFromStart;
     p.pass = 1;
-    return launch_pass<T, VEC, CONV, TRAP>(p, sc, tm, sms, stream);
+    return launch_pass<T, VEC, CONV, TRAP, STATES>(p, sc, tm, sms, stream);
 }
 
 // SMs of the current device (the schedule, and so the workspace size, depend on it)
@@ -194,13 +197,13 @@ size_t fwd_workspace_bytes(const FwdParams &p, int sms) {
 }
 
 // One forward call on the caller's workspace: zero its flag words, then the kernels.
-template <typename T, bool VEC, bool CONV, bool TRAP = false>
+template <typename T, bool VEC, bool CONV, bool TRAP = false, bool STATES = false>
 int launch_fwd(FwdParams p, void *ws, size_t ws_bytes, int sms, bool force_chained, cudaStream_t stream) {
     const int64_t groups = ((p.dim + 31) / 32) * p.batch;
     const int64_t segs = force_chained ? 0 : parallel_segments(p, sms, &p.seg_steps);
     if (ws_bytes < fwd_scratch_bytes(groups, segs)) return SSM_ERR_INVALID_ARG;
     if (cudaMemsetAsync(ws, 0, fwd_scratch_flag_bytes(groups), stream) != cudaSuccess) return SSM_ERR_CUDA;
-    return launch_fwd_kernels<T, VEC, CONV, TRAP>(p, ws, segs, sms, stream);
+    return launch_fwd_kernels<T, VEC, CONV, TRAP, STATES>(p, ws, segs, sms, stream);
 }
 
 // The convolution in front of the scan, when a forward call has one.
@@ -414,6 +417,11 @@ int dispatch_fwd(const FwdParams &p, size_t es, int act_dtype, void *ws, size_t 
                          : launch_fwd<bf16raw, false, false, true>(p, ws, ws_bytes, sms, force_chained, s))
                   : (vec ? launch_fwd<float, true, false, true>(p, ws, ws_bytes, sms, force_chained, s)
                          : launch_fwd<float, false, false, true>(p, ws, ws_bytes, sms, force_chained, s));
+    if (!p.out)  // the states alone (the backward entry's checkpoint pass)
+        return bf ? (vec ? launch_fwd<bf16raw, true, false, false, true>(p, ws, ws_bytes, sms, force_chained, s)
+                         : launch_fwd<bf16raw, false, false, false, true>(p, ws, ws_bytes, sms, force_chained, s))
+                  : (vec ? launch_fwd<float, true, false, false, true>(p, ws, ws_bytes, sms, force_chained, s)
+                         : launch_fwd<float, false, false, false, true>(p, ws, ws_bytes, sms, force_chained, s));
     return bf ? (vec ? launch_fwd<bf16raw, true, false>(p, ws, ws_bytes, sms, force_chained, s)
                      : launch_fwd<bf16raw, false, false>(p, ws, ws_bytes, sms, force_chained, s))
               : (vec ? launch_fwd<float, true, false>(p, ws, ws_bytes, sms, force_chained, s)
@@ -640,7 +648,7 @@ int ssm_scan_bwd(const void *x, const void *delta, const float *delta_bias, int 
     p.batch = batch; p.seqlen = L; p.dim = dim; p.softplus = softplus ? 1 : 0;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     // the checkpoints: the forward scan with no output, storing its state every
-    // 32 steps (its scratch at the start of the workspace)
+    // kCkptSteps steps (its scratch at the start of the workspace)
     FwdParams f = bwd_ckpt_params(batch, L, dim);
     f.x = x; f.delta = delta; f.B = B; f.C = C;
     f.delta_bias = delta_bias; f.A = A; f.h0 = h0;

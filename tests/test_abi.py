@@ -247,10 +247,10 @@ def test_bwd_rejects_bad_arguments(lib):
     need = ctypes.c_size_t(0)
     assert lib.ssm_scan_bwd_workspace_size(_dims(m), ctypes.byref(need)) == 0
     # the checkpoint pass's forward scratch (sized for 256 SMs), then one 64-byte
-    # state per channel and 32-step segment
+    # state per channel and 16-step segment
     fwd = ctypes.c_size_t(0)
     assert lib.ssm_scan_fwd_workspace_size(_dims(m), 256, ctypes.byref(fwd)) == 0
-    segments = -(-64 // 32)
+    segments = -(-64 // 16)
     assert need.value == (fwd.value + 255) // 256 * 256 + (2 * 128 * segments * 16 * 4 + 255) // 256 * 256
 
     def bwd(**over):

@@ -262,7 +262,7 @@ int ssm_scan_bwd_workspace_size(const ssm_dims_t *dims, size_t *bytes);
  * every input, given dout = dL/dout and dh_last = dL/dh_last.  As Appendix D
  * "Memory" describes, the intermediate states are not stored by the forward
  * pass: the call first runs the forward scan without output, storing the state
- * at the start of every 32-step segment, and recomputes each segment's states
+ * at the start of every 16-step segment, and recomputes each segment's states
  * from it while it runs the adjoint recurrence
  *   g_t = C_t dy_t + Abar_{t+1} g_{t+1},  dy_t = dout_t silu(z_t)
  * backwards through the chunk.

@@ -430,7 +430,7 @@ int dispatch_fwd(const FwdParams &p, size_t es, int act_dtype, void *ws, size_t 
 
 // Workspace of the backward pass: first the scratch of the forward pass that
 // stores the checkpoints (so ssm_scan_fwd_status reads its error word), then
-// the states at every segment start (64 B per channel and segment of 32 steps).
+// the states at every segment start (64 B per channel and segment of kCkptSteps steps).
 FwdParams bwd_ckpt_params(int64_t batch, int64_t L, int64_t dim) {
     FwdParams f;
     memset(&f, 0, sizeof f);

@@ -22,11 +22,15 @@
 //   MMA2 Yd = (L o G) X (128 x 64 x 128) and MMA4 ST = B^T (w o X) (128 x 64 x 128);
 //   epilogue 2 writes y and updates the state.
 // Operands are bf16 in the 128-byte-swizzled canonical layouts; the ones that
-// are products (L o G, w o X, S) are split into a bf16 high part and a low part
-// (two MMAs each), so they keep about 16 bits.  C, B and X arrive by TMA into
-// one of two buffers, the next chunk's while this one is computed.  One thread
-// issues the MMAs; tcgen05.commit arrives on an mbarrier that every thread
-// waits on (bounded); each thread reads its TMEM lane with tcgen05.ld.
+// are products (L o G, w o X, S) are split into a bf16 high part and a low part,
+// so they keep about 16 bits: the two parts of S^T and of w o X form one N = 128
+// operand (the low tile is its second 64-column atom), L o G's two parts two
+// MMAs, and each product's halves land side by side in TMEM and are added in
+// the epilogue.  C, B and X arrive by TMA into one of two buffers, the next
+// chunk's while this one is computed.  Single threads issue the MMAs (MMA2's
+// halves and MMA4 from three threads at once); tcgen05.commit arrives on one
+// mbarrier per MMA group that every thread waits on (bounded); each thread reads
+// its TMEM lane with tcgen05.ld.
 #pragma once
 
 #include <cuda.h>

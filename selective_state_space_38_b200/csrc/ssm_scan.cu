@@ -224,8 +224,7 @@ struct TrapArgs {
 
 template <typename T, bool CONV, bool TRAP = false>
 int launch_step(const StepParams &p, cudaStream_t stream) {
-    const int64_t threads = p.batch * p.dim * 4;
-    const int64_t blocks = (threads + kStepThreads - 1) / kStepThreads;
+    const int64_t blocks = (p.batch * p.dim + kStepTile - 1) / kStepTile;
     if (blocks > INT_MAX) return SSM_ERR_UNSUPPORTED;
     if (p.batch * p.dim < (int64_t(1) << 31))
         scan_step_kernel<T, true, CONV, TRAP><<<static_cast<unsigned>(blocks), kStepThreads, 0, stream>>>(p);

@@ -96,12 +96,11 @@ __global__ void __launch_bounds__(kStepThreads) scan_step_kernel(const StepParam
         const int64_t c = chan < nchan ? chan : nchan - 1;
         step_copy16(&hs[k][tid], p.state + c * kNState + q * 4, chan < nchan ? 16u : 0u);
     }
-#pragma unroll
-    for (int k = 0; k < kStepPasses; ++k) {
-        const int64_t chan = base + k * (kStepThreads / 4);
-        const bool active = chan < nchan;
-        const int64_t c = active ? chan : nchan - 1;  // inactive lanes still join the shuffles
-        int64_t b, d;
+    // (b, d) of the first pass's channel by one division; the later passes' by
+    // stepping kStepThreads / 4 channels on (inactive lanes keep the last channel)
+    int64_t b, d;
+    {
+        const int64_t c = base < nchan ? base : nchan - 1;
         if constexpr (SMALL) {
             const uint32_t c32 = static_cast<uint32_t>(c), dim32 = static_cast<uint32_t>(p.dim);
             b = c32 / dim32;
@@ -109,6 +108,24 @@ __global__ void __launch_bounds__(kStepThreads) scan_step_kernel(const StepParam
         } else {
             b = c / p.dim;
             d = c % p.dim;
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < kStepPasses; ++k) {
+        const int64_t chan = base + k * (kStepThreads / 4);
+        const bool active = chan < nchan;
+        const int64_t c = active ? chan : nchan - 1;  // inactive lanes still join the shuffles
+        if (k > 0) {
+            if (active) {
+                d += kStepThreads / 4;
+                while (d >= p.dim) {  // once at most when dim >= kStepThreads / 4
+                    d -= p.dim;
+                    ++b;
+                }
+            } else {
+                b = (nchan - 1) / p.dim;
+                d = (nchan - 1) - b * p.dim;
+            }
         }
         const float4 a = *reinterpret_cast<const float4 *>(p.A + d * kNState + q * 4);
         float xf = AT::load(p.x, c);

@@ -372,6 +372,21 @@ int ssm_debug_fwd_flag_timeout(const void *x, const void *delta, const float *de
                                void *workspace, size_t workspace_bytes, uint32_t spin_limit,
                                const ssm_dims_t *dims, ssm_stream_t stream);
 
+/*
+ * Test support, not part of the operation: ssm_ssd_fwd where every CTA that
+ * continues a sequence split between two CTAs waits for a hand-off flag value
+ * that no flag ever reaches and gives up after `spin_limit` polls (0: at
+ * once).  Only a call that splits sequences (more sequences than SMs, and a
+ * workspace of ssm_ssd_fwd_workspace_size bytes) waits at all.  The kernel
+ * still ends normally; ssm_scan_fwd_status then reports SSM_ERR_TIMEOUT.
+ * Arguments as for ssm_ssd_fwd.
+ */
+int ssm_debug_ssd_flag_timeout(const void *x, const void *dt, const float *dt_bias, int softplus,
+                               const float *A, const void *B, const void *C, const float *D,
+                               const float *h0, void *y, float *h_last, void *workspace,
+                               size_t workspace_bytes, uint32_t spin_limit, const ssm_ssd_dims_t *dims,
+                               ssm_stream_t stream);
+
 /* Static, human-readable text for an SSM_* code (never NULL). */
 const char *ssm_strerror(int code);
 

@@ -73,6 +73,9 @@ def _load():
     lib.ssm_ssd_fwd_workspace_size.argtypes = [ctypes.POINTER(SsdDims), I, ctypes.POINTER(S)]
     lib.ssm_ssd_fwd_workspace_size.restype = I
     lib.ssm_ssd_fwd.argtypes = [P, P, P, I, P, P, P, P, P, P, P, P, S, ctypes.POINTER(SsdDims), P]
+    lib.ssm_debug_ssd_flag_timeout.argtypes = [P, P, P, I, P, P, P, P, P, P, P, P, S, ctypes.c_uint32,
+                                               ctypes.POINTER(SsdDims), P]
+    lib.ssm_debug_ssd_flag_timeout.restype = I
     lib.ssm_ssd_fwd.restype = I
     lib.ssm_scan_step.argtypes = [P, P, P, P, I, P, P, P, P, P, P, DP, P]
     lib.ssm_scan_step.restype = I
@@ -98,7 +101,7 @@ EXPORTS = ("ssm_scan_fwd_workspace_size", "ssm_scan_fwd", "ssm_scan_fwd_status",
            "ssm_conv_scan_fwd", "ssm_conv_scan_step", "ssm_trap_scan_fwd", "ssm_trap_scan_step",
            "ssm_scan_bwd_workspace_size", "ssm_scan_bwd", "ssm_ssd_fwd_workspace_size", "ssm_ssd_fwd",
            "ssm_scan_fwd_noalloc",
-           "ssm_debug_fwd_flag_timeout",
+           "ssm_debug_fwd_flag_timeout", "ssm_debug_ssd_flag_timeout",
            "ssm_strerror", "ssm_version")
 
 

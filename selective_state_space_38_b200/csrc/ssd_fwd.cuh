@@ -64,6 +64,8 @@ struct SsdParams {
     float *slots;
     int64_t batch, seqlen, heads, groups;
     int64_t units_per_cta;       // chunks a CTA walks (the chunk count of a sequence without splits)
+    uint32_t flag_want;          // a hand-off flag is set when it reaches this (1; larger: test support)
+    uint32_t spin_limit;         // polls of a hand-off flag before the wait gives up
     int softplus;
 };
 
@@ -342,8 +344,8 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
         if (tid == 0) {
             got = false;
             const uint32_t *flag = p.flags + (kcta - 1);
-            for (uint32_t n = 0; n < kSsdFlagLimit; ++n) {
-                if (ld_acquire(flag) != 0) {
+            for (uint32_t n = 0; n < p.spin_limit; ++n) {
+                if (ld_acquire(flag) >= p.flag_want) {
                     got = true;
                     break;
                 }

@@ -679,9 +679,11 @@ int ssm_ssd_fwd_workspace_size(const ssm_ssd_dims_t *dims, int sm_count, size_t 
     return SSM_OK;
 }
 
-int ssm_ssd_fwd(const void *x, const void *dt, const float *dt_bias, int softplus, const float *A, const void *B,
-                const void *C, const float *D, const float *h0, void *y, float *h_last, void *workspace,
-                size_t workspace_bytes, const ssm_ssd_dims_t *dims, ssm_stream_t stream) {
+// ssm_ssd_fwd with the hand-off flag value and the poll bound of the waits
+static int ssd_fwd_impl(const void *x, const void *dt, const float *dt_bias, int softplus, const float *A,
+                        const void *B, const void *C, const float *D, const float *h0, void *y, float *h_last,
+                        void *workspace, size_t workspace_bytes, const ssm_ssd_dims_t *dims, ssm_stream_t stream,
+                        uint32_t flag_want, uint32_t spin_limit) {
     if (!dims || !x || !dt || !A || !B || !C || !y || !workspace) return SSM_ERR_INVALID_ARG;
     const int64_t batch = dims->batch, L = dims->seqlen, H = dims->heads, P = dims->headdim, G = dims->groups,
                   N = dims->dstate;
@@ -729,6 +731,8 @@ int ssm_ssd_fwd(const void *x, const void *dt, const float *dt_bias, int softplu
     prm.flags = ctas ? reinterpret_cast<uint32_t *>(wb + kSsdFlagOff) : nullptr;
     prm.slots = ctas ? reinterpret_cast<float *>(wb + kSsdSlotOff) : nullptr;
     prm.units_per_cta = per_cta;
+    prm.flag_want = flag_want;
+    prm.spin_limit = spin_limit;
     prm.dt = dt;
     prm.dt_bias = dt_bias; prm.A = A; prm.D = D; prm.h0 = h0;
     prm.y = y; prm.h_last = h_last;
@@ -747,6 +751,21 @@ int ssm_ssd_fwd(const void *x, const void *dt, const float *dt_bias, int softplu
         return SSM_ERR_CUDA;
     ssd_fwd_kernel<<<static_cast<unsigned>(ctas ? ctas : nseq), kSsdThreads, smem, s>>>(prm, tm);
     return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+int ssm_ssd_fwd(const void *x, const void *dt, const float *dt_bias, int softplus, const float *A, const void *B,
+                const void *C, const float *D, const float *h0, void *y, float *h_last, void *workspace,
+                size_t workspace_bytes, const ssm_ssd_dims_t *dims, ssm_stream_t stream) {
+    return ssd_fwd_impl(x, dt, dt_bias, softplus, A, B, C, D, h0, y, h_last, workspace, workspace_bytes, dims,
+                        stream, 1u, kSsdFlagLimit);
+}
+
+int ssm_debug_ssd_flag_timeout(const void *x, const void *dt, const float *dt_bias, int softplus, const float *A,
+                               const void *B, const void *C, const float *D, const float *h0, void *y,
+                               float *h_last, void *workspace, size_t workspace_bytes, uint32_t spin_limit,
+                               const ssm_ssd_dims_t *dims, ssm_stream_t stream) {
+    return ssd_fwd_impl(x, dt, dt_bias, softplus, A, B, C, D, h0, y, h_last, workspace, workspace_bytes, dims,
+                        stream, 1u << 30, spin_limit);  // no hand-off flag ever reaches this
 }
 
 int ssm_conv_scan_step(void *conv_state, float *state, const void *x, const float *conv_w,

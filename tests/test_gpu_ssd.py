@@ -119,3 +119,38 @@ def test_split_sequences(orc, L):
     # a chunk's arithmetic does not depend on which CTA runs it, and the handed-on
     # state is the float32 state itself: both launches agree bit for bit
     assert torch.equal(got[0][0], got[1][0]) and torch.equal(got[0][1], got[1][1])
+
+
+@pytest.mark.parametrize("spin_limit", [0, 2000])
+def test_handoff_wait_timeout_is_reported(orc, spin_limit):
+    """A hand-off wait of the split launch that gives up is reported, and the
+    kernel still ends.  The test entry point makes every CTA that continues a
+    split sequence wait for a flag value that nothing writes; with a bound of
+    0 (or 2000 polls) the wait gives up, the status call returns
+    SSM_ERR_TIMEOUT, and the next ordinary call on the same workspace is
+    correct and reports success."""
+    import ctypes
+    import selective_state_space_38_b200 as ssm
+    if torch.cuda.get_device_properties(0).multi_processor_count >= 3 * 64:
+        pytest.skip("the launch splits sequences only with more sequences than SMs")
+    lib = ssm.get_lib()
+    inp = ssd_inputs(3, 300, 64, 2, seed=51, h0=True)
+    t = {k: to_dev(v) for k, v in inp.items() if isinstance(v, np.ndarray)}
+    ws = torch.empty(ssm.ssm_ssd_fwd_workspace_size(3, 64, t["x"].device), dtype=torch.uint8, device="cuda")
+    y = torch.empty_like(t["x"])
+    hl = torch.empty(t["h0"].shape, dtype=torch.float32, device="cuda")
+    dims = ssm.SsdDims(3, 300, 64, 64, 2, 128, ssm.SSM_BF16)
+    stream = torch.cuda.current_stream()
+    rc = lib.ssm_debug_ssd_flag_timeout(
+        t["x"].data_ptr(), t["dt"].data_ptr(), t["dt_bias"].data_ptr(), 1, t["A"].data_ptr(), t["B"].data_ptr(),
+        t["C"].data_ptr(), t["D"].data_ptr(), t["h0"].data_ptr(), y.data_ptr(), hl.data_ptr(), ws.data_ptr(),
+        ws.numel(), spin_limit, ctypes.byref(dims), stream.cuda_stream)
+    assert rc == 0, ssm.ssm_strerror(rc)
+    assert ssm.ssm_scan_fwd_status(ws, stream) == 5
+    torch.cuda.synchronize()  # the context is still usable
+    y2, hl2 = ssm.ssm_ssd_fwd(t["x"], t["dt"], t["dt_bias"], True, t["A"], t["B"], t["C"], t["D"], t["h0"],
+                              workspace=ws, check=True)
+    torch.cuda.synchronize()
+    ry, rh = _ref(orc, inp)
+    check(to_np64(y2), ry, "bf16", "ssd y after a timed-out call")
+    check(to_np64(hl2), rh, "bf16", "ssd h_last after a timed-out call")

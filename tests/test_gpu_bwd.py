@@ -42,7 +42,9 @@ def _run(orc, inp, what):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("L", [1, 7, 128, 129, 300, 1000])
+# 17, 48, 49: a last chunk of 17, 16 and 17 steps around the checkpoint inside a
+# 32-step chunk (bf16), and segments of one step
+@pytest.mark.parametrize("L", [1, 7, 17, 48, 49, 128, 129, 300, 1000])
 def test_small_shapes(orc, dtype, L):
     """Ragged chunks (L not a multiple of 128) and a ragged channel block (70
     channels = 2 blocks of 32 + 6)."""

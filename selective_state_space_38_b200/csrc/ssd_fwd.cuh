@@ -42,7 +42,8 @@ namespace ssm {
 constexpr int kSsdQ = 128;  // chunk length
 constexpr int kSsdP = 64;   // head dimension
 constexpr int kSsdN = 128;  // state dimension
-constexpr int kSsdThreads = 256;
+constexpr int kSsdConsumers = 256;               // epilogue threads (8 warps)
+constexpr int kSsdThreads = kSsdConsumers + 32;  // + the producer warp
 constexpr uint32_t kSsdWaitLimit = 1u << 24;
 constexpr uint32_t kSsdFlagLimit = 1u << 20;  // polls of a hand-off flag, 64 ns apart at least
 
@@ -266,10 +267,32 @@ __device__ __forceinline__ void split_pair(float a, float b, uint32_t &hi, uint3
     lo = pack_bf16x2(a - __uint_as_float(hi << 16), b - __uint_as_float(hi & 0xffff0000u));
 }
 
-// grid: one CTA per range of units (SsdRange); block: 256 threads.  Thread
-// (quad, half, lane) owns row 32 quad + lane of every [128][..] tile (its TMEM
-// lane) and the half `half` of that row's columns.
-__global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams p, const __grid_constant__ SsdMaps tm) {
+// Barrier 1 among the kSsdConsumers epilogue threads (the producer warp is not
+// part of it): a plain sync, and one that returns the AND of a predicate.
+__device__ __forceinline__ void ssd_cbar() { asm volatile("bar.sync 1, %0;" ::"n"(kSsdConsumers) : "memory"); }
+__device__ __forceinline__ bool ssd_cbar_and(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbarrier.cta.red.and.pred q, 1, %2, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(v)), "n"(kSsdConsumers)
+        : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ void ssd_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// grid: one CTA per range of units (SsdRange); block: kSsdConsumers epilogue
+// threads and one producer warp.  Epilogue thread (quad, half, lane) owns row
+// 32 quad + lane of every [128][..] tile (its TMEM lane) and the half `half` of
+// that row's columns.  One lane of the producer warp issues every TMA load and
+// every MMA; the epilogue threads hand it their results through two mbarriers
+// (epilogue 1 done; the next unit's S^T in shared memory) and wait for its
+// commits, so no epilogue thread is held while the tensor core takes an MMA.
+__global__ void __launch_bounds__(kSsdThreads, 1)
+    ssd_fwd_kernel(const SsdParams p, const __grid_constant__ SsdMaps tm) {
     extern __shared__ __align__(1024) uint8_t ssd_smem_raw[];
     uint8_t *sm = ssd_smem_raw + ((1024u - (smem_u32(ssd_smem_raw) & 1023u)) & 1023u);
     using S = SsdSmem;
@@ -278,17 +301,21 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
     float *Fs = dts + 128;  // F_j = exp(-cs_j) dt_j, when every |cs| of the chunk is at most 80
     float *wsum = Fs + 128;
     uint64_t *lbar = reinterpret_cast<uint64_t *>(sm + S::kBar);  // [2] input buffer landed
-    uint64_t *mbar = lbar + 2;  // [0] MMA1 (G), [1] MMA2 high, [2] MMA3 (Yo), [3] MMA4 (ST), [4] MMA2 low done
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(mbar + 5);
+    uint64_t *mG = lbar + 2, *mYo = lbar + 3, *m24 = lbar + 4;    // MMA1; MMA3; MMA2 and MMA4 done
+    uint64_t *cE1 = lbar + 5, *cS = lbar + 6;  // epilogue 1 done; S^T of a unit ready (kSsdConsumers arrivals)
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(lbar + 7);
     uint32_t *korder = tslot + 1;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, half = warp >> 2;
+    const bool producer = tid >= kSsdConsumers;
+    const int quad = warp & 3, half = (warp >> 2) & 1;
     const int row = quad * 32 + lane;
     const int64_t L = p.seqlen, H = p.heads, per_group = p.heads / p.groups;
     const int64_t chunks = (L + kSsdQ - 1) / kSsdQ;
 
     if (tid == 0) {
-        for (int i = 0; i < 7; ++i) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(lbar + i)));
+        for (int i = 0; i < 5; ++i) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(lbar + i)));
+        for (int i = 5; i < 7; ++i)
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(lbar + i)), "n"(kSsdConsumers));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         // with split sequences a CTA's range is its place in the order of start
         *korder = p.order ? atomicAdd(p.order, 1u) : blockIdx.x;
@@ -304,223 +331,303 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
     const int64_t kcta = *reinterpret_cast<volatile uint32_t *>(korder);
     const SsdRange rg(kcta, p.units_per_cta, p.batch * H, chunks, H, per_group);
     const int64_t units = rg.units();
-    // TMEM columns: G then L o G (128); Yd (128: the products of the high and of
-    // the low part of L o G side by side); Yo (128: the same for S^T); ST (128:
-    // the same for w o X)
-    const uint32_t tG = tbase, tYd = tbase + 128, tYo = tbase + 256, tST = tbase + 384;
-    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-
-    // the inputs of unit u (x) into buffer u & 1 (one thread)
-    auto load = [&](const SsdUnit &x, int64_t u) {
-        uint8_t *in = sm + (u & 1) * S::kInBytes;
-        uint64_t *bar = lbar + (u & 1);
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_arrive_expect_tx(bar, S::kInBytes);
-        const int t0 = static_cast<int>(x.c * kSsdQ), bi = static_cast<int>(x.b), gi = static_cast<int>(x.g);
-        tma_load_4d(in + S::kInC, &tm.C, 0, gi, t0, bi, bar);
-        tma_load_4d(in + S::kInC + S::kTile, &tm.C, 64, gi, t0, bi, bar);
-        tma_load_4d(in + S::kInB, &tm.B, 0, gi, t0, bi, bar);
-        tma_load_4d(in + S::kInB + S::kTile, &tm.B, 64, gi, t0, bi, bar);
-        tma_load_4d(in + S::kInX, &tm.x, 0, static_cast<int>(x.h), t0, bi, bar);
-    };
-    // raw dt of this thread's step of unit x (zero past the end)
-    auto load_dt = [&](const SsdUnit &x) -> float {
-        const int64_t t = x.c * kSsdQ + tid;
-        return t < L ? Act<bf16raw>::load(p.dt, (x.b * L + t) * H + x.h) : 0.0f;
-    };
-
-    // this thread's share of the state: S[p][n] for n = row, p in [32 half, 32 half + 32)
-    float st[32];
-    // the state a part starts from: h0 (or zero) at a sequence start, else the
-    // one the previous CTA handed on (a bounded wait on its flag)
-    auto begin_part = [&](int64_t seq, int64_t c) -> bool {
-        if (c == 0) {
-#pragma unroll
-            for (int q = 0; q < 32; ++q)
-                st[q] = p.h0 ? p.h0[(seq * kSsdP + 32 * half + q) * kSsdN + row] : 0.0f;
-            return true;
-        }
-        bool got = true;
-        if (tid == 0) {
-            got = false;
-            const uint32_t *flag = p.flags + (kcta - 1);
-            for (uint32_t n = 0; n < p.spin_limit; ++n) {
-                if (ld_acquire(flag) >= p.flag_want) {
-                    got = true;
-                    break;
-                }
-                if ((n & 255u) == 255u && *reinterpret_cast<volatile uint32_t *>(p.error) != 0) break;
-                __nanosleep(64);
-            }
-            if (!got && *reinterpret_cast<volatile uint32_t *>(p.error) == 0) atomicOr(p.error, 2u);
-        }
-        if (!__syncthreads_and(got)) return false;
-        const float *src = p.slots + (kcta - 1) * (kSsdP * kSsdN);
-#pragma unroll
-        for (int q = 0; q < 32; ++q) st[q] = __ldcg(src + (32 * half + q) * kSsdN + row);
-        return true;
-    };
-    // the state at the end of a part: h_last at a sequence end, else to this
-    // CTA's hand-off slot, then its flag (release)
-    auto end_part = [&](int64_t seq, bool handoff) {
-        if (handoff) {
-            float *dst = p.slots + kcta * (kSsdP * kSsdN);
-#pragma unroll
-            for (int q = 0; q < 32; ++q) dst[(32 * half + q) * kSsdN + row] = st[q];
-            __syncthreads();
-            if (tid == 0) {
-                __threadfence();
-                st_release(p.flags + kcta, 1u);
-            }
-        } else if (p.h_last) {
-#pragma unroll
-            for (int q = 0; q < 32; ++q) p.h_last[(seq * kSsdP + 32 * half + q) * kSsdN + row] = st[q];
-        }
-    };
-    // S^T [n][p] as bf16 high and low tiles (the B operand of MMA3, N = p contiguous)
-    auto write_state = [&]() {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            uint32_t hi[4], lo[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) split_pair(st[8 * k + 2 * e], st[8 * k + 2 * e + 1], hi[e], lo[e]);
-            const uint32_t o = ssd_sw128(row, 32 * half + 8 * k);
-            *reinterpret_cast<uint4 *>(sm + S::kS + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-            *reinterpret_cast<uint4 *>(sm + S::kS + S::kTile + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-        }
-    };
-
-    // Chunks overlap on the tensor core: unit u + 1's G = C B^T is issued as soon as
-    // unit u's MMA2/4 have read L o G out of its TMEM columns, and runs during
-    // unit u's epilogue 2; unit u's Yo = C S^T is issued before its epilogue 1,
-    // which does not need it.  Each MMA group commits to its own mbarrier, one
-    // phase per unit; the counts below let a walk that gives up drain them.
-    int64_t loads_issued = 0, loads_waited = 0;
-    uint32_t committed[5] = {0, 0, 0, 0, 0}, waited[5] = {0, 0, 0, 0, 0};
-    // the running sums of unit x's chunk: first dt and the running sum within each
-    // warp (threads 0..127; the warp's total to wsum), then, after a barrier, the
-    // sums of the warps before it; cs, dt and F to their tables.  Returns whether
-    // this thread's |cs| is at most 80 (threads 128.. return true).
-    float s = 0.0f, dtv = 0.0f;
-    auto sums_in_warp = [&](const SsdUnit &x, float raw, float bias_x, float A_x) {
-        if (tid < kSsdQ) {
-            dtv = 0.0f;
-            if (static_cast<int64_t>(x.c) * kSsdQ + tid < L) {
-                const float v = raw + bias_x;
-                dtv = p.softplus ? softplus_fast(v) : v;
-            }
-            s = dtv * A_x;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float o = __shfl_up_sync(0xffffffffu, s, off);
-                if (lane >= off) s += o;
-            }
-            if (lane == 31) wsum[warp] = s;
-        }
-    };
-    auto sums_across_warps = [&]() -> bool {
-        if (tid >= kSsdQ) return true;
-        for (int w = 0; w < warp; ++w) s += wsum[w];
-        cs[tid] = s;
-        dts[tid] = dtv;
-        Fs[tid] = __expf(-s) * dtv;
-        return fabsf(s) <= 80.0f;
-    };
-
-    // Per unit u: cur is unit u, nxt unit u + 1, nn unit u + 2 (whose dt is loaded
-    // while u runs); the cs tables hold unit u's, and unit u + 1's are formed while
-    // u's MMA2 and MMA4 run (epilogue 2 keeps what it needs in registers).
-    SsdUnit cur = rg.first_unit(), nxt = cur;
-    if (units > 1) rg.advance(nxt, 0);
-    bool ok = units > 0;
-    if (ok) {
-        if (tid == 0) load(cur, 0);
-        loads_issued = 1;
-    }
-    // the head's A, dt bias and D (the next unit's are loaded a unit ahead)
-    float Ah = p.A[cur.h], bias = p.dt_bias ? p.dt_bias[cur.h] : 0.0f, Dh = p.D ? p.D[cur.h] : 0.0f;
-    float dt_raw = ok && tid < kSsdQ ? load_dt(cur) : 0.0f;
-    bool factored = true;  // every |cs| of the unit's chunk at most 80: exp(cs_i - cs_j) = exp(cs_i) exp(-cs_j)
-    if (ok) {
-        ok = begin_part(cur.seq, cur.c);
-        write_state();
-        sums_in_warp(cur, dt_raw, bias, Ah);
-        if (units > 1 && tid < kSsdQ) dt_raw = load_dt(nxt);
-        __syncthreads();
-        factored = __syncthreads_and(sums_across_warps()) != 0;
-    }
-
+    // TMEM columns: G then L o G (128); Yd and Yo (64 each: the products of the
+    // high and the low operand parts accumulated, in issue order); ST (128: the
+    // products with w o X high and low side by side, one N = 128 MMA); the
+    // carried state S (64: lane n holds S[p][n] in column p)
+    const uint32_t tG = tbase, tYd = tbase + 128, tYo = tbase + 192, tST = tbase + 256, tS = tbase + 384;
     const uint32_t a_s = smem_u32(sm + S::kS), a_xw = smem_u32(sm + S::kXw);
-    // a descriptor of base + off is the base's plus off / 16 (no carry: every
-    // shared-memory address is below 2^18)
-    auto issue_g = [&](int64_t u) {  // MMA1: G = C B^T of unit u
-        uint8_t *in = sm + (u & 1) * S::kInBytes;
-        constexpr uint32_t i1 = ssd_idesc(128, 128, 0, 0);
-        const uint64_t dC = ssd_desc(smem_u32(in + S::kInC), 16, 1024), dB = ssd_desc(smem_u32(in + S::kInB), 16, 1024);
+
+    if (producer) {
+        if (lane == 0 && units > 0) {
+            // the inputs of unit u (x) into buffer u & 1
+            auto load = [&](const SsdUnit &x, int64_t u) {
+                uint8_t *in = sm + (u & 1) * S::kInBytes;
+                uint64_t *bar = lbar + (u & 1);
+                mbar_arrive_expect_tx(bar, S::kInBytes);
+                const int t0 = static_cast<int>(x.c * kSsdQ), bi = static_cast<int>(x.b), gi = static_cast<int>(x.g);
+                tma_load_4d(in + S::kInC, &tm.C, 0, gi, t0, bi, bar);
+                tma_load_4d(in + S::kInC + S::kTile, &tm.C, 64, gi, t0, bi, bar);
+                tma_load_4d(in + S::kInB, &tm.B, 0, gi, t0, bi, bar);
+                tma_load_4d(in + S::kInB + S::kTile, &tm.B, 64, gi, t0, bi, bar);
+                tma_load_4d(in + S::kInX, &tm.x, 0, static_cast<int>(x.h), t0, bi, bar);
+            };
+            // a descriptor of base + off is the base's plus off / 16 (no carry: every
+            // shared-memory address is below 2^18)
+            SsdUnit x1 = rg.first_unit();  // the unit whose inputs are loaded next
+            int64_t loads = 0, loads_waited = 0, nG = 0, nYo = 0, n24 = 0, w24 = 0;
+            auto issue_g = [&](int64_t u) {  // MMA1: G = C B^T of unit u
+                uint8_t *in = sm + (u & 1) * S::kInBytes;
+                constexpr uint32_t i1 = ssd_idesc(128, 128, 0, 0);
+                const uint64_t dC = ssd_desc(smem_u32(in + S::kInC), 16, 1024),
+                               dB = ssd_desc(smem_u32(in + S::kInB), 16, 1024);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const uint32_t ko = ((k / 4) * S::kTile + (k % 4) * 32) >> 4;
-            ssd_mma(tG, dC + ko, dB + ko, i1, k > 0);
-        }
-        ssd_commit(mbar);
-    };
-    // a bounded wait that every thread takes the same way, and its bookkeeping
-    auto wait_all = [&](uint64_t *bar, uint32_t parity) -> bool {
-        return __syncthreads_and(ssd_wait(bar, parity, p.error)) != 0;
-    };
-    if (ok) ok = wait_all(lbar, 0u);
-    if (ok) {
-        loads_waited = 1;
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        if (tid == 0) issue_g(0);
-        committed[0] = 1;
-    }
-    for (int64_t u = 0; ok && u < units; ++u) {
-        SsdUnit nn = nxt;
-        if (u + 2 < units) rg.advance(nn, u + 1);
-        float nAh = Ah, nbias = bias, nDh = Dh;
-        if (u + 1 < units && nxt.h != cur.h) {
-            nAh = p.A[nxt.h];
-            nbias = p.dt_bias ? p.dt_bias[nxt.h] : 0.0f;
-            nDh = p.D ? p.D[nxt.h] : 0.0f;
-        }
-        const int64_t b = cur.b, h = cur.h, c = cur.c;
-        const int64_t t0 = c * kSsdQ;
-        const uint32_t ph = static_cast<uint32_t>(u & 1);
-        uint8_t *in = sm + (u & 1) * S::kInBytes;
-        const uint32_t a_c = smem_u32(in + S::kInC), a_b = smem_u32(in + S::kInB), a_x = smem_u32(in + S::kInX);
-        // the next chunk's inputs go to the other buffer, whose last readers (the
-        // previous unit's MMAs and epilogue 1) have finished; a warp that has no
-        // other work here issues them
-        if (tid == kSsdThreads - 1 && u + 1 < units) load(nxt, u + 1);
-        if (u + 1 < units) loads_issued = u + 2;
-        // S^T (written at the end of the previous unit) visible to the tensor core
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-        __syncthreads();
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        // ---- MMA3: Yo = C [S^T high | S^T low] (N = 128: the low tile is the
-        // operand's second 64-column atom, one tile on); epilogue 2 needs it
-        if (tid == 0) {
-            constexpr uint32_t i3 = ssd_idesc(128, 128, 0, 1);
-            const uint64_t dC = ssd_desc(a_c, 16, 1024), dS = ssd_desc(a_s, S::kTile, 1024);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint32_t ka = ((k / 4) * S::kTile + (k % 4) * 32) >> 4;
-                ssd_mma(tYo, dC + ka, dS + ((2048 * k) >> 4), i3, k > 0);
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t ko = ((k / 4) * S::kTile + (k % 4) * 32) >> 4;
+                    ssd_mma(tG, dC + ko, dB + ko, i1, k > 0);
+                }
+                ssd_commit(mG);
+                nG = u + 1;
+            };
+            load(x1, 0);
+            loads = 1;
+            if (units > 1) rg.advance(x1, 0);
+            bool pok = ssd_wait(lbar, 0u, p.error);
+            if (pok) {
+                loads_waited = 1;
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                issue_g(0);
             }
-            ssd_commit(mbar + 2);
+            for (int64_t u = 0; pok && u < units; ++u) {
+                const uint32_t ph = static_cast<uint32_t>(u & 1);
+                uint8_t *in = sm + (u & 1) * S::kInBytes;
+                // S^T of unit u is written, and the previous unit's epilogue 2 is done
+                // with Yo, Yd, ST and its X: the other buffer takes unit u + 1's
+                // inputs (the tensor core read them before MMA2/MMA4 of the previous
+                // unit completed)
+                if (!ssd_wait(cS, ph, p.error)) break;
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                if (u + 1 < units) {
+                    load(x1, u + 1);
+                    loads = u + 2;
+                    if (u + 2 < units) rg.advance(x1, u + 1);
+                }
+                // MMA3: Yo = C S^T, the high tile then the low one accumulated
+                {
+                    constexpr uint32_t i3 = ssd_idesc(128, 64, 0, 1);
+                    const uint64_t dC = ssd_desc(smem_u32(in + S::kInC), 16, 1024), dS = ssd_desc(a_s, S::kTile, 1024);
+#pragma unroll
+                    for (int part = 0; part < 2; ++part)
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            const uint32_t ka = ((k / 4) * S::kTile + (k % 4) * 32) >> 4;
+                            ssd_mma(tYo, dC + ka, dS + ((part * S::kTile + 2048 * k) >> 4), i3, part > 0 || k > 0);
+                        }
+                    ssd_commit(mYo);
+                    nYo = u + 1;
+                }
+                // MMA2: Yd = (L o G) X, A from TMEM, the high part then the low one
+                // accumulated; MMA4: ST = B^T [w o X high | w o X low] (N = 128: the low
+                // tile is the operand's second 64-column atom); once epilogue 1 is done
+                if (!ssd_wait(cE1, ph, p.error)) break;
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                {
+                    constexpr uint32_t i2 = ssd_idesc(128, 64, 0, 1), i4 = ssd_idesc(128, 128, 1, 1);
+                    const uint64_t dX = ssd_desc(smem_u32(in + S::kInX), S::kTile, 1024);
+                    const uint64_t dBt = ssd_desc(smem_u32(in + S::kInB), S::kTile, 1024),
+                                   dXw = ssd_desc(a_xw, S::kTile, 1024);
+#pragma unroll
+                    for (int part = 0; part < 2; ++part)
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            // K step k covers j in [16 k, 16 k + 16): column half k / 4,
+                            // 32-column block (k % 4) / 2, high or low 16 columns, 8
+                            // columns per 16 j
+                            const uint32_t acol = 64 * (k / 4) + 32 * ((k % 4) / 2) + 16 * part + 8 * (k % 2);
+                            ssd_mma_ts(tYd, tG + acol, dX + ((2048 * k) >> 4), i2, part > 0 || k > 0);
+                        }
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        ssd_mma(tST, dBt + ((2048 * k) >> 4), dXw + ((2048 * k) >> 4), i4, k > 0);
+                    ssd_commit(m24);
+                    n24 = u + 1;
+                }
+                // the next unit's G once MMA2 has read L o G out of its columns (it
+                // runs during this unit's epilogue 2)
+                if (u + 1 < units) {
+                    if (!ssd_wait(m24, ph, p.error)) break;
+                    w24 = u + 1;
+                    if (!ssd_wait(lbar + ((u + 1) & 1), static_cast<uint32_t>(((u + 1) >> 1) & 1), p.error)) break;
+                    loads_waited = u + 2;
+                    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                    issue_g(u + 1);
+                }
+            }
+            // nothing in flight when the CTA ends (at most the newest phase of each
+            // commit barrier is open: the tensor core completes MMAs in order, and
+            // G(u + 1) is issued after MMA2/MMA4(u) are done)
+            if (nG > 0) ssd_drain(mG, static_cast<uint32_t>((nG - 1) & 1), p.error);
+            if (nYo > 0) ssd_drain(mYo, static_cast<uint32_t>((nYo - 1) & 1), p.error);
+            if (n24 > w24) ssd_drain(m24, static_cast<uint32_t>((n24 - 1) & 1), p.error);
+            for (int64_t c = loads_waited; c < loads; ++c)
+                ssd_drain(lbar + (c & 1), static_cast<uint32_t>((c >> 1) & 1), p.error);
         }
-        committed[2] = static_cast<uint32_t>(u + 1);
-        // ---- G of this chunk (issued during the previous chunk's epilogue 2)
-        if (!wait_all(mbar, ph)) {
-            ok = false;
-            break;
+        __syncwarp();
+    } else {
+        const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+        // raw dt of this thread's step of unit x (zero past the end)
+        auto load_dt = [&](const SsdUnit &x) -> float {
+            const int64_t t = x.c * kSsdQ + tid;
+            return t < L ? Act<bf16raw>::load(p.dt, (x.b * L + t) * H + x.h) : 0.0f;
+        };
+        // a bounded wait that every epilogue thread takes the same way
+        auto cwait = [&](uint64_t *bar, uint32_t parity) -> bool {
+            return ssd_cbar_and(ssd_wait(bar, parity, p.error));
+        };
+
+        // This thread's share of the state, S[p][n] for n = row and p in [32 half,
+        // 32 half + 32), lives in its TMEM lane, columns tS + p; it moves through
+        // registers 16 values at a time.
+        const uint32_t t_s = tS + lane_off + 32 * half;
+        auto put_state = [&](int q0, const float (&v)[16]) {
+            uint32_t r[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(v[e]);
+            ssd_st16(t_s + q0, r);
+        };
+        // S^T [n][p] high and low tiles, columns q0 .. q0 + 15 of this thread's half
+        auto put_state_tiles = [&](int q0, const float (&v)[16]) {
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) split_pair(v[8 * k + 2 * e], v[8 * k + 2 * e + 1], hi[e], lo[e]);
+                const uint32_t o = ssd_sw128(row, 32 * half + q0 + 8 * k);
+                *reinterpret_cast<uint4 *>(sm + S::kS + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4 *>(sm + S::kS + S::kTile + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+        };
+        // S^T of the state in TMEM to shared memory; then the producer may issue MMA3
+        auto write_state = [&]() {
+#pragma unroll
+            for (int q0 = 0; q0 < 32; q0 += 16) {
+                float v[16];
+                ssd_ld16(t_s + q0, v);
+                put_state_tiles(q0, v);
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+            ssd_arrive(cS);
+        };
+        // the state a part starts from: h0 (or zero) at a sequence start, else the
+        // one the previous CTA handed on (a bounded wait on its flag); into TMEM
+        auto begin_part = [&](int64_t seq, int64_t c) -> bool {
+            const float *src = nullptr;
+            if (c == 0) {
+                src = p.h0 ? p.h0 + seq * kSsdP * kSsdN : nullptr;
+            } else {
+                bool got = true;
+                if (tid == 0) {
+                    got = false;
+                    const uint32_t *flag = p.flags + (kcta - 1);
+                    for (uint32_t n = 0; n < p.spin_limit; ++n) {
+                        if (ld_acquire(flag) >= p.flag_want) {
+                            got = true;
+                            break;
+                        }
+                        if ((n & 255u) == 255u && *reinterpret_cast<volatile uint32_t *>(p.error) != 0) break;
+                        __nanosleep(64);
+                    }
+                    if (!got && *reinterpret_cast<volatile uint32_t *>(p.error) == 0) atomicOr(p.error, 2u);
+                }
+                if (!ssd_cbar_and(got)) return false;
+                src = p.slots + (kcta - 1) * (kSsdP * kSsdN);
+            }
+#pragma unroll
+            for (int q0 = 0; q0 < 32; q0 += 16) {
+                float v[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) v[e] = src ? __ldcg(src + (32 * half + q0 + e) * kSsdN + row) : 0.0f;
+                put_state(q0, v);
+            }
+            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+            return true;
+        };
+        // the state at the end of a part (from TMEM): h_last at a sequence end, else
+        // to this CTA's hand-off slot, then its flag (release)
+        auto end_part = [&](int64_t seq, bool handoff) {
+            float *dst = handoff ? p.slots + kcta * (kSsdP * kSsdN) : p.h_last ? p.h_last + seq * kSsdP * kSsdN : nullptr;
+            if (dst) {
+#pragma unroll
+                for (int q0 = 0; q0 < 32; q0 += 16) {
+                    float v[16];
+                    ssd_ld16(t_s + q0, v);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) dst[(32 * half + q0 + e) * kSsdN + row] = v[e];
+                }
+            }
+            if (handoff) {
+                ssd_cbar();
+                if (tid == 0) {
+                    __threadfence();
+                    st_release(p.flags + kcta, 1u);
+                }
+            }
+        };
+        // the running sums of unit x's chunk: first dt and the running sum within
+        // each warp (threads 0..127; the warp's total to wsum), then, after a
+        // barrier, the sums of the warps before it; cs, dt and F to their tables.
+        // Returns whether this thread's |cs| is at most 80 (threads 128.. true).
+        float s = 0.0f, dtv = 0.0f;
+        auto sums_in_warp = [&](const SsdUnit &x, float raw, float bias_x, float A_x) {
+            if (tid < kSsdQ) {
+                dtv = 0.0f;
+                if (static_cast<int64_t>(x.c) * kSsdQ + tid < L) {
+                    const float v = raw + bias_x;
+                    dtv = p.softplus ? softplus_fast(v) : v;
+                }
+                s = dtv * A_x;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float o = __shfl_up_sync(0xffffffffu, s, off);
+                    if (lane >= off) s += o;
+                }
+                if (lane == 31) wsum[warp] = s;
+            }
+        };
+        auto sums_across_warps = [&]() -> bool {
+            if (tid >= kSsdQ) return true;
+            for (int w = 0; w < warp; ++w) s += wsum[w];
+            cs[tid] = s;
+            dts[tid] = dtv;
+            Fs[tid] = __expf(-s) * dtv;
+            return fabsf(s) <= 80.0f;
+        };
+
+        // Per unit u: cur is unit u, nxt unit u + 1, nn unit u + 2 (whose dt is
+        // loaded while u runs); the cs tables hold unit u's, and unit u + 1's are
+        // formed while u's MMA2 and MMA4 run (epilogue 2 keeps what it needs in
+        // registers).
+        SsdUnit cur = rg.first_unit(), nxt = cur;
+        if (units > 1) rg.advance(nxt, 0);
+        bool ok = units > 0;
+        // the head's A, dt bias and D (the next unit's are loaded a unit ahead)
+        float Ah = 0.0f, bias = 0.0f, Dh = 0.0f;
+        float dt_raw = 0.0f;
+        bool factored = true;  // every |cs| of the chunk at most 80: exp(cs_i - cs_j) = exp(cs_i) exp(-cs_j)
+        if (ok) {
+            Ah = p.A[cur.h];
+            bias = p.dt_bias ? p.dt_bias[cur.h] : 0.0f;
+            Dh = p.D ? p.D[cur.h] : 0.0f;
+            if (tid < kSsdQ) dt_raw = load_dt(cur);
+            ok = begin_part(cur.seq, cur.c);
+            if (ok) write_state();
+            sums_in_warp(cur, dt_raw, bias, Ah);
+            if (units > 1 && tid < kSsdQ) dt_raw = load_dt(nxt);
+            ssd_cbar();
+            factored = ssd_cbar_and(sums_across_warps());
         }
-        waited[0] = static_cast<uint32_t>(u + 1);
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        for (int64_t u = 0; ok && u < units; ++u) {
+            SsdUnit nn = nxt;
+            if (u + 2 < units) rg.advance(nn, u + 1);
+            float nAh = Ah, nbias = bias, nDh = Dh;
+            if (u + 1 < units && nxt.h != cur.h) {
+                nAh = p.A[nxt.h];
+                nbias = p.dt_bias ? p.dt_bias[nxt.h] : 0.0f;
+                nDh = p.D ? p.D[nxt.h] : 0.0f;
+            }
+            const int64_t b = cur.b, h = cur.h, c = cur.c;
+            const int64_t t0 = c * kSsdQ;
+            const uint32_t ph = static_cast<uint32_t>(u & 1);
+            uint8_t *in = sm + (u & 1) * S::kInBytes;
+            // G of this unit, and its inputs (X for epilogue 1)
+            if (!ssd_cbar_and(ssd_wait(mG, ph, p.error) &&
+                              ssd_wait(lbar + (u & 1), static_cast<uint32_t>((u >> 1) & 1), p.error))) {
+                ok = false;
+                break;
+            }
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         const float total = cs[kSsdQ - 1];
-        float dx[32];  // D x of this thread's row and column half, kept for epilogue 2
         float ecs;     // exp(cs) of this thread's row, kept for epilogue 2
         {
             // ---- epilogue 1a: row i of L o G, columns j in [64 half, 64 half + 64), 32
@@ -529,7 +636,7 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
             const int i = row;
             const float csi = cs[i], Ei = __expf(csi);
             ecs = Ei;
-#pragma unroll
+#pragma unroll 1
             for (int jp = 0; jp < 2; ++jp) {
                 const uint32_t col = tG + lane_off + 64 * half + 32 * jp;
                 float v[32];
@@ -566,7 +673,7 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
                 ssd_st16(col, mh);
                 ssd_st16(col + 16, ml);
             }
-            // ---- epilogue 1b: row t of w o X (high and low tiles) and D x, p in [32 half, 32 half + 32)
+            // ---- epilogue 1b: row t of w o X (high and low tiles), p in [32 half, 32 half + 32)
             const int t = row;
             const float w = __expf(total - cs[t]) * dts[t];
 #pragma unroll
@@ -578,8 +685,6 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float x0 = __uint_as_float(xw[e] << 16), x1 = __uint_as_float(xw[e] & 0xffff0000u);
-                    dx[8 * k + 2 * e] = Dh * x0;
-                    dx[8 * k + 2 * e + 1] = Dh * x1;
                     split_pair(w * x0, w * x1, hi[e], lo[e]);
                 }
                 *reinterpret_cast<uint4 *>(sm + S::kXw + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
@@ -589,71 +694,30 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-        __syncthreads();
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        // ---- MMA2: Yd = (L o G high) X | (L o G low) X, A from TMEM, by threads 0
-        // and 64; MMA4: ST = B^T [w o X high | w o X low] (N = 128), by thread 32:
-        // three threads issue at once
-        if (tid == 0 || tid == 64) {
-            const int part = tid >> 6;
-            constexpr uint32_t i2 = ssd_idesc(128, 64, 0, 1);
-            const uint64_t dX = ssd_desc(a_x, S::kTile, 1024);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                // K step k covers j in [16 k, 16 k + 16): column half k / 4, 32-column
-                // block (k % 4) / 2, high or low 16 columns, 8 columns per 16 j
-                const uint32_t acol = 64 * (k / 4) + 32 * ((k % 4) / 2) + 16 * part + 8 * (k % 2);
-                ssd_mma_ts(tYd + 64 * part, tG + acol, dX + ((2048 * k) >> 4), i2, k > 0);
-            }
-            ssd_commit(mbar + (part ? 4 : 1));
-        } else if (tid == 32) {
-            constexpr uint32_t i4 = ssd_idesc(128, 128, 1, 1);
-            const uint64_t dBt = ssd_desc(a_b, S::kTile, 1024), dXw = ssd_desc(a_xw, S::kTile, 1024);
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-                ssd_mma(tST, dBt + ((2048 * k) >> 4), dXw + ((2048 * k) >> 4), i4, k > 0);
-            ssd_commit(mbar + 3);
-        }
-        committed[1] = committed[3] = committed[4] = static_cast<uint32_t>(u + 1);
-        // ---- meanwhile the next unit's running sums (its dt loaded a unit ago)
+        ssd_arrive(cE1);
+        // ---- meanwhile the next unit's running sums (its dt loaded a unit ago),
+        // once every epilogue thread is done with this unit's tables
+        ssd_cbar();
         if (u + 1 < units) {
             sums_in_warp(nxt, dt_raw, nbias, nAh);
             if (u + 2 < units && tid < kSsdQ) dt_raw = load_dt(nn);
         }
-        if (!wait_all(mbar + 1, ph)) {
-            ok = false;
-            break;
-        }
-        waited[1] = static_cast<uint32_t>(u + 1);
-        // the tables are free: epilogue 1 has read them, epilogue 2 needs none
+        ssd_cbar();
         const bool fac_next = u + 1 < units ? sums_across_warps() : true;
         bool factored_next = true;
         {
-            // the other three MMA groups, and whether every |cs| of the next unit is
+            // Yo, Yd and ST of this unit, and whether every |cs| of the next unit is
             // at most 80, in one barrier (two more only when that is not so)
-            const bool w = ssd_wait(mbar + 4, ph, p.error) && ssd_wait(mbar + 3, ph, p.error) &&
-                           ssd_wait(mbar + 2, ph, p.error);
-            if (!__syncthreads_and(w && fac_next)) {
-                factored_next = __syncthreads_and(fac_next) != 0;
-                if (!__syncthreads_and(w)) {
+            const bool w = ssd_wait(mYo, ph, p.error) && ssd_wait(m24, ph, p.error);
+            if (!ssd_cbar_and(w && fac_next)) {
+                factored_next = ssd_cbar_and(fac_next);
+                if (!ssd_cbar_and(w)) {
                     ok = false;
                     break;
                 }
             }
         }
-        waited[2] = waited[3] = waited[4] = static_cast<uint32_t>(u + 1);
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        // ---- the next chunk's G: its inputs have landed and G's columns are read
-        if (u + 1 < units) {
-            if (!wait_all(lbar + ((u + 1) & 1), static_cast<uint32_t>(((u + 1) >> 1) & 1))) {
-                ok = false;
-                break;
-            }
-            loads_waited = u + 2;
-            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            if (tid == 0) issue_g(u + 1);
-            committed[0] = static_cast<uint32_t>(u + 2);
-        }
         // ---- epilogue 2: y row i, p in [32 half, 32 half + 32); state row n, same p
         {
             const int i = row;
@@ -662,40 +726,47 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
 #pragma unroll
             for (int q0 = 0; q0 < 32; q0 += 16) {
                 float yd[16], yo[16];
-                {
-                    float lo[16];
-                    ssd_ld16(tYo + lane_off + 32 * half + q0, yo);
-                    ssd_ld16(tYo + 64 + lane_off + 32 * half + q0, lo);
+                ssd_ld16(tYo + lane_off + 32 * half + q0, yo);
+                ssd_ld16(tYd + lane_off + 32 * half + q0, yd);
+                // D x of the row's 16 columns, from the X tile (not overwritten before
+                // this unit's epilogue 2 is done)
+                float dx[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) yo[e] += lo[e];
-                }
-                {
-                    float lo[16];
-                    ssd_ld16(tYd + lane_off + 32 * half + q0, yd);
-                    ssd_ld16(tYd + 64 + lane_off + 32 * half + q0, lo);
+                for (int k = 0; k < 2; ++k) {
+                    const uint4 xv = *reinterpret_cast<const uint4 *>(in + S::kInX + ssd_sw128(i, 32 * half + q0 + 8 * k));
+                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) yd[e] += lo[e];
+                    for (int e = 0; e < 4; ++e) {
+                        dx[8 * k + 2 * e] = Dh * __uint_as_float(xw[e] << 16);
+                        dx[8 * k + 2 * e + 1] = Dh * __uint_as_float(xw[e] & 0xffff0000u);
+                    }
                 }
                 uint32_t pk[8];
 #pragma unroll
                 for (int e = 0; e < 16; e += 2)
-                    pk[e / 2] = pack_bf16x2(fmaf(ecs, yo[e], yd[e]) + dx[q0 + e],
-                                            fmaf(ecs, yo[e + 1], yd[e + 1]) + dx[q0 + e + 1]);
+                    pk[e / 2] = pack_bf16x2(fmaf(ecs, yo[e], yd[e]) + dx[e],
+                                            fmaf(ecs, yo[e + 1], yd[e + 1]) + dx[e + 1]);
                 if (t < L) {
                     uint4 *dst = reinterpret_cast<uint4 *>(yg + ((b * L + t) * H + h) * kSsdP + 32 * half + q0);
                     dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                     dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
                 }
             }
+            // S <- exp(cs_last) S + ST, in TMEM
             const float et = __expf(total);
 #pragma unroll
             for (int q0 = 0; q0 < 32; q0 += 16) {
-                float v[16], lo[16];
+                float v[16], sv[16];
                 ssd_ld16(tST + lane_off + 32 * half + q0, v);
-                ssd_ld16(tST + 64 + lane_off + 32 * half + q0, lo);
+                ssd_ld16(tST + 64 + lane_off + 32 * half + q0, sv);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) st[q0 + e] = fmaf(et, st[q0 + e], v[e] + lo[e]);
+                for (int e = 0; e < 16; ++e) v[e] += sv[e];
+                ssd_ld16(t_s + q0, sv);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) sv[e] = fmaf(et, sv[e], v[e]);
+                put_state(q0, sv);
             }
+            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
         }
         // the end of a part (h_last, or the hand-off to the next CTA); the state the
         // next unit starts from, as MMA3's operand
@@ -713,15 +784,9 @@ __global__ void __launch_bounds__(kSsdThreads, 1) ssd_fwd_kernel(const SsdParams
         bias = nbias;
         Dh = nDh;
         factored = factored_next;
-        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+        }
     }
-    // a wait that gave up leaves no load or MMA running when the CTA ends
-    if (!ok && tid == 0) {
-        for (int g = 0; g < 5; ++g)
-            for (uint32_t n = waited[g]; n < committed[g]; ++n) ssd_drain(mbar + g, n & 1u, p.error);
-        for (int64_t c = loads_waited; c < loads_issued; ++c)
-            ssd_drain(lbar + (c & 1), static_cast<uint32_t>((c >> 1) & 1), p.error);
-    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tbase));

@@ -87,52 +87,48 @@ __global__ void __launch_bounds__(kStepThreads) scan_step_kernel(const StepParam
     using AT = Act<T>;
     constexpr bool kAccurate = AT::kBytes == 4;
     __shared__ __align__(16) float4 hs[kStepPasses][kStepThreads];
+    // channel indices in 32 bits when every one fits (offsets widen once, at the pointer)
+    using Ix = std::conditional_t<SMALL, uint32_t, int64_t>;
     const int tid = threadIdx.x, q = tid & 3;
-    const int64_t nchan = p.batch * p.dim;
-    const int64_t base = static_cast<int64_t>(blockIdx.x) * kStepTile + (tid >> 2);
+    const Ix nchan = static_cast<Ix>(p.batch * p.dim), dim = static_cast<Ix>(p.dim);
+    const Ix base = static_cast<Ix>(blockIdx.x) * kStepTile + static_cast<Ix>(tid >> 2);
 #pragma unroll
     for (int k = 0; k < kStepPasses; ++k) {
-        const int64_t chan = base + k * (kStepThreads / 4);
-        const int64_t c = chan < nchan ? chan : nchan - 1;
-        step_copy16(&hs[k][tid], p.state + c * kNState + q * 4, chan < nchan ? 16u : 0u);
+        const Ix chan = base + k * (kStepThreads / 4);
+        const Ix c = chan < nchan ? chan : nchan - 1;
+        step_copy16(&hs[k][tid], p.state + static_cast<uint64_t>(c) * kNState + q * 4, chan < nchan ? 16u : 0u);
     }
     // (b, d) of the first pass's channel by one division; the later passes' by
     // stepping kStepThreads / 4 channels on (inactive lanes keep the last channel)
-    int64_t b, d;
+    Ix b, d;
     {
-        const int64_t c = base < nchan ? base : nchan - 1;
-        if constexpr (SMALL) {
-            const uint32_t c32 = static_cast<uint32_t>(c), dim32 = static_cast<uint32_t>(p.dim);
-            b = c32 / dim32;
-            d = c32 - static_cast<uint32_t>(b) * dim32;
-        } else {
-            b = c / p.dim;
-            d = c % p.dim;
-        }
+        const Ix c = base < nchan ? base : nchan - 1;
+        b = c / dim;
+        d = c - b * dim;
     }
 #pragma unroll
     for (int k = 0; k < kStepPasses; ++k) {
-        const int64_t chan = base + k * (kStepThreads / 4);
+        const Ix chan = base + k * (kStepThreads / 4);
         const bool active = chan < nchan;
-        const int64_t c = active ? chan : nchan - 1;  // inactive lanes still join the shuffles
+        const Ix c = active ? chan : nchan - 1;  // inactive lanes still join the shuffles
         if (k > 0) {
             if (active) {
                 d += kStepThreads / 4;
-                while (d >= p.dim) {  // once at most when dim >= kStepThreads / 4
-                    d -= p.dim;
+                while (d >= dim) {  // once at most when dim >= kStepThreads / 4
+                    d -= dim;
                     ++b;
                 }
             } else {
-                b = (nchan - 1) / p.dim;
-                d = (nchan - 1) - b * p.dim;
+                b = (nchan - 1) / dim;
+                d = (nchan - 1) - b * dim;
             }
         }
-        const float4 a = *reinterpret_cast<const float4 *>(p.A + d * kNState + q * 4);
+        const float4 a = *reinterpret_cast<const float4 *>(p.A + static_cast<uint64_t>(d) * kNState + q * 4);
         float xf = AT::load(p.x, c);
         float v = AT::load(p.delta, c);
         const float zf = p.z && q == 0 ? AT::load(p.z, c) : 0.0f;
         if (p.delta_bias) v += p.delta_bias[d];
-        const int64_t bn = b * kNState + q * 4;
+        const int64_t bn = static_cast<int64_t>(static_cast<uint64_t>(b) * kNState) + q * 4;
         const float4 Bv = load4<T>(p.B, bn), Cv = load4<T>(p.C, bn);
         if constexpr (CONV) {
             float window[3] = {0.0f, 0.0f, 0.0f};
@@ -182,7 +178,7 @@ __global__ void __launch_bounds__(kStepThreads) scan_step_kernel(const StepParam
         y += __shfl_xor_sync(0xffffffffu, y, 2);
 
         if (active) {
-            *reinterpret_cast<float4 *>(p.state + c * kNState + q * 4) = h;
+            *reinterpret_cast<float4 *>(p.state + static_cast<uint64_t>(c) * kNState + q * 4) = h;
             if (q == 0) {
                 if (p.D) y += p.D[d] * xf;
                 if (p.z) y *= kAccurate ? silu_accurate(zf) : silu_fast(zf);

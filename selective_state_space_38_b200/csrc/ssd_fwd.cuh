@@ -460,10 +460,6 @@ __global__ void __launch_bounds__(kSsdThreads, 1)
             const int64_t t = x.c * kSsdQ + tid;
             return t < L ? Act<bf16raw>::load(p.dt, (x.b * L + t) * H + x.h) : 0.0f;
         };
-        // a bounded wait that every epilogue thread takes the same way
-        auto cwait = [&](uint64_t *bar, uint32_t parity) -> bool {
-            return ssd_cbar_and(ssd_wait(bar, parity, p.error));
-        };
 
         // This thread's share of the state, S[p][n] for n = row and p in [32 half,
         // 32 half + 32), lives in its TMEM lane, columns tS + p; it moves through
